@@ -1,0 +1,374 @@
+"""Benchmark of the hard-routed sparse MoE layer forward on B200.
+
+One step = one whole-layer forward (router logits, softmax/top-k, row sort,
+grouped gate|up + SwiGLU, grouped down, combine) over one batch of seeded
+synthetic input already resident in HBM, through the C ABI (moe_forward,
+captured once in a CUDA graph and replayed).
+
+Default workload: the 2,048-token prefill chunk (T=2048, d=2048, E=512,
+top-10, F=512, 4-bit affine group-64 experts, bf16 activations). The decode
+layer at T=1 and T=32 is timed in the same run and reported under
+"decode".
+
+Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank runs an
+independent replica on its own tokens (no collective on the data path);
+value = all ranks' tokens / max-over-ranks device time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU fp64 oracle on host cores
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ accounting
+
+def expert_bytes(ex) -> int:
+    return ex.nbytes_per_expert()
+
+
+def gate_up_bytes(ex) -> int:
+    tot = ex.w_gu[0].numel() * ex.w_gu.element_size()
+    for t in (ex.s_gu, ex.b_gu):
+        if t is not None:
+            tot += t[0].numel() * t.element_size()
+    return tot
+
+
+def kernels_per_forward(T, k, regime_tc: bool) -> int:
+    R = T * k
+    sort = 1 if R <= 1024 else 3
+    return 2 + sort + 2 + 1   # router logits + top-k, sort, gate|up, down, combine
+
+
+# ------------------------------------------------------------------ timing
+
+def time_device(fn, steps, warmup, flush):
+    """Per-step CUDA-event time (ms) of fn() on the current stream; the L2 is
+    flushed (a 256 MB write) before every step, outside the timed events."""
+    for _ in range(warmup):
+        fn()
+    s = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.add_(1)
+        starts[i].record(s)
+        fn()
+        ends[i].record(s)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in zip(starts, ends)]
+
+
+def run_ours(args, rank, world, local_rank):
+    import sparse_mixture_experts_top_b200 as moe
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+    wl = mi.WORKLOADS[args.workload]
+    layer = mi.make_layer(wl, seed=args.seed + 1000 * rank, device=dev)
+    ex = layer.experts
+    k, T = wl.k, wl.T
+    ws = moe.forward_workspace(layer.x, ex, k)
+    y = torch.empty(T, wl.d, dtype=layer.x.dtype, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    L = moe.forward_layout(T, wl.d, wl.E, k, wl.F, layer.x.dtype)
+
+    def fwd():
+        moe.forward(layer.x, layer.w_router, layer.router_bias, ex, k, ws=ws, out=y)
+
+    fwd()
+    torch.cuda.synchronize()
+    # CUDA graph of one forward
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    torch.cuda.synchronize()
+
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    ms = time_device(g.replay, args.steps, args.warmup, flush)
+    clocks = sampler.stop()
+    ms_eager = time_device(fwd, args.steps, 1, flush)
+    if world > 1:
+        torch.distributed.barrier()
+
+    # dominant kernel: the gate|up (SwiGLU) stage, timed alone through its C call
+    st = moe.SortTables(*(
+        ws[off:off + n * 4].view(dt) for off, n, dt in (
+            (L.order, T * k, torch.uint32), (L.inv_order, T * k, torch.uint32),
+            (L.row_map, T * k, torch.uint32), (L.counts, wl.E, torch.int32),
+            (L.row_off, wl.E + 1, torch.int32), (L.tile_off, wl.E + 1, torch.int32))), L.BM)
+    h = ws[L.h:L.h + T * k * wl.F * 2].view(torch.bfloat16).view(T * k, wl.F) \
+        if layer.x.dtype == torch.bfloat16 else None
+    regime = L.regime
+
+    def swiglu():
+        moe.lib.moe_grouped_swiglu(
+            moe._ptr(layer.x), moe._dt(layer.x), moe._ptr(st.row_map), moe._ptr(st.row_off),
+            moe._ptr(st.tile_off), L.BM, T, k, __import__("ctypes").byref(moe.experts_struct(ex)),
+            moe._ptr(h), regime, moe._stream())
+
+    fwd()
+    ms_swiglu = time_device(swiglu, args.steps, args.warmup, flush)
+    counts = st.counts.cpu().numpy()
+    active = int((counts > 0).sum())
+    gu_bytes = active * gate_up_bytes(ex) + T * wl.d * 2 + T * k * wl.F * 2
+    sw_s = statistics.mean(ms_swiglu) * 1e-3
+    achieved_gbs = gu_bytes / sw_s / 1e9
+    gu_flops = 2.0 * T * k * wl.d * 2 * wl.F
+    tflops = gu_flops / sw_s / 1e12
+
+    # end-to-end through the C ABI with host buffers: pinned x -> device,
+    # forward, y -> pinned host, inside the timed region
+    x_host = layer.x.cpu().pin_memory()
+    y_host = torch.empty(T, wl.d, dtype=layer.x.dtype).pin_memory()
+
+    def e2e():
+        layer.x.copy_(x_host, non_blocking=True)
+        g.replay()
+        y_host.copy_(y, non_blocking=True)
+
+    ms_e2e = time_device(e2e, args.steps, args.warmup, flush)
+
+    # decode rows (T = 1 and T = 32), same procedure
+    decode = {}
+    if not args.no_decode:
+        for name in ("decode_t1", "decode_t32"):
+            dl = mi.make_layer(name, seed=args.seed + 1000 * rank, device=dev)
+            dws = moe.forward_workspace(dl.x, dl.experts, dl.wl.k)
+            dy = torch.empty(dl.wl.T, dl.wl.d, dtype=dl.x.dtype, device=dev)
+            f2 = lambda: moe.forward(dl.x, dl.w_router, dl.router_bias, dl.experts, dl.wl.k,
+                                     ws=dws, out=dy)
+            f2()
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                f2()
+            torch.cuda.synchronize()
+            dms = statistics.mean(time_device(g2.replay, max(args.steps, 20), args.warmup, flush))
+            dL = moe.forward_layout(dl.wl.T, dl.wl.d, dl.wl.E, dl.wl.k, dl.wl.F, dl.x.dtype)
+            dcounts = dws[dL.counts:dL.counts + dl.wl.E * 4].view(torch.int32).cpu().numpy()
+            dbytes = int((dcounts > 0).sum()) * expert_bytes(dl.experts) + 2 * dl.wl.T * dl.wl.d * 2
+            decode[name] = {"tokens_per_s": dl.wl.T / (dms * 1e-3), "us_per_layer": dms * 1e3,
+                            "selected_expert_bytes": dbytes,
+                            "hbm_frac": dbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+            del dl, dws, g2
+
+    step_ms = statistics.mean(ms)
+    res = {"ms": step_ms, "ms_eager": statistics.mean(ms_eager), "ms_e2e": statistics.mean(ms_e2e),
+           "ms_swiglu": statistics.mean(ms_swiglu), "achieved_gbs": achieved_gbs,
+           "tflops_swiglu": tflops, "gu_bytes": gu_bytes, "clocks": clocks, "decode": decode,
+           "active": active, "regime": regime, "BM": L.BM, "pk": pk, "pk_kind": pk_kind,
+           "layer_bytes": active * expert_bytes(ex) + 2 * T * wl.d * 2,
+           "layer_flops": 6.0 * T * k * wl.d * wl.F}
+    return res, layer
+
+
+def cpu_baseline(layer, budget_s=12.0):
+    """The oracle as it stands, on this host's cores, on a bounded sample of
+    the workload's tokens (the layer is token-independent, so tokens/s of a
+    sample is the workload's rate)."""
+    import oracle
+    wl = layer.wl
+    x = layer.x.cpu()
+    wr = layer.w_router.cpu()
+    b = None if layer.router_bias is None else layer.router_bias.cpu()
+    ex = layer.experts.to("cpu")
+    nth = oracle.default_threads()
+    n = min(4, wl.T)
+    total_t, total_tok = 0.0, 0
+    while True:
+        lo = total_tok % wl.T
+        xs = x[lo: lo + n]
+        t0 = time.perf_counter()
+        oracle.forward(xs, wr, b, ex, wl.k, nthreads=nth)
+        dt = time.perf_counter() - t0
+        total_t += dt
+        total_tok += xs.shape[0]
+        if total_t >= budget_s or total_tok >= wl.T:
+            break
+        rate = xs.shape[0] / max(dt, 1e-3)
+        n = int(max(1, min(wl.T - total_tok, rate * (budget_s - total_t))))
+    return {"value": total_tok / total_t, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+            "sample": f"{total_tok} of {wl.T} tokens of the {wl.name} workload (whole layer per "
+                      f"token, fp64, {nth} threads), {total_t:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = mi.WORKLOADS[args.workload]
+    metric = "MoE-layer tokens/s"
+    config = {"workload": f"{wl.name}: T={wl.T} d={wl.d} E={wl.E} top-{wl.k} F={wl.F} "
+                          f"{wl.wfmt} experts, {wl.act} activations"
+                          + (f", router bias {wl.bias}" if wl.bias != "none" else ""),
+              "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "F": wl.F, "weights": wl.wfmt,
+              "l2": "flushed before every timed step (256 MB write, outside the events)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        layer = mi.make_layer(wl, seed=args.seed, device="cpu")
+        cb = cpu_baseline(layer, budget_s=min(60.0, max(5.0, 1.0 * args.steps)))
+        line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", timeout=__import__("datetime").timedelta(seconds=120),
+            device_id=torch.device("cuda", local_rank))
+    res, layer = run_ours(args, rank, world, local_rank)
+    ms = res["ms"]
+    ms_e2e = res["ms_e2e"]
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+    if rank == 0:
+        pk = res["pk"]
+        sw_s = res["ms_swiglu"] * 1e-3
+        line = {
+            "metric": metric, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; shapes and distributions of the workload)",
+            "config": dict(config, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                           regime={1: "gemv", 2: "tcgen05"}.get(res["regime"], "?"), BM=res["BM"],
+                           active_experts=res["active"], cuda_graph=True),
+            "roofline": {"kernel": "grouped gate|up + SwiGLU (moe_grouped_swiglu)",
+                         "bound": "hbm", "achieved": res["achieved_gbs"],
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": res["achieved_gbs"] / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": res["pk_kind"],
+                         "us_per_launch": res["ms_swiglu"] * 1e3,
+                         "tensor_tflops": res["tflops_swiglu"],
+                         "tensor_frac": res["tflops_swiglu"] / pk["bf16_tflops"]},
+            "layer_roofline": {
+                "bytes": res["layer_bytes"], "flops": res["layer_flops"],
+                "hbm_frac": res["layer_bytes"] / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "tensor_frac": res["layer_flops"] / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
+            "ms_per_step_eager": res["ms_eager"],
+            "e2e": {"value": world * wl.T / (ms_e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": wl.T * wl.d * 2, "d2h_bytes_per_step": wl.T * wl.d * 2},
+            "gpu_launches": kernels_per_forward(wl.T, wl.k, res["regime"] == 2) * args.steps,
+            "clocks": res["clocks"],
+            "decode": res["decode"],
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(layer)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) hard-routed sparse MoE layer forward.
+ *
+ * The layer, for T tokens x [T][d], E experts, top-k routing and expert
+ * hidden size F (SwiGLU experts):
+ *
+ *   logits  L = x . W_r + b                                    (moe_route)
+ *   top-k   idx[t][0..k-1], w[t][j] = softmax over the selected (moe_route / moe_topk)
+ *   sort    routed slots r = t*k + j sorted by expert           (moe_sort_rows)
+ *   gate|up h[i] = silu(x[row_map[i]] Wg_e^T) * (x[row_map[i]] Wu_e^T)
+ *                                                               (moe_grouped_swiglu)
+ *   down    ys[i] = h[i] Wd_e^T                                 (moe_grouped_down)
+ *   combine y[t] = sum_j w[t][j] * ys[inv_order[t*k + j]]       (moe_combine)
+ *
+ * and all of it in one call (moe_forward).
+ *
+ * Sources of the operations (the web pages the method is taken from):
+ *   - "5.5 real sparse MoE kernels (Metal)" (posttrainllm PRD), section
+ *     "Scope -- in": top-K routing kernel (routing_logits -> top_k_indices,
+ *     top_k_weights, no host round trip), expert dispatch, post-expert combine.
+ *   - mlxcel PR #275, "What it does": out[h] = sum_k scores[k] *
+ *     down_k(silu(gate_k(x)) * up_k(x))[h], with affine dequantised experts.
+ *   - mlx-lm PR #2044, "What" and "When it applies": experts grouped by expert
+ *     so each expert's weights are read and dequantised once per tile; affine
+ *     4-bit, group 64; a small-batch regime when tokens per expert T*k/E <= 8.
+ *   - DS4Server issue #112, "Current upstream route" and "Kernel contract":
+ *     sort_rows (argsort of flattened expert ids, inv_order = argsort(order),
+ *     row_map = order // top_k as uint32), swiglu_rows reading token rows in
+ *     place through row_map, sorted down projection, _scatter_unsort;
+ *     per-expert tile and row prefix tables with the expert found by binary
+ *     search; 32-bit row positions.
+ *   - MOE_OPTIMIZATION_COMPLETE.md (markbaseengine), "Mega Kernel
+ *     Architecture": router matmul, softmax, top-K and dispatch on the GPU
+ *     with no CPU wait in between.
+ *
+ * Conventions shared by every call:
+ *   - Pointers marked (device) are CUDA device pointers owned by the caller;
+ *     the library never allocates, frees, or keeps them after the call.
+ *     Pointers marked (host) are read before the call returns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream). The library never synchronises the stream and
+ *     never reads device data on the host.
+ *   - Argument errors are detected on the host before any launch and returned
+ *     synchronously; nothing is launched then. MOE_ERR_CUDA reports a launch
+ *     error (cudaGetLastError after the launches).
+ *   - Device-side errors (a bounded wait that ran out) are recorded in a
+ *     device status word; read and clear it with moe_device_status().
+ *   - T = 0 is valid: the call returns MOE_OK and launches nothing.
+ *   - Preconditions: 1 <= k <= min(E, 32); E <= 1024; d and F multiples of 64;
+ *     q4 and bf16 expert weights need bf16 activations, f32 weights need f32
+ *     activations. Violations return MOE_ERR_INVALID_ARG or
+ *     MOE_ERR_UNSUPPORTED.
+ *   - All layouts are row-major with the stated shapes; buffers must be
+ *     16-byte aligned.
+ *   - Calls are reentrant; the library holds no per-call state.
+ *
+ * Regimes: moe_grouped_swiglu / moe_grouped_down / moe_forward take a regime.
+ *   MOE_REGIME_GEMV: weight-streaming kernels, every selected expert's bytes
+ *     read once per step, for few tokens per expert (decode);
+ *   MOE_REGIME_TC: tensor-core grouped GEMM (tcgen05 / TMEM, TMA-staged
+ *     operands) for many tokens per expert (prefill); bf16 activations only;
+ *   MOE_REGIME_AUTO: GEMV when T*k <= 8*E, else TC (bf16) or GEMV (f32).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, k > E, misaligned ... */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but not implemented (dims, dtype/format mix) */
+  MOE_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required */
+  MOE_ERR_CUDA = 4,        /* a CUDA launch failed */
+  MOE_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out (device status) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype; /* activations */
+
+typedef enum { MOE_W_F32 = 0, MOE_W_BF16 = 1, MOE_W_Q4G64 = 2 } moe_wfmt;
+
+typedef enum { MOE_REGIME_AUTO = 0, MOE_REGIME_GEMV = 1, MOE_REGIME_TC = 2 } moe_regime;
+
+/* Expert weights (all device, read-only, caller-owned).
+ *   MOE_W_F32 / MOE_W_BF16:
+ *     w_gu [E][2F][d]  rows 0..F-1 gate, rows F..2F-1 up (fused [gate|up])
+ *     w_dn [E][d][F]
+ *     s_* and b_* unused (may be NULL)
+ *   MOE_W_Q4G64 (4-bit affine, group 64 along the input dimension;
+ *   mlx-lm PR #2044 "When it applies"):
+ *     w_gu uint32 [E][2F][d/8], s_gu, b_gu bf16 [E][2F][d/64]
+ *     w_dn uint32 [E][d][F/8],  s_dn, b_dn bf16 [E][d][F/64]
+ *     element j of a word sits in bits [4j, 4j+3] (low nibble first);
+ *     value = scale[group] * q + bias[group]. */
+typedef struct {
+  int32_t fmt; /* moe_wfmt */
+  int32_t E, d, F;
+  const void* w_gu;
+  const void* s_gu;
+  const void* b_gu;
+  const void* w_dn;
+  const void* s_dn;
+  const void* b_dn;
+} moe_experts;
+
+/* Router: logits, softmax, top-k, renormalised weights.
+ * ("5.5 real sparse MoE kernels (Metal)", Scope -- in; "Mega Kernel
+ * Architecture" phases 1-3.)
+ *   x          (device) [T][d], dtype dt
+ *   w_router   (device) [E][d], dtype dt: row e is column e of W_r [d][E]
+ *   router_bias(device) [E] fp32, or NULL; added to the logits before the
+ *              softmax and the selection
+ *   logits     (device, out) [T][E] fp32: x . W_r + b, fp32 accumulation
+ *   topk_idx   (device, out) [T][k] int32: selected experts, best first;
+ *              ties go to the lowest expert index, -0.0 == +0.0, NaN last
+ *   topk_w     (device, out) [T][k] fp32: exp(L_j - max) / sum over selected
+ *              (= softmax over all E renormalised over the selection) */
+moe_status moe_route(const void* x, moe_dtype dt, const void* w_router, const float* router_bias,
+                     int T, int d, int E, int k, float* logits, int32_t* topk_idx, float* topk_w,
+                     moe_stream_t stream);
+
+/* Softmax / top-k step alone, from given fp32 logits [T][E] (device).
+ * Same outputs and rules as moe_route. */
+moe_status moe_topk(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
+                    moe_stream_t stream);
+
+/* Dispatch: stable counting sort of the R = T*k routed slots r = t*k + j by
+ * expert id (DS4Server issue #112, "Current upstream route": sort_rows;
+ * "Kernel contract": per-expert tile and row prefix tables).
+ *   topk_idx  (device) [T][k] int32, values in [0, E)
+ *   BM        rows per tile for tile_off (>= 1)
+ *   order     (device, out) [R] uint32: order[i] = slot r of sorted row i;
+ *             rows grouped by expert (ascending), slots ascending within one
+ *   inv_order (device, out) [R] uint32: inv_order[order[i]] = i
+ *   row_map   (device, out) [R] uint32: row_map[i] = order[i] / k (token)
+ *   counts    (device, out) [E] int32: rows per expert
+ *   row_off   (device, out) [E+1] int32: exclusive scan of counts
+ *   tile_off  (device, out) [E+1] int32: exclusive scan of ceil(counts/BM)
+ *   ws        (device) scratch of moe_sort_rows_workspace(T, k, E) bytes
+ *             (contents on entry do not matter)
+ * Ids outside [0, E) are a caller error; the kernels clamp them so that no
+ * access leaves the buffers, and the result is then unspecified. */
+size_t moe_sort_rows_workspace(int T, int k, int E);
+moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, uint32_t* order,
+                         uint32_t* inv_order, uint32_t* row_map, int32_t* counts, int32_t* row_off,
+                         int32_t* tile_off, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped gate|up projection with the SwiGLU epilogue over sorted rows,
+ * reading token rows in place through row_map (DS4Server issue #112,
+ * swiglu_rows; mlxcel PR #275 "What it does").
+ *   x        (device) [T][d], dtype dt
+ *   row_map, row_off, tile_off: as written by moe_sort_rows with the same BM
+ *   h        (device, out) [T*k][F], dtype dt:
+ *            h[i][f] = silu(g) * u, g = x[row_map[i]] . w_gu[e][f],
+ *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
+ * fp32 accumulation; h rounded once to dt. */
+moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
+                              const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
+                              const moe_experts* experts, void* h, moe_regime regime,
+                              moe_stream_t stream);
+
+/* Grouped down projection over rows already sorted by expert (DS4Server
+ * issue #112, switch_linear with sorted indices).
+ *   h        (device) [T*k][F], dtype dt
+ *   ys       (device, out) [T*k][d], dtype dt: ys[i][o] = h[i] . w_dn[e][o] */
+moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
+                            const int32_t* tile_off, int BM, int T, int k,
+                            const moe_experts* experts, void* ys, moe_regime regime,
+                            moe_stream_t stream);
+
+/* Score-weighted unsort back to token order, atomic-free (DS4Server issue
+ * #112, _scatter_unsort; "5.5 real sparse MoE kernels (Metal)", scatter_add
+ * equivalent): y[t][o] = sum_{j=0..k-1} w[t][j] * ys[inv_order[t*k+j]][o],
+ * summed in fp32 in j order, rounded once to dt.
+ *   ys (device) [T*k][d], inv_order (device) [T*k], topk_w (device) [T][k]
+ *   y  (device, out) [T][d] */
+moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* topk_w, int T, int k,
+                       int d, moe_dtype dt, void* y, moe_stream_t stream);
+
+/* The whole layer in one call, on one stream, no host synchronisation
+ * (MOE_OPTIMIZATION_COMPLETE.md, "Mega Kernel Architecture": no CPU wait
+ * between router and experts).
+ *   x, w_router, router_bias: as for moe_route; experts: as above
+ *   y   (device, out) [T][d], dtype dt
+ *   ws  (device) workspace of moe_forward_workspace(...) bytes; it holds the
+ *       intermediates at the offsets moe_forward_layout() reports */
+size_t moe_forward_workspace(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime);
+moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const float* router_bias,
+                       const moe_experts* experts, int T, int k, void* y, void* ws,
+                       size_t ws_bytes, moe_regime regime, moe_stream_t stream);
+
+/* Where moe_forward keeps each intermediate inside its workspace (byte
+ * offsets), the regime it resolves to and the BM it sorts with. */
+typedef struct {
+  size_t logits, topk_idx, topk_w, order, inv_order, row_map, counts, row_off, tile_off;
+  size_t sort_ws, h, ys, total;
+  int32_t regime; /* resolved: MOE_REGIME_GEMV or MOE_REGIME_TC */
+  int32_t BM;
+} moe_ws_layout;
+moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime,
+                              moe_ws_layout* out /* (host, out) */);
+
+/* Read the device status word (MOE_OK or the first device-side error since
+ * the last read) and reset it. Synchronises the current device. */
+moe_status moe_device_status(void);
+
+const char* moe_status_str(moe_status s);
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

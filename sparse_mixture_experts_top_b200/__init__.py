@@ -1,0 +1,252 @@
+"""Python binding of libmoe_b200.so, the sm_100a hard-routed sparse MoE
+layer forward.
+
+Argument marshalling only: every function here checks shapes and dtypes,
+allocates outputs with PyTorch on the inputs' device, passes raw device
+pointers and the current CUDA stream to the C ABI (``include/moe.h``), and
+raises on a non-OK status. All arithmetic runs in the library's CUDA
+kernels; there is no CPU path. Importing this module fails loudly if the
+library is missing or cannot be loaded.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+F32, BF16 = 0, 1
+W_F32, W_BF16, W_Q4G64 = 0, 1, 2
+REGIME_AUTO, REGIME_GEMV, REGIME_TC = 0, 1, 2
+
+EXPORTS = ("moe_route", "moe_topk", "moe_sort_rows_workspace", "moe_sort_rows",
+           "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward_workspace",
+           "moe_forward", "moe_forward_layout", "moe_device_status", "moe_status_str",
+           "moe_version")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_str(status)} (status {status})")
+        self.status = status
+
+
+class Experts(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("F", ctypes.c_int32), ("w_gu", ctypes.c_void_p), ("s_gu", ctypes.c_void_p),
+                ("b_gu", ctypes.c_void_p), ("w_dn", ctypes.c_void_p), ("s_dn", ctypes.c_void_p),
+                ("b_dn", ctypes.c_void_p)]
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("logits", "topk_idx", "topk_w", "order", "inv_order", "row_map", "counts",
+                 "row_off", "tile_off", "sort_ws", "h", "ys", "total")] + \
+               [("regime", ctypes.c_int32), ("BM", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_mixture_experts_top_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.moe_route.argtypes = [P, I, P, P, I, I, I, I, P, P, P, P]
+    L.moe_topk.argtypes = [P, I, I, I, P, P, P]
+    L.moe_sort_rows_workspace.argtypes = [I, I, I]
+    L.moe_sort_rows_workspace.restype = S
+    L.moe_sort_rows.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, S, P]
+    L.moe_grouped_swiglu.argtypes = [P, I, P, P, P, I, I, I, ctypes.POINTER(Experts), P, I, P]
+    L.moe_grouped_down.argtypes = [P, I, P, P, I, I, I, ctypes.POINTER(Experts), P, I, P]
+    L.moe_combine.argtypes = [P, P, P, I, I, I, I, P, P]
+    L.moe_forward_workspace.argtypes = [I, I, I, I, I, I, I]
+    L.moe_forward_workspace.restype = S
+    L.moe_forward.argtypes = [P, I, P, P, ctypes.POINTER(Experts), I, I, P, P, S, I, P]
+    L.moe_forward_layout.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(WsLayout)]
+    L.moe_device_status.argtypes = []
+    L.moe_status_str.argtypes = [I]
+    L.moe_status_str.restype = ctypes.c_char_p
+    L.moe_version.restype = ctypes.c_char_p
+    for name in ("moe_route", "moe_topk", "moe_sort_rows", "moe_grouped_swiglu",
+                 "moe_grouped_down", "moe_combine", "moe_forward", "moe_forward_layout",
+                 "moe_device_status"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def status_str(s: int) -> str:
+    return lib.moe_status_str(s).decode()
+
+
+def version() -> str:
+    return lib.moe_version().decode()
+
+
+def _check(st: int, what: str):
+    if st != OK:
+        raise MoeError(st, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"activations must be bfloat16 or float32, got {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and (t.device.type != "cuda" or not t.is_contiguous()):
+            raise ValueError("inputs must be contiguous CUDA tensors")
+
+
+_FMT = {"f32": W_F32, "bf16": W_BF16, "q4": W_Q4G64}
+
+
+def experts_struct(ex) -> Experts:
+    """C view of an expert-weight set (any object with fmt, E, d, F, w_gu,
+    s_gu, b_gu, w_dn, s_dn, b_dn, tensors on the device)."""
+    _dev(ex.w_gu, ex.w_dn, ex.s_gu, ex.b_gu, ex.s_dn, ex.b_dn)
+    fmt = _FMT[ex.fmt] if isinstance(ex.fmt, str) else int(ex.fmt)
+    return Experts(fmt, ex.E, ex.d, ex.F, _ptr(ex.w_gu), _ptr(ex.s_gu), _ptr(ex.b_gu),
+                   _ptr(ex.w_dn), _ptr(ex.s_dn), _ptr(ex.b_dn))
+
+
+# ------------------------------------------------------------------ stages
+
+def route(x, w_router, router_bias, k, stream=None):
+    """-> (logits fp32 [T,E], topk_idx int32 [T,k], topk_w fp32 [T,k])"""
+    _dev(x, w_router, router_bias)
+    T, d = x.shape
+    E = w_router.shape[0]
+    dev = x.device
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    _check(lib.moe_route(_ptr(x), _dt(x), _ptr(w_router), _ptr(router_bias), T, d, E, k,
+                         _ptr(logits), _ptr(idx), _ptr(w), _stream(stream)), "moe_route")
+    return logits, idx, w
+
+
+def topk(logits, k, stream=None):
+    """-> (topk_idx int32 [T,k], topk_w fp32 [T,k]) from fp32 logits [T,E]"""
+    _dev(logits)
+    T, E = logits.shape
+    idx = torch.empty(T, k, dtype=torch.int32, device=logits.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
+    _check(lib.moe_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(w), _stream(stream)), "moe_topk")
+    return idx, w
+
+
+@dataclass
+class SortTables:
+    order: torch.Tensor
+    inv_order: torch.Tensor
+    row_map: torch.Tensor
+    counts: torch.Tensor
+    row_off: torch.Tensor
+    tile_off: torch.Tensor
+    BM: int
+
+
+def sort_rows(topk_idx, E, BM, stream=None) -> SortTables:
+    _dev(topk_idx)
+    T, k = topk_idx.shape
+    R = T * k
+    dev = topk_idx.device
+    u32 = lambda n: torch.empty(n, dtype=torch.uint32, device=dev)
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device=dev)
+    order, inv, rmap = u32(R), u32(R), u32(R)
+    counts, roff, toff = i32(E), i32(E + 1), i32(E + 1)
+    nws = lib.moe_sort_rows_workspace(T, k, E)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    _check(lib.moe_sort_rows(_ptr(topk_idx), T, k, E, BM, _ptr(order), _ptr(inv), _ptr(rmap),
+                             _ptr(counts), _ptr(roff), _ptr(toff), _ptr(ws), nws,
+                             _stream(stream)), "moe_sort_rows")
+    return SortTables(order, inv, rmap, counts, roff, toff, BM)
+
+
+def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, stream=None):
+    """-> h [T*k, F] in x's dtype"""
+    _dev(x)
+    T = x.shape[0]
+    ex = experts_struct(experts)
+    h = torch.empty(T * k, experts.F, dtype=x.dtype, device=x.device)
+    _check(lib.moe_grouped_swiglu(_ptr(x), _dt(x), _ptr(tables.row_map), _ptr(tables.row_off),
+                                  _ptr(tables.tile_off), tables.BM, T, k, ctypes.byref(ex),
+                                  _ptr(h), regime, _stream(stream)), "moe_grouped_swiglu")
+    return h
+
+
+def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, stream=None):
+    """-> ys [T*k, d] in h's dtype"""
+    _dev(h)
+    ex = experts_struct(experts)
+    ys = torch.empty(T * k, experts.d, dtype=h.dtype, device=h.device)
+    _check(lib.moe_grouped_down(_ptr(h), _dt(h), _ptr(tables.row_off), _ptr(tables.tile_off),
+                                tables.BM, T, k, ctypes.byref(ex), _ptr(ys), regime,
+                                _stream(stream)), "moe_grouped_down")
+    return ys
+
+
+def combine(ys, inv_order, topk_w, T, k, stream=None):
+    """-> y [T, d] in ys's dtype"""
+    _dev(ys, inv_order, topk_w)
+    d = ys.shape[1]
+    y = torch.empty(T, d, dtype=ys.dtype, device=ys.device)
+    _check(lib.moe_combine(_ptr(ys), _ptr(inv_order), _ptr(topk_w), T, k, d, _dt(ys), _ptr(y),
+                           _stream(stream)), "moe_combine")
+    return y
+
+
+# ------------------------------------------------------------------ forward
+
+def forward_layout(T, d, E, k, F, dtype, regime=REGIME_AUTO) -> WsLayout:
+    L = WsLayout()
+    dt = BF16 if dtype == torch.bfloat16 else F32
+    _check(lib.moe_forward_layout(T, d, E, k, F, dt, regime, ctypes.byref(L)), "moe_forward_layout")
+    return L
+
+
+def forward_workspace(x, experts, k, regime=REGIME_AUTO):
+    """A workspace tensor large enough for moe_forward on these shapes."""
+    L = forward_layout(x.shape[0], experts.d, experts.E, k, experts.F, x.dtype, regime)
+    return torch.empty(max(L.total, 256), dtype=torch.uint8, device=x.device)
+
+
+def forward(x, w_router, router_bias, experts, k, regime=REGIME_AUTO, ws=None, out=None,
+            stream=None):
+    """The whole layer: y [T, d] in x's dtype."""
+    _dev(x, w_router, router_bias)
+    T = x.shape[0]
+    ex = experts_struct(experts)
+    if ws is None:
+        ws = forward_workspace(x, experts, k, regime)
+    y = out if out is not None else torch.empty(T, experts.d, dtype=x.dtype, device=x.device)
+    _check(lib.moe_forward(_ptr(x), _dt(x), _ptr(w_router), _ptr(router_bias), ctypes.byref(ex),
+                           T, k, _ptr(y), _ptr(ws), ws.numel(), regime, _stream(stream)),
+           "moe_forward")
+    return y
+
+
+def device_status() -> int:
+    """Status word of device-side errors since the last read (resets it)."""
+    return lib.moe_device_status()

@@ -1,0 +1,329 @@
+// C ABI entry points: argument checks, workspace carving, launch sequences.
+// Every check runs on the host before the first launch; nothing here reads
+// device memory or synchronises a stream (except moe_device_status).
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+__device__ int g_moe_status;   // first device-side error since the last read
+
+static int* status_ptr() {
+  static std::mutex mu;
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static inline size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+static inline size_t act_size(int dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+static moe_status launched(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
+  return MOE_ERR_CUDA;
+}
+
+static moe_status check_dims(int T, int d, int E, int k) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (k > 32 || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if ((long long)T * k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+static moe_status check_experts(const moe_experts* ex, int dt) {
+  if (!ex) return MOE_ERR_INVALID_ARG;
+  if (ex->E <= 0 || ex->d <= 0 || ex->F <= 0) return MOE_ERR_INVALID_ARG;
+  if (ex->d % 64 || ex->F % 64) return MOE_ERR_UNSUPPORTED;
+  if (!ex->w_gu || !ex->w_dn) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ex->w_gu) || !aligned16(ex->w_dn)) return MOE_ERR_INVALID_ARG;
+  switch (ex->fmt) {
+    case MOE_W_F32:
+      if (dt != MOE_F32) return MOE_ERR_UNSUPPORTED;
+      break;
+    case MOE_W_BF16:
+      if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      break;
+    case MOE_W_Q4G64:
+      if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
+      break;
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16; }
+
+// The regime a call runs: AUTO picks the weight-streaming kernels when there
+// are at most 8 routed rows per expert on average, or for fp32 activations
+// (the tensor-core kernels take bf16 operands).
+static int resolve_regime(int regime, long long R, int E, int dt) {
+  if (regime == MOE_REGIME_GEMV || regime == MOE_REGIME_TC) return regime;
+  (void)R; (void)E; (void)dt;
+  return MOE_REGIME_GEMV;   // tensor-core kernels not built yet
+}
+
+static int block_m_for(int regime, long long R, int E) {
+  if (regime == MOE_REGIME_TC) return tc_block_m();
+  return (R <= 8LL * E) ? 8 : 32;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+const char* moe_status_str(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape, dtype or format";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA launch error";
+    case MOE_ERR_TIMEOUT: return "device-side bounded wait ran out";
+  }
+  return "unknown status";
+}
+
+moe_status moe_device_status(void) {
+  int* p = status_ptr();
+  if (!p) return MOE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+  return (moe_status)v;
+}
+
+moe_status moe_topk(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
+                    moe_stream_t stream) {
+  moe_status st = check_dims(T, 64, E, k);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  return launched(launch_topk(logits, T, E, k, topk_idx, topk_w, (cudaStream_t)stream));
+}
+
+moe_status moe_route(const void* x, moe_dtype dt, const void* w_router, const float* router_bias,
+                     int T, int d, int E, int k, float* logits, int32_t* topk_idx, float* topk_w,
+                     moe_stream_t stream) {
+  moe_status st = check_dims(T, d, E, k);
+  if (st != MOE_OK) return st;
+  if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  if (d % 64) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaErrorNotSupported;
+  if (dt == MOE_BF16) e = launch_router_logits_tc(x, w_router, router_bias, T, d, E, logits,
+                                                  status_ptr(), s);
+  if (e == cudaErrorNotSupported)
+    e = launch_router_logits(x, dt, w_router, router_bias, T, d, E, logits, s);
+  if (e != cudaSuccess) return launched(e);
+  return launched(launch_topk(logits, T, E, k, topk_idx, topk_w, s));
+}
+
+size_t moe_sort_rows_workspace(int T, int k, int E) {
+  if (T < 0 || k <= 0 || E <= 0) return 0;
+  return sort_workspace_bytes((int)((long long)T * k), E);
+}
+
+moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, uint32_t* order,
+                         uint32_t* inv_order, uint32_t* row_map, int32_t* counts, int32_t* row_off,
+                         int32_t* tile_off, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_dims(T, 64, E, k);
+  if (st != MOE_OK) return st;
+  if (BM < 1) return MOE_ERR_INVALID_ARG;
+  if (!counts || !row_off || !tile_off) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !order || !inv_order || !row_map)) return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * k;
+  if (R > 1024) {
+    if (!ws) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < moe_sort_rows_workspace(T, k, E)) return MOE_ERR_WORKSPACE;
+  }
+  return launched(launch_sort_rows(topk_idx, T, k, E, BM, order, inv_order, row_map, counts,
+                                   row_off, tile_off, ws, (cudaStream_t)stream));
+}
+
+moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
+                              const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
+                              const moe_experts* experts, void* h, moe_regime regime,
+                              moe_stream_t stream) {
+  if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_experts(experts, dt);
+  if (st != MOE_OK) return st;
+  st = check_dims(T, experts->d, experts->E, k);
+  if (st != MOE_OK) return st;
+  if (BM < 1) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !row_map || !row_off || !tile_off || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * k;
+  const int rg = resolve_regime(regime, R, experts->E, dt);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rg == MOE_REGIME_TC) {
+    if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
+    return launched(launch_swiglu_tc(x, row_map, row_off, tile_off, (int)R, *experts, h,
+                                     status_ptr(), s));
+  }
+  return launched(launch_swiglu_gemv(x, dt, row_map, row_off, tile_off, BM, (int)R, *experts, h, s));
+}
+
+moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
+                            const int32_t* tile_off, int BM, int T, int k,
+                            const moe_experts* experts, void* ys, moe_regime regime,
+                            moe_stream_t stream) {
+  if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_experts(experts, dt);
+  if (st != MOE_OK) return st;
+  st = check_dims(T, experts->d, experts->E, k);
+  if (st != MOE_OK) return st;
+  if (BM < 1) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!h || !row_off || !tile_off || !ys) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(ys)) return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * k;
+  const int rg = resolve_regime(regime, R, experts->E, dt);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rg == MOE_REGIME_TC) {
+    if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
+    return launched(launch_down_tc(h, row_off, tile_off, (int)R, *experts, ys, status_ptr(), s));
+  }
+  return launched(launch_down_gemv(h, dt, row_off, tile_off, BM, (int)R, *experts, ys, s));
+}
+
+moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* topk_w, int T, int k,
+                       int d, moe_dtype dt, void* y, moe_stream_t stream) {
+  if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || k <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (k > 32) return MOE_ERR_UNSUPPORTED;
+  if (d % 64) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!ys || !inv_order || !topk_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ys) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  return launched(launch_combine(ys, inv_order, topk_w, T, k, d, dt, y, (cudaStream_t)stream));
+}
+
+moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime,
+                              moe_ws_layout* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_dims(T, d, E, k);
+  if (st != MOE_OK) return st;
+  if (F <= 0) return MOE_ERR_INVALID_ARG;
+  if (regime != MOE_REGIME_AUTO && regime != MOE_REGIME_GEMV && regime != MOE_REGIME_TC)
+    return MOE_ERR_INVALID_ARG;
+  const long long R = (long long)T * k;
+  const size_t a = act_size(dt);
+  moe_ws_layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = up256(off + bytes);
+    return at;
+  };
+  L.logits = take((size_t)T * E * 4);
+  L.topk_idx = take((size_t)R * 4);
+  L.topk_w = take((size_t)R * 4);
+  L.order = take((size_t)R * 4);
+  L.inv_order = take((size_t)R * 4);
+  L.row_map = take((size_t)R * 4);
+  L.counts = take((size_t)E * 4);
+  L.row_off = take((size_t)(E + 1) * 4);
+  L.tile_off = take((size_t)(E + 1) * 4);
+  L.sort_ws = take(sort_workspace_bytes((int)R, E));
+  L.h = take((size_t)R * F * a);
+  L.ys = take((size_t)R * d * a);
+  L.total = off;
+  L.regime = resolve_regime(regime, R, E, dt);
+  L.BM = block_m_for(L.regime, R, E);
+  *out = L;
+  return MOE_OK;
+}
+
+size_t moe_forward_workspace(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime) {
+  moe_ws_layout L;
+  if (moe_forward_layout(T, d, E, k, F, dt, regime, &L) != MOE_OK) return 0;
+  return L.total;
+}
+
+moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const float* router_bias,
+                       const moe_experts* experts, int T, int k, void* y, void* ws,
+                       size_t ws_bytes, moe_regime regime, moe_stream_t stream) {
+  if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_experts(experts, dt);
+  if (st != MOE_OK) return st;
+  const int d = experts->d, E = experts->E, F = experts->F;
+  st = check_dims(T, d, E, k);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_ws_layout L;
+  st = moe_forward_layout(T, d, E, k, F, dt, regime, &L);
+  if (st != MOE_OK) return st;
+  if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (L.regime == MOE_REGIME_TC && dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+
+  char* base = static_cast<char*>(ws);
+  float* logits = (float*)(base + L.logits);
+  int32_t* idx = (int32_t*)(base + L.topk_idx);
+  float* w = (float*)(base + L.topk_w);
+  uint32_t* order = (uint32_t*)(base + L.order);
+  uint32_t* inv = (uint32_t*)(base + L.inv_order);
+  uint32_t* rmap = (uint32_t*)(base + L.row_map);
+  int32_t* counts = (int32_t*)(base + L.counts);
+  int32_t* roff = (int32_t*)(base + L.row_off);
+  int32_t* toff = (int32_t*)(base + L.tile_off);
+  void* sws = base + L.sort_ws;
+  void* h = base + L.h;
+  void* ys = base + L.ys;
+  const long long R = (long long)T * k;
+  cudaStream_t s = (cudaStream_t)stream;
+  int* stp = status_ptr();
+
+  cudaError_t e = cudaErrorNotSupported;
+  if (dt == MOE_BF16) e = launch_router_logits_tc(x, w_router, router_bias, T, d, E, logits, stp, s);
+  if (e == cudaErrorNotSupported)
+    e = launch_router_logits(x, dt, w_router, router_bias, T, d, E, logits, s);
+  if (e != cudaSuccess) return launched(e);
+  if ((e = launch_topk(logits, T, E, k, idx, w, s)) != cudaSuccess) return launched(e);
+  if ((e = launch_sort_rows(idx, T, k, E, L.BM, order, inv, rmap, counts, roff, toff, sws, s)) !=
+      cudaSuccess)
+    return launched(e);
+  if (L.regime == MOE_REGIME_TC) {
+    if ((e = launch_swiglu_tc(x, rmap, roff, toff, (int)R, *experts, h, stp, s)) != cudaSuccess)
+      return launched(e);
+    if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s)) != cudaSuccess)
+      return launched(e);
+  } else {
+    if ((e = launch_swiglu_gemv(x, dt, rmap, roff, toff, L.BM, (int)R, *experts, h, s)) !=
+        cudaSuccess)
+      return launched(e);
+    if ((e = launch_down_gemv(h, dt, roff, toff, L.BM, (int)R, *experts, ys, s)) != cudaSuccess)
+      return launched(e);
+  }
+  return launched(launch_combine(ys, inv, w, T, k, d, dt, y, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,53 @@
+// Host-side launchers of the MoE forward kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Router logits L[T][E] = x[T][d] . w_router[E][d]^T + bias, fp32 out.
+cudaError_t launch_router_logits(const void* x, int dt, const void* w_router, const float* bias,
+                                 int T, int d, int E, float* logits, cudaStream_t s);
+// Tensor-core router (bf16 only); returns cudaErrorNotSupported when the
+// shape is outside what the kernel tiles (caller then uses the SIMT one).
+cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const float* bias, int T,
+                                    int d, int E, float* logits, int* status, cudaStream_t s);
+
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
+                        cudaStream_t s);
+
+size_t sort_workspace_bytes(int R, int E);
+cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, uint32_t* order,
+                             uint32_t* inv_order, uint32_t* row_map, int32_t* counts,
+                             int32_t* row_off, int32_t* tile_off, void* ws, cudaStream_t s);
+
+// Upper bound of tile_off[E] for R rows, E experts and BM rows per tile.
+inline long long max_tiles(long long R, int E, int BM) {
+  long long a = (R + BM - 1) / BM + (R < E ? R : E);
+  return a < R ? a : R;
+}
+
+// Weight-streaming grouped kernels (any format, any BM).
+cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
+                               const int32_t* row_off, const int32_t* tile_off, int BM, int R,
+                               const moe_experts& ex, void* h, cudaStream_t s);
+cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
+                             const int32_t* tile_off, int BM, int R, const moe_experts& ex,
+                             void* ys, cudaStream_t s);
+
+// Tensor-core grouped kernels (bf16 activations; bf16 or q4 weights).
+// BM must equal tc_block_m().
+int tc_block_m();
+cudaError_t launch_swiglu_tc(const void* x, const uint32_t* row_map, const int32_t* row_off,
+                             const int32_t* tile_off, int R, const moe_experts& ex, void* h,
+                             int* status, cudaStream_t s);
+cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
+                           const moe_experts& ex, void* ys, int* status, cudaStream_t s);
+
+cudaError_t launch_combine(const void* ys, const uint32_t* inv_order, const float* w, int T, int k,
+                           int d, int dt, void* y, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,69 @@
+"""Comparison rules shared by the GPU parity tests (test-side only)."""
+import numpy as np
+import torch
+
+# bf16 activations: max |gpu - oracle| <= 2e-2 * RMS(oracle)
+TOL_BF16 = 2e-2
+# fp32 activations and weights throughout: fp32 accumulation and one fp32
+# rounding per stored value, against fp64 -> 1e-4 * RMS leaves > 100x margin
+TOL_F32 = 1e-4
+
+
+def to_np(t):
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu()
+        if t.dtype == torch.bfloat16:
+            t = t.float()
+        if t.dtype == torch.uint32:
+            return t.view(torch.int32).numpy().view(np.uint32)
+        return t.numpy()
+    return np.asarray(t)
+
+
+def rms(a) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    return float(np.sqrt(np.mean(a * a))) if a.size else 0.0
+
+
+def assert_close_rms(gpu, ref, tol, what="", rounded_to=None):
+    """max |gpu - ref| <= tol * RMS(ref). With rounded_to="bf16" (an
+    intermediate the kernel stores in bf16) each element may in addition
+    differ by one bf16 rounding of its own value, 2^-8 * |ref| (twice the
+    half-ulp bound, for the fp32 error it is added to)."""
+    g = to_np(gpu).astype(np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
+    if r.size == 0:
+        return 0.0
+    err = np.abs(g - r)
+    bound = tol * rms(r)
+    if rounded_to == "bf16":
+        excess = err - (bound + 2.0 ** -8 * np.abs(r))
+        i = int(np.argmax(excess))
+        assert excess.flat[i] <= 0, (f"{what}: |err| {err.flat[i]:.3e} at {i} (ref {r.flat[i]:.4e}) > "
+                                     f"{tol} * RMS {rms(r):.3e} + 2^-8 |ref|")
+    else:
+        e = float(err.max())
+        assert e <= bound, f"{what}: max|err| {e:.3e} > {tol} * RMS {rms(r):.3e} = {bound:.3e}"
+    return float(err.max()) / max(rms(r), 1e-300)
+
+
+def topk_ref(logits_np, k):
+    """Top-k by (value descending, index ascending), -0 == +0, NaN last;
+    Python's sorted, for property checks of GPU output."""
+    T, E = logits_np.shape
+    out = np.empty((T, k), np.int32)
+    for t in range(T):
+        row = logits_np[t]
+        key = lambda e: (1, 0.0, e) if np.isnan(row[e]) else (0, -float(row[e]), e)
+        out[t] = sorted(range(E), key=key)[:k]
+    return out
+
+
+def kth_gap(logits_np, k):
+    """Gap between the k-th and (k+1)-th largest logit of each token."""
+    s = -np.sort(-logits_np.astype(np.float64), axis=1)
+    if logits_np.shape[1] <= k:
+        return np.full(logits_np.shape[0], np.inf)
+    return s[:, k - 1] - s[:, k]

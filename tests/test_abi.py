@@ -1,0 +1,122 @@
+"""The C ABI library: it loads, exports every symbol include/moe.h declares,
+and rejects bad arguments on the host before any launch (runs without a GPU:
+none of these calls reaches the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from sparse_mixture_experts_top_b200 import build as b
+    b.build()
+    import sparse_mixture_experts_top_b200 as m
+    return m
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("moe_route", "moe_topk", "moe_sort_rows", "moe_grouped_swiglu", "moe_grouped_down",
+              "moe_combine", "moe_forward", "moe_forward_workspace"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(moe):
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_names_match_exports(moe):
+    assert sorted(moe.EXPORTS) == _declared()
+
+
+def test_status_strings(moe):
+    for s in range(6):
+        assert moe.status_str(s)
+    assert "sm_100a" in moe.version()
+
+
+P = None   # null pointer
+
+
+def _ex(moe, fmt=2, E=8, d=128, F=256, w=0x1000):
+    return moe.Experts(fmt, E, d, F, w, w, w, w, w, w)
+
+
+def test_forward_rejects_bad_arguments_without_launching(moe):
+    L = moe.lib
+    ex = _ex(moe)
+    fake = ctypes.c_void_p(0x10000)
+    # null x
+    assert L.moe_forward(P, moe.BF16, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # k > E
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 4, 9, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # k = 0
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 4, 0, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # negative T
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), -1, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # d not a multiple of 64
+    bad = _ex(moe, d=100)
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(bad), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
+    # q4 weights with fp32 activations
+    assert L.moe_forward(fake, moe.F32, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
+    # unknown weight format
+    bad = _ex(moe, fmt=7)
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(bad), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # workspace too small / missing
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 16, 0, P) == moe.ERR_WORKSPACE
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 4, 2, fake, P, 1 << 30, 0, P) == moe.ERR_WORKSPACE
+    # misaligned x
+    assert L.moe_forward(ctypes.c_void_p(0x10008), moe.BF16, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # E too large, k too large
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(_ex(moe, E=2048)), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(_ex(moe, E=64)), 4, 33, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
+    # T = 0 is a no-op
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 0, 2, fake, fake, 0, 0, P) == moe.OK
+
+
+def test_stage_calls_reject_bad_arguments(moe):
+    L = moe.lib
+    fake = ctypes.c_void_p(0x10000)
+    ex = _ex(moe)
+    assert L.moe_topk(P, 4, 8, 2, fake, fake, P) == moe.ERR_INVALID_ARG
+    assert L.moe_topk(fake, 4, 8, 9, fake, fake, P) == moe.ERR_INVALID_ARG
+    assert L.moe_topk(fake, 0, 8, 2, fake, fake, P) == moe.OK
+    assert L.moe_route(fake, 5, fake, P, 4, 128, 8, 2, fake, fake, fake, P) == moe.ERR_INVALID_ARG
+    assert L.moe_route(fake, moe.BF16, fake, P, 4, 100, 8, 2, fake, fake, fake, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_sort_rows(fake, 4, 2, 8, 0, fake, fake, fake, fake, fake, fake, fake, 1 << 20, P) == moe.ERR_INVALID_ARG
+    assert L.moe_sort_rows(fake, 4000, 2, 8, 8, fake, fake, fake, fake, fake, fake, P, 0, P) == moe.ERR_WORKSPACE
+    assert L.moe_sort_rows(fake, 4000, 2, 8, 8, fake, fake, fake, fake, fake, fake, fake, 8, P) == moe.ERR_WORKSPACE
+    assert L.moe_grouped_swiglu(fake, moe.BF16, P, fake, fake, 8, 4, 2, ctypes.byref(ex), fake, 0, P) == moe.ERR_INVALID_ARG
+    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 0, 4, 2, ctypes.byref(ex), fake, 0, P) == moe.ERR_INVALID_ARG
+    assert L.moe_grouped_down(fake, moe.BF16, fake, fake, 8, 4, 2, P, fake, 0, P) == moe.ERR_INVALID_ARG
+    # the tensor-core regime takes bf16 activations only
+    exf = _ex(moe, fmt=0)
+    assert L.moe_grouped_down(fake, moe.F32, fake, fake, 128, 4, 2, ctypes.byref(exf), fake, 2, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_combine(fake, fake, fake, 4, 2, 100, moe.BF16, fake, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_combine(P, fake, fake, 4, 2, 128, moe.BF16, fake, P) == moe.ERR_INVALID_ARG
+    assert L.moe_combine(fake, fake, fake, 0, 2, 128, moe.BF16, fake, P) == moe.OK
+
+
+def test_forward_layout_is_consistent(moe):
+    for (T, d, E, k, F) in [(1, 2048, 128, 8, 768), (2048, 2048, 512, 10, 512), (16, 128, 8, 2, 256)]:
+        L = moe.forward_layout(T, d, E, k, F, __import__("torch").bfloat16)
+        offs = [L.logits, L.topk_idx, L.topk_w, L.order, L.inv_order, L.row_map, L.counts,
+                L.row_off, L.tile_off, L.sort_ws, L.h, L.ys]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert L.ys + T * k * d * 2 <= L.total
+        assert L.h + T * k * F * 2 <= L.ys
+        assert L.BM >= 1 and L.regime in (moe.REGIME_GEMV, moe.REGIME_TC)
+        assert moe.lib.moe_forward_workspace(T, d, E, k, F, moe.BF16, 0) == L.total
