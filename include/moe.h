@@ -169,7 +169,9 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
 /* Grouped down projection over rows already sorted by expert (DS4Server
  * issue #112, switch_linear with sorted indices).
  *   h        (device) [T*k][F], dtype dt
- *   ys       (device, out) [T*k][d], dtype dt: ys[i][o] = h[i] . w_dn[e][o] */
+ *   ys       (device, out) [T*k][d] fp32: ys[i][o] = h[i] . w_dn[e][o]
+ *            (kept in fp32 so the only rounding after the expert matmuls is
+ *            the final one of y) */
 moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
                             const int32_t* tile_off, int BM, int T, int k,
                             const moe_experts* experts, void* ys, moe_regime regime,
@@ -179,8 +181,8 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
  * #112, _scatter_unsort; "5.5 real sparse MoE kernels (Metal)", scatter_add
  * equivalent): y[t][o] = sum_{j=0..k-1} w[t][j] * ys[inv_order[t*k+j]][o],
  * summed in fp32 in j order, rounded once to dt.
- *   ys (device) [T*k][d], inv_order (device) [T*k], topk_w (device) [T][k]
- *   y  (device, out) [T][d] */
+ *   ys (device) [T*k][d] fp32, inv_order (device) [T*k], topk_w (device) [T][k]
+ *   y  (device, out) [T][d], dtype dt */
 moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* topk_w, int T, int k,
                        int d, moe_dtype dt, void* y, moe_stream_t stream);
 

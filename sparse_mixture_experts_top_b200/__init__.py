@@ -197,22 +197,25 @@ def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, stream
 
 
 def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, stream=None):
-    """-> ys [T*k, d] in h's dtype"""
+    """-> ys [T*k, d] fp32"""
     _dev(h)
     ex = experts_struct(experts)
-    ys = torch.empty(T * k, experts.d, dtype=h.dtype, device=h.device)
+    ys = torch.empty(T * k, experts.d, dtype=torch.float32, device=h.device)
     _check(lib.moe_grouped_down(_ptr(h), _dt(h), _ptr(tables.row_off), _ptr(tables.tile_off),
                                 tables.BM, T, k, ctypes.byref(ex), _ptr(ys), regime,
                                 _stream(stream)), "moe_grouped_down")
     return ys
 
 
-def combine(ys, inv_order, topk_w, T, k, stream=None):
-    """-> y [T, d] in ys's dtype"""
+def combine(ys, inv_order, topk_w, T, k, dtype=torch.bfloat16, stream=None):
+    """-> y [T, d] in `dtype` from fp32 ys [T*k, d]"""
     _dev(ys, inv_order, topk_w)
+    if ys.dtype != torch.float32:
+        raise TypeError("ys must be float32")
     d = ys.shape[1]
-    y = torch.empty(T, d, dtype=ys.dtype, device=ys.device)
-    _check(lib.moe_combine(_ptr(ys), _ptr(inv_order), _ptr(topk_w), T, k, d, _dt(ys), _ptr(y),
+    y = torch.empty(T, d, dtype=dtype, device=ys.device)
+    _check(lib.moe_combine(_ptr(ys), _ptr(inv_order), _ptr(topk_w), T, k, d,
+                           BF16 if dtype == torch.bfloat16 else F32, _ptr(y),
                            _stream(stream)), "moe_combine")
     return y
 

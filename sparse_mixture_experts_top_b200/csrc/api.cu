@@ -69,10 +69,13 @@ static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16; }
 // The regime a call runs: AUTO picks the weight-streaming kernels when there
 // are at most 8 routed rows per expert on average, or for fp32 activations
 // (the tensor-core kernels take bf16 operands).
-static int resolve_regime(int regime, long long R, int E, int dt) {
+static int resolve_regime(int regime, long long R, int E, int dt, int d = 128, int F = 128,
+                          int fmt = MOE_W_Q4G64) {
   if (regime == MOE_REGIME_GEMV || regime == MOE_REGIME_TC) return regime;
-  (void)R; (void)E; (void)dt;
-  return MOE_REGIME_GEMV;   // tensor-core kernels not built yet
+  // the tensor-core kernels tile d and F by 128 and take bf16 or q4 weights
+  if (d % 128 || F % 128 || fmt == MOE_W_F32) return MOE_REGIME_GEMV;
+  if (dt != MOE_BF16) return MOE_REGIME_GEMV;
+  return (R <= 8LL * E) ? MOE_REGIME_GEMV : MOE_REGIME_TC;
 }
 
 static int block_m_for(int regime, long long R, int E) {
@@ -176,12 +179,12 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
   if (!x || !row_map || !row_off || !tile_off || !h) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
   const long long R = (long long)T * k;
-  const int rg = resolve_regime(regime, R, experts->E, dt);
+  const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt);
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
     if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
-    return launched(launch_swiglu_tc(x, row_map, row_off, tile_off, (int)R, *experts, h,
+    return launched(launch_swiglu_tc(x, T, row_map, row_off, tile_off, (int)R, *experts, h,
                                      status_ptr(), s));
   }
   return launched(launch_swiglu_gemv(x, dt, row_map, row_off, tile_off, BM, (int)R, *experts, h, s));
@@ -201,7 +204,7 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
   if (!h || !row_off || !tile_off || !ys) return MOE_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(ys)) return MOE_ERR_INVALID_ARG;
   const long long R = (long long)T * k;
-  const int rg = resolve_regime(regime, R, experts->E, dt);
+  const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt);
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
     if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
@@ -252,9 +255,9 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.tile_off = take((size_t)(E + 1) * 4);
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
   L.h = take((size_t)R * F * a);
-  L.ys = take((size_t)R * d * a);
+  L.ys = take((size_t)R * d * 4);
   L.total = off;
-  L.regime = resolve_regime(regime, R, E, dt);
+  L.regime = resolve_regime(regime, R, E, dt, d, F);
   L.BM = block_m_for(L.regime, R, E);
   *out = L;
   return MOE_OK;
@@ -312,7 +315,7 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
       cudaSuccess)
     return launched(e);
   if (L.regime == MOE_REGIME_TC) {
-    if ((e = launch_swiglu_tc(x, rmap, roff, toff, (int)R, *experts, h, stp, s)) != cudaSuccess)
+    if ((e = launch_swiglu_tc(x, T, rmap, roff, toff, (int)R, *experts, h, stp, s)) != cudaSuccess)
       return launched(e);
     if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s)) != cudaSuccess)
       return launched(e);

@@ -11,13 +11,14 @@
 
 namespace moe {
 
-// One thread per 16 bytes of output (8 bf16 or 4 fp32 values).
+// One thread per 8 consecutive outputs of one token: k gathers of 32 bytes
+// of fp32 ys, fp32 fused multiply-adds in j order, one rounding to TA.
 template <typename TA>
-__global__ void __launch_bounds__(256) combine_kernel(const TA* __restrict__ ys,
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ ys,
                                                       const uint32_t* __restrict__ inv_order,
                                                       const float* __restrict__ w, int T, int k,
                                                       int d, TA* __restrict__ y) {
-  constexpr int V = 16 / sizeof(TA);
+  constexpr int V = 8;
   const int per_row = d / V;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= (long long)T * per_row) return;
@@ -28,22 +29,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const TA* __restrict__ ys,
   for (int i = 0; i < V; ++i) acc[i] = 0.f;
   for (int j = 0; j < k; ++j) {
     const float wj = __ldg(w + (size_t)t * k + j);
-    const TA* src = ys + (size_t)__ldg(inv_order + (size_t)t * k + j) * d + o;
-    uint4 raw = ldg_v4(src);
-    if constexpr (sizeof(TA) == 2) {
-      const uint32_t v[4] = {raw.x, raw.y, raw.z, raw.w};
+    const float* src = ys + (size_t)__ldg(inv_order + (size_t)t * k + j) * d + o;
+    const float4 a = *reinterpret_cast<const float4*>(src);
+    const float4 b = *reinterpret_cast<const float4*>(src + 4);
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 p = bf16x2_to_f32x2(v[i]);
-        acc[2 * i] = fmaf(wj, p.x, acc[2 * i]);
-        acc[2 * i + 1] = fmaf(wj, p.y, acc[2 * i + 1]);
-      }
-    } else {
-      const float v[4] = {__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
-                          __uint_as_float(raw.w)};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
-    }
+    for (int i = 0; i < V; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
   }
   TA* dst = y + (size_t)t * d + o;
   if constexpr (sizeof(TA) == 2) {
@@ -55,18 +46,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const TA* __restrict__ ys,
     *reinterpret_cast<uint4*>(dst) = out;
   } else {
     *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
 cudaError_t launch_combine(const void* ys, const uint32_t* inv_order, const float* w, int T, int k,
                            int d, int dt, void* y, cudaStream_t s) {
-  const int V = dt == MOE_BF16 ? 8 : 4;
-  const long long n = (long long)T * (d / V);
+  const long long n = (long long)T * (d / 8);
   if (n == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (dt == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        (const __nv_bfloat16*)ys, inv_order, w, T, k, d, (__nv_bfloat16*)y);
+    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const float*)ys, inv_order, w, T, k, d,
+                                                         (__nv_bfloat16*)y);
   else
     combine_kernel<float><<<blocks, 256, 0, s>>>((const float*)ys, inv_order, w, T, k, d,
                                                  (float*)y);

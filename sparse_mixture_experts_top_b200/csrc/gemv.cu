@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
     const TA* __restrict__ hin, const int32_t* __restrict__ row_off,
     const int32_t* __restrict__ tile_off, int BM, int E, int d, int F,
     const uint32_t* __restrict__ wdn, const uint16_t* __restrict__ sdn,
-    const uint16_t* __restrict__ bdn, TA* __restrict__ ys) {
+    const uint16_t* __restrict__ bdn, float* __restrict__ ys) {
   using D = WDecode<FMT>;
   constexpr int EPW = D::EPW;
   const int tau = blockIdx.y;
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
 #pragma unroll
     for (int j = 0; j < kRowsPerPass; ++j) {
       const float v = warp_sum(acc[j]);
-      if (lane == 0 && j < nr) Act<TA>::store(ys, (size_t)(rb + j) * d + o, v);
+      if (lane == 0 && j < nr) ys[(size_t)(rb + j) * d + o] = v;
     }
   }
 }
@@ -247,7 +247,7 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
   const uint16_t* bi = (const uint16_t*)ex.b_dn;
 #define MOE_DOWN(TA, FMT)                                                                    \
   down_gemv_kernel<TA, FMT><<<grid, 256, 0, s>>>((const TA*)h, row_off, tile_off, BM, ex.E, \
-                                                 ex.d, ex.F, w, sc, bi, (TA*)ys)
+                                                 ex.d, ex.F, w, sc, bi, (float*)ys)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_DOWN(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);

@@ -41,7 +41,7 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
 // Tensor-core grouped kernels (bf16 activations; bf16 or q4 weights).
 // BM must equal tc_block_m().
 int tc_block_m();
-cudaError_t launch_swiglu_tc(const void* x, const uint32_t* row_map, const int32_t* row_off,
+cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
                              int* status, cudaStream_t s);
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,

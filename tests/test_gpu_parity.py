@@ -67,7 +67,8 @@ def test_topk_signed_zero_and_nan(moe, orc):
 # ------------------------------------------------------------------ route
 
 @pytest.mark.parametrize("name,T", [("tiny", 16), ("decode_t1", 1), ("decode_t32", 32),
-                                    ("prefill", 256), ("skewed", 64), ("acceptance", 100)])
+                                    ("prefill", 256), ("skewed", 64), ("acceptance", 100),
+                                    ("prefill", 2048), ("skewed", 520), ("acceptance", 512)])
 def test_route_logits_and_selection(moe, orc, name, T):
     wl = mi.workload(name, T=T)
     g = torch.Generator().manual_seed(11)
@@ -127,12 +128,21 @@ def test_sort_all_rows_to_one_expert(moe, orc):
 # ------------------------------------------------------------------ experts
 
 STAGE_CASES = [
-    # workload, T override, regime, BM, skew
+    # workload, T override, regime (1 = weight-streaming, 2 = tensor core), BM, skew
     ("tiny", 16, 1, 8, 0.0),
     ("decode_t1", 1, 1, 8, 0.0),
     ("decode_t32", 32, 1, 8, 0.0),
     ("acceptance", 64, 1, 32, 0.0),
     ("prefill", 96, 1, 8, 0.02),
+    # tensor-core kernels: bf16 weights; q4 weights; one row per tile (N = 16);
+    # skewed routing with experts above 128 rows (several token tiles) and
+    # empty experts; the large-d workload
+    ("acceptance", 300, 2, 128, 0.0),
+    ("decode_t32", 32, 2, 128, 0.0),
+    ("decode_t1", 1, 2, 128, 0.0),
+    ("prefill", 200, 2, 128, 0.0),
+    ("prefill", 600, 2, 128, 0.5),
+    ("skewed", 24, 2, 128, 0.3),
 ]
 
 
@@ -162,7 +172,8 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
     ys = moe.grouped_down(hin.to(DEV), st, T, wl.k, layer.experts, regime=regime)
     ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
     yref = orc.expert_down(hin.double().numpy(), ref_st.row_off, _host(layer.experts))
-    assert_close_rms(ys, yref, _tol(wl.act), f"ys[{name}]", rounded_to=_rounded(wl.act))
+    assert ys.dtype == torch.float32
+    assert_close_rms(ys, yref, _tol(wl.act), f"ys[{name}]")
 
 
 @pytest.mark.parametrize("T,k,d,dt", [(1, 8, 2048, torch.bfloat16), (16, 2, 128, torch.float32),
@@ -171,16 +182,18 @@ def test_combine_parity(moe, orc, T, k, d, dt):
     E = max(k, 16)
     idx = mi.random_topk_idx(T, E, k, seed=31)
     st = orc.sort_rows(idx.numpy(), E, 8)
-    ys = mi.random_ys(T * k, d, seed=32, dtype=dt)
+    ys = mi.random_ys(T * k, d, seed=32, dtype=torch.float32)
     w = mi.random_weights(T, k, seed=33)
     inv = torch.from_numpy(st.inv_order.view(np.int32)).view(torch.uint32)
-    y = moe.combine(ys.to(DEV), inv.to(DEV), w.to(DEV), T, k)
+    y = moe.combine(ys.to(DEV), inv.to(DEV), w.to(DEV), T, k, dtype=dt)
     yref = orc.combine(ys.double().numpy(), st.inv_order, w.double().numpy(), T, k)
     g = to_np(y).astype(np.float64)
-    # one rounding of an fp32 sum of k terms to the output dtype
-    u = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -23
-    bound = u * np.abs(yref) + (k + 1) * 2.0 ** -24 * (np.abs(w.double().numpy()) @ np.ones((k, 1))) * np.abs(ys.double().numpy()).max()
-    assert (np.abs(g - yref) <= bound + 1e-30).all()
+    # an fp32 sum of k products (each rounding <= 2^-24 relative of the
+    # partial sum), then one rounding to the output dtype
+    u = 2.0 ** -9 if dt == torch.bfloat16 else 2.0 ** -24
+    mag = np.abs(w.double().numpy())[:, :, None] * np.abs(ys.double().numpy()[st.inv_order.reshape(T, k)])
+    bound = u * np.abs(yref) + (k + 1) * 2.0 ** -24 * mag.sum(axis=1) * (1 + u)
+    assert (np.abs(g - yref) <= bound).all()
 
 
 # ------------------------------------------------------------------ forward
@@ -220,10 +233,18 @@ def test_forward_parity_acceptance(moe, orc):
     _forward_and_compare(moe, orc, layer, sample=np.arange(0, 512, 4))
 
 
-def test_forward_parity_prefill_sampled(moe, orc):
+@pytest.mark.parametrize("regime", [0, 1])
+def test_forward_parity_prefill_sampled(moe, orc, regime):
     layer = mi.make_layer("prefill", seed=0, device=DEV)
     rng = np.random.default_rng(0)
-    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(2048, 96, replace=False)))
+    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(2048, 96, replace=False)),
+                         regime=regime)
+    assert moe.device_status() == moe.OK
+
+
+def test_forward_parity_decode_t32_tensor_core(moe, orc):
+    layer = mi.make_layer("decode_t32", seed=1, device=DEV)
+    _forward_and_compare(moe, orc, layer, regime=2)
 
 
 @pytest.mark.slow
