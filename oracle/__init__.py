@@ -15,6 +15,8 @@ the layer (see the header of ``moe_oracle.c`` for the passage each follows):
 * ``sort_rows``      -- stable sort of routed slots, row and tile tables
 * ``expert_swiglu``  -- h = silu(x W_g^T) * (x W_u^T) over sorted rows
 * ``expert_down``    -- ys = h W_d^T over sorted rows
+* ``expert_gate_up`` / ``expert_down_abs`` -- pre-activations and sums of
+  absolute products, used by the tests to bound rounding errors
 * ``combine``        -- y[t] = sum_j w[t,j] ys[inv_order[t k + j]]
 * ``forward``        -- the whole layer
 """
@@ -64,6 +66,8 @@ def lib():
         L.orc_combine.argtypes = [P, P, P, I, I, I, P]
         L.orc_forward.argtypes = [P, I, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P,
                                   P, P, P, P, P, P, I]
+        L.orc_expert_gate_up.argtypes = [P, I, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
+        L.orc_expert_down_abs.argtypes = [P, P, I, I, I, I, P, P, P, P, I]
         L.orc_weight_value.argtypes = [I, P, P, P, I, I, I, I, I]
         L.orc_weight_value.restype = D
         _lib = L
@@ -204,6 +208,33 @@ def expert_swiglu(x, row_map, row_off, experts, nthreads=None):
                                    experts.F, WFMT[experts.fmt], _p(w), _p(s), _p(b), _p(h),
                                    nthreads or default_threads()), "expert_swiglu")
     return h
+
+
+def expert_gate_up(x, row_map, row_off, experts, nthreads=None):
+    """(g, u, |x|.|w_gate|, |x|.|w_up|), each fp64 [R, F], for sorted rows."""
+    xa = _np(x)
+    rm = _np(row_map, np.uint32)
+    ro = _np(row_off, np.int32)
+    w, s, b = _wargs(experts, "gu")
+    R = rm.shape[0]
+    out = [np.empty((R, experts.F), np.float64) for _ in range(4)]
+    _check(lib().orc_expert_gate_up(_p(xa), _act_code(xa), _p(rm), _p(ro), experts.E, experts.d,
+                                    experts.F, WFMT[experts.fmt], _p(w), _p(s), _p(b),
+                                    *[_p(o) for o in out], nthreads or default_threads()),
+           "expert_gate_up")
+    return tuple(out)
+
+
+def expert_down_abs(h, row_off, experts, nthreads=None):
+    """|h[i]| . |w_dn[e][o]| for sorted rows, fp64 [R, d]."""
+    ha = _np(h).astype(np.float64)
+    ro = _np(row_off, np.int32)
+    w, s, b = _wargs(experts, "dn")
+    out = np.empty((ha.shape[0], experts.d), np.float64)
+    _check(lib().orc_expert_down_abs(_p(ha), _p(ro), experts.E, experts.d, experts.F,
+                                     WFMT[experts.fmt], _p(w), _p(s), _p(b), _p(out),
+                                     nthreads or default_threads()), "expert_down_abs")
+    return out
 
 
 def expert_down(h, row_off, experts, nthreads=None):

@@ -299,6 +299,53 @@ int orc_expert_swiglu(const void* x, int xdt, const uint32_t* row_map, const int
     return 0;
 }
 
+/* Pre-activations of the same rows, for error bounds in the tests: g and u
+ * as above, and the sums of absolute products |x| . |w_gate| and |x| . |w_up|
+ * (each output [R][F]). */
+typedef struct {
+    const void* x; int xdt; const uint32_t* row_map; const int32_t* row_off;
+    orc_wmat gu; int d, F; double *g, *u, *ga, *ua;
+} gate_up_ctx;
+
+static void gate_up_range(void* p, int lo, int hi) {
+    gate_up_ctx* c = (gate_up_ctx*)p;
+    double* wg = (double*)malloc(sizeof(double) * c->d);
+    double* wu = (double*)malloc(sizeof(double) * c->d);
+    for (int e = lo; e < hi; ++e) {
+        int r0 = c->row_off[e], r1 = c->row_off[e + 1];
+        if (r0 == r1) continue;
+        for (int f = 0; f < c->F; ++f) {
+            weight_row(&c->gu, e, f, wg);
+            weight_row(&c->gu, e, c->F + f, wu);
+            for (int i = r0; i < r1; ++i) {
+                size_t t = c->row_map[i];
+                double g = 0.0, u = 0.0, ga = 0.0, ua = 0.0;
+                for (int a = 0; a < c->d; ++a) {
+                    double xv = act_value(c->x, c->xdt, t * c->d + a);
+                    g += xv * wg[a];
+                    u += xv * wu[a];
+                    ga += fabs(xv * wg[a]);
+                    ua += fabs(xv * wu[a]);
+                }
+                size_t o = (size_t)i * c->F + f;
+                c->g[o] = g; c->u[o] = u; c->ga[o] = ga; c->ua[o] = ua;
+            }
+        }
+    }
+    free(wg);
+    free(wu);
+}
+
+int orc_expert_gate_up(const void* x, int xdt, const uint32_t* row_map, const int32_t* row_off,
+                       int E, int d, int F, int wfmt, const void* w_gu, const uint16_t* s_gu,
+                       const uint16_t* b_gu, double* g, double* u, double* ga, double* ua,
+                       int nthreads) {
+    gate_up_ctx c = {x, xdt, row_map, row_off, {wfmt, w_gu, s_gu, b_gu, 2 * F, d}, d, F,
+                     g, u, ga, ua};
+    orc_parallel(gate_up_range, &c, E, nthreads);
+    return 0;
+}
+
 /* ---------------------------------------------------------------- 5. down */
 
 typedef struct {
@@ -330,6 +377,37 @@ int orc_expert_down(const double* h, const int32_t* row_off, int E, int d, int F
                     int nthreads) {
     down_ctx c = {h, row_off, {wfmt, w_dn, s_dn, b_dn, d, F}, d, F, ys};
     orc_parallel(down_range, &c, E, nthreads);
+    return 0;
+}
+
+/* Sums of absolute products |h[i]| . |w_dn[e][o]| (for error bounds). */
+typedef struct {
+    const double* h; const int32_t* row_off; orc_wmat dn; int d, F; double* out;
+} down_abs_ctx;
+
+static void down_abs_range(void* p, int lo, int hi) {
+    down_abs_ctx* c = (down_abs_ctx*)p;
+    double* wd = (double*)malloc(sizeof(double) * c->F);
+    for (int e = lo; e < hi; ++e) {
+        int r0 = c->row_off[e], r1 = c->row_off[e + 1];
+        if (r0 == r1) continue;
+        for (int o = 0; o < c->d; ++o) {
+            weight_row(&c->dn, e, o, wd);
+            for (int i = r0; i < r1; ++i) {
+                double acc = 0.0;
+                for (int f = 0; f < c->F; ++f) acc += fabs(c->h[(size_t)i * c->F + f] * wd[f]);
+                c->out[(size_t)i * c->d + o] = acc;
+            }
+        }
+    }
+    free(wd);
+}
+
+int orc_expert_down_abs(const double* h, const int32_t* row_off, int E, int d, int F, int wfmt,
+                        const void* w_dn, const uint16_t* s_dn, const uint16_t* b_dn, double* out,
+                        int nthreads) {
+    down_abs_ctx c = {h, row_off, {wfmt, w_dn, s_dn, b_dn, d, F}, d, F, out};
+    orc_parallel(down_abs_range, &c, E, nthreads);
     return 0;
 }
 

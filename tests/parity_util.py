@@ -67,3 +67,46 @@ def kth_gap(logits_np, k):
     if logits_np.shape[1] <= k:
         return np.full(logits_np.shape[0], np.inf)
     return s[:, k - 1] - s[:, k]
+
+
+def assert_h_close(h_gpu, href, g, u, ga, ua, d, wfmt, tol, what=""):
+    """h = silu(g) * u stored in bf16 by a kernel that multiplies in bf16 on
+    the tensor cores: dequantised q4 weights are rounded to bf16 (relative
+    2^-9 each, so |dg| <= 2^-9 * sum |x w|), products accumulate in fp32
+    (d * 2^-24 * sum |x w|), and h is rounded once to bf16 (2^-9 |h|). The
+    first-order bound per element is
+        tol * RMS(h) + 2^-8 |h| + |u silu'(g)| dg + |silu(g)| du,
+    with the factor 2 of margin folded into the 2^-8 terms."""
+    gh = to_np(h_gpu).astype(np.float64)
+    assert gh.shape == href.shape, (what, gh.shape, href.shape)
+    assert np.isfinite(gh).all(), f"{what}: non-finite GPU output"
+    if href.size == 0:
+        return 0.0
+    wr = 2.0 ** -8 if wfmt == "q4" else 0.0
+    acc = 2.0 * d * 2.0 ** -24
+    dg = (wr + acc) * ga
+    du = (wr + acc) * ua
+    sig = 1.0 / (1.0 + np.exp(-g))
+    bound = (tol * rms(href) + 2.0 ** -8 * np.abs(href)
+             + np.abs(u * sig * (1.0 + g * (1.0 - sig))) * dg + np.abs(g * sig) * du)
+    err = np.abs(gh - href)
+    i = int(np.argmax(err - bound))
+    assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "
+                                          f"(ref {href.flat[i]:.4e}) > bound {bound.flat[i]:.3e}")
+    return float(err.max()) / max(rms(href), 1e-300)
+
+
+def assert_ys_close(ys_gpu, yref, habs, wfmt, tol, what=""):
+    """ys = h . W_d^T kept in fp32: q4 weights rounded to bf16 inside the
+    tensor-core kernel add at most 2^-9 * sum |h w| (2^-8 with margin)."""
+    g = to_np(ys_gpu).astype(np.float64)
+    assert g.shape == yref.shape and np.isfinite(g).all(), what
+    if yref.size == 0:
+        return 0.0
+    wr = 2.0 ** -8 if wfmt == "q4" else 0.0
+    bound = tol * rms(yref) + wr * habs
+    err = np.abs(g - yref)
+    i = int(np.argmax(err - bound))
+    assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "
+                                          f"(ref {yref.flat[i]:.4e}) > bound {bound.flat[i]:.3e}")
+    return float(err.max()) / max(rms(yref), 1e-300)

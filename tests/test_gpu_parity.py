@@ -14,7 +14,8 @@ import pytest
 import torch
 
 import moe_inputs as mi
-from parity_util import TOL_BF16, TOL_F32, assert_close_rms, kth_gap, to_np, topk_ref
+from parity_util import (TOL_BF16, TOL_F32, assert_close_rms, assert_h_close, assert_ys_close,
+                         kth_gap, to_np, topk_ref)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,10 +32,6 @@ def moe():
 
 def _tol(act):
     return TOL_F32 if act == "f32" else TOL_BF16
-
-
-def _rounded(act):
-    return "bf16" if act == "bf16" else None
 
 
 def _host(ex):
@@ -159,8 +156,13 @@ def test_grouped_swiglu_parity(moe, orc, name, T, regime, BM, skew):
     st = moe.sort_rows(idx.to(DEV), wl.E, BM)
     h = moe.grouped_swiglu(layer.x, st, wl.k, layer.experts, regime=regime)
     ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
-    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, _host(layer.experts))
-    assert_close_rms(h, href, _tol(wl.act), f"h[{name}]", rounded_to=_rounded(wl.act))
+    hx = _host(layer.experts)
+    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    if wl.act == "f32":
+        assert_close_rms(h, href, TOL_F32, f"h[{name}]")
+    else:
+        g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+        assert_h_close(h, href, g, u, ga, ua, wl.d, wl.wfmt, TOL_BF16, f"h[{name}]")
 
 
 @pytest.mark.parametrize("name,T,regime,BM,skew", STAGE_CASES)
@@ -171,9 +173,11 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
     hin = mi.random_rows(T * wl.k, wl.F, seed=23, dtype=mi._act_dtype(wl.act))
     ys = moe.grouped_down(hin.to(DEV), st, T, wl.k, layer.experts, regime=regime)
     ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
-    yref = orc.expert_down(hin.double().numpy(), ref_st.row_off, _host(layer.experts))
+    hx = _host(layer.experts)
+    yref = orc.expert_down(hin.double().numpy(), ref_st.row_off, hx)
     assert ys.dtype == torch.float32
-    assert_close_rms(ys, yref, _tol(wl.act), f"ys[{name}]")
+    habs = orc.expert_down_abs(hin.double().numpy(), ref_st.row_off, hx)
+    assert_ys_close(ys, yref, habs, wl.wfmt, _tol(wl.act), f"ys[{name}]")
 
 
 @pytest.mark.parametrize("T,k,d,dt", [(1, 8, 2048, torch.bfloat16), (16, 2, 128, torch.float32),
