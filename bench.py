@@ -122,22 +122,29 @@ def gate_up_bytes(ex) -> int:
 def kernels_per_forward(T, k, regime_tc: bool) -> int:
     R = T * k
     sort = 1 if R <= 1024 else 3
-    return 2 + sort + 2 + 1   # router logits + top-k, sort, gate|up, down, combine
+    conv = 1 if regime_tc else 0   # x -> fp16 for the tensor-core expert GEMMs
+    return 2 + sort + conv + 2 + 1   # router + top-k, sort, [x16], gate|up, down, combine
 
 
 # ------------------------------------------------------------------ timing
 
 def time_device(fn, steps, warmup, flush):
-    """Per-step CUDA-event time (ms) of fn() on the current stream; the L2 is
-    flushed (a 256 MB write) before every step, outside the timed events."""
+    """Per-step CUDA-event time (ms) of fn() on the current stream. Before
+    every step, outside the timed events, the L2 is flushed: a 256 MB buffer
+    is written, then a second 256 MB buffer is read, so the dirty lines the
+    write leaves are written back before the step starts and the step begins
+    with a cold, clean L2."""
+    wbuf, rbuf = flush
     for _ in range(warmup):
         fn()
     s = torch.cuda.current_stream()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    sink = torch.empty((), dtype=torch.float32, device=wbuf.device)
     torch.cuda.synchronize()
     for i in range(steps):
-        flush.add_(1)
+        wbuf.add_(1)
+        torch.sum(rbuf, out=sink)
         starts[i].record(s)
         fn()
         ends[i].record(s)
@@ -156,7 +163,8 @@ def run_ours(args, rank, world, local_rank):
     k, T = wl.k, wl.T
     ws = moe.forward_workspace(layer.x, ex, k)
     y = torch.empty(T, wl.d, dtype=layer.x.dtype, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = (torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+             torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev))
     L = moe.forward_layout(T, wl.d, wl.E, k, wl.F, layer.x.dtype)
 
     def fwd():
@@ -187,15 +195,16 @@ def run_ours(args, rank, world, local_rank):
             (L.order, T * k, torch.uint32), (L.inv_order, T * k, torch.uint32),
             (L.row_map, T * k, torch.uint32), (L.counts, wl.E, torch.int32),
             (L.row_off, wl.E + 1, torch.int32), (L.tile_off, wl.E + 1, torch.int32))), L.BM)
-    h = ws[L.h:L.h + T * k * wl.F * 2].view(torch.bfloat16).view(T * k, wl.F) \
-        if layer.x.dtype == torch.bfloat16 else None
+    h = ws[L.h:L.h + T * k * wl.F * 2].view(torch.float16).view(T * k, wl.F)
+    x16 = ws[L.x16:L.x16 + T * wl.d * 2]
     regime = L.regime
+    exs = moe.experts_struct(ex)
 
     def swiglu():
         moe.lib.moe_grouped_swiglu(
             moe._ptr(layer.x), moe._dt(layer.x), moe._ptr(st.row_map), moe._ptr(st.row_off),
-            moe._ptr(st.tile_off), L.BM, T, k, __import__("ctypes").byref(moe.experts_struct(ex)),
-            moe._ptr(h), regime, moe._stream())
+            moe._ptr(st.tile_off), L.BM, T, k, __import__("ctypes").byref(exs),
+            moe._ptr(h), moe._ptr(x16), x16.numel(), regime, moe._stream())
 
     fwd()
     ms_swiglu = time_device(swiglu, args.steps, args.warmup, flush)
@@ -304,7 +313,8 @@ def main():
                           f"{wl.wfmt} experts, {wl.act} activations"
                           + (f", router bias {wl.bias}" if wl.bias != "none" else ""),
               "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "F": wl.F, "weights": wl.wfmt,
-              "l2": "flushed before every timed step (256 MB write, outside the events)"}
+              "l2": "flushed before every timed step, outside the events: 256 MB written, then "
+                    "256 MB read so the write-back finishes before the step"}
 
     if args.impl == "reference":
         if rank != 0:

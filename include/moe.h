@@ -79,7 +79,9 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2, /* valid but not implemented (dims, dtype/format mix) */
   MOE_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required */
   MOE_ERR_CUDA = 4,        /* a CUDA launch failed */
-  MOE_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out (device status) */
+  MOE_ERR_TIMEOUT = 5,     /* a device-side bounded wait ran out (device status) */
+  MOE_ERR_RANGE = 6        /* a value outside the fp16 range of the expert GEMMs'
+                              operands (|x| or |h| >= 65520; device status) */
 } moe_status;
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype; /* activations */
@@ -157,18 +159,27 @@ moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, u
  * swiglu_rows; mlxcel PR #275 "What it does").
  *   x        (device) [T][d], dtype dt
  *   row_map, row_off, tile_off: as written by moe_sort_rows with the same BM
- *   h        (device, out) [T*k][F], dtype dt:
+ *            (the tensor-core regime needs BM = 128)
+ *   h        (device, out) [T*k][F]: fp16 for bf16 activations, fp32 for fp32:
  *            h[i][f] = silu(g) * u, g = x[row_map[i]] . w_gu[e][f],
  *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
- * fp32 accumulation; h rounded once to dt. */
+ *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, d, dt) bytes,
+ *            used by the tensor-core regime (x converted to fp16); may be NULL
+ *            in the weight-streaming regime
+ * fp32 accumulation; h rounded once. The tensor-core regime multiplies fp16
+ * operands (x converted exactly from bf16 when |x| < 65520, weights
+ * dequantised to fp16); values outside fp16 range are reported as
+ * MOE_ERR_RANGE in the device status. */
+size_t moe_grouped_swiglu_workspace(int T, int d, moe_dtype dt);
 moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
                               const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
-                              const moe_experts* experts, void* h, moe_regime regime,
-                              moe_stream_t stream);
+                              const moe_experts* experts, void* h, void* ws, size_t ws_bytes,
+                              moe_regime regime, moe_stream_t stream);
 
 /* Grouped down projection over rows already sorted by expert (DS4Server
  * issue #112, switch_linear with sorted indices).
- *   h        (device) [T*k][F], dtype dt
+ *   h        (device) [T*k][F]: fp16 for bf16 activations (dt = MOE_BF16),
+ *            fp32 for fp32 -- as moe_grouped_swiglu writes it
  *   ys       (device, out) [T*k][d] fp32: ys[i][o] = h[i] . w_dn[e][o]
  *            (kept in fp32 so the only rounding after the expert matmuls is
  *            the final one of y) */
@@ -202,7 +213,7 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
  * offsets), the regime it resolves to and the BM it sorts with. */
 typedef struct {
   size_t logits, topk_idx, topk_w, order, inv_order, row_map, counts, row_off, tile_off;
-  size_t sort_ws, h, ys, total;
+  size_t sort_ws, h, ys, x16, total;
   int32_t regime; /* resolved: MOE_REGIME_GEMV or MOE_REGIME_TC */
   int32_t BM;
 } moe_ws_layout;

@@ -19,13 +19,14 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(7)
 F32, BF16 = 0, 1
 W_F32, W_BF16, W_Q4G64 = 0, 1, 2
 REGIME_AUTO, REGIME_GEMV, REGIME_TC = 0, 1, 2
 
 EXPORTS = ("moe_route", "moe_topk", "moe_sort_rows_workspace", "moe_sort_rows",
-           "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward_workspace",
+           "moe_grouped_swiglu_workspace", "moe_grouped_swiglu", "moe_grouped_down",
+           "moe_combine", "moe_forward_workspace",
            "moe_forward", "moe_forward_layout", "moe_device_status", "moe_status_str",
            "moe_version")
 
@@ -46,7 +47,7 @@ class Experts(ctypes.Structure):
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("logits", "topk_idx", "topk_w", "order", "inv_order", "row_map", "counts",
-                 "row_off", "tile_off", "sort_ws", "h", "ys", "total")] + \
+                 "row_off", "tile_off", "sort_ws", "h", "ys", "x16", "total")] + \
                [("regime", ctypes.c_int32), ("BM", ctypes.c_int32)]
 
 
@@ -61,7 +62,10 @@ def _load():
     L.moe_sort_rows_workspace.argtypes = [I, I, I]
     L.moe_sort_rows_workspace.restype = S
     L.moe_sort_rows.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, S, P]
-    L.moe_grouped_swiglu.argtypes = [P, I, P, P, P, I, I, I, ctypes.POINTER(Experts), P, I, P]
+    L.moe_grouped_swiglu_workspace.argtypes = [I, I, I]
+    L.moe_grouped_swiglu_workspace.restype = S
+    L.moe_grouped_swiglu.argtypes = [P, I, P, P, P, I, I, I, ctypes.POINTER(Experts), P, P, S, I,
+                                     P]
     L.moe_grouped_down.argtypes = [P, I, P, P, I, I, I, ctypes.POINTER(Experts), P, I, P]
     L.moe_combine.argtypes = [P, P, P, I, I, I, I, P, P]
     L.moe_forward_workspace.argtypes = [I, I, I, I, I, I, I]
@@ -184,15 +188,20 @@ def sort_rows(topk_idx, E, BM, stream=None) -> SortTables:
     return SortTables(order, inv, rmap, counts, roff, toff, BM)
 
 
-def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, stream=None):
-    """-> h [T*k, F] in x's dtype"""
+def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, ws=None, stream=None):
+    """-> h [T*k, F]: fp16 for bf16 x, fp32 for fp32 x"""
     _dev(x)
     T = x.shape[0]
     ex = experts_struct(experts)
-    h = torch.empty(T * k, experts.F, dtype=x.dtype, device=x.device)
+    hdt = torch.float16 if x.dtype == torch.bfloat16 else torch.float32
+    h = torch.empty(T * k, experts.F, dtype=hdt, device=x.device)
+    nws = lib.moe_grouped_swiglu_workspace(T, experts.d, _dt(x))
+    if ws is None:
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=x.device)
     _check(lib.moe_grouped_swiglu(_ptr(x), _dt(x), _ptr(tables.row_map), _ptr(tables.row_off),
                                   _ptr(tables.tile_off), tables.BM, T, k, ctypes.byref(ex),
-                                  _ptr(h), regime, _stream(stream)), "moe_grouped_swiglu")
+                                  _ptr(h), _ptr(ws), ws.numel(), regime, _stream(stream)),
+           "moe_grouped_swiglu")
     return h
 
 
@@ -201,7 +210,9 @@ def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, strea
     _dev(h)
     ex = experts_struct(experts)
     ys = torch.empty(T * k, experts.d, dtype=torch.float32, device=h.device)
-    _check(lib.moe_grouped_down(_ptr(h), _dt(h), _ptr(tables.row_off), _ptr(tables.tile_off),
+    # h is fp16 exactly when the activations are bf16
+    adt = BF16 if h.dtype == torch.float16 else F32
+    _check(lib.moe_grouped_down(_ptr(h), adt, _ptr(tables.row_off), _ptr(tables.tile_off),
                                 tables.BM, T, k, ctypes.byref(ex), _ptr(ys), regime,
                                 _stream(stream)), "moe_grouped_down")
     return ys

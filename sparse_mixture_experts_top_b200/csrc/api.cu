@@ -99,6 +99,7 @@ const char* moe_status_str(moe_status s) {
     case MOE_ERR_WORKSPACE: return "workspace missing or too small";
     case MOE_ERR_CUDA: return "CUDA launch error";
     case MOE_ERR_TIMEOUT: return "device-side bounded wait ran out";
+    case MOE_ERR_RANGE: return "value outside the fp16 range of the expert GEMM operands";
   }
   return "unknown status";
 }
@@ -165,10 +166,15 @@ moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, u
                                    row_off, tile_off, ws, (cudaStream_t)stream));
 }
 
+size_t moe_grouped_swiglu_workspace(int T, int d, moe_dtype dt) {
+  if (T < 0 || d <= 0) return 0;
+  return dt == MOE_BF16 ? up256((size_t)T * d * 2) : 0;
+}
+
 moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
                               const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
-                              const moe_experts* experts, void* h, moe_regime regime,
-                              moe_stream_t stream) {
+                              const moe_experts* experts, void* h, void* ws, size_t ws_bytes,
+                              moe_regime regime, moe_stream_t stream) {
   if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_experts(experts, dt);
   if (st != MOE_OK) return st;
@@ -184,10 +190,13 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
   if (rg == MOE_REGIME_TC) {
     if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
-    return launched(launch_swiglu_tc(x, T, row_map, row_off, tile_off, (int)R, *experts, h,
+    if (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, experts->d, dt))
+      return MOE_ERR_WORKSPACE;
+    return launched(launch_swiglu_tc(x, T, row_map, row_off, tile_off, (int)R, *experts, h, ws,
                                      status_ptr(), s));
   }
-  return launched(launch_swiglu_gemv(x, dt, row_map, row_off, tile_off, BM, (int)R, *experts, h, s));
+  return launched(launch_swiglu_gemv(x, dt, row_map, row_off, tile_off, BM, (int)R, *experts, h,
+                                     status_ptr(), s));
 }
 
 moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
@@ -254,8 +263,9 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.row_off = take((size_t)(E + 1) * 4);
   L.tile_off = take((size_t)(E + 1) * 4);
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
-  L.h = take((size_t)R * F * a);
+  L.h = take((size_t)R * F * a);      // fp16 (bf16 activations) or fp32
   L.ys = take((size_t)R * d * 4);
+  L.x16 = take(dt == MOE_BF16 ? (size_t)T * d * 2 : 0);
   L.total = off;
   L.regime = resolve_regime(regime, R, E, dt, d, F);
   L.BM = block_m_for(L.regime, R, E);
@@ -301,6 +311,7 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
   void* sws = base + L.sort_ws;
   void* h = base + L.h;
   void* ys = base + L.ys;
+  void* x16 = base + L.x16;
   const long long R = (long long)T * k;
   cudaStream_t s = (cudaStream_t)stream;
   int* stp = status_ptr();
@@ -315,12 +326,13 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
       cudaSuccess)
     return launched(e);
   if (L.regime == MOE_REGIME_TC) {
-    if ((e = launch_swiglu_tc(x, T, rmap, roff, toff, (int)R, *experts, h, stp, s)) != cudaSuccess)
+    if ((e = launch_swiglu_tc(x, T, rmap, roff, toff, (int)R, *experts, h, x16, stp, s)) !=
+        cudaSuccess)
       return launched(e);
     if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s)) != cudaSuccess)
       return launched(e);
   } else {
-    if ((e = launch_swiglu_gemv(x, dt, rmap, roff, toff, L.BM, (int)R, *experts, h, s)) !=
+    if ((e = launch_swiglu_gemv(x, dt, rmap, roff, toff, L.BM, (int)R, *experts, h, stp, s)) !=
         cudaSuccess)
       return launched(e);
     if ((e = launch_down_gemv(h, dt, roff, toff, L.BM, (int)R, *experts, ys, s)) != cudaSuccess)

@@ -13,6 +13,10 @@
 // dequantises in registers, and accumulates all the tile's token rows in
 // fp32, then warp-reduces. Every selected expert's bytes are read once per
 // call when BM covers the expert's rows.
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -46,10 +50,31 @@ template <> struct WDecode<MOE_W_Q4G64> {
   }
 };
 
+// The hidden rows h between the two projections: fp16 for bf16 activations
+// (the tensor-core operand format, 11-bit precision), fp32 for fp32.
+template <typename TA> struct HType { using T = float; };
+template <> struct HType<__nv_bfloat16> { using T = __half; };
+
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
 // N consecutive activations starting at p (16-, 8- or 4-byte aligned) as floats.
 template <typename TA, int N>
 __device__ __forceinline__ void load_act(const TA* p, float* out) {
-  if constexpr (sizeof(TA) == 2) {
+  if constexpr (std::is_same<TA, __half>::value) {
+    static_assert(N == 2 || N == 8, "fp16 rows come in words of 2 or 8");
+    if constexpr (N == 8) {
+      uint4 v = ldg_v4(p);
+      float2 a = f16x2_to_f32x2(v.x), b = f16x2_to_f32x2(v.y);
+      float2 c = f16x2_to_f32x2(v.z), d = f16x2_to_f32x2(v.w);
+      out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+      out[4] = c.x; out[5] = c.y; out[6] = d.x; out[7] = d.y;
+    } else {
+      float2 a = f16x2_to_f32x2(*reinterpret_cast<const uint32_t*>(p));
+      out[0] = a.x; out[1] = a.y;
+    }
+  } else if constexpr (sizeof(TA) == 2) {
     static_assert(N == 2 || N == 8, "bf16 activations come in words of 2 or 8");
     if constexpr (N == 8) {
       uint4 v = ldg_v4(p);
@@ -92,7 +117,8 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
     const TA* __restrict__ x, const uint32_t* __restrict__ row_map,
     const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E, int d,
     int F, const uint32_t* __restrict__ wgu, const uint16_t* __restrict__ sgu,
-    const uint16_t* __restrict__ bgu, TA* __restrict__ h) {
+    const uint16_t* __restrict__ bgu, typename HType<TA>::T* __restrict__ h, int* status) {
+  using TH = typename HType<TA>::T;
   using D = WDecode<FMT>;
   constexpr int EPW = D::EPW;
   const int tau = blockIdx.y;
@@ -151,7 +177,15 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
     for (int j = 0; j < kRowsPerPass; ++j) {
       const float g = warp_sum(ag[j]);
       const float u = warp_sum(au[j]);
-      if (lane == 0 && j < nr) Act<TA>::store(h, (size_t)(rb + j) * F + f, swiglu(g, u));
+      if (lane == 0 && j < nr) {
+        const float v = swiglu(g, u);
+        if constexpr (std::is_same<TH, __half>::value) {
+          if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
+          h[(size_t)(rb + j) * F + f] = __float2half_rn(v);
+        } else {
+          h[(size_t)(rb + j) * F + f] = v;
+        }
+      }
     }
   }
 }
@@ -160,7 +194,7 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
 
 template <typename TA, int FMT>
 __global__ void __launch_bounds__(256) down_gemv_kernel(
-    const TA* __restrict__ hin, const int32_t* __restrict__ row_off,
+    const typename HType<TA>::T* __restrict__ hin, const int32_t* __restrict__ row_off,
     const int32_t* __restrict__ tile_off, int BM, int E, int d, int F,
     const uint32_t* __restrict__ wdn, const uint16_t* __restrict__ sdn,
     const uint16_t* __restrict__ bdn, float* __restrict__ ys) {
@@ -197,7 +231,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
         for (int j = 0; j < kRowsPerPass; ++j) {
           if (j < nr) {
             float hv[EPW];
-            load_act<TA, EPW>(hin + (size_t)(rb + j) * F + elem, hv);
+            load_act<typename HType<TA>::T, EPW>(hin + (size_t)(rb + j) * F + elem, hv);
 #pragma unroll
             for (int i = 0; i < EPW; ++i) acc[j] = fmaf(hv[i], wv[i], acc[j]);
           }
@@ -216,7 +250,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
 
 cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
                                const int32_t* row_off, const int32_t* tile_off, int BM, int R,
-                               const moe_experts& ex, void* h, cudaStream_t s) {
+                               const moe_experts& ex, void* h, int* status, cudaStream_t s) {
   const long long tiles = max_tiles(R, ex.E, BM);
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 65535) return cudaErrorInvalidConfiguration;
@@ -226,7 +260,8 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
   const uint16_t* bi = (const uint16_t*)ex.b_gu;
 #define MOE_SWIGLU(TA, FMT)                                                                    \
   swiglu_gemv_kernel<TA, FMT><<<grid, 256, 0, s>>>((const TA*)x, row_map, row_off, tile_off, BM, \
-                                                   ex.E, ex.d, ex.F, w, sc, bi, (TA*)h)
+                                                   ex.E, ex.d, ex.F, w, sc, bi,                  \
+                                                   (typename HType<TA>::T*)h, status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_SWIGLU(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_SWIGLU(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q4G64);
@@ -246,8 +281,9 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
   const uint16_t* sc = (const uint16_t*)ex.s_dn;
   const uint16_t* bi = (const uint16_t*)ex.b_dn;
 #define MOE_DOWN(TA, FMT)                                                                    \
-  down_gemv_kernel<TA, FMT><<<grid, 256, 0, s>>>((const TA*)h, row_off, tile_off, BM, ex.E, \
-                                                 ex.d, ex.F, w, sc, bi, (float*)ys)
+  down_gemv_kernel<TA, FMT><<<grid, 256, 0, s>>>((const typename HType<TA>::T*)h, row_off,    \
+                                                 tile_off, BM, ex.E, ex.d, ex.F, w, sc, bi,     \
+                                                 (float*)ys)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_DOWN(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);

@@ -33,7 +33,7 @@ inline long long max_tiles(long long R, int E, int BM) {
 // Weight-streaming grouped kernels (any format, any BM).
 cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
                                const int32_t* row_off, const int32_t* tile_off, int BM, int R,
-                               const moe_experts& ex, void* h, cudaStream_t s);
+                               const moe_experts& ex, void* h, int* status, cudaStream_t s);
 cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
                              const int32_t* tile_off, int BM, int R, const moe_experts& ex,
                              void* ys, cudaStream_t s);
@@ -41,9 +41,10 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
 // Tensor-core grouped kernels (bf16 activations; bf16 or q4 weights).
 // BM must equal tc_block_m().
 int tc_block_m();
+// x16: T*d fp16 scratch that receives x converted from bf16
 cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
-                             int* status, cudaStream_t s);
+                             void* x16, int* status, cudaStream_t s);
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
                            const moe_experts& ex, void* ys, int* status, cudaStream_t s);
 

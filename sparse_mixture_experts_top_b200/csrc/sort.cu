@@ -12,9 +12,10 @@
 //   1. count   -- one block per chunk of 1024 slots counts ids per expert
 //   2. scan    -- one block: counts, row_off, tile_off, and each chunk's
 //                 starting position per expert (chunks in slot order)
-//   3. scatter -- one block per chunk; its 32 warps take their 32 slots in
-//                 slot order, ranking equal ids inside a warp with
-//                 __match_any_sync, so positions follow slot order exactly.
+//   3. scatter -- one block per chunk: per-warp counts of every id, a scan of
+//                 each id's counts over the chunk's 32 warps, and the rank
+//                 among equal ids inside a warp (__match_any_sync) place each
+//                 slot at once, in slot order.
 // When all slots fit one chunk the three steps run in a single block
 // (decode), so a whole dispatch is one launch there.
 #include "common.cuh"
@@ -72,27 +73,39 @@ __device__ void block_exclusive_scan(int* v, int n, int* total, int* warp_tmp) {
   __syncthreads();
 }
 
-// Scatter the slots of one chunk in slot order. cursor[e] holds the next
-// sorted position of expert e for this chunk and is advanced.
+// Scatter the slots of one chunk in slot order. cursor[e] holds the first
+// sorted position of expert e for this chunk. wtab is a [32][E] uint16
+// table in shared memory: each warp's count of every id, then (in place)
+// the number of equal ids in the earlier warps of the chunk; with the rank
+// among equal ids inside the warp (__match_any_sync) that gives every slot
+// its position at once, in slot order.
 __device__ void scatter_chunk(const int32_t* __restrict__ idx, long long r0, long long R, int k,
-                              int E, int* cursor, uint32_t* __restrict__ order,
-                              uint32_t* __restrict__ inv_order, uint32_t* __restrict__ row_map) {
+                              int E, const int* cursor, uint16_t* wtab,
+                              uint32_t* __restrict__ order, uint32_t* __restrict__ inv_order,
+                              uint32_t* __restrict__ row_map) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wtab[i] = 0;
+  __syncthreads();
   const long long r = r0 + warp * 32 + lane;
   const int e = (r < R) ? clamp_id(idx[r], E) : -1;
   const unsigned peers = __match_any_sync(0xffffffffu, e);
   const int rank = __popc(peers & ((1u << lane) - 1u));
-  const int leader_last = 31 - __clz(peers);           // highest lane of the group
-  for (int w = 0; w < 32; ++w) {
-    if (warp == w && e >= 0) {
-      const int pos = cursor[e] + rank;
-      order[pos] = (uint32_t)r;
-      inv_order[r] = (uint32_t)pos;
-      row_map[pos] = (uint32_t)(r / k);
-      __syncwarp(peers);
-      if (lane == leader_last) cursor[e] += __popc(peers);
+  if (e >= 0 && rank == 0) wtab[warp * E + e] = (uint16_t)__popc(peers);
+  __syncthreads();
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {     // exclusive scan over warps
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wtab[w * E + x];
+      wtab[w * E + x] = (uint16_t)run;
+      run += c;
     }
-    __syncthreads();
+  }
+  __syncthreads();
+  if (e >= 0) {
+    const int pos = cursor[e] + wtab[warp * E + e] + rank;
+    order[pos] = (uint32_t)r;
+    inv_order[r] = (uint32_t)pos;
+    row_map[pos] = (uint32_t)(r / k);
   }
 }
 
@@ -104,6 +117,7 @@ __global__ void __launch_bounds__(1024) sort_single_kernel(
   extern __shared__ int sm[];
   int* cnt = sm;            // [E]
   int* tiles = sm + E;      // [E]
+  uint16_t* wtab = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [32][E]
   __shared__ int warp_tmp[32];
   __shared__ int totals[2];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -126,7 +140,7 @@ __global__ void __launch_bounds__(1024) sort_single_kernel(
     tile_off[E] = totals[1];
   }
   __syncthreads();
-  scatter_chunk(idx, 0, R, k, E, cnt, order, inv_order, row_map);
+  scatter_chunk(idx, 0, R, k, E, cnt, wtab, order, inv_order, row_map);
 }
 
 __global__ void __launch_bounds__(1024) sort_count_kernel(const int32_t* __restrict__ idx, long long R,
@@ -181,10 +195,12 @@ __global__ void __launch_bounds__(1024) sort_scatter_kernel(
     const int32_t* __restrict__ chunk_base, uint32_t* __restrict__ order,
     uint32_t* __restrict__ inv_order, uint32_t* __restrict__ row_map) {
   extern __shared__ int cursor[];
+  uint16_t* wtab = reinterpret_cast<uint16_t*>(cursor + E);   // [32][E]
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     cursor[e] = chunk_base[(size_t)blockIdx.x * E + e];
   __syncthreads();
-  scatter_chunk(idx, (long long)blockIdx.x * kChunk, R, k, E, cursor, order, inv_order, row_map);
+  scatter_chunk(idx, (long long)blockIdx.x * kChunk, R, k, E, cursor, wtab, order, inv_order,
+                row_map);
 }
 
 cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, uint32_t* order,
@@ -192,9 +208,12 @@ cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, ui
                              int32_t* row_off, int32_t* tile_off, void* ws, cudaStream_t s) {
   const long long R = (long long)T * k;
   const size_t smem2 = (size_t)2 * E * sizeof(int);
+  const size_t wtab = (size_t)32 * E * sizeof(uint16_t);
   if (R <= kChunk) {
-    sort_single_kernel<<<1, 1024, smem2, s>>>(idx, (int)R, k, E, BM, order, inv_order, row_map,
-                                              counts, row_off, tile_off);
+    cudaFuncSetAttribute(sort_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)(smem2 + wtab));
+    sort_single_kernel<<<1, 1024, smem2 + wtab, s>>>(idx, (int)R, k, E, BM, order, inv_order,
+                                                     row_map, counts, row_off, tile_off);
     return cudaGetLastError();
   }
   const int nch = num_chunks(R);
@@ -203,8 +222,10 @@ cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, ui
   sort_count_kernel<<<nch, 1024, E * sizeof(int), s>>>(idx, R, E, chunk_cnt);
   sort_scan_kernel<<<1, 1024, smem2, s>>>(chunk_cnt, nch, E, BM, chunk_base, counts, row_off,
                                           tile_off);
-  sort_scatter_kernel<<<nch, 1024, E * sizeof(int), s>>>(idx, R, k, E, chunk_base, order,
-                                                         inv_order, row_map);
+  cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)(E * sizeof(int) + wtab));
+  sort_scatter_kernel<<<nch, 1024, E * sizeof(int) + wtab, s>>>(idx, R, k, E, chunk_base, order,
+                                                                inv_order, row_map);
   return cudaGetLastError();
 }
 

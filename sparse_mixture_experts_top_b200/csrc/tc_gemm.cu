@@ -23,13 +23,19 @@
 //   * warp 1 (MMA): one thread issues tcgen05.mma (A from TMEM, B from
 //     shared memory) into fp32 accumulators in TMEM; gate and up accumulate
 //     side by side so one token tile feeds both;
-//   * warps 4..7 (epilogue): tcgen05.ld of the accumulators, SwiGLU to bf16
+//   * warps 4..7 (epilogue): tcgen05.ld of the accumulators, SwiGLU to fp16
 //     (gate|up) or an fp32 store (down projection; router logits + bias).
+// The expert GEMMs multiply fp16 operands (x converted once from bf16,
+// weights dequantised to fp16, h stored in fp16): 11-bit operands keep the
+// rounding of the dequantised weights and of h 8x below bf16's; values
+// outside the fp16 range are reported as MOE_ERR_RANGE. The router keeps its
+// bf16 operands, which are exact there.
 // Every mbarrier wait is bounded (about a second): on expiry the kernel
 // records MOE_ERR_TIMEOUT in the status word, all roles leave their loops,
 // copies in flight are waited for (bounded), TMEM is freed, and it returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -42,7 +48,9 @@ namespace tc {
 constexpr int BN = 128;        // token rows per tile (the sort tables' BM)
 constexpr int BMW = 128;       // weight rows per tile (MMA M)
 constexpr int KA = 64;         // K elements per A stage (one q4 group)
-constexpr int NB = 4;          // token-row (B) stages
+constexpr int NB = 6;          // token-row (B) stages
+constexpr int kMaxE = 1024;    // tile / row tables cached in shared memory
+constexpr int kScaleAhead = 4; // raw stages of scales/biases loaded ahead
 constexpr int kThreads = 512;
 constexpr int kEpiWarp0 = 4;
 constexpr int kDqWarp0 = 8;
@@ -68,7 +76,8 @@ struct Cfg {
   // warps that write one A stage: NMAT == 2: 4 gate + 4 up warps;
   // NMAT == 1: q4 -- the 4 warps of one half; bf16 -- all 8 (half the columns each)
   static constexpr int A_ARRIVALS = NMAT == 2 ? 8 : (Q4 ? 4 : 8);
-  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024;
+  static constexpr int TABLES = 2 * (kMaxE + 1) * 4;       // tile_off, row_off copies
+  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES;
 };
 
 struct Params {
@@ -188,9 +197,11 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   return d;
 }
 
-// M = 128, N = n, bf16 x bf16 -> fp32, both K-major
-__device__ __forceinline__ uint32_t idesc_bf16(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+// M = 128, N = n, fp32 accumulate, both operands K-major; operand format
+// fp16 (code 0) or bf16 (code 1)
+__device__ __forceinline__ uint32_t idesc_mma(int n, bool f16) {
+  const uint32_t ab = f16 ? 0u : 1u;
+  return (1u << 4) | (ab << 7) | (ab << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(BMW >> 4) << 24);
 }
 
@@ -221,33 +232,48 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 // ------------------------------------------------------------------ dequant
 
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
-__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+__device__ __forceinline__ uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
+}
+// (lo, hi) floats -> packed fp16 pair, lo in the low half, round to nearest
+__device__ __forceinline__ uint32_t f16x2_pack(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// a bf16 value (low 16 bits of v) as an fp16 pair holding it twice
+__device__ __forceinline__ uint32_t f16x2_from_bf16(uint32_t v) {
+  const float f = __uint_as_float(v << 16);
+  return f16x2_pack(f, f);
+}
+// two bf16 values (element 2c low, 2c+1 high) -> the same pair in fp16
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return f16x2_pack(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
-// 8 nibbles of one word (element j in bits [4j, 4j+3]) -> 4 bf16 pairs
+// 8 nibbles of one word (element j in bits [4j, 4j+3]) -> 4 fp16 pairs
 // (element 2c in the low half of out[c]), value = s * q + b rounded once.
-// Each nibble q is placed in the mantissa of bf16 128.0 (0x4300 | q = 128 + q,
-// exact), 128 is subtracted exactly, then one fused multiply-add applies the
-// group's scale and bias.
+// Each nibble q is placed in the mantissa of fp16 1024.0 (0x6400 | q =
+// 1024 + q, exact), 1024 is subtracted exactly, then one fused multiply-add
+// applies the group's scale and bias (s2, b2: fp16 pairs).
 __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* out) {
   const uint32_t lo = w & 0x0F0F0F0Fu;           // elements 0, 2, 4, 6
   const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;    // elements 1, 3, 5, 7
   const uint32_t p0 = __byte_perm(lo, hi, 0x5140);   // e0 e1 e2 e3
   const uint32_t p1 = __byte_perm(lo, hi, 0x7362);   // e4 e5 e6 e7
-  const uint32_t M = 0x43434343u;
-  const uint32_t c128 = 0x43004300u;
-  out[0] = bf16x2_fma(bf16x2_sub(__byte_perm(p0, M, 0x4140), c128), s2, b2);
-  out[1] = bf16x2_fma(bf16x2_sub(__byte_perm(p0, M, 0x4342), c128), s2, b2);
-  out[2] = bf16x2_fma(bf16x2_sub(__byte_perm(p1, M, 0x4140), c128), s2, b2);
-  out[3] = bf16x2_fma(bf16x2_sub(__byte_perm(p1, M, 0x4342), c128), s2, b2);
+  const uint32_t M = 0x64646464u;
+  const uint32_t c1024 = 0x64006400u;
+  out[0] = f16x2_fma(f16x2_sub(__byte_perm(p0, M, 0x4140), c1024), s2, b2);
+  out[1] = f16x2_fma(f16x2_sub(__byte_perm(p0, M, 0x4342), c1024), s2, b2);
+  out[2] = f16x2_fma(f16x2_sub(__byte_perm(p1, M, 0x4140), c1024), s2, b2);
+  out[3] = f16x2_fma(f16x2_sub(__byte_perm(p1, M, 0x4342), c1024), s2, b2);
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -260,9 +286,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 
 // ------------------------------------------------------------------ tiles
 
+// Tile tau -> (expert e, first sorted row r0, valid rows nv), with the
+// prefix tables read from their shared-memory copies.
 template <bool ROUTER>
-__device__ __forceinline__ void decode_tile(const Params& p, int u, int& e, int& mb, int& r0,
-                                            int& nv) {
+__device__ __forceinline__ void decode_tile(const Params& p, const int* s_toff, const int* s_roff,
+                                            int u, int& e, int& mb, int& r0, int& nv) {
   const int tau = u / p.n_mb;
   mb = u - tau * p.n_mb;
   if (ROUTER) {
@@ -270,16 +298,21 @@ __device__ __forceinline__ void decode_tile(const Params& p, int u, int& e, int&
     r0 = tau * BN;
     nv = min(BN, p.n_rows - r0);
   } else {
-    e = expert_of_tile(p.tile_off, p.E, tau);
-    r0 = __ldg(p.row_off + e) + (tau - __ldg(p.tile_off + e)) * BN;
-    nv = min(BN, __ldg(p.row_off + e + 1) - r0);
+    int lo = 0, hi = p.E - 1;      // largest e with tile_off[e] <= tau
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_toff[mid] <= tau) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    r0 = s_roff[e] + (tau - s_toff[e]) * BN;
+    nv = min(BN, s_roff[e + 1] - r0);
   }
 }
 
 template <bool ROUTER>
-__device__ __forceinline__ int total_units(const Params& p) {
+__device__ __forceinline__ int total_units(const Params& p, const int* s_toff) {
   if (ROUTER) return ((p.n_rows + BN - 1) / BN) * p.n_mb;
-  return __ldg(p.tile_off + p.E) * p.n_mb;
+  return s_toff[p.E] * p.n_mb;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -306,6 +339,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_toff = reinterpret_cast<int*>(smem + C::NR * C::RAW_BYTES + NB * C::B_BYTES + 1024);
+  int* s_roff = s_toff + kMaxE + 1;
+  if (!ROUTER) {
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+      s_toff[i] = __ldg(p.tile_off + i);
+      s_roff[i] = __ldg(p.row_off + i);
+    }
+  }
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -342,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int total = total_units<ROUTER>(p);
+  const int total = total_units<ROUTER>(p, s_toff);
   const int nkr = p.K / C::KR;           // raw stages per tile
   const int nka = p.K / KA;              // A stages per tile
 
@@ -352,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, u, e, mb, r0, nv);
+      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
       const int wrow = (ROUTER ? 0 : e * p.rows_per_group) + mb * BMW;
       int trow[BN / 32];
       if (GATHER) {
@@ -419,9 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
         int e, mb, r0, nv;
-        decode_tile<ROUTER>(p, u, e, mb, r0, nv);
+        decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
         const int n_mma = max(16, (nv + 15) & ~15);
-        const uint32_t idesc = idesc_bf16(n_mma);
+        const uint32_t idesc = idesc_mma(n_mma, !ROUTER);
         if (tcount > 0) {
           ok = mbar_wait(smem_u32(acc_empty), (tcount - 1) & 1, abort_flag, p.status);
           if (!ok) break;
@@ -464,9 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = q * 32 + lane;                      // weight row of this thread
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t tcount = 0;
+    bool range_ok = true;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, u, e, mb, r0, nv);
+      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
       if (!mbar_wait_warp(smem_u32(acc_full), tcount & 1, abort_flag, p.status)) break;
       tc_fence_after();
       const int orow = mb * BMW + m;                  // output feature
@@ -478,13 +520,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t uu[16];
           tmem_ld16(tl + BN + c0, uu);
           tmem_ld_wait();
-          __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+          __half* h = reinterpret_cast<__half*>(p.out);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
-            if (n < nv)
-              h[(size_t)(r0 + n) * p.out_ld + orow] =
-                  __float2bfloat16_rn(swiglu(__uint_as_float(g[j]), __uint_as_float(uu[j])));
+            if (n < nv) {
+              const float v = swiglu(__uint_as_float(g[j]), __uint_as_float(uu[j]));
+              range_ok &= fabsf(v) < 65520.f;    // rounds to a finite fp16
+              h[(size_t)(r0 + n) * p.out_ld + orow] = __float2half_rn(v);
+            }
           }
         } else {
           tmem_ld_wait();
@@ -502,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(smem_u32(acc_empty));
       ++tcount;
     }
+    if (!__all_sync(0xffffffffu, range_ok) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------ dequant
     const int dw = warp - kDqWarp0;                   // 0..7
@@ -511,29 +556,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t raw_it = 0, a_it = 0;
     bool ok = true;
+    // q4 scales/biases: a queue of the next kScaleAhead raw stages, filled by
+    // a cursor that walks the same (tile, raw stage) sequence ahead of the
+    // consumer, across tile boundaries
+    const int sub = C::NMAT == 2 ? 0 : part;        // group within the raw stage (NMAT 1)
+    int pf_u = blockIdx.x, pf_kr = 0;
+    const uint16_t* pf_s = nullptr;
+    const uint16_t* pf_b = nullptr;
+    auto pf_row = [&]() {
+      if (!C::Q4 || pf_u >= total) return;
+      int e2, mb2, r02, nv2;
+      decode_tile<ROUTER>(p, s_toff, s_roff, pf_u, e2, mb2, r02, nv2);
+      const size_t grow = (size_t)(ROUTER ? 0 : e2 * p.rows_per_group) +
+                          (C::NMAT == 2 ? part * p.up_off : 0) + mb2 * BMW + m;
+      pf_s = p.scales + grow * p.G;
+      pf_b = p.biases + grow * p.G;
+    };
+    auto pf_load = [&](uint32_t& sv, uint32_t& bv) {
+      sv = bv = 0;
+      if (!C::Q4 || pf_u >= total) return;
+      if (C::NMAT == 2) {   // both groups of the raw stage: 2 x bf16
+        sv = __ldg(reinterpret_cast<const uint32_t*>(pf_s + 2 * pf_kr));
+        bv = __ldg(reinterpret_cast<const uint32_t*>(pf_b + 2 * pf_kr));
+      } else {
+        sv = __ldg(pf_s + 2 * pf_kr + sub);
+        bv = __ldg(pf_b + 2 * pf_kr + sub);
+      }
+      if (++pf_kr == nkr) {
+        pf_kr = 0;
+        pf_u += gridDim.x;
+        pf_row();
+      }
+    };
+    uint32_t sq[kScaleAhead], bq[kScaleAhead];
+    pf_row();
+#pragma unroll
+    for (int i = 0; i < kScaleAhead; ++i) pf_load(sq[i], bq[i]);
+
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, u, e, mb, r0, nv);
-      const int grow = (ROUTER ? 0 : e * p.rows_per_group) + (C::NMAT == 2 ? part * p.up_off : 0) +
-                       mb * BMW + m;
-      // q4: scales/biases of the next raw stage are loaded one stage ahead
-      uint32_t sc_next = 0, bi_next = 0;
-      const uint16_t* srow = C::Q4 ? p.scales + (size_t)grow * p.G : nullptr;
-      const uint16_t* brow = C::Q4 ? p.biases + (size_t)grow * p.G : nullptr;
-      auto load_sb = [&](int kr, uint32_t& s, uint32_t& b) {
-        if (C::NMAT == 2) {   // both groups of the raw stage: 2 x bf16
-          s = __ldg(reinterpret_cast<const uint32_t*>(srow + 2 * kr));
-          b = __ldg(reinterpret_cast<const uint32_t*>(brow + 2 * kr));
-        } else {              // this half's group, replicated
-          const uint32_t sv = __ldg(srow + 2 * kr + part), bv = __ldg(brow + 2 * kr + part);
-          s = sv | (sv << 16);
-          b = bv | (bv << 16);
-        }
-      };
-      if (C::Q4) load_sb(0, sc_next, bi_next);
+      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
       for (int kr = 0; kr < nkr && ok; ++kr) {
-        const uint32_t sc = sc_next, bi = bi_next;
-        if (C::Q4 && kr + 1 < nkr) load_sb(kr + 1, sc_next, bi_next);
+        const uint32_t sc = sq[0], bi = bq[0];
+#pragma unroll
+        for (int i = 0; i + 1 < kScaleAhead; ++i) {
+          sq[i] = sq[i + 1];
+          bq[i] = bq[i + 1];
+        }
+        pf_load(sq[kScaleAhead - 1], bq[kScaleAhead - 1]);
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status);
         if (!ok) break;
@@ -558,13 +628,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int st = 0; st < nst && ok; ++st) {
             uint32_t s2, b2;
             if (C::NMAT == 2) {
-              const uint32_t sv = st ? (sc >> 16) : (sc & 0xFFFFu);
-              const uint32_t bv = st ? (bi >> 16) : (bi & 0xFFFFu);
-              s2 = sv | (sv << 16);
-              b2 = bv | (bv << 16);
+              s2 = f16x2_from_bf16(st ? (sc >> 16) : (sc & 0xFFFFu));
+              b2 = f16x2_from_bf16(st ? (bi >> 16) : (bi & 0xFFFFu));
             } else {
-              s2 = sc;
-              b2 = bi;
+              s2 = f16x2_from_bf16(sc & 0xFFFFu);
+              b2 = f16x2_from_bf16(bi & 0xFFFFu);
             }
             const uint4 w0 = wv[2 * st], w1 = wv[2 * st + 1];
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -592,10 +660,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nc = C::NMAT == 2 ? 8 : 4;
           for (int c = 0; c < nc; ++c) {
             const uint4 v = lds128(rowa + (((c0 + c) ^ sw) << 4));
-            vals[4 * c + 0] = v.x;
-            vals[4 * c + 1] = v.y;
-            vals[4 * c + 2] = v.z;
-            vals[4 * c + 3] = v.w;
+            if (ROUTER) {
+              vals[4 * c + 0] = v.x;
+              vals[4 * c + 1] = v.y;
+              vals[4 * c + 2] = v.z;
+              vals[4 * c + 3] = v.w;
+            } else {
+              vals[4 * c + 0] = bf16x2_to_f16x2(v.x);
+              vals[4 * c + 1] = bf16x2_to_f16x2(v.y);
+              vals[4 * c + 2] = bf16x2_to_f16x2(v.z);
+              vals[4 * c + 3] = bf16x2_to_f16x2(v.w);
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
@@ -676,10 +751,34 @@ static bool weight_map(CUtensorMap* m, int fmt, const void* w, long long rows, i
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// token-row map: rows of K bf16, box of `box_rows` rows
-static bool rows_map(CUtensorMap* m, const void* x, long long rows, int K, int box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, rows, (uint64_t)K * 2, 64, box_rows,
-                  CU_TENSOR_MAP_SWIZZLE_128B);
+// token-row map: rows of K 16-bit values (fp16 or bf16), box of `box_rows` rows
+static bool rows_map(CUtensorMap* m, const void* x, long long rows, int K, int box_rows, bool f16) {
+  return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x,
+                  K, rows, (uint64_t)K * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// bf16 -> fp16, 8 values per thread; values that do not round to a finite
+// fp16 are reported as MOE_ERR_RANGE (they become +-inf).
+__global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ in,
+                                                     uint4* __restrict__ out, long long n8,
+                                                     int* status) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  bool ok = true;
+  if (i < n8) {
+    const uint4 v = in[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+      ok &= fabsf(a) < 65520.f && fabsf(b) < 65520.f;
+      uint32_t d;
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(b), "f"(a));
+      o[j] = d;
+    }
+    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (!__all_sync(0xffffffffu, ok) && (threadIdx.x & 31) == 0) report_status(status, MOE_ERR_RANGE);
 }
 
 template <int FMT, int EPI, bool GATHER, bool ROUTER>
@@ -706,12 +805,18 @@ int tc_block_m() { return tc::BN; }
 
 cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
-                             int* status, cudaStream_t s) {
+                             void* x16, int* status, cudaStream_t s) {
   using namespace tc;
   if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
+  // the expert GEMMs take fp16 operands: x is converted once into x16 [T][d]
+  const long long n8 = (long long)T * ex.d / 8;
+  to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const uint4*)x, (uint4*)x16, n8,
+                                                             status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   CUtensorMap ta, tb;
   if (!weight_map(&ta, ex.fmt, ex.w_gu, (long long)ex.E * 2 * ex.F, ex.d)) return cudaErrorInvalidValue;
-  if (!rows_map(&tb, x, T, ex.d, 1)) return cudaErrorInvalidValue;
+  if (!rows_map(&tb, x16, T, ex.d, 1, true)) return cudaErrorInvalidValue;
   Params p{};
   p.row_off = row_off;
   p.tile_off = tile_off;
@@ -739,7 +844,7 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
   CUtensorMap ta, tb;
   if (!weight_map(&ta, ex.fmt, ex.w_dn, (long long)ex.E * ex.d, ex.F)) return cudaErrorInvalidValue;
-  if (!rows_map(&tb, h, R, ex.F, BN)) return cudaErrorInvalidValue;
+  if (!rows_map(&tb, h, R, ex.F, BN, true)) return cudaErrorInvalidValue;
   Params p{};
   p.row_off = row_off;
   p.tile_off = tile_off;
@@ -767,7 +872,7 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
   if (T < 256 || d % 64 != 0) return cudaErrorNotSupported;
   CUtensorMap ta, tb;
   if (!weight_map(&ta, MOE_W_BF16, w_router, E, d)) return cudaErrorInvalidValue;
-  if (!rows_map(&tb, x, T, d, BN)) return cudaErrorInvalidValue;
+  if (!rows_map(&tb, x, T, d, BN, false)) return cudaErrorInvalidValue;
   Params p{};
   p.E = 1;
   p.n_rows = T;

@@ -43,7 +43,7 @@ def test_binding_names_match_exports(moe):
 
 
 def test_status_strings(moe):
-    for s in range(6):
+    for s in range(7):
         assert moe.status_str(s)
     assert "sm_100a" in moe.version()
 
@@ -99,8 +99,11 @@ def test_stage_calls_reject_bad_arguments(moe):
     assert L.moe_sort_rows(fake, 4, 2, 8, 0, fake, fake, fake, fake, fake, fake, fake, 1 << 20, P) == moe.ERR_INVALID_ARG
     assert L.moe_sort_rows(fake, 4000, 2, 8, 8, fake, fake, fake, fake, fake, fake, P, 0, P) == moe.ERR_WORKSPACE
     assert L.moe_sort_rows(fake, 4000, 2, 8, 8, fake, fake, fake, fake, fake, fake, fake, 8, P) == moe.ERR_WORKSPACE
-    assert L.moe_grouped_swiglu(fake, moe.BF16, P, fake, fake, 8, 4, 2, ctypes.byref(ex), fake, 0, P) == moe.ERR_INVALID_ARG
-    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 0, 4, 2, ctypes.byref(ex), fake, 0, P) == moe.ERR_INVALID_ARG
+    assert L.moe_grouped_swiglu(fake, moe.BF16, P, fake, fake, 8, 4, 2, ctypes.byref(ex), fake, fake, 1 << 20, 0, P) == moe.ERR_INVALID_ARG
+    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 0, 4, 2, ctypes.byref(ex), fake, fake, 1 << 20, 0, P) == moe.ERR_INVALID_ARG
+    # the tensor-core regime needs its fp16 staging workspace
+    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 128, 4, 2, ctypes.byref(ex), fake, P, 0, 2, P) == moe.ERR_WORKSPACE
+    assert L.moe_grouped_swiglu_workspace(4, 128, moe.BF16) >= 4 * 128 * 2
     assert L.moe_grouped_down(fake, moe.BF16, fake, fake, 8, 4, 2, P, fake, 0, P) == moe.ERR_INVALID_ARG
     # the tensor-core regime takes bf16 activations only
     exf = _ex(moe, fmt=0)
@@ -114,9 +117,10 @@ def test_forward_layout_is_consistent(moe):
     for (T, d, E, k, F) in [(1, 2048, 128, 8, 768), (2048, 2048, 512, 10, 512), (16, 128, 8, 2, 256)]:
         L = moe.forward_layout(T, d, E, k, F, __import__("torch").bfloat16)
         offs = [L.logits, L.topk_idx, L.topk_w, L.order, L.inv_order, L.row_map, L.counts,
-                L.row_off, L.tile_off, L.sort_ws, L.h, L.ys]
+                L.row_off, L.tile_off, L.sort_ws, L.h, L.ys, L.x16]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
-        assert L.ys + T * k * d * 2 <= L.total
+        assert L.ys + T * k * d * 4 <= L.x16
+        assert L.x16 + T * d * 2 <= L.total
         assert L.h + T * k * F * 2 <= L.ys
         assert L.BM >= 1 and L.regime in (moe.REGIME_GEMV, moe.REGIME_TC)
         assert moe.lib.moe_forward_workspace(T, d, E, k, F, moe.BF16, 0) == L.total
