@@ -154,6 +154,29 @@ moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, u
                          uint32_t* inv_order, uint32_t* row_map, int32_t* counts, int32_t* row_off,
                          int32_t* tile_off, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_sort_rows for callers that cannot allocate device memory: the same
+ * outputs, bit for bit, with no workspace argument. The source pages have no
+ * counterpart to this call. It is meant for code that runs inside a host
+ * framework which owns all device memory and hands an operator no allocator
+ * or workspace (a plugin or custom-op interface), and for code that must not
+ * allocate at the point where it sorts.
+ *   Scratch: a static device array inside the library (256 KiB, held by every
+ *     GPU that loads the library until the process exits), so sizes are
+ *     limited: T*k <= 32768 and E <= 1024, else MOE_ERR_UNSUPPORTED. It calls
+ *     no cudaMalloc, cudaFree or any allocating routine.
+ *   Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture. MOE_ERR_CUDA if the lookup fails.
+ *   Sharing: every call uses the same array. Calls that may overlap on the
+ *     GPU (other streams, other host threads) race and corrupt each other's
+ *     result; serialise them. The array keeps the last call's contents; the
+ *     sort writes every entry it reads first, so nothing needs clearing.
+ * Other arguments and errors: as moe_sort_rows. */
+moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, int BM,
+                                 uint32_t* order, uint32_t* inv_order, uint32_t* row_map,
+                                 int32_t* counts, int32_t* row_off, int32_t* tile_off,
+                                 moe_stream_t stream);
+
 /* Grouped gate|up projection with the SwiGLU epilogue over sorted rows,
  * reading token rows in place through row_map (DS4Server issue #112,
  * swiglu_rows; mlxcel PR #275 "What it does").

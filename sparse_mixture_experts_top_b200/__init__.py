@@ -25,6 +25,7 @@ W_F32, W_BF16, W_Q4G64 = 0, 1, 2
 REGIME_AUTO, REGIME_GEMV, REGIME_TC = 0, 1, 2
 
 EXPORTS = ("moe_route", "moe_topk", "moe_sort_rows_workspace", "moe_sort_rows",
+           "moe_sort_rows_noalloc",
            "moe_grouped_swiglu_workspace", "moe_grouped_swiglu", "moe_grouped_down",
            "moe_combine", "moe_forward_workspace",
            "moe_forward", "moe_forward_layout", "moe_device_status", "moe_status_str",
@@ -76,7 +77,8 @@ def _load():
     L.moe_status_str.argtypes = [I]
     L.moe_status_str.restype = ctypes.c_char_p
     L.moe_version.restype = ctypes.c_char_p
-    for name in ("moe_route", "moe_topk", "moe_sort_rows", "moe_grouped_swiglu",
+    for name in ("moe_route", "moe_topk", "moe_sort_rows", "moe_sort_rows_noalloc",
+                 "moe_grouped_swiglu",
                  "moe_grouped_down", "moe_combine", "moe_forward", "moe_forward_layout",
                  "moe_device_status"):
         getattr(L, name).restype = ctypes.c_int

@@ -171,6 +171,20 @@ size_t moe_grouped_swiglu_workspace(int T, int d, moe_dtype dt) {
   return dt == MOE_BF16 ? up256((size_t)T * d * 2) : 0;
 }
 
+moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, int BM,
+                                 uint32_t* order, uint32_t* inv_order, uint32_t* row_map,
+                                 int32_t* counts, int32_t* row_off, int32_t* tile_off,
+                                 moe_stream_t stream) {
+  moe_status st = check_dims(T, 64, E, k);
+  if (st != MOE_OK) return st;
+  if (BM < 1) return MOE_ERR_INVALID_ARG;
+  if (!counts || !row_off || !tile_off) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !order || !inv_order || !row_map)) return MOE_ERR_INVALID_ARG;
+  if (!noalloc_sort_fits((long long)T * k, E)) return MOE_ERR_UNSUPPORTED;
+  return launched(launch_sort_rows_noalloc(topk_idx, T, k, E, BM, order, inv_order, row_map,
+                                           counts, row_off, tile_off, (cudaStream_t)stream));
+}
+
 moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
                               const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
                               const moe_experts* experts, void* h, void* ws, size_t ws_bytes,

@@ -24,6 +24,13 @@ cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, ui
                              uint32_t* inv_order, uint32_t* row_map, int32_t* counts,
                              int32_t* row_off, int32_t* tile_off, void* ws, cudaStream_t s);
 
+// The same sort with its scratch in a static device array (no allocation).
+bool noalloc_sort_fits(long long R, int E);
+cudaError_t launch_sort_rows_noalloc(const int32_t* idx, int T, int k, int E, int BM,
+                                     uint32_t* order, uint32_t* inv_order, uint32_t* row_map,
+                                     int32_t* counts, int32_t* row_off, int32_t* tile_off,
+                                     cudaStream_t s);
+
 // Upper bound of tile_off[E] for R rows, E experts and BM rows per tile.
 inline long long max_tiles(long long R, int E, int BM) {
   long long a = (R + BM - 1) / BM + (R < E ? R : E);

@@ -18,6 +18,8 @@
 //                 slot at once, in slot order.
 // When all slots fit one chunk the three steps run in a single block
 // (decode), so a whole dispatch is one launch there.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -227,6 +229,53 @@ cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, ui
   sort_scatter_kernel<<<nch, 1024, E * sizeof(int) + wtab, s>>>(idx, R, k, E, chunk_base, order,
                                                                 inv_order, row_map);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ no-alloc
+
+// Scratch for moe_sort_rows_noalloc: the per-chunk counts and bases of the
+// multi-block sort, sized for up to kNoAllocMaxRows routed rows and
+// kNoAllocMaxExperts experts (2 * 32 * 1024 int32 = 256 KiB). It is a
+// file-scope device array, so every GPU that loads this library holds it for
+// the life of the process. Host code must not pass the symbol itself to a
+// kernel (on the host it only names a stand-in); it passes the device address
+// looked up once per device below.
+constexpr int kNoAllocMaxRows = 32768;
+constexpr int kNoAllocMaxExperts = 1024;
+constexpr int kNoAllocChunks = (kNoAllocMaxRows + kChunk - 1) / kChunk;
+static __device__ __align__(256) int32_t g_noalloc_sort_scratch[2 * kNoAllocChunks *
+                                                                kNoAllocMaxExperts];
+
+// Device address of the scratch on the current device, looked up on first use
+// with that device current; nullptr when the lookup fails.
+static int32_t* noalloc_scratch_ptr() {
+  static std::mutex mu;
+  static int32_t* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    int32_t* p = nullptr;
+    if (cudaGetSymbolAddress((void**)&p, g_noalloc_sort_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+bool noalloc_sort_fits(long long R, int E) {
+  return R <= kNoAllocMaxRows && E <= kNoAllocMaxExperts;
+}
+
+cudaError_t launch_sort_rows_noalloc(const int32_t* idx, int T, int k, int E, int BM,
+                                     uint32_t* order, uint32_t* inv_order, uint32_t* row_map,
+                                     int32_t* counts, int32_t* row_off, int32_t* tile_off,
+                                     cudaStream_t s) {
+  int32_t* scratch = noalloc_scratch_ptr();
+  if (!scratch) return cudaErrorUnknown;
+  // every chunk count and base the sort reads is written by the same call
+  // first, so the scratch needs no clearing between calls
+  return launch_sort_rows(idx, T, k, E, BM, order, inv_order, row_map, counts, row_off, tile_off,
+                          scratch, s);
 }
 
 }  // namespace moe
