@@ -144,7 +144,7 @@ def time_device(fn, steps, warmup, flush):
     torch.cuda.synchronize()
     for i in range(steps):
         wbuf.add_(1)
-        torch.sum(rbuf, out=sink)
+        torch.sum(rbuf, dim=0, out=sink)
         starts[i].record(s)
         fn()
         ends[i].record(s)

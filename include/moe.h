@@ -186,9 +186,9 @@ moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, i
  *   h        (device, out) [T*k][F]: fp16 for bf16 activations, fp32 for fp32:
  *            h[i][f] = silu(g) * u, g = x[row_map[i]] . w_gu[e][f],
  *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
- *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, d, dt) bytes,
- *            used by the tensor-core regime (x converted to fp16); may be NULL
- *            in the weight-streaming regime
+ *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, d, dt) bytes
+ *            (x converted to fp16); required for bf16 activations, may be
+ *            NULL for fp32
  * fp32 accumulation; h rounded once. The tensor-core regime multiplies fp16
  * operands (x converted exactly from bf16 when |x| < 65520, weights
  * dequantised to fp16); values outside fp16 range are reported as

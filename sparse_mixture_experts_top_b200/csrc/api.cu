@@ -80,7 +80,28 @@ static int resolve_regime(int regime, long long R, int E, int dt, int d = 128, i
 
 static int block_m_for(int regime, long long R, int E) {
   if (regime == MOE_REGIME_TC) return tc_block_m();
-  return (R <= 8LL * E) ? 8 : 32;
+  return (R <= 8LL * E) ? 16 : 32;
+}
+
+// gate|up in the weight-streaming regime: the q4 tensor-core GEMV when it
+// applies (x converted to fp16 into x16 first), else the SIMT kernel
+static cudaError_t swiglu_gemv(const void* x, int dt, int T, const uint32_t* rmap,
+                               const int32_t* roff, const int32_t* toff, int BM, int R,
+                               const moe_experts& ex, void* h, void* x16, int* stp,
+                               cudaStream_t s) {
+  if (gemv_q4_mma_ok(ex, dt, BM) && x16) {
+    cudaError_t e = launch_to_f16(x, (long long)T * ex.d, x16, stp, s);
+    if (e != cudaSuccess) return e;
+    return launch_swiglu_q4_mma(x16, rmap, roff, toff, BM, R, ex, h, stp, s);
+  }
+  return launch_swiglu_gemv(x, dt, rmap, roff, toff, BM, R, ex, h, stp, s);
+}
+
+static cudaError_t down_gemv(const void* h, int dt, const int32_t* roff, const int32_t* toff,
+                             int BM, int R, const moe_experts& ex, void* ys, int* stp,
+                             cudaStream_t s) {
+  if (gemv_q4_mma_ok(ex, dt, BM)) return launch_down_q4_mma(h, roff, toff, BM, R, ex, ys, stp, s);
+  return launch_down_gemv(h, dt, roff, toff, BM, R, ex, ys, s);
 }
 
 }  // namespace moe
@@ -209,8 +230,11 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
     return launched(launch_swiglu_tc(x, T, row_map, row_off, tile_off, (int)R, *experts, h, ws,
                                      status_ptr(), s));
   }
-  return launched(launch_swiglu_gemv(x, dt, row_map, row_off, tile_off, BM, (int)R, *experts, h,
-                                     status_ptr(), s));
+  if (dt == MOE_BF16 &&
+      (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, experts->d, dt)))
+    return MOE_ERR_WORKSPACE;
+  return launched(swiglu_gemv(x, dt, T, row_map, row_off, tile_off, BM, (int)R, *experts, h, ws,
+                              status_ptr(), s));
 }
 
 moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
@@ -234,7 +258,7 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
     return launched(launch_down_tc(h, row_off, tile_off, (int)R, *experts, ys, status_ptr(), s));
   }
-  return launched(launch_down_gemv(h, dt, row_off, tile_off, BM, (int)R, *experts, ys, s));
+  return launched(down_gemv(h, dt, row_off, tile_off, BM, (int)R, *experts, ys, status_ptr(), s));
 }
 
 moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* topk_w, int T, int k,
@@ -346,10 +370,10 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
     if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s)) != cudaSuccess)
       return launched(e);
   } else {
-    if ((e = launch_swiglu_gemv(x, dt, rmap, roff, toff, L.BM, (int)R, *experts, h, stp, s)) !=
-        cudaSuccess)
+    if ((e = swiglu_gemv(x, dt, T, rmap, roff, toff, L.BM, (int)R, *experts, h,
+                         dt == MOE_BF16 ? x16 : nullptr, stp, s)) != cudaSuccess)
       return launched(e);
-    if ((e = launch_down_gemv(h, dt, roff, toff, L.BM, (int)R, *experts, ys, s)) != cudaSuccess)
+    if ((e = down_gemv(h, dt, roff, toff, L.BM, (int)R, *experts, ys, stp, s)) != cudaSuccess)
       return launched(e);
   }
   return launched(launch_combine(ys, inv, w, T, k, d, dt, y, s));

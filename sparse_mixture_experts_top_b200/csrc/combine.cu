@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const uint32_t* __restrict__ inv_order,
                                                       const float* __restrict__ w, int T, int k,
                                                       int d, TA* __restrict__ y) {
+  pdl_wait();
+  pdl_launch();
   constexpr int V = 8;
   const int per_row = d / V;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -56,10 +58,10 @@ cudaError_t launch_combine(const void* ys, const uint32_t* inv_order, const floa
   if (n == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (dt == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const float*)ys, inv_order, w, T, k, d,
+    launch_pdl(combine_kernel<__nv_bfloat16>, blocks, 256, 0, s, (const float*)ys, inv_order, w, T, k, d,
                                                          (__nv_bfloat16*)y);
   else
-    combine_kernel<float><<<blocks, 256, 0, s>>>((const float*)ys, inv_order, w, T, k, d,
+    launch_pdl(combine_kernel<float>, blocks, 256, 0, s, (const float*)ys, inv_order, w, T, k, d,
                                                  (float*)y);
   return cudaGetLastError();
 }

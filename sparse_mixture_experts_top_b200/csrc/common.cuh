@@ -90,6 +90,51 @@ __device__ __forceinline__ int expert_of_tile(const int32_t* tile_off, int E, in
   return lo;
 }
 
+// ---------------------------------------------------------------- launches
+
+// Programmatic dependent launch. Every kernel of the library waits, before
+// it reads anything an earlier kernel in the stream wrote, until those
+// kernels have completed and their memory is visible (griddepcontrol.wait),
+// then lets the next kernel be scheduled (launch_dependents); launches carry
+// the programmatic-serialization attribute, so a kernel's launch and prologue
+// overlap the tail of the one before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// The same search by one warp in two dependent loads (E <= 1024): the lanes
+// first read every ceil(E/32)-th entry, then the entries of the segment the
+// first round picked. All lanes return the same expert.
+__device__ __forceinline__ int expert_of_tile_warp(const int32_t* tile_off, int E, int tau) {
+  const int lane = threadIdx.x & 31;
+  const int stride = (E + 31) >> 5;
+  const int i0 = lane * stride;
+  const bool ok0 = i0 < E && __ldg(tile_off + i0) <= tau;
+  const unsigned m0 = __ballot_sync(0xffffffffu, ok0);   // lane 0 always qualifies
+  const int base = (31 - __clz(m0)) * stride;
+  const int i1 = base + lane;
+  const bool ok1 = lane < stride && i1 < E && __ldg(tile_off + i1) <= tau;
+  const unsigned m1 = __ballot_sync(0xffffffffu, ok1);
+  return base + (31 - __clz(m1));
+}
+
 // ---------------------------------------------------------------- status
 
 // Record the first device-side error in the status word `st` (a device

@@ -118,12 +118,14 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
     const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E, int d,
     int F, const uint32_t* __restrict__ wgu, const uint16_t* __restrict__ sgu,
     const uint16_t* __restrict__ bgu, typename HType<TA>::T* __restrict__ h, int* status) {
+  pdl_wait();
+  pdl_launch();
   using TH = typename HType<TA>::T;
   using D = WDecode<FMT>;
   constexpr int EPW = D::EPW;
   const int tau = blockIdx.y;
   if (tau >= __ldg(tile_off + E)) return;
-  const int e = expert_of_tile(tile_off, E, tau);
+  const int e = expert_of_tile_warp(tile_off, E, tau);
   const int r0 = __ldg(row_off + e) + (tau - __ldg(tile_off + e)) * BM;
   const int r1 = min(__ldg(row_off + e + 1), r0 + BM);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,11 +200,13 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
     const int32_t* __restrict__ tile_off, int BM, int E, int d, int F,
     const uint32_t* __restrict__ wdn, const uint16_t* __restrict__ sdn,
     const uint16_t* __restrict__ bdn, float* __restrict__ ys) {
+  pdl_wait();
+  pdl_launch();
   using D = WDecode<FMT>;
   constexpr int EPW = D::EPW;
   const int tau = blockIdx.y;
   if (tau >= __ldg(tile_off + E)) return;
-  const int e = expert_of_tile(tile_off, E, tau);
+  const int e = expert_of_tile_warp(tile_off, E, tau);
   const int r0 = __ldg(row_off + e) + (tau - __ldg(tile_off + e)) * BM;
   const int r1 = min(__ldg(row_off + e + 1), r0 + BM);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -259,7 +263,7 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
   const uint16_t* sc = (const uint16_t*)ex.s_gu;
   const uint16_t* bi = (const uint16_t*)ex.b_gu;
 #define MOE_SWIGLU(TA, FMT)                                                                    \
-  swiglu_gemv_kernel<TA, FMT><<<grid, 256, 0, s>>>((const TA*)x, row_map, row_off, tile_off, BM, \
+  launch_pdl(swiglu_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const TA*)x, row_map, row_off, tile_off, BM, \
                                                    ex.E, ex.d, ex.F, w, sc, bi,                  \
                                                    (typename HType<TA>::T*)h, status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_SWIGLU(float, MOE_W_F32);
@@ -281,7 +285,7 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
   const uint16_t* sc = (const uint16_t*)ex.s_dn;
   const uint16_t* bi = (const uint16_t*)ex.b_dn;
 #define MOE_DOWN(TA, FMT)                                                                    \
-  down_gemv_kernel<TA, FMT><<<grid, 256, 0, s>>>((const typename HType<TA>::T*)h, row_off,    \
+  launch_pdl(down_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const typename HType<TA>::T*)h, row_off,    \
                                                  tile_off, BM, ex.E, ex.d, ex.F, w, sc, bi,     \
                                                  (float*)ys)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
@@ -289,6 +293,236 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
   else return cudaErrorInvalidValue;
 #undef MOE_DOWN
+  return cudaGetLastError();
+}
+
+
+// ===================================================================
+// q4 weights, bf16 activations: tensor-core GEMV (mma.sync m16n8k16, fp16
+// operands, fp32 accumulate) for tiles of at most 16 token rows.
+//
+// A CTA of 4 warps owns one block of 16 weight rows of one tile -- for the
+// gate|up projection rows g and g+8 of the block are gate row f0+g and up
+// row f0+g, so SwiGLU happens in the lane that holds both accumulators; for
+// the down projection they are output rows o0+g and o0+8+g. K is walked in
+// steps of 128 elements, dealt round-robin to the 4 warps and reduced
+// through shared memory at the end.
+//
+// In a step, lane (g = lane/4, c = lane%4) loads 16 bytes (32 nibbles,
+// elements c*32 .. c*32+31 of the step) of each of its two rows, and the same
+// 32 elements of its token row(s) from fp16 activations. Inside the 16-wide
+// K slice of MMA m (m = 0..7) the element order is permuted identically for
+// A and B: fragment columns (2c, 2c+1) and (2c+8, 2c+9) are elements
+// c*32 + 4m + (0, 1) and c*32 + 4m + (2, 3). Those are consecutive nibbles of
+// word m/2 and consecutive activations, so both fragments are contiguous
+// loads and the dequantised pairs come out in fragment order.
+
+constexpr int kMmaWarps = 4;
+constexpr int kMmaMaxRows = 16;            // token rows per tile (two n8 groups)
+
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_from_bf16(uint32_t v16) {
+  const float f = __uint_as_float(v16 << 16);
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(f));
+  return d;
+}
+// nibbles of one word -> fp16 pairs (e0,e1) (e2,e3) (e4,e5) (e6,e7) of
+// s*q + b, one rounding: q goes into the mantissa of fp16 1024.0 (exact),
+// 1024 is subtracted exactly, one fused multiply-add applies scale and bias
+__device__ __forceinline__ void q4_word_f16(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* o) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t p0 = __byte_perm(lo, hi, 0x5140), p1 = __byte_perm(lo, hi, 0x7362);
+  const uint32_t M = 0x64646464u, c1024 = 0x64006400u;
+  o[0] = h2_fma(h2_sub(__byte_perm(p0, M, 0x4140), c1024), s2, b2);
+  o[1] = h2_fma(h2_sub(__byte_perm(p0, M, 0x4342), c1024), s2, b2);
+  o[2] = h2_fma(h2_sub(__byte_perm(p1, M, 0x4140), c1024), s2, b2);
+  o[3] = h2_fma(h2_sub(__byte_perm(p1, M, 0x4342), c1024), s2, b2);
+}
+
+// SWIGLU: x16 [T][d] fp16 activations through row_map, w = w_gu, out = h fp16
+// else:   x16 = h [R][F] fp16 rows (contiguous), w = w_dn, out = ys fp32
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
+    const __half* __restrict__ x16, const uint32_t* __restrict__ row_map,
+    const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E,
+    int d, int F, const uint32_t* __restrict__ w, const uint16_t* __restrict__ sc,
+    const uint16_t* __restrict__ bi, void* __restrict__ out, int* status) {
+  pdl_wait();
+  pdl_launch();
+  __shared__ float red[kMmaWarps - 1][32][8];
+  const int tau = blockIdx.y;
+  if (tau >= __ldg(tile_off + E)) return;
+  const int e = expert_of_tile_warp(tile_off, E, tau);
+  const int r0 = __ldg(row_off + e) + (tau - __ldg(tile_off + e)) * BM;
+  const int nv = min(__ldg(row_off + e + 1), r0 + BM) - r0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int K = SWIGLU ? d : F;                 // reduction length
+  const int rows_e = SWIGLU ? 2 * F : d;        // weight rows per expert
+  const int blk = blockIdx.x;                   // block of 16 weight rows
+  const size_t row_lo = (size_t)e * rows_e + (SWIGLU ? blk * 8 + g : blk * 16 + g);
+  const size_t row_hi = SWIGLU ? row_lo + F : row_lo + 8;
+  const int words = K / 8, G = K / 64;
+  const uint32_t* wlo = w + row_lo * words;
+  const uint32_t* whi = w + row_hi * words;
+  // token rows of this lane's B fragment: tokens g (group 0) and 8+g (group 1)
+  const __half* xr[2];
+  bool tok_ok[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int n = t * 8 + g;
+    tok_ok[t] = n < nv;
+    const size_t row = tok_ok[t] ? (SWIGLU ? (size_t)__ldg(row_map + r0 + n) : (size_t)(r0 + n)) : 0;
+    xr[t] = x16 + row * K;
+  }
+  const bool two = nv > 8;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  const int nsteps = K / 128;
+
+  // one step's operands: this lane's 32 elements of both rows, their group's
+  // scales and biases, and the same 32 activations of its two token rows
+  struct Step {
+    uint4 wl, wh;
+    uint16_t sl, bl, sh, bh;
+    uint4 xv[2][4];
+  };
+  auto load = [&](Step& S, int st) {
+    const int k0 = st * 128 + c * 32;
+    S.wl = ldg_nc_v4(wlo + k0 / 8);
+    S.wh = ldg_nc_v4(whi + k0 / 8);
+    const int grp = k0 / 64;
+    S.sl = __ldg(sc + row_lo * G + grp);
+    S.bl = __ldg(bi + row_lo * G + grp);
+    S.sh = __ldg(sc + row_hi * G + grp);
+    S.bh = __ldg(bi + row_hi * G + grp);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        S.xv[t][q] = (tok_ok[t] && (t == 0 || two)) ? ldg_v4(xr[t] + k0 + q * 8)
+                                                    : make_uint4(0, 0, 0, 0);
+  };
+  auto compute = [&](const Step& S) {
+    const uint32_t sl = h2_from_bf16(S.sl), bl = h2_from_bf16(S.bl);
+    const uint32_t sh = h2_from_bf16(S.sh), bh = h2_from_bf16(S.bh);
+    const uint32_t wlw[4] = {S.wl.x, S.wl.y, S.wl.z, S.wl.w};
+    const uint32_t whw[4] = {S.wh.x, S.wh.y, S.wh.z, S.wh.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {               // word q: MMAs m = 2q, 2q+1
+      uint32_t dl[4], dh[4];
+      q4_word_f16(wlw[q], sl, bl, dl);
+      q4_word_f16(whw[q], sh, bh, dh);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t a[4] = {dl[2 * half], dh[2 * half], dl[2 * half + 1], dh[2 * half + 1]};
+        // activations c*32 + 4m + (0..3) with m = 2q + half: uint32 words
+        // 2m and 2m+1 of this lane's 64 bytes
+        const int m = 2 * q + half;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (t == 1 && !two) break;
+          const uint4 v = S.xv[t][m >> 1];
+          mma_16816(acc[t], a, (m & 1) ? v.z : v.x, (m & 1) ? v.w : v.y);
+        }
+      }
+    }
+  };
+  // steps warp, warp + 4, ...: the next step's loads are in flight while the
+  // current one is dequantised and multiplied (two register buffers used in
+  // turn -- never copied into each other, which would wait for the loads)
+  Step b0, b1;
+  int st = warp;
+  if (st < nsteps) load(b0, st);
+  while (st < nsteps) {
+    if (st + kMmaWarps < nsteps) load(b1, st + kMmaWarps);
+    compute(b0);
+    st += kMmaWarps;
+    if (st >= nsteps) break;
+    if (st + kMmaWarps < nsteps) load(b0, st + kMmaWarps);
+    compute(b1);
+    st += kMmaWarps;
+  }
+  // reduce the 4 warps' partial sums (warp 0 keeps the result)
+  if (warp > 0) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[warp - 1][lane][t * 4 + i] = acc[t][i];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll
+  for (int wv = 0; wv < kMmaWarps - 1; ++wv)
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[t][i] += red[wv][lane][t * 4 + i];
+  // lane (g, c) holds rows g and g+8 for tokens t*8 + 2c and t*8 + 2c + 1
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int n = t * 8 + 2 * c + j;
+      if (n >= nv) continue;
+      if (SWIGLU) {
+        const float v = swiglu(acc[t][j], acc[t][2 + j]);
+        if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
+        reinterpret_cast<__half*>(out)[(size_t)(r0 + n) * F + blk * 8 + g] = __float2half_rn(v);
+      } else {
+        float* ys = reinterpret_cast<float*>(out);
+        ys[(size_t)(r0 + n) * d + blk * 16 + g] = acc[t][j];
+        ys[(size_t)(r0 + n) * d + blk * 16 + 8 + g] = acc[t][2 + j];
+      }
+    }
+  }
+}
+
+bool gemv_q4_mma_ok(const moe_experts& ex, int dt, int BM) {
+  return ex.fmt == MOE_W_Q4G64 && dt == MOE_BF16 && BM <= kMmaMaxRows && ex.d % 128 == 0 &&
+         ex.F % 128 == 0;
+}
+
+cudaError_t launch_swiglu_q4_mma(const void* x16, const uint32_t* row_map, const int32_t* row_off,
+                                 const int32_t* tile_off, int BM, int R, const moe_experts& ex,
+                                 void* h, int* status, cudaStream_t s) {
+  const long long tiles = max_tiles(R, ex.E, BM);
+  if (tiles <= 0) return cudaSuccess;
+  if (tiles > 65535) return cudaErrorInvalidConfiguration;
+  dim3 grid(ex.F / 8, (unsigned)tiles);
+  launch_pdl(gemv_q4_mma_kernel<true>, grid, kMmaWarps * 32, 0, s, 
+      (const __half*)x16, row_map, row_off, tile_off, BM, ex.E, ex.d, ex.F,
+      (const uint32_t*)ex.w_gu, (const uint16_t*)ex.s_gu, (const uint16_t*)ex.b_gu, h, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_down_q4_mma(const void* h, const int32_t* row_off, const int32_t* tile_off,
+                               int BM, int R, const moe_experts& ex, void* ys, int* status,
+                               cudaStream_t s) {
+  const long long tiles = max_tiles(R, ex.E, BM);
+  if (tiles <= 0) return cudaSuccess;
+  if (tiles > 65535) return cudaErrorInvalidConfiguration;
+  dim3 grid(ex.d / 16, (unsigned)tiles);
+  launch_pdl(gemv_q4_mma_kernel<false>, grid, kMmaWarps * 32, 0, s, 
+      (const __half*)h, nullptr, row_off, tile_off, BM, ex.E, ex.d, ex.F,
+      (const uint32_t*)ex.w_dn, (const uint16_t*)ex.s_dn, (const uint16_t*)ex.b_dn, ys, status);
   return cudaGetLastError();
 }
 

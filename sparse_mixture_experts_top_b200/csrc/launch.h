@@ -45,6 +45,19 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
                              const int32_t* tile_off, int BM, int R, const moe_experts& ex,
                              void* ys, cudaStream_t s);
 
+// q4 weights with bf16 activations and at most 16 rows per tile: mma.sync
+// fp16 GEMV (x16: activations converted to fp16; h fp16 in, ys fp32 out).
+bool gemv_q4_mma_ok(const moe_experts& ex, int dt, int BM);
+cudaError_t launch_swiglu_q4_mma(const void* x16, const uint32_t* row_map, const int32_t* row_off,
+                                 const int32_t* tile_off, int BM, int R, const moe_experts& ex,
+                                 void* h, int* status, cudaStream_t s);
+cudaError_t launch_down_q4_mma(const void* h, const int32_t* row_off, const int32_t* tile_off,
+                               int BM, int R, const moe_experts& ex, void* ys, int* status,
+                               cudaStream_t s);
+// bf16 -> fp16 copy of n values (n a multiple of 8); out-of-range values
+// are reported as MOE_ERR_RANGE
+cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cudaStream_t s);
+
 // Tensor-core grouped kernels (bf16 activations; bf16 or q4 weights).
 // BM must equal tc_block_m().
 int tc_block_m();

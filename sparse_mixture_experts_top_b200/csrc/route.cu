@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const T* __restrict__ 
                                                           const T* __restrict__ wr,
                                                           const float* __restrict__ bias, int Tn,
                                                           int d, int E, float* __restrict__ out) {
+  pdl_wait();
+  pdl_launch();
   constexpr int TG = 8;                         // tokens per warp
   constexpr int VE = 16 / sizeof(T);            // elements per 16-byte load
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -67,6 +69,8 @@ __global__ void __launch_bounds__(256) router_tile_kernel(const T* __restrict__ 
                                                           const T* __restrict__ wr,
                                                           const float* __restrict__ bias, int Tn,
                                                           int d, int E, float* __restrict__ out) {
+  pdl_wait();
+  pdl_launch();
   constexpr int BT = 64, BE = 64, BK = 32;
   __shared__ float As[BK][BT + 4];
   __shared__ float Bs[BK][BE + 4];
@@ -114,18 +118,18 @@ cudaError_t launch_router_logits(const void* x, int dt, const void* w_router, co
     int warps = E * ((T + 7) / 8);
     int blocks = (warps * 32 + 255) / 256;
     if (dt == MOE_BF16)
-      router_gemv_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+      launch_pdl(router_gemv_kernel<__nv_bfloat16>, blocks, 256, 0, s, 
           (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, T, d, E, logits);
     else
-      router_gemv_kernel<float><<<blocks, 256, 0, s>>>((const float*)x, (const float*)w_router,
+      launch_pdl(router_gemv_kernel<float>, blocks, 256, 0, s, (const float*)x, (const float*)w_router,
                                                        bias, T, d, E, logits);
   } else {
     dim3 grid((E + 63) / 64, (T + 63) / 64);
     if (dt == MOE_BF16)
-      router_tile_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+      launch_pdl(router_tile_kernel<__nv_bfloat16>, grid, 256, 0, s, 
           (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, T, d, E, logits);
     else
-      router_tile_kernel<float><<<grid, 256, 0, s>>>((const float*)x, (const float*)w_router,
+      launch_pdl(router_tile_kernel<float>, grid, 256, 0, s, (const float*)x, (const float*)w_router,
                                                      bias, T, d, E, logits);
   }
   return cudaGetLastError();
@@ -156,6 +160,8 @@ template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
                                                    int k, int32_t* __restrict__ idx_out,
                                                    float* __restrict__ w_out) {
+  pdl_wait();
+  pdl_launch();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -195,12 +201,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
                         cudaStream_t s) {
   const int blocks = (T * 32 + 255) / 256;
-  if (E <= 32) topk_kernel<1><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, w);
-  else if (E <= 64) topk_kernel<2><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, w);
-  else if (E <= 128) topk_kernel<4><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, w);
-  else if (E <= 256) topk_kernel<8><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, w);
-  else if (E <= 512) topk_kernel<16><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, w);
-  else if (E <= 1024) topk_kernel<32><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, w);
+  if (E <= 32) launch_pdl(topk_kernel<1>, blocks, 256, 0, s, logits, T, E, k, idx, w);
+  else if (E <= 64) launch_pdl(topk_kernel<2>, blocks, 256, 0, s, logits, T, E, k, idx, w);
+  else if (E <= 128) launch_pdl(topk_kernel<4>, blocks, 256, 0, s, logits, T, E, k, idx, w);
+  else if (E <= 256) launch_pdl(topk_kernel<8>, blocks, 256, 0, s, logits, T, E, k, idx, w);
+  else if (E <= 512) launch_pdl(topk_kernel<16>, blocks, 256, 0, s, logits, T, E, k, idx, w);
+  else if (E <= 1024) launch_pdl(topk_kernel<32>, blocks, 256, 0, s, logits, T, E, k, idx, w);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }

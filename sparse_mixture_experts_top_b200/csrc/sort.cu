@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(1024) sort_single_kernel(
     const int32_t* __restrict__ idx, int R, int k, int E, int BM, uint32_t* __restrict__ order,
     uint32_t* __restrict__ inv_order, uint32_t* __restrict__ row_map, int32_t* __restrict__ counts,
     int32_t* __restrict__ row_off, int32_t* __restrict__ tile_off) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ int sm[];
   int* cnt = sm;            // [E]
   int* tiles = sm + E;      // [E]
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(1024) sort_single_kernel(
 
 __global__ void __launch_bounds__(1024) sort_count_kernel(const int32_t* __restrict__ idx, long long R,
                                                           int E, int32_t* __restrict__ chunk_cnt) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -162,6 +166,8 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ row_off,
                                                          int32_t* __restrict__ tile_off) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ int sm[];
   int* cnt = sm;
   int* tiles = sm + E;
@@ -196,6 +202,8 @@ __global__ void __launch_bounds__(1024) sort_scatter_kernel(
     const int32_t* __restrict__ idx, long long R, int k, int E,
     const int32_t* __restrict__ chunk_base, uint32_t* __restrict__ order,
     uint32_t* __restrict__ inv_order, uint32_t* __restrict__ row_map) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ int cursor[];
   uint16_t* wtab = reinterpret_cast<uint16_t*>(cursor + E);   // [32][E]
   for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -214,19 +222,19 @@ cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, ui
   if (R <= kChunk) {
     cudaFuncSetAttribute(sort_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)(smem2 + wtab));
-    sort_single_kernel<<<1, 1024, smem2 + wtab, s>>>(idx, (int)R, k, E, BM, order, inv_order,
+    launch_pdl(sort_single_kernel, 1, 1024, smem2 + wtab, s, idx, (int)R, k, E, BM, order, inv_order,
                                                      row_map, counts, row_off, tile_off);
     return cudaGetLastError();
   }
   const int nch = num_chunks(R);
   int32_t* chunk_cnt = reinterpret_cast<int32_t*>(ws);
   int32_t* chunk_base = chunk_cnt + (size_t)nch * E;
-  sort_count_kernel<<<nch, 1024, E * sizeof(int), s>>>(idx, R, E, chunk_cnt);
-  sort_scan_kernel<<<1, 1024, smem2, s>>>(chunk_cnt, nch, E, BM, chunk_base, counts, row_off,
+  launch_pdl(sort_count_kernel, nch, 1024, E * sizeof(int), s, idx, R, E, chunk_cnt);
+  launch_pdl(sort_scan_kernel, 1, 1024, smem2, s, chunk_cnt, nch, E, BM, chunk_base, counts, row_off,
                                           tile_off);
   cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)(E * sizeof(int) + wtab));
-  sort_scatter_kernel<<<nch, 1024, E * sizeof(int) + wtab, s>>>(idx, R, k, E, chunk_base, order,
+  launch_pdl(sort_scatter_kernel, nch, 1024, E * sizeof(int) + wtab, s, idx, R, k, E, chunk_base, order,
                                                                 inv_order, row_map);
   return cudaGetLastError();
 }

@@ -11,10 +11,11 @@
 //   * swap-AB: the MMA's M = 128 weight rows (output features), N = the
 //     tile's token rows (<= 128, rounded up to 16 per tile at run time), so
 //     a tile with few rows costs proportionally few tensor cycles;
-//   * warp 0 (producer): TMA loads of the raw weight tile (packed q4 words or
-//     bf16) into a shared-memory ring, and of the tile's token rows -- one
-//     single-row TMA per row through row_map (gather), or one box when rows
-//     are contiguous -- into a 128B-swizzled K-major ring;
+//   * warp 0: TMA loads of the raw weight tile (packed q4 words or bf16,
+//     128-byte rows) into a shared-memory ring;
+//   * warp 2: cp.async copies of the tile's token rows -- through row_map
+//     (gather) or contiguous -- into a 128B-swizzled K-major ring (per-row
+//     TMA loads cost ~30 ns of issue each, which starved the tensor core);
 //   * warps 8..15 (dequant): each thread owns one weight row (one TMEM lane):
 //     reads its packed words from shared memory, dequantises w = s*q + b to
 //     bf16 pairs and writes them into TMEM with tcgen05.st, where the MMA
@@ -48,9 +49,15 @@ namespace tc {
 constexpr int BN = 128;        // token rows per tile (the sort tables' BM)
 constexpr int BMW = 128;       // weight rows per tile (MMA M)
 constexpr int KA = 64;         // K elements per A stage (one q4 group)
-constexpr int NB = 6;          // token-row (B) stages
+#ifndef MOE_TC_NB
+#define MOE_TC_NB 6
+#endif
+#ifndef MOE_TC_BLAG
+#define MOE_TC_BLAG 5
+#endif
+constexpr int NB = MOE_TC_NB;  // token-row (B) stages
 constexpr int kMaxE = 1024;    // tile / row tables cached in shared memory
-constexpr int kScaleAhead = 4; // raw stages of scales/biases loaded ahead
+constexpr int kBLag = MOE_TC_BLAG;  // token-row stages in flight before one is signalled
 constexpr int kThreads = 512;
 constexpr int kEpiWarp0 = 4;
 constexpr int kDqWarp0 = 8;
@@ -62,22 +69,29 @@ template <int FMT, int EPI>
 struct Cfg {
   static constexpr int NMAT = EPI == EPI_SWIGLU ? 2 : 1;
   static constexpr bool Q4 = FMT == MOE_W_Q4G64;
-  static constexpr int KR = Q4 ? 128 : 64;                  // K elements per raw stage
-  static constexpr int RAW_ROW = Q4 ? 64 : 128;             // bytes per weight row per raw stage
+  static constexpr int KR = Q4 ? 256 : 64;                  // K elements per raw stage
+  static constexpr int RAW_ROW = 128;                       // bytes per weight row per raw stage
   static constexpr int RAW_MAT = BMW * RAW_ROW;
   static constexpr int RAW_BYTES = NMAT * RAW_MAT;
-  static constexpr int A_PER_RAW = KR / KA;
-  static constexpr int NR_FIT = (96 * 1024) / RAW_BYTES;
+  static constexpr int A_PER_RAW = KR / KA;                 // 4 (q4) or 1 (bf16)
+#ifndef MOE_TC_RAW_KB
+#define MOE_TC_RAW_KB 96
+#endif
+  static constexpr int NR_FIT = (MOE_TC_RAW_KB * 1024) / RAW_BYTES;
   static constexpr int NR = NR_FIT > 8 ? 8 : NR_FIT;
   static constexpr int ACC_COLS = NMAT * BN;
   static constexpr int A_COLS = NMAT * (KA / 2);            // 32-bit TMEM columns per A stage
   static constexpr int NA = (512 - ACC_COLS) / A_COLS;
   static constexpr int B_BYTES = BN * 128;
   // warps that write one A stage: NMAT == 2: 4 gate + 4 up warps;
-  // NMAT == 1: q4 -- the 4 warps of one half; bf16 -- all 8 (half the columns each)
+  // NMAT == 1: q4 -- the 4 warps of one half of the raw row; bf16 -- all 8
+  // (half the columns each)
   static constexpr int A_ARRIVALS = NMAT == 2 ? 8 : (Q4 ? 4 : 8);
-  static constexpr int TABLES = 2 * (kMaxE + 1) * 4;       // tile_off, row_off copies
-  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES;
+  // q4 scales and biases of a raw stage: [NMAT][128 rows][4 groups] bf16 each
+  static constexpr int SCL_BYTES = Q4 ? NMAT * BMW * 4 * 2 * 2 : 0;
+  static constexpr int TABLES = 2 * (kMaxE + 1) * 4 + BN * 4;  // tile/row tables, tile rows
+  static_assert(kBLag >= 1 && kBLag < NB && kBLag <= 8, "loader lag must leave a free stage");
+  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
 };
 
 struct Params {
@@ -92,7 +106,8 @@ struct Params {
   int G;               // q4 groups per weight row (K / 64)
   const uint16_t* scales;
   const uint16_t* biases;
-  const uint32_t* row_map;
+  const uint32_t* row_map;  // token of each sorted row (gather), or null
+  const void* b_src;        // token rows: [rows][K] 16-bit (x16, h or x)
   void* out;
   int out_ld;          // elements per output row
   int m_limit;         // valid weight rows per group (router: E)
@@ -319,8 +334,9 @@ __device__ __forceinline__ int total_units(const Params& p, const int* s_toff) {
 
 template <int FMT, int EPI, bool GATHER, bool ROUTER>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA,
-                      const __grid_constant__ CUtensorMap tmB) {
+    grouped_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA) {
+  pdl_wait();
+  pdl_launch();
   using C = Cfg<FMT, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -341,19 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_toff = reinterpret_cast<int*>(smem + C::NR * C::RAW_BYTES + NB * C::B_BYTES + 1024);
   int* s_roff = s_toff + kMaxE + 1;
-  if (!ROUTER) {
-    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
-      s_toff[i] = __ldg(p.tile_off + i);
-      s_roff[i] = __ldg(p.row_off + i);
-    }
-  }
+  int* s_trow = s_roff + kMaxE + 1;     // [BN] source rows of the loader's current tile
+  // q4 scale ring: raw stage rs holds scales [NMAT][128][4] then biases [NMAT][128][4]
+  const uint32_t scl_base = smem_u32(s_trow + BN);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NR; ++i) {
-      mbar_init(smem_u32(raw_full + i), 1);
+      // q4: the TMA arrive + the 32 lanes' cp.async arrivals for the scales
+      mbar_init(smem_u32(raw_full + i), C::Q4 ? 33 : 1);
       mbar_init(smem_u32(raw_empty + i), 8);
     }
     for (int i = 0; i < C::NA; ++i) {
@@ -361,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(a_empty + i), 1);
     }
     for (int i = 0; i < NB; ++i) {
-      mbar_init(smem_u32(b_full + i), 1);
+      mbar_init(smem_u32(b_full + i), 1);   // the loader warp's lane 0
       mbar_init(smem_u32(b_empty + i), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
@@ -370,13 +384,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                      smem_u32(tmem_slot))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // the prologue above overlaps the previous kernel; everything below reads
+  // what earlier kernels wrote
+  pdl_wait();
+  pdl_launch();
+  if (!ROUTER) {
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+      s_toff[i] = __ldg(p.tile_off + i);
+      s_roff[i] = __ldg(p.row_off + i);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -388,26 +411,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nka = p.K / KA;              // A stages per tile
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    uint32_t raw_it = 0, b_it = 0;
+    // ------------------------------------------------------------ raw weights (TMA)
+    uint32_t raw_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int e, mb, r0, nv;
       decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
       const int wrow = (ROUTER ? 0 : e * p.rows_per_group) + mb * BMW;
-      int trow[BN / 32];
-      if (GATHER) {
-#pragma unroll
-        for (int j = 0; j < BN / 32; ++j) {
-          const int n = lane + 32 * j;
-          trow[j] = n < nv ? (int)__ldg(p.row_map + r0 + n) : 0;
-        }
-      }
       for (int kr = 0; kr < nkr && ok; ++kr) {
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_empty + rs), ((raw_it / C::NR) & 1) ^ 1, abort_flag,
                             p.status);
         if (!ok) break;
+        if (C::Q4) {
+          // the stage's scales and biases (4 groups of each weight row), 8
+          // bytes per row and array, copied by the 32 lanes; each lane's
+          // arrival fires when its copies have landed
+          const uint32_t sdst = scl_base + rs * C::SCL_BYTES;
+#pragma unroll
+          for (int mat = 0; mat < C::NMAT; ++mat)
+#pragma unroll
+            for (int j = 0; j < BMW / 32; ++j) {
+              const int m = lane + 32 * j;
+              const size_t grow = (size_t)wrow + (mat ? p.up_off : 0) + m;
+              const uint32_t o = (uint32_t)((mat * BMW + m) * 8);
+              asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sdst + o),
+                           "l"(p.scales + grow * p.G + 4 * kr)
+                           : "memory");
+              asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                               sdst + C::SCL_BYTES / 2 + o),
+                           "l"(p.biases + grow * p.G + 4 * kr)
+                           : "memory");
+            }
+          asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                           smem_u32(raw_full + rs))
+                       : "memory");
+        }
         if (lane == 0) {
           const uint32_t dst = raw_base + rs * C::RAW_BYTES;
           const uint32_t bar = smem_u32(raw_full + rs);
@@ -417,41 +456,70 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (C::NMAT == 2) tma_load_2d(dst + C::RAW_MAT, &tmA, x, wrow + p.up_off, bar);
         }
         ++raw_it;
-        for (int a = 0; a < C::A_PER_RAW; ++a) {
-          const int kb = kr * C::A_PER_RAW + a;
-          const int bs = b_it % NB;
-          ok = mbar_wait_warp(smem_u32(b_empty + bs), ((b_it / NB) & 1) ^ 1, abort_flag, p.status);
-          if (!ok) break;
-          const uint32_t dst = b_base + bs * C::B_BYTES;
-          const uint32_t bar = smem_u32(b_full + bs);
-          if (GATHER) {
-            if (lane == 0) mbar_arrive_tx(bar, (uint32_t)nv * 128u);
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < BN / 32; ++j) {
-              const int n = lane + 32 * j;
-              if (n < nv) tma_load_2d(dst + n * 128, &tmB, kb * KA, trow[j], bar);
-            }
-          } else if (lane == 0) {
-            mbar_arrive_tx(bar, C::B_BYTES);
-            tma_load_2d(dst, &tmB, kb * KA, r0, bar);
-          }
-          ++b_it;
-        }
       }
     }
     // copies in flight: wait (bounded, also when aborting) for the last
     // phase issued on every stage before the CTA may exit
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       for (uint32_t i = 0; i < (uint32_t)C::NR && i < raw_it; ++i) {
         const uint32_t last = raw_it - 1 - i;
         mbar_wait(smem_u32(raw_full + last % C::NR), (last / C::NR) & 1, abort_flag, p.status, false);
       }
-      for (uint32_t i = 0; i < (uint32_t)NB && i < b_it; ++i) {
-        const uint32_t last = b_it - 1 - i;
-        mbar_wait(smem_u32(b_full + last % NB), (last / NB) & 1, abort_flag, p.status, false);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ token rows (cp.async)
+    // Lane l copies 16-byte chunks l, l + 32, ... of the tile's rows (chunk c
+    // of row n lands at n*128 + ((c ^ (n & 7)) * 16): the 128B-swizzled
+    // K-major layout the MMA reads). A stage is signalled kBLag stages after
+    // its copies were issued, once they are complete and made visible to the
+    // tensor core's (async proxy) reads.
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(p.b_src);
+    uint32_t b_it = 0, signalled = 0;
+    bool ok = true;
+    auto signal_oldest = [&](int keep) {
+      // complete all but the newest `keep` groups, then signal the oldest stage
+      switch (keep) {
+        case 7: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(b_full + signalled % NB));
+      ++signalled;
+    };
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int e, mb, r0, nv;
+      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
+      __syncwarp();
+      for (int n = lane; n < nv; n += 32) s_trow[n] = GATHER ? (int)__ldg(p.row_map + r0 + n) : r0 + n;
+      __syncwarp();
+      for (int kb = 0; kb < nka && ok; ++kb) {
+        const int bs = b_it % NB;
+        ok = mbar_wait_warp(smem_u32(b_empty + bs), ((b_it / NB) & 1) ^ 1, abort_flag, p.status);
+        if (!ok) break;
+        const uint32_t dst = b_base + bs * C::B_BYTES;
+        for (int i = lane; i < nv * 8; i += 32) {
+          const int n = i >> 3, c = i & 7;
+          const uint16_t* g = src + (size_t)s_trow[n] * p.K + kb * KA + c * 8;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                           dst + n * 128 + ((c ^ (n & 7)) << 4)),
+                       "l"(g)
+                       : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        ++b_it;
+        if (b_it - signalled == (uint32_t)kBLag) signal_oldest(kBLag - 1);
       }
     }
+    while (signalled < b_it) signal_oldest((int)(b_it - signalled) - 1);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -556,89 +624,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t raw_it = 0, a_it = 0;
     bool ok = true;
-    // q4 scales/biases: a queue of the next kScaleAhead raw stages, filled by
-    // a cursor that walks the same (tile, raw stage) sequence ahead of the
-    // consumer, across tile boundaries
-    const int sub = C::NMAT == 2 ? 0 : part;        // group within the raw stage (NMAT 1)
-    int pf_u = blockIdx.x, pf_kr = 0;
-    const uint16_t* pf_s = nullptr;
-    const uint16_t* pf_b = nullptr;
-    auto pf_row = [&]() {
-      if (!C::Q4 || pf_u >= total) return;
-      int e2, mb2, r02, nv2;
-      decode_tile<ROUTER>(p, s_toff, s_roff, pf_u, e2, mb2, r02, nv2);
-      const size_t grow = (size_t)(ROUTER ? 0 : e2 * p.rows_per_group) +
-                          (C::NMAT == 2 ? part * p.up_off : 0) + mb2 * BMW + m;
-      pf_s = p.scales + grow * p.G;
-      pf_b = p.biases + grow * p.G;
-    };
-    auto pf_load = [&](uint32_t& sv, uint32_t& bv) {
-      sv = bv = 0;
-      if (!C::Q4 || pf_u >= total) return;
-      if (C::NMAT == 2) {   // both groups of the raw stage: 2 x bf16
-        sv = __ldg(reinterpret_cast<const uint32_t*>(pf_s + 2 * pf_kr));
-        bv = __ldg(reinterpret_cast<const uint32_t*>(pf_b + 2 * pf_kr));
-      } else {
-        sv = __ldg(pf_s + 2 * pf_kr + sub);
-        bv = __ldg(pf_b + 2 * pf_kr + sub);
-      }
-      if (++pf_kr == nkr) {
-        pf_kr = 0;
-        pf_u += gridDim.x;
-        pf_row();
-      }
-    };
-    uint32_t sq[kScaleAhead], bq[kScaleAhead];
-    pf_row();
-#pragma unroll
-    for (int i = 0; i < kScaleAhead; ++i) pf_load(sq[i], bq[i]);
-
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int e, mb, r0, nv;
       decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
       for (int kr = 0; kr < nkr && ok; ++kr) {
-        const uint32_t sc = sq[0], bi = bq[0];
-#pragma unroll
-        for (int i = 0; i + 1 < kScaleAhead; ++i) {
-          sq[i] = sq[i + 1];
-          bq[i] = bq[i + 1];
-        }
-        pf_load(sq[kScaleAhead - 1], bq[kScaleAhead - 1]);
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status);
         if (!ok) break;
         const uint32_t rbase = raw_base + rs * C::RAW_BYTES;
         uint32_t vals[32];
+        // q4: this row's 4 groups of scales and biases (bf16 pairs)
+        uint32_t sc[2] = {0, 0}, bi[2] = {0, 0};
         if (C::Q4) {
-          // my row: 64 bytes = 4 chunks of 16 B, 64-byte swizzle
-          const uint32_t rowa = rbase + (C::NMAT == 2 ? part * C::RAW_MAT : 0) + m * 64;
-          const int sw = (m >> 1) & 3;
-          uint4 wv[4];
-          if (C::NMAT == 2) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) wv[c] = lds128(rowa + ((c ^ sw) << 4));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) wv[c] = lds128(rowa + (((2 * part + c) ^ sw) << 4));
+          const uint32_t so = scl_base + rs * C::SCL_BYTES +
+                              (uint32_t)(((C::NMAT == 2 ? part : 0) * BMW + m) * 8);
+          asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(sc[0]), "=r"(sc[1]) : "r"(so));
+          asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                       : "=r"(bi[0]), "=r"(bi[1])
+                       : "r"(so + C::SCL_BYTES / 2));
+          if (C::NMAT == 1 && part) {   // half 1: groups 2, 3
+            sc[0] = sc[1];
+            bi[0] = bi[1];
           }
+        }
+        if (C::Q4) {
+          // my row: 128 bytes = 8 chunks of 16 B (128-byte swizzle): chunk pair
+          // (2j, 2j+1) holds the 64 elements of A stage j (group 4kr + j).
+          // NMAT 2: this thread converts all 4 A stages of its matrix;
+          // NMAT 1: half `part` converts A stages 2*part and 2*part + 1.
+          const uint32_t rowa = rbase + (C::NMAT == 2 ? part * C::RAW_MAT : 0) + m * 128;
+          const int sw = m & 7;
+          constexpr int nst = C::NMAT == 2 ? 4 : 2;    // A stages this thread converts
+          const int cbase = C::NMAT == 2 ? 0 : 4 * part;  // its first 16-byte chunk
+          uint4 wv[2 * nst];
+#pragma unroll
+          for (int c = 0; c < 2 * nst; ++c) wv[c] = lds128(rowa + (((cbase + c) ^ sw) << 4));
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
-          // NMAT 2: words 0..7 -> A stage 0 (group 2kr), words 8..15 -> A stage 1
-          const int nst = C::NMAT == 2 ? 2 : 1;
-          for (int st = 0; st < nst && ok; ++st) {
-            uint32_t s2, b2;
-            if (C::NMAT == 2) {
-              s2 = f16x2_from_bf16(st ? (sc >> 16) : (sc & 0xFFFFu));
-              b2 = f16x2_from_bf16(st ? (bi >> 16) : (bi & 0xFFFFu));
-            } else {
-              s2 = f16x2_from_bf16(sc & 0xFFFFu);
-              b2 = f16x2_from_bf16(bi & 0xFFFFu);
-            }
+#pragma unroll
+          for (int st = 0; st < nst; ++st) {
+            if (!ok) break;
+            const int j = (C::NMAT == 2 ? 0 : 2 * part) + st;   // A stage within the raw stage
+            const uint32_t sv = C::NMAT == 2 ? sc[st >> 1] : sc[0];
+            const uint32_t bv = C::NMAT == 2 ? bi[st >> 1] : bi[0];
+            const uint32_t s2 = f16x2_from_bf16((st & 1) ? (sv >> 16) : (sv & 0xFFFFu));
+            const uint32_t b2 = f16x2_from_bf16((st & 1) ? (bv >> 16) : (bv & 0xFFFFu));
             const uint4 w0 = wv[2 * st], w1 = wv[2 * st + 1];
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) dequant_word(ws[i], s2, b2, vals + 4 * i);
-            const uint32_t stage = a_it + (C::NMAT == 2 ? st : part);
+            const uint32_t stage = a_it + j;
             const int as = stage % C::NA;
             ok = mbar_wait_warp(smem_u32(a_empty + as), ((stage / C::NA) & 1) ^ 1, abort_flag,
                                 p.status);
@@ -745,16 +780,10 @@ static int num_sms() {
 // raw weight-tile map over a stack of `rows` weight rows of K elements
 static bool weight_map(CUtensorMap* m, int fmt, const void* w, long long rows, int K) {
   if (fmt == MOE_W_Q4G64)
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / 8, rows, (uint64_t)K / 2, 16, BMW,
-                    CU_TENSOR_MAP_SWIZZLE_64B);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / 8, rows, (uint64_t)K / 2, 32, BMW,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, rows, (uint64_t)K * 2, 64, BMW,
                   CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-// token-row map: rows of K 16-bit values (fp16 or bf16), box of `box_rows` rows
-static bool rows_map(CUtensorMap* m, const void* x, long long rows, int K, int box_rows, bool f16) {
-  return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x,
-                  K, rows, (uint64_t)K * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // bf16 -> fp16, 8 values per thread; values that do not round to a finite
@@ -762,6 +791,8 @@ static bool rows_map(CUtensorMap* m, const void* x, long long rows, int K, int b
 __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ in,
                                                      uint4* __restrict__ out, long long n8,
                                                      int* status) {
+  pdl_wait();
+  pdl_launch();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   bool ok = true;
   if (i < n8) {
@@ -782,26 +813,35 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ i
 }
 
 template <int FMT, int EPI, bool GATHER, bool ROUTER>
-static cudaError_t run(const Params& p, const CUtensorMap& a, const CUtensorMap& b,
-                       long long units_ub, cudaStream_t s) {
+static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub, cudaStream_t s) {
   using C = Cfg<FMT, EPI>;
   auto kern = grouped_tc_kernel<FMT, EPI, GATHER, ROUTER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const long long grid = units_ub < num_sms() ? units_ub : num_sms();
   if (grid <= 0) return cudaSuccess;
-  kern<<<(unsigned)grid, kThreads, C::SMEM, s>>>(p, a, b);
+  launch_pdl(kern, (unsigned)grid, kThreads, C::SMEM, s, p, a);
   return cudaGetLastError();
 }
 
+// the kernels tile d and F by 128 rows; q4 raw stages span 256 elements of K
 static bool tc_shape_ok(const moe_experts& ex) {
-  return ex.d % 128 == 0 && ex.F % 128 == 0 &&
-         (ex.fmt == MOE_W_Q4G64 || ex.fmt == MOE_W_BF16);
+  if (ex.d % 128 || ex.F % 128) return false;
+  if (ex.fmt == MOE_W_Q4G64) return ex.d % 256 == 0 && ex.F % 256 == 0;
+  return ex.fmt == MOE_W_BF16;
 }
 
 }  // namespace tc
 
 int tc_block_m() { return tc::BN; }
+
+cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cudaStream_t s) {
+  const long long n8 = n / 8;
+  if (n8 <= 0) return cudaSuccess;
+  launch_pdl(tc::to_f16_kernel, (unsigned)((n8 + 255) / 256), 256, 0, s, (const uint4*)x, (uint4*)x16, n8,
+                                                                 status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
@@ -809,14 +849,10 @@ cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, cons
   using namespace tc;
   if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
   // the expert GEMMs take fp16 operands: x is converted once into x16 [T][d]
-  const long long n8 = (long long)T * ex.d / 8;
-  to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const uint4*)x, (uint4*)x16, n8,
-                                                             status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_to_f16(x, (long long)T * ex.d, x16, status, s);
   if (e != cudaSuccess) return e;
-  CUtensorMap ta, tb;
+  CUtensorMap ta;
   if (!weight_map(&ta, ex.fmt, ex.w_gu, (long long)ex.E * 2 * ex.F, ex.d)) return cudaErrorInvalidValue;
-  if (!rows_map(&tb, x16, T, ex.d, 1, true)) return cudaErrorInvalidValue;
   Params p{};
   p.row_off = row_off;
   p.tile_off = tile_off;
@@ -829,22 +865,22 @@ cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, cons
   p.scales = (const uint16_t*)ex.s_gu;
   p.biases = (const uint16_t*)ex.b_gu;
   p.row_map = row_map;
+  p.b_src = x16;
   p.out = h;
   p.out_ld = ex.F;
   p.m_limit = ex.F;
   p.status = status;
   const long long ub = max_tiles(R, ex.E, BN) * p.n_mb;
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_SWIGLU, true, false>(p, ta, tb, ub, s);
-  return run<MOE_W_BF16, EPI_SWIGLU, true, false>(p, ta, tb, ub, s);
+  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_SWIGLU, true, false>(p, ta, ub, s);
+  return run<MOE_W_BF16, EPI_SWIGLU, true, false>(p, ta, ub, s);
 }
 
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
                            const moe_experts& ex, void* ys, int* status, cudaStream_t s) {
   using namespace tc;
   if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
-  CUtensorMap ta, tb;
+  CUtensorMap ta;
   if (!weight_map(&ta, ex.fmt, ex.w_dn, (long long)ex.E * ex.d, ex.F)) return cudaErrorInvalidValue;
-  if (!rows_map(&tb, h, R, ex.F, BN, true)) return cudaErrorInvalidValue;
   Params p{};
   p.row_off = row_off;
   p.tile_off = tile_off;
@@ -856,13 +892,14 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.G = ex.F / 64;
   p.scales = (const uint16_t*)ex.s_dn;
   p.biases = (const uint16_t*)ex.b_dn;
+  p.b_src = h;
   p.out = ys;
   p.out_ld = ex.d;
   p.m_limit = ex.d;
   p.status = status;
   const long long ub = max_tiles(R, ex.E, BN) * p.n_mb;
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE_F32, false, false>(p, ta, tb, ub, s);
-  return run<MOE_W_BF16, EPI_STORE_F32, false, false>(p, ta, tb, ub, s);
+  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE_F32, false, false>(p, ta, ub, s);
+  return run<MOE_W_BF16, EPI_STORE_F32, false, false>(p, ta, ub, s);
 }
 
 cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const float* bias, int T,
@@ -870,9 +907,8 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
   using namespace tc;
   // few tokens: the weight-streaming kernel is faster than a 128-row tile
   if (T < 256 || d % 64 != 0) return cudaErrorNotSupported;
-  CUtensorMap ta, tb;
+  CUtensorMap ta;
   if (!weight_map(&ta, MOE_W_BF16, w_router, E, d)) return cudaErrorInvalidValue;
-  if (!rows_map(&tb, x, T, d, BN, false)) return cudaErrorInvalidValue;
   Params p{};
   p.E = 1;
   p.n_rows = T;
@@ -882,9 +918,10 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
   p.out_ld = E;
   p.m_limit = E;
   p.bias = bias;
+  p.b_src = x;
   p.status = status;
   const long long ub = (long long)((T + BN - 1) / BN) * p.n_mb;
-  return run<MOE_W_BF16, EPI_STORE_F32, false, true>(p, ta, tb, ub, s);
+  return run<MOE_W_BF16, EPI_STORE_F32, false, true>(p, ta, ub, s);
 }
 
 }  // namespace moe
