@@ -49,15 +49,7 @@ namespace tc {
 constexpr int BN = 128;        // token rows per tile (the sort tables' BM)
 constexpr int BMW = 128;       // weight rows per tile (MMA M)
 constexpr int KA = 64;         // K elements per A stage (one q4 group)
-#ifndef MOE_TC_NB
-#define MOE_TC_NB 6
-#endif
-#ifndef MOE_TC_BLAG
-#define MOE_TC_BLAG 5
-#endif
-constexpr int NB = MOE_TC_NB;  // token-row (B) stages
 constexpr int kMaxE = 1024;    // tile / row tables cached in shared memory
-constexpr int kBLag = MOE_TC_BLAG;  // token-row stages in flight before one is signalled
 constexpr int kThreads = 512;
 constexpr int kEpiWarp0 = 4;
 constexpr int kDqWarp0 = 8;
@@ -81,7 +73,10 @@ struct Cfg {
   static constexpr int NR = NR_FIT > 8 ? 8 : NR_FIT;
   static constexpr int ACC_COLS = NMAT * BN;
   static constexpr int A_COLS = NMAT * (KA / 2);            // 32-bit TMEM columns per A stage
-  static constexpr int NA = (512 - ACC_COLS) / A_COLS;
+  // k-block stages: stage s = A slot s (TMEM) + B slot s (shared memory).
+  // The MMA releases stages in pairs (one commit per two k-blocks: each
+  // tcgen05.commit costs the tensor pipe ~200 cycles), so NS is even.
+  static constexpr int NS = NMAT == 2 ? 4 : 6;
   static constexpr int B_BYTES = BN * 128;
   // warps that write one A stage: NMAT == 2: 4 gate + 4 up warps;
   // NMAT == 1: q4 -- the 4 warps of one half of the raw row; bf16 -- all 8
@@ -90,8 +85,8 @@ struct Cfg {
   // q4 scales and biases of a raw stage: [NMAT][128 rows][4 groups] bf16 each
   static constexpr int SCL_BYTES = Q4 ? NMAT * BMW * 4 * 2 * 2 : 0;
   static constexpr int TABLES = 2 * (kMaxE + 1) * 4 + BN * 4;  // tile/row tables, tile rows
-  static_assert(kBLag >= 1 && kBLag < NB && kBLag <= 8, "loader lag must leave a free stage");
-  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
+  static_assert(NS % 2 == 0 && ACC_COLS + NS * A_COLS <= 512, "stages must fit TMEM in pairs");
+  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NS * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
 };
 
 struct Params {
@@ -195,6 +190,60 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, u
       "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The MMAs of one 64-deep k-block (4 K-steps of 16) for one or two
+// accumulators, in a single statement: A columns a (+8 per K-step), B
+// descriptor low word blo (+2 per K-step, i.e. +32 bytes inside the 128-byte
+// swizzle atom), accumulate unless `first`. Keeping the issue path to a few
+// instructions per MMA matters: the tensor core takes a K=16 step of an
+// M=128 tile in ~80 cycles, and the single issuing thread must keep up.
+__device__ __forceinline__ void mma_kblock2(uint32_t d0, uint32_t d1, uint32_t a0, uint32_t a1,
+                                            uint32_t blo, uint32_t bhi, uint32_t idesc,
+                                            uint32_t first) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b64 b0, b1, b2, b3;\n\t"
+      "setp.eq.b32 pf, %7, 0;\n\t"
+      "setp.ne.b32 pt, %6, 0;\n\t"
+      "mov.b64 b0, {%4, %5};\n\t"
+      "add.u32 %4, %4, 2;\n\tmov.b64 b1, {%4, %5};\n\t"
+      "add.u32 %4, %4, 2;\n\tmov.b64 b2, {%4, %5};\n\t"
+      "add.u32 %4, %4, 2;\n\tmov.b64 b3, {%4, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b0, %6, pf;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b0, %6, pf;\n\t"
+      "add.u32 %2, %2, 8;\n\tadd.u32 %3, %3, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b1, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b1, %6, pt;\n\t"
+      "add.u32 %2, %2, 8;\n\tadd.u32 %3, %3, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b2, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b2, %6, pt;\n\t"
+      "add.u32 %2, %2, 8;\n\tadd.u32 %3, %3, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b3, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b3, %6, pt;\n\t}\n"
+      : "+r"(d0), "+r"(d1), "+r"(a0), "+r"(a1), "+r"(blo), "+r"(bhi)
+      : "r"(idesc), "r"(first)
+      : "memory");
+}
+__device__ __forceinline__ void mma_kblock1(uint32_t d0, uint32_t a0, uint32_t blo, uint32_t bhi,
+                                            uint32_t idesc, uint32_t first) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b64 b0, b1, b2, b3;\n\t"
+      "setp.eq.b32 pf, %5, 0;\n\t"
+      "setp.ne.b32 pt, %4, 0;\n\t"
+      "mov.b64 b0, {%2, %3};\n\t"
+      "add.u32 %2, %2, 2;\n\tmov.b64 b1, {%2, %3};\n\t"
+      "add.u32 %2, %2, 2;\n\tmov.b64 b2, {%2, %3};\n\t"
+      "add.u32 %2, %2, 2;\n\tmov.b64 b3, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b0, %4, pf;\n\t"
+      "add.u32 %1, %1, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b1, %4, pt;\n\t"
+      "add.u32 %1, %1, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b2, %4, pt;\n\t"
+      "add.u32 %1, %1, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b3, %4, pt;\n\t}\n"
+      : "+r"(d0), "+r"(a0), "+r"(blo), "+r"(bhi)
+      : "r"(idesc), "r"(first)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -343,19 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~(uintptr_t)1023);
   const uint32_t raw_base = smem_u32(smem);
   const uint32_t b_base = raw_base + C::NR * C::RAW_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NR * C::RAW_BYTES + NB * C::B_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NR * C::RAW_BYTES + C::NS * C::B_BYTES);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + C::NR;
   uint64_t* a_full = raw_empty + C::NR;
-  uint64_t* a_empty = a_full + C::NA;
-  uint64_t* b_full = a_empty + C::NA;
-  uint64_t* b_empty = b_full + NB;
-  uint64_t* acc_full = b_empty + NB;
+  uint64_t* b_full = a_full + C::NS;
+  uint64_t* s_empty = b_full + C::NS;    // [NS / 2]: stage pair released by the MMA
+  uint64_t* acc_full = s_empty + C::NS / 2;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_toff = reinterpret_cast<int*>(smem + C::NR * C::RAW_BYTES + NB * C::B_BYTES + 1024);
+  int* s_toff = reinterpret_cast<int*>(smem + C::NR * C::RAW_BYTES + C::NS * C::B_BYTES + 1024);
   int* s_roff = s_toff + kMaxE + 1;
   int* s_trow = s_roff + kMaxE + 1;     // [BN] source rows of the loader's current tile
   // q4 scale ring: raw stage rs holds scales [NMAT][128][4] then biases [NMAT][128][4]
@@ -370,14 +418,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(raw_full + i), C::Q4 ? 33 : 1);
       mbar_init(smem_u32(raw_empty + i), 8);
     }
-    for (int i = 0; i < C::NA; ++i) {
+    for (int i = 0; i < C::NS; ++i) {
       mbar_init(smem_u32(a_full + i), C::A_ARRIVALS);
-      mbar_init(smem_u32(a_empty + i), 1);
+      mbar_init(smem_u32(b_full + i), 32);  // the loader's 32 lanes, as their copies land
     }
-    for (int i = 0; i < NB; ++i) {
-      mbar_init(smem_u32(b_full + i), 1);   // the loader warp's lane 0
-      mbar_init(smem_u32(b_empty + i), 1);
-    }
+    for (int i = 0; i < C::NS / 2; ++i) mbar_init(smem_u32(s_empty + i), 1);
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(acc_empty), 4);
     mbar_init(smem_u32(drain), 1);
@@ -472,29 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ token rows (cp.async)
     // Lane l copies 16-byte chunks l, l + 32, ... of the tile's rows (chunk c
     // of row n lands at n*128 + ((c ^ (n & 7)) * 16): the 128B-swizzled
-    // K-major layout the MMA reads). A stage is signalled kBLag stages after
-    // its copies were issued, once they are complete and made visible to the
-    // tensor core's (async proxy) reads.
+    // K-major layout the MMA reads). Each lane then arms a hardware arrival
+    // on the stage's barrier that fires once its copies have landed, so the
+    // loader never waits for its own copies; the MMA thread, after the
+    // barrier, fences the async proxy before the tensor core reads them.
     const uint16_t* src = reinterpret_cast<const uint16_t*>(p.b_src);
-    uint32_t b_it = 0, signalled = 0;
+    uint32_t b_it = 0;
     bool ok = true;
-    auto signal_oldest = [&](int keep) {
-      // complete all but the newest `keep` groups, then signal the oldest stage
-      switch (keep) {
-        case 7: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(b_full + signalled % NB));
-      ++signalled;
-    };
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int e, mb, r0, nv;
       decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
@@ -502,8 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = lane; n < nv; n += 32) s_trow[n] = GATHER ? (int)__ldg(p.row_map + r0 + n) : r0 + n;
       __syncwarp();
       for (int kb = 0; kb < nka && ok; ++kb) {
-        const int bs = b_it % NB;
-        ok = mbar_wait_warp(smem_u32(b_empty + bs), ((b_it / NB) & 1) ^ 1, abort_flag, p.status);
+        const int bs = b_it % C::NS;
+        ok = mbar_wait_warp(smem_u32(s_empty + (bs >> 1)), ((b_it / C::NS) & 1) ^ 1, abort_flag,
+                            p.status);
         if (!ok) break;
         const uint32_t dst = b_base + bs * C::B_BYTES;
         for (int i = lane; i < nv * 8; i += 32) {
@@ -514,18 +544,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                        "l"(g)
                        : "memory");
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                         smem_u32(b_full + bs))
+                     : "memory");
         ++b_it;
-        if (b_it - signalled == (uint32_t)kBLag) signal_oldest(kBLag - 1);
       }
     }
-    while (signalled < b_it) signal_oldest((int)(b_it - signalled) - 1);
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t a_it = 0, b_it = 0, tcount = 0;
+      uint32_t tcount = 0;
+      uint32_t ss = 0, sph = 0;                       // stage slot and its phase
       bool ok = true;
+      // descriptor of B stage 0 (low word: start address / 16 and the
+      // leading offset; high word: stride offset, version, swizzle)
+      const uint64_t d0 = desc_sw128(b_base);
+      const uint32_t blo0 = (uint32_t)d0, bhi = (uint32_t)(d0 >> 32);
+      const uint32_t a_col0 = tmem + C::ACC_COLS;
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
         int e, mb, r0, nv;
         decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
@@ -537,26 +574,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         for (int kb = 0; kb < nka && ok; ++kb) {
-          const int as = a_it % C::NA;
-          const int bs = b_it % NB;
-          ok = mbar_wait(smem_u32(a_full + as), (a_it / C::NA) & 1, abort_flag, p.status) &&
-               mbar_wait(smem_u32(b_full + bs), (b_it / NB) & 1, abort_flag, p.status);
+          ok = mbar_wait(smem_u32(a_full + ss), sph, abort_flag, p.status) &&
+               mbar_wait(smem_u32(b_full + ss), sph, abort_flag, p.status);
           if (!ok) break;
+          // the token rows were written by cp.async (generic proxy); the
+          // tensor core reads them through the async proxy
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           tc_fence_after();
-          const uint32_t bsmem = b_base + bs * C::B_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < KA / 16; ++kk) {
-            const uint64_t bdesc = desc_sw128(bsmem + kk * 32);
-#pragma unroll
-            for (int mat = 0; mat < C::NMAT; ++mat) {
-              const uint32_t acol = C::ACC_COLS + as * C::A_COLS + mat * (KA / 2) + kk * 8;
-              mma_ts(tmem + mat * BN, tmem + acol, bdesc, idesc, (kb | kk) != 0);
-            }
-          }
-          mma_commit(smem_u32(a_empty + as));
-          mma_commit(smem_u32(b_empty + bs));
-          ++a_it;
-          ++b_it;
+          const uint32_t blo = blo0 + ss * (uint32_t)(C::B_BYTES >> 4);
+          const uint32_t acol = a_col0 + ss * (uint32_t)C::A_COLS;
+          if (C::NMAT == 2)
+            mma_kblock2(tmem, tmem + BN, acol, acol + KA / 2, blo, bhi, idesc, kb == 0);
+          else
+            mma_kblock1(tmem, acol, blo, bhi, idesc, kb == 0);
+          // K is a multiple of 128, so a tile has an even number of
+          // k-blocks and the pairs never straddle tiles
+          if (ss & 1) mma_commit(smem_u32(s_empty + (ss >> 1)));
+          if (++ss == (uint32_t)C::NS) { ss = 0; sph ^= 1; }
         }
         if (!ok) break;
         mma_commit(smem_u32(acc_full));
@@ -674,8 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) dequant_word(ws[i], s2, b2, vals + 4 * i);
             const uint32_t stage = a_it + j;
-            const int as = stage % C::NA;
-            ok = mbar_wait_warp(smem_u32(a_empty + as), ((stage / C::NA) & 1) ^ 1, abort_flag,
+            const int as = stage % C::NS;
+            ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / C::NS) & 1) ^ 1, abort_flag,
                                 p.status);
             if (!ok) break;
             tc_fence_after();
@@ -710,8 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
           const uint32_t stage = a_it;
-          const int as = stage % C::NA;
-          ok = mbar_wait_warp(smem_u32(a_empty + as), ((stage / C::NA) & 1) ^ 1, abort_flag,
+          const int as = stage % C::NS;
+          ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / C::NS) & 1) ^ 1, abort_flag,
                               p.status);
           if (!ok) break;
           tc_fence_after();
@@ -906,7 +940,7 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
                                     int d, int E, float* logits, int* status, cudaStream_t s) {
   using namespace tc;
   // few tokens: the weight-streaming kernel is faster than a 128-row tile
-  if (T < 256 || d % 64 != 0) return cudaErrorNotSupported;
+  if (T < 256 || d % 128 != 0) return cudaErrorNotSupported;
   CUtensorMap ta;
   if (!weight_map(&ta, MOE_W_BF16, w_router, E, d)) return cudaErrorInvalidValue;
   Params p{};
