@@ -196,7 +196,7 @@ def run_ours(args, rank, world, local_rank):
             (L.row_map, T * k, torch.uint32), (L.counts, wl.E, torch.int32),
             (L.row_off, wl.E + 1, torch.int32), (L.tile_off, wl.E + 1, torch.int32))), L.BM)
     h = ws[L.h:L.h + T * k * wl.F * 2].view(torch.float16).view(T * k, wl.F)
-    x16 = ws[L.x16:L.x16 + T * wl.d * 2]
+    x16 = ws[L.x16:L.total]
     regime = L.regime
     exs = moe.experts_struct(ex)
 

@@ -58,8 +58,11 @@
  *   MOE_REGIME_GEMV: weight-streaming kernels, every selected expert's bytes
  *     read once per step, for few tokens per expert (decode);
  *   MOE_REGIME_TC: tensor-core grouped GEMM (tcgen05 / TMEM, TMA-staged
- *     operands) for many tokens per expert (prefill); bf16 activations only;
- *   MOE_REGIME_AUTO: GEMV when T*k <= 8*E, else TC (bf16) or GEMV (f32).
+ *     operands) for many tokens per expert (prefill); bf16 activations,
+ *     bf16 or q4 weights, d a multiple of 256, F of 128 (q4: of 256);
+ *     other shapes return MOE_ERR_UNSUPPORTED;
+ *   MOE_REGIME_AUTO: GEMV when T*k <= 8*E or the shape is not one the
+ *     tensor-core kernels tile, else TC (bf16) or GEMV (f32).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -186,14 +189,15 @@ moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, i
  *   h        (device, out) [T*k][F]: fp16 for bf16 activations, fp32 for fp32:
  *            h[i][f] = silu(g) * u, g = x[row_map[i]] . w_gu[e][f],
  *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
- *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, d, dt) bytes
- *            (x converted to fp16); required for bf16 activations, may be
- *            NULL for fp32
+ *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, k, d, dt)
+ *            bytes (the token rows in fp16: x converted, or, in the
+ *            tensor-core regime, gathered into sorted row order); required
+ *            for bf16 activations, may be NULL for fp32
  * fp32 accumulation; h rounded once. The tensor-core regime multiplies fp16
  * operands (x converted exactly from bf16 when |x| < 65520, weights
  * dequantised to fp16); values outside fp16 range are reported as
  * MOE_ERR_RANGE in the device status. */
-size_t moe_grouped_swiglu_workspace(int T, int d, moe_dtype dt);
+size_t moe_grouped_swiglu_workspace(int T, int k, int d, moe_dtype dt);
 moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
                               const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
                               const moe_experts* experts, void* h, void* ws, size_t ws_bytes,

@@ -63,7 +63,7 @@ def _load():
     L.moe_sort_rows_workspace.argtypes = [I, I, I]
     L.moe_sort_rows_workspace.restype = S
     L.moe_sort_rows.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, S, P]
-    L.moe_grouped_swiglu_workspace.argtypes = [I, I, I]
+    L.moe_grouped_swiglu_workspace.argtypes = [I, I, I, I]
     L.moe_grouped_swiglu_workspace.restype = S
     L.moe_grouped_swiglu.argtypes = [P, I, P, P, P, I, I, I, ctypes.POINTER(Experts), P, P, S, I,
                                      P]
@@ -197,7 +197,7 @@ def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, ws=Non
     ex = experts_struct(experts)
     hdt = torch.float16 if x.dtype == torch.bfloat16 else torch.float32
     h = torch.empty(T * k, experts.F, dtype=hdt, device=x.device)
-    nws = lib.moe_grouped_swiglu_workspace(T, experts.d, _dt(x))
+    nws = lib.moe_grouped_swiglu_workspace(T, k, experts.d, _dt(x))
     if ws is None:
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=x.device)
     _check(lib.moe_grouped_swiglu(_ptr(x), _dt(x), _ptr(tables.row_map), _ptr(tables.row_off),

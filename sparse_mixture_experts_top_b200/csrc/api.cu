@@ -72,8 +72,8 @@ static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16; }
 static int resolve_regime(int regime, long long R, int E, int dt, int d = 128, int F = 128,
                           int fmt = MOE_W_Q4G64) {
   if (regime == MOE_REGIME_GEMV || regime == MOE_REGIME_TC) return regime;
-  // the tensor-core kernels tile d and F by 128 and take bf16 or q4 weights
-  if (d % 128 || F % 128 || fmt == MOE_W_F32) return MOE_REGIME_GEMV;
+  // the tensor-core kernels tile d by 256 and F by 128 and take bf16 or q4 weights
+  if (!tc_shape_supported(d, F, fmt)) return MOE_REGIME_GEMV;
   if (dt != MOE_BF16) return MOE_REGIME_GEMV;
   return (R <= 8LL * E) ? MOE_REGIME_GEMV : MOE_REGIME_TC;
 }
@@ -187,9 +187,11 @@ moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, u
                                    row_off, tile_off, ws, (cudaStream_t)stream));
 }
 
-size_t moe_grouped_swiglu_workspace(int T, int d, moe_dtype dt) {
-  if (T < 0 || d <= 0) return 0;
-  return dt == MOE_BF16 ? up256((size_t)T * d * 2) : 0;
+size_t moe_grouped_swiglu_workspace(int T, int k, int d, moe_dtype dt) {
+  if (T < 0 || k < 1 || d <= 0) return 0;
+  // fp16 token rows: T rows (weight-streaming regime) or the T*k rows in
+  // sorted order (tensor-core regime)
+  return dt == MOE_BF16 ? up256((size_t)T * k * d * 2) : 0;
 }
 
 moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, int BM,
@@ -224,14 +226,15 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
     if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!tc_shape_supported(experts->d, experts->F, experts->fmt)) return MOE_ERR_UNSUPPORTED;
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, experts->d, dt))
+    if (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, k, experts->d, dt))
       return MOE_ERR_WORKSPACE;
     return launched(launch_swiglu_tc(x, T, row_map, row_off, tile_off, (int)R, *experts, h, ws,
                                      status_ptr(), s));
   }
   if (dt == MOE_BF16 &&
-      (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, experts->d, dt)))
+      (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, k, experts->d, dt)))
     return MOE_ERR_WORKSPACE;
   return launched(swiglu_gemv(x, dt, T, row_map, row_off, tile_off, BM, (int)R, *experts, h, ws,
                               status_ptr(), s));
@@ -255,6 +258,7 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
     if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!tc_shape_supported(experts->d, experts->F, experts->fmt)) return MOE_ERR_UNSUPPORTED;
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
     return launched(launch_down_tc(h, row_off, tile_off, (int)R, *experts, ys, status_ptr(), s));
   }
@@ -303,10 +307,12 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
   L.h = take((size_t)R * F * a);      // fp16 (bf16 activations) or fp32
   L.ys = take((size_t)R * d * 4);
-  L.x16 = take(dt == MOE_BF16 ? (size_t)T * d * 2 : 0);
-  L.total = off;
   L.regime = resolve_regime(regime, R, E, dt, d, F);
   L.BM = block_m_for(L.regime, R, E);
+  // fp16 token rows: x converted (weight-streaming) or gathered in sorted
+  // row order (tensor cores)
+  L.x16 = take(dt != MOE_BF16 ? 0 : (size_t)(L.regime == MOE_REGIME_TC ? R : T) * d * 2);
+  L.total = off;
   *out = L;
   return MOE_OK;
 }
@@ -335,6 +341,13 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
   if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   if (L.regime == MOE_REGIME_TC && dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  // the layout assumes q4 weights; other formats the tensor-core kernels do
+  // not tile take the weight-streaming kernels (which accept any BM)
+  int regime_run = L.regime;
+  if (regime_run == MOE_REGIME_TC && !tc_shape_supported(d, F, experts->fmt)) {
+    if (regime == MOE_REGIME_TC) return MOE_ERR_UNSUPPORTED;
+    regime_run = MOE_REGIME_GEMV;
+  }
 
   char* base = static_cast<char*>(ws);
   float* logits = (float*)(base + L.logits);
@@ -363,7 +376,7 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
   if ((e = launch_sort_rows(idx, T, k, E, L.BM, order, inv, rmap, counts, roff, toff, sws, s)) !=
       cudaSuccess)
     return launched(e);
-  if (L.regime == MOE_REGIME_TC) {
+  if (regime_run == MOE_REGIME_TC) {
     if ((e = launch_swiglu_tc(x, T, rmap, roff, toff, (int)R, *experts, h, x16, stp, s)) !=
         cudaSuccess)
       return launched(e);

@@ -61,10 +61,13 @@ cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cu
 // Tensor-core grouped kernels (bf16 activations; bf16 or q4 weights).
 // BM must equal tc_block_m().
 int tc_block_m();
-// x16: T*d fp16 scratch that receives x converted from bf16
+// whether the tensor-core kernels tile these expert shapes
+bool tc_shape_supported(int d, int F, int fmt);
+// xs16: R*d fp16 scratch that receives the token rows of the R sorted rows,
+// gathered through row_map and converted from bf16
 cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
-                             void* x16, int* status, cudaStream_t s);
+                             void* xs16, int* status, cudaStream_t s);
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
                            const moe_experts& ex, void* ys, int* status, cudaStream_t s);
 

@@ -2,30 +2,33 @@
 //
 // DS4Server issue #112, "Kernel contract": work is split into tiles that own
 // sorted rows of one expert, found from per-expert tile and row prefix tables
-// by binary search; gate|up reads token rows in place through row_map and
-// writes silu(gate) * up; the down projection reads rows already sorted by
-// expert. mlx-lm PR #2044, "What": each expert's weights are read and
-// dequantised once per tile instead of once per (token, slot).
+// by binary search; gate|up takes the token rows of each sorted row (gathered
+// through row_map) and writes silu(gate) * up; the down projection reads rows
+// already sorted by expert. mlx-lm PR #2044, "What": each expert's weights are
+// read and dequantised once per tile instead of once per (token, slot).
 //
-// B200 design (one persistent CTA per SM, 16 warps):
-//   * swap-AB: the MMA's M = 128 weight rows (output features), N = the
-//     tile's token rows (<= 128, rounded up to 16 per tile at run time), so
-//     a tile with few rows costs proportionally few tensor cycles;
-//   * warp 0: TMA loads of the raw weight tile (packed q4 words or bf16,
-//     128-byte rows) into a shared-memory ring;
-//   * warp 2: cp.async copies of the tile's token rows -- through row_map
-//     (gather) or contiguous -- into a 128B-swizzled K-major ring (per-row
-//     TMA loads cost ~30 ns of issue each, which starved the tensor core);
-//   * warps 8..15 (dequant): each thread owns one weight row (one TMEM lane):
-//     reads its packed words from shared memory, dequantises w = s*q + b to
-//     bf16 pairs and writes them into TMEM with tcgen05.st, where the MMA
-//     takes them as its A operand -- the dequantised tile never goes back
-//     through shared memory;
-//   * warp 1 (MMA): one thread issues tcgen05.mma (A from TMEM, B from
-//     shared memory) into fp32 accumulators in TMEM; gate and up accumulate
-//     side by side so one token tile feeds both;
-//   * warps 4..7 (epilogue): tcgen05.ld of the accumulators, SwiGLU to fp16
-//     (gate|up) or an fp32 store (down projection; router logits + bias).
+// B200 design (one persistent CTA per SM, 16 warps). A unit of work is one
+// token tile x two 128-row weight matrices: gate and up rows of the same
+// features (gate|up), or two adjacent 128-row blocks (down, router).
+//   * swap-AB: the MMA's M = 128 weight rows, N = the tile's token rows
+//     (<= 128, rounded up to 16 per tile), so few rows cost few tensor cycles;
+//   * warp 0: TMA of the raw weight tiles (q4 words or bf16, 128-byte rows)
+//     of both matrices, and cp.async of the q4 scales and biases;
+//   * warp 2: one TMA per k-block of the tile's token rows, from a row-sorted
+//     16-bit copy (x gathered through row_map, or h, or x for the router),
+//     with one tensor map per tile height (16, 32, ..., 128 rows);
+//   * warps 8..15 (dequant, 4 per matrix): each thread owns one weight row
+//     (one TMEM lane), dequantises w = s*q + b to fp16 and writes it into
+//     TMEM with tcgen05.st, where the MMA takes it as its A operand -- the
+//     dequantised tile never goes back through shared memory;
+//   * warps 1 and 3 (MMA): one thread each issues the tcgen05.mma of one
+//     matrix (A from TMEM, B from shared memory) into its own fp32
+//     accumulator. Two issuers, because at small N one thread cannot issue
+//     MMAs as fast as the tensor core completes them;
+//   * warps 4..7 (epilogue): tcgen05.ld of both accumulators, SwiGLU to fp16
+//     (gate|up) or fp32 stores (down; router logits + bias). Tiles of at most
+//     64 rows alternate between two accumulator buffers, so the epilogue of
+//     one overlaps the MMAs of the next.
 // The expert GEMMs multiply fp16 operands (x converted once from bf16,
 // weights dequantised to fp16, h stored in fp16): 11-bit operands keep the
 // rounding of the dequantised weights and of h 8x below bf16's; values
@@ -46,9 +49,12 @@
 namespace moe {
 namespace tc {
 
-constexpr int BN = 128;        // token rows per tile (the sort tables' BM)
-constexpr int BMW = 128;       // weight rows per tile (MMA M)
-constexpr int KA = 64;         // K elements per A stage (one q4 group)
+constexpr int BN = 128;        // token rows per tile (the sort tables' BM; MMA N at most)
+constexpr int BMW = 128;       // weight rows per matrix (MMA M)
+constexpr int KA = 64;         // K elements per k-block (one q4 group)
+constexpr int NS = 4;          // k-block stages of A in TMEM, released in pairs
+constexpr int NB = 6;          // token-row (B) stages in shared memory
+constexpr int NBOX = BN / 16;  // token-row tensor maps: tile heights 16, 32, ..., 128
 constexpr int kMaxE = 1024;    // tile / row tables cached in shared memory
 constexpr int kThreads = 512;
 constexpr int kEpiWarp0 = 4;
@@ -57,52 +63,41 @@ constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at the B200's clocks
 
 enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };   // fp32 store adds p.bias when set
 
-template <int FMT, int EPI>
+template <int FMT>
 struct Cfg {
-  static constexpr int NMAT = EPI == EPI_SWIGLU ? 2 : 1;
   static constexpr bool Q4 = FMT == MOE_W_Q4G64;
   static constexpr int KR = Q4 ? 256 : 64;                  // K elements per raw stage
-  static constexpr int RAW_ROW = 128;                       // bytes per weight row per raw stage
-  static constexpr int RAW_MAT = BMW * RAW_ROW;
-  static constexpr int RAW_BYTES = NMAT * RAW_MAT;
+  static constexpr int RAW_MAT = BMW * 128;                 // one matrix: 128 rows x 128 bytes
+  static constexpr int RAW_BYTES = 2 * RAW_MAT;
   static constexpr int A_PER_RAW = KR / KA;                 // 4 (q4) or 1 (bf16)
-#ifndef MOE_TC_RAW_KB
-#define MOE_TC_RAW_KB 96
-#endif
-  static constexpr int NR_FIT = (MOE_TC_RAW_KB * 1024) / RAW_BYTES;
-  static constexpr int NR = NR_FIT > 8 ? 8 : NR_FIT;
-  static constexpr int ACC_COLS = NMAT * BN;
-  static constexpr int A_COLS = NMAT * (KA / 2);            // 32-bit TMEM columns per A stage
-  // k-block stages: stage s = A slot s (TMEM) + B slot s (shared memory).
-  // The MMA releases stages in pairs (one commit per two k-blocks: each
-  // tcgen05.commit costs the tensor pipe ~200 cycles), so NS is even.
-  static constexpr int NS = NMAT == 2 ? 4 : 6;
+  static constexpr int NR = 3;                              // raw stages
+  static constexpr int ACC_COLS = 2 * BN;                   // two accumulators of up to 128 columns
+  static constexpr int A_COLS = 2 * (KA / 2);               // TMEM columns of one A stage (2 matrices)
   static constexpr int B_BYTES = BN * 128;
-  // warps that write one A stage: NMAT == 2: 4 gate + 4 up warps;
-  // NMAT == 1: q4 -- the 4 warps of one half of the raw row; bf16 -- all 8
-  // (half the columns each)
-  static constexpr int A_ARRIVALS = NMAT == 2 ? 8 : (Q4 ? 4 : 8);
-  // q4 scales and biases of a raw stage: [NMAT][128 rows][4 groups] bf16 each
-  static constexpr int SCL_BYTES = Q4 ? NMAT * BMW * 4 * 2 * 2 : 0;
-  static constexpr int TABLES = 2 * (kMaxE + 1) * 4 + BN * 4;  // tile/row tables, tile rows
-  static_assert(NS % 2 == 0 && ACC_COLS + NS * A_COLS <= 512, "stages must fit TMEM in pairs");
-  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NS * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
+  // q4 scales then biases of a raw stage: [2 arrays][2 matrices][128 rows][4 groups] bf16
+  static constexpr int SCL_BYTES = Q4 ? 2 * 2 * BMW * 4 * 2 : 0;
+  static constexpr int TABLES = 2 * (kMaxE + 1) * 4;
+  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
+  static_assert(ACC_COLS + NS * A_COLS <= 512, "accumulators and A stages must fit TMEM");
+  static_assert(NS % 2 == 0, "A stages are released in pairs");
+  static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 struct Params {
+  CUtensorMap tmB[NBOX];     // token rows [rows][K] 16-bit; map i: box 64 x 16(i+1), 128B swizzle
   const int32_t* row_off;
   const int32_t* tile_off;
   int E;               // groups (experts); 1 for the router
   int n_rows;          // router: tokens T
-  int n_mb;            // weight-row blocks per group
+  int n_units;         // units (pairs of weight matrices) per token tile
+  int unit_rows;       // weight rows from one unit to the next
+  int mat_off;         // row offset of matrix 1 from matrix 0 inside a unit
   int K;               // reduction length
   int rows_per_group;  // weight rows per expert in the stacked tensor
-  int up_off;          // row offset of the up matrix inside an expert
   int G;               // q4 groups per weight row (K / 64)
+  long long w_rows;    // rows of the stacked weight tensor
   const uint16_t* scales;
   const uint16_t* biases;
-  const uint32_t* row_map;  // token of each sorted row (gather), or null
-  const void* b_src;        // token rows: [rows][K] 16-bit (x16, h or x)
   void* out;
   int out_ld;          // elements per output row
   int m_limit;         // valid weight rows per group (router: E)
@@ -180,48 +175,14 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate)
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
-      "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// The MMAs of one 64-deep k-block (4 K-steps of 16) for one or two
-// accumulators, in a single statement: A columns a (+8 per K-step), B
-// descriptor low word blo (+2 per K-step, i.e. +32 bytes inside the 128-byte
-// swizzle atom), accumulate unless `first`. Keeping the issue path to a few
-// instructions per MMA matters: the tensor core takes a K=16 step of an
-// M=128 tile in ~80 cycles, and the single issuing thread must keep up.
-__device__ __forceinline__ void mma_kblock2(uint32_t d0, uint32_t d1, uint32_t a0, uint32_t a1,
-                                            uint32_t blo, uint32_t bhi, uint32_t idesc,
-                                            uint32_t first) {
-  asm volatile(
-      "{\n\t.reg .pred pf, pt;\n\t.reg .b64 b0, b1, b2, b3;\n\t"
-      "setp.eq.b32 pf, %7, 0;\n\t"
-      "setp.ne.b32 pt, %6, 0;\n\t"
-      "mov.b64 b0, {%4, %5};\n\t"
-      "add.u32 %4, %4, 2;\n\tmov.b64 b1, {%4, %5};\n\t"
-      "add.u32 %4, %4, 2;\n\tmov.b64 b2, {%4, %5};\n\t"
-      "add.u32 %4, %4, 2;\n\tmov.b64 b3, {%4, %5};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b0, %6, pf;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b0, %6, pf;\n\t"
-      "add.u32 %2, %2, 8;\n\tadd.u32 %3, %3, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b1, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b1, %6, pt;\n\t"
-      "add.u32 %2, %2, 8;\n\tadd.u32 %3, %3, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b2, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b2, %6, pt;\n\t"
-      "add.u32 %2, %2, 8;\n\tadd.u32 %3, %3, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], b3, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%3], b3, %6, pt;\n\t}\n"
-      : "+r"(d0), "+r"(d1), "+r"(a0), "+r"(a1), "+r"(blo), "+r"(bhi)
-      : "r"(idesc), "r"(first)
-      : "memory");
-}
+// The four MMAs of one 64-deep k-block (K-steps of 16) into one accumulator,
+// in a single statement: D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (fp16 or
+// bf16 operands, fp32 accumulation). A columns advance 8 per K-step, the B
+// descriptor's start address 32 bytes (+2 in 16-byte units) inside the
+// 128-byte swizzle atom; accumulate unless `first`. The issuing thread is
+// on the critical path: at small N a tcgen05.mma from one thread is accepted
+// only every ~50-80 cycles and nothing queues behind it, so every other
+// instruction it executes adds to the tile's time.
 __device__ __forceinline__ void mma_kblock1(uint32_t d0, uint32_t a0, uint32_t blo, uint32_t bhi,
                                             uint32_t idesc, uint32_t first) {
   asm volatile(
@@ -350,13 +311,13 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 
 // ------------------------------------------------------------------ tiles
 
-// Tile tau -> (expert e, first sorted row r0, valid rows nv), with the
-// prefix tables read from their shared-memory copies.
+// Work item u -> (unit within the tile, first sorted row r0, valid rows nv,
+// expert e), with the prefix tables read from their shared-memory copies.
 template <bool ROUTER>
-__device__ __forceinline__ void decode_tile(const Params& p, const int* s_toff, const int* s_roff,
-                                            int u, int& e, int& mb, int& r0, int& nv) {
-  const int tau = u / p.n_mb;
-  mb = u - tau * p.n_mb;
+__device__ __forceinline__ void decode_unit(const Params& p, const int* s_toff, const int* s_roff,
+                                            int u, int& unit, int& r0, int& nv, int& e) {
+  const int tau = u / p.n_units;
+  unit = u - tau * p.n_units;
   if (ROUTER) {
     e = 0;
     r0 = tau * BN;
@@ -375,39 +336,39 @@ __device__ __forceinline__ void decode_tile(const Params& p, const int* s_toff, 
 
 template <bool ROUTER>
 __device__ __forceinline__ int total_units(const Params& p, const int* s_toff) {
-  if (ROUTER) return ((p.n_rows + BN - 1) / BN) * p.n_mb;
-  return s_toff[p.E] * p.n_mb;
+  if (ROUTER) return ((p.n_rows + BN - 1) / BN) * p.n_units;
+  return s_toff[p.E] * p.n_units;
 }
+
+// MMA N of a tile: its rows rounded up to 16
+__device__ __forceinline__ int mma_n(int nv) { return max(16, (nv + 15) & ~15); }
 
 // ------------------------------------------------------------------ kernel
 
-template <int FMT, int EPI, bool GATHER, bool ROUTER>
+template <int FMT, int EPI, bool ROUTER>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA) {
-  pdl_wait();
-  pdl_launch();
-  using C = Cfg<FMT, EPI>;
+  using C = Cfg<FMT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const uint32_t raw_base = smem_u32(smem);
   const uint32_t b_base = raw_base + C::NR * C::RAW_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NR * C::RAW_BYTES + C::NS * C::B_BYTES);
-  uint64_t* raw_full = bars;
-  uint64_t* raw_empty = raw_full + C::NR;
-  uint64_t* a_full = raw_empty + C::NR;
-  uint64_t* b_full = a_full + C::NS;
-  uint64_t* s_empty = b_full + C::NS;    // [NS / 2]: stage pair released by the MMA
-  uint64_t* acc_full = s_empty + C::NS / 2;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint8_t* bar_area = smem + C::NR * C::RAW_BYTES + NB * C::B_BYTES;
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(bar_area);   // [NR]
+  uint64_t* raw_empty = raw_full + C::NR;                        // [NR]
+  uint64_t* a_full = raw_empty + C::NR;                          // [2 matrices][NS]
+  uint64_t* b_full = a_full + 2 * NS;                            // [NB]
+  uint64_t* s_empty = b_full + NB;                               // [NS / 2] stage pairs
+  uint64_t* acc_full = s_empty + NS / 2;                         // [2] accumulator buffers
+  uint64_t* acc_empty = acc_full + 2;                            // [2]
+  uint64_t* drain = acc_empty + 2;                               // [2] one per issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_toff = reinterpret_cast<int*>(smem + C::NR * C::RAW_BYTES + C::NS * C::B_BYTES + 1024);
+  int* s_toff = reinterpret_cast<int*>(bar_area + 1024);
   int* s_roff = s_toff + kMaxE + 1;
-  int* s_trow = s_roff + kMaxE + 1;     // [BN] source rows of the loader's current tile
-  // q4 scale ring: raw stage rs holds scales [NMAT][128][4] then biases [NMAT][128][4]
-  const uint32_t scl_base = smem_u32(s_trow + BN);
+  // q4 scale ring: raw stage rs holds scales [2][128][4] then biases [2][128][4]
+  const uint32_t scl_base = smem_u32(s_roff + kMaxE + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -416,16 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < C::NR; ++i) {
       // q4: the TMA arrive + the 32 lanes' cp.async arrivals for the scales
       mbar_init(smem_u32(raw_full + i), C::Q4 ? 33 : 1);
-      mbar_init(smem_u32(raw_empty + i), 8);
+      mbar_init(smem_u32(raw_empty + i), 8);   // the 8 dequant warps
     }
-    for (int i = 0; i < C::NS; ++i) {
-      mbar_init(smem_u32(a_full + i), C::A_ARRIVALS);
-      mbar_init(smem_u32(b_full + i), 32);  // the loader's 32 lanes, as their copies land
+    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), 4);   // a matrix's 4 warps
+    for (int i = 0; i < NB; ++i) mbar_init(smem_u32(b_full + i), 1);
+    for (int i = 0; i < NS / 2; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(acc_full + i), 2);    // both issuers
+      mbar_init(smem_u32(acc_empty + i), 4);   // the 4 epilogue warps
+      mbar_init(smem_u32(drain + i), 1);
     }
-    for (int i = 0; i < C::NS / 2; ++i) mbar_init(smem_u32(s_empty + i), 1);
-    mbar_init(smem_u32(acc_full), 1);
-    mbar_init(smem_u32(acc_empty), 4);
-    mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -452,17 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   const int total = total_units<ROUTER>(p, s_toff);
-  const int nkr = p.K / C::KR;           // raw stages per tile
-  const int nka = p.K / KA;              // A stages per tile
+  const int nkr = p.K / C::KR;           // raw stages per unit
+  const int nka = p.K / KA;              // k-blocks per unit (even: K % 128 == 0)
 
   if (warp == 0) {
     // ------------------------------------------------------------ raw weights (TMA)
     uint32_t raw_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
-      const int wrow = (ROUTER ? 0 : e * p.rows_per_group) + mb * BMW;
+      int unit, r0, nv, e;
+      decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+      const long long wrow0 = (ROUTER ? 0LL : (long long)e * p.rows_per_group) +
+                              (long long)unit * p.unit_rows;
+      const long long wrow1 = wrow0 + p.mat_off;
       for (int kr = 0; kr < nkr && ok; ++kr) {
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_empty + rs), ((raw_it / C::NR) & 1) ^ 1, abort_flag,
@@ -471,14 +434,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (C::Q4) {
           // the stage's scales and biases (4 groups of each weight row), 8
           // bytes per row and array, copied by the 32 lanes; each lane's
-          // arrival fires when its copies have landed
+          // arrival fires when its copies have landed. Rows past the end of
+          // the stacked tensor (never stored) read the last row instead.
           const uint32_t sdst = scl_base + rs * C::SCL_BYTES;
 #pragma unroll
-          for (int mat = 0; mat < C::NMAT; ++mat)
+          for (int mat = 0; mat < 2; ++mat)
 #pragma unroll
             for (int j = 0; j < BMW / 32; ++j) {
               const int m = lane + 32 * j;
-              const size_t grow = (size_t)wrow + (mat ? p.up_off : 0) + m;
+              long long grow = (mat ? wrow1 : wrow0) + m;
+              if (grow >= p.w_rows) grow = p.w_rows - 1;
               const uint32_t o = (uint32_t)((mat * BMW + m) * 8);
               asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sdst + o),
                            "l"(p.scales + grow * p.G + 4 * kr)
@@ -493,12 +458,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                        : "memory");
         }
         if (lane == 0) {
+          // rows past the end of the tensor are filled with zeros by the TMA
           const uint32_t dst = raw_base + rs * C::RAW_BYTES;
           const uint32_t bar = smem_u32(raw_full + rs);
           const int x = kr * (C::Q4 ? C::KR / 8 : C::KR);
           mbar_arrive_tx(bar, C::RAW_BYTES);
-          tma_load_2d(dst, &tmA, x, wrow, bar);
-          if (C::NMAT == 2) tma_load_2d(dst + C::RAW_MAT, &tmA, x, wrow + p.up_off, bar);
+          tma_load_2d(dst, &tmA, x, (int)wrow0, bar);
+          tma_load_2d(dst + C::RAW_MAT, &tmA, x, (int)wrow1, bar);
         }
         ++raw_it;
       }
@@ -514,249 +480,233 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ------------------------------------------------------------ token rows (cp.async)
-    // Lane l copies 16-byte chunks l, l + 32, ... of the tile's rows (chunk c
-    // of row n lands at n*128 + ((c ^ (n & 7)) * 16): the 128B-swizzled
-    // K-major layout the MMA reads). Each lane then arms a hardware arrival
-    // on the stage's barrier that fires once its copies have landed, so the
-    // loader never waits for its own copies; the MMA thread, after the
-    // barrier, fences the async proxy before the tensor core reads them.
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(p.b_src);
-    uint32_t b_it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
-      __syncwarp();
-      for (int n = lane; n < nv; n += 32) s_trow[n] = GATHER ? (int)__ldg(p.row_map + r0 + n) : r0 + n;
-      __syncwarp();
-      for (int kb = 0; kb < nka && ok; ++kb) {
-        const int bs = b_it % C::NS;
-        ok = mbar_wait_warp(smem_u32(s_empty + (bs >> 1)), ((b_it / C::NS) & 1) ^ 1, abort_flag,
-                            p.status);
-        if (!ok) break;
-        const uint32_t dst = b_base + bs * C::B_BYTES;
-        for (int i = lane; i < nv * 8; i += 32) {
-          const int n = i >> 3, c = i & 7;
-          const uint16_t* g = src + (size_t)s_trow[n] * p.K + kb * KA + c * 8;
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                           dst + n * 128 + ((c ^ (n & 7)) << 4)),
-                       "l"(g)
-                       : "memory");
+    // ------------------------------------------------------------ token rows (TMA)
+    // One copy per k-block: rows r0 .. r0 + n - 1 (n = the tile's MMA N) of
+    // the row-sorted 16-bit operand, 64 elements (128 bytes) each, landing in
+    // the 128B-swizzled K-major layout the MMA reads. Rows past the tile
+    // belong to the next tile (their columns are never stored) or lie past
+    // the end (zero fill). B stage j is reused by k-block j + NB once the A
+    // stage pair that holds k-block j has been released by both issuers.
+    if (lane == 0) {
+      uint32_t j = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        int unit, r0, nv, e;
+        decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+        const int n = mma_n(nv);
+        const CUtensorMap* tm = &p.tmB[n / 16 - 1];
+        for (int kb = 0; kb < nka && ok; ++kb) {
+          const int bs = j % NB;
+          if (j >= (uint32_t)NB) {
+            const uint32_t jj = j - NB;
+            ok = mbar_wait(smem_u32(s_empty + ((jj % NS) >> 1)), (jj / NS) & 1, abort_flag,
+                           p.status);
+            if (!ok) break;
+          }
+          const uint32_t bar = smem_u32(b_full + bs);
+          mbar_arrive_tx(bar, (uint32_t)n * 128u);
+          tma_load_2d(b_base + bs * C::B_BYTES, tm, kb * KA, r0, bar);
+          ++j;
         }
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                         smem_u32(b_full + bs))
-                     : "memory");
-        ++b_it;
+      }
+      for (uint32_t i = 0; i < (uint32_t)NB && i < j; ++i) {
+        const uint32_t last = j - 1 - i;
+        mbar_wait(smem_u32(b_full + last % NB), (last / NB) & 1, abort_flag, p.status, false);
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 1 issues matrix 0, warp 3 matrix 1, each into its own accumulator
     if (lane == 0) {
-      uint32_t tcount = 0;
-      uint32_t ss = 0, sph = 0;                       // stage slot and its phase
+      const int q = warp >> 1;
+      uint32_t ss = 0, sph = 0, bs = 0, bph = 0;      // A and B stage slots and phases
+      uint32_t nb = 0, uses0 = 0, uses1 = 0;          // accumulator buffers
       bool ok = true;
       // descriptor of B stage 0 (low word: start address / 16 and the
       // leading offset; high word: stride offset, version, swizzle)
       const uint64_t d0 = desc_sw128(b_base);
       const uint32_t blo0 = (uint32_t)d0, bhi = (uint32_t)(d0 >> 32);
-      const uint32_t a_col0 = tmem + C::ACC_COLS;
+      const uint32_t a_col0 = tmem + C::ACC_COLS + q * (KA / 2);
+      const uint32_t afull0 = smem_u32(a_full + q * NS);
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        int e, mb, r0, nv;
-        decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
-        const int n_mma = max(16, (nv + 15) & ~15);
-        const uint32_t idesc = idesc_mma(n_mma, !ROUTER);
-        if (tcount > 0) {
-          ok = mbar_wait(smem_u32(acc_empty), (tcount - 1) & 1, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-        }
+        int unit, r0, nv, e;
+        decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+        const int n = mma_n(nv);
+        const uint32_t idesc = idesc_mma(n, !ROUTER);
+        // tiles of <= 64 rows alternate between the two 128-column buffers
+        // (matrix q at +64q); larger ones take both (matrix q at +128q)
+        const bool small = n <= 64;
+        const uint32_t b = small ? nb : 0u;
+        const bool use0 = !small || b == 0, use1 = !small || b == 1;
+        // the epilogue has drained the buffers' previous tiles
+        if (use0 && uses0 > 0)
+          ok = mbar_wait(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status);
+        if (ok && use1 && uses1 > 0)
+          ok = mbar_wait(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t dcol = tmem + (small ? b * 128u + q * 64u : q * 128u);
         for (int kb = 0; kb < nka && ok; ++kb) {
-          ok = mbar_wait(smem_u32(a_full + ss), sph, abort_flag, p.status) &&
-               mbar_wait(smem_u32(b_full + ss), sph, abort_flag, p.status);
+          ok = mbar_wait(afull0 + ss * 8, sph, abort_flag, p.status) &&
+               mbar_wait(smem_u32(b_full + bs), bph, abort_flag, p.status);
           if (!ok) break;
-          // the token rows were written by cp.async (generic proxy); the
-          // tensor core reads them through the async proxy
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           tc_fence_after();
-          const uint32_t blo = blo0 + ss * (uint32_t)(C::B_BYTES >> 4);
-          const uint32_t acol = a_col0 + ss * (uint32_t)C::A_COLS;
-          if (C::NMAT == 2)
-            mma_kblock2(tmem, tmem + BN, acol, acol + KA / 2, blo, bhi, idesc, kb == 0);
-          else
-            mma_kblock1(tmem, acol, blo, bhi, idesc, kb == 0);
-          // K is a multiple of 128, so a tile has an even number of
-          // k-blocks and the pairs never straddle tiles
+          mma_kblock1(dcol, a_col0 + ss * (uint32_t)C::A_COLS,
+                      blo0 + bs * (uint32_t)(C::B_BYTES >> 4), bhi, idesc, kb == 0);
+          // a unit has an even number of k-blocks, so the pairs never
+          // straddle units
           if (ss & 1) mma_commit(smem_u32(s_empty + (ss >> 1)));
-          if (++ss == (uint32_t)C::NS) { ss = 0; sph ^= 1; }
+          if (++ss == (uint32_t)NS) { ss = 0; sph ^= 1; }
+          if (++bs == (uint32_t)NB) { bs = 0; bph ^= 1; }
         }
         if (!ok) break;
-        mma_commit(smem_u32(acc_full));
-        ++tcount;
+        if (use0) { mma_commit(smem_u32(acc_full + 0)); ++uses0; }
+        if (use1) { mma_commit(smem_u32(acc_full + 1)); ++uses1; }
+        if (small) nb ^= 1u;
       }
       // all MMAs issued by this thread complete before TMEM is released
-      mma_commit(smem_u32(drain));
-      mbar_wait(smem_u32(drain), 0, abort_flag, p.status, false);
+      mma_commit(smem_u32(drain + q));
+      mbar_wait(smem_u32(drain + q), 0, abort_flag, p.status, false);
     }
     __syncwarp();
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const int m = q * 32 + lane;                      // weight row of this thread
-    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-    uint32_t tcount = 0;
+    const int qd = warp & 3;
+    const int m = qd * 32 + lane;                     // weight row of this thread
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    uint32_t nb = 0, uses0 = 0, uses1 = 0;
     bool range_ok = true;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
-      if (!mbar_wait_warp(smem_u32(acc_full), tcount & 1, abort_flag, p.status)) break;
+      int unit, r0, nv, e;
+      decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+      const bool small = mma_n(nv) <= 64;
+      const uint32_t b = small ? nb : 0u;
+      const bool use0 = !small || b == 0, use1 = !small || b == 1;
+      if (use0 && !mbar_wait_warp(smem_u32(acc_full + 0), uses0 & 1, abort_flag, p.status)) break;
+      if (use1 && !mbar_wait_warp(smem_u32(acc_full + 1), uses1 & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      const int orow = mb * BMW + m;                  // output feature
-      const bool mok = orow < p.m_limit;
-      for (int c0 = 0; c0 < nv; c0 += 16) {
-        uint32_t g[16];
-        tmem_ld16(tl + c0, g);
-        if (EPI == EPI_SWIGLU) {
-          uint32_t uu[16];
-          tmem_ld16(tl + BN + c0, uu);
+      const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
+      const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
+      if (EPI == EPI_SWIGLU) {
+        const int orow = unit * p.unit_rows + m;          // feature of this thread
+        __half* h = reinterpret_cast<__half*>(p.out);
+        for (int n0 = 0; n0 < nv; n0 += 16) {
+          uint32_t g[16], uu[16];
+          tmem_ld16(c0 + n0, g);
+          tmem_ld16(c1 + n0, uu);
           tmem_ld_wait();
-          __half* h = reinterpret_cast<__half*>(p.out);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
+            const int n = n0 + j;
             if (n < nv) {
               const float v = swiglu(__uint_as_float(g[j]), __uint_as_float(uu[j]));
               range_ok &= fabsf(v) < 65520.f;    // rounds to a finite fp16
               h[(size_t)(r0 + n) * p.out_ld + orow] = __float2half_rn(v);
             }
           }
-        } else {
+        }
+      } else {
+        float* o = reinterpret_cast<float*>(p.out);
+        const int orow0 = unit * p.unit_rows + m;
+        const int orow1 = orow0 + BMW;
+        const bool ok0 = orow0 < p.m_limit, ok1 = orow1 < p.m_limit;
+        const float bv0 = (ok0 && p.bias) ? __ldg(p.bias + orow0) : 0.f;
+        const float bv1 = (ok1 && p.bias) ? __ldg(p.bias + orow1) : 0.f;
+        for (int n0 = 0; n0 < nv; n0 += 16) {
+          uint32_t g0[16], g1[16];
+          tmem_ld16(c0 + n0, g0);
+          tmem_ld16(c1 + n0, g1);
           tmem_ld_wait();
-          float* o = reinterpret_cast<float*>(p.out);
-          const float bv = (mok && p.bias) ? __ldg(p.bias + orow) : 0.f;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < nv && mok) o[(size_t)(r0 + n) * p.out_ld + orow] = __uint_as_float(g[j]) + bv;
+            const int n = n0 + j;
+            if (n < nv) {
+              float* orow = o + (size_t)(r0 + n) * p.out_ld;
+              if (ok0) orow[orow0] = __uint_as_float(g0[j]) + bv0;
+              if (ok1) orow[orow1] = __uint_as_float(g1[j]) + bv1;
+            }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(acc_empty));
-      ++tcount;
+      if (lane == 0) {
+        if (use0) mbar_arrive(smem_u32(acc_empty + 0));
+        if (use1) mbar_arrive(smem_u32(acc_empty + 1));
+      }
+      if (use0) ++uses0;
+      if (use1) ++uses1;
+      if (small) nb ^= 1u;
     }
     if (!__all_sync(0xffffffffu, range_ok) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------ dequant
     const int dw = warp - kDqWarp0;                   // 0..7
-    const int q = warp & 3;                           // TMEM lane quadrant
-    const int m = q * 32 + lane;                      // weight row of this thread
-    const int part = dw >> 2;                         // matrix (NMAT 2) or half (NMAT 1)
-    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const int q = dw >> 2;                            // matrix
+    const int qd = warp & 3;                          // TMEM lane quadrant
+    const int m = qd * 32 + lane;                     // weight row of this thread
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    const uint32_t afull = smem_u32(a_full + q * NS);
     uint32_t raw_it = 0, a_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      int e, mb, r0, nv;
-      decode_tile<ROUTER>(p, s_toff, s_roff, u, e, mb, r0, nv);
       for (int kr = 0; kr < nkr && ok; ++kr) {
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status);
         if (!ok) break;
-        const uint32_t rbase = raw_base + rs * C::RAW_BYTES;
-        uint32_t vals[32];
-        // q4: this row's 4 groups of scales and biases (bf16 pairs)
+        // my row: 128 bytes = 8 chunks of 16 B in the 128-byte swizzle
+        const uint32_t rowa = raw_base + rs * C::RAW_BYTES + q * C::RAW_MAT + m * 128;
+        const int sw = m & 7;
+        uint4 wv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) wv[c] = lds128(rowa + ((c ^ sw) << 4));
         uint32_t sc[2] = {0, 0}, bi[2] = {0, 0};
         if (C::Q4) {
-          const uint32_t so = scl_base + rs * C::SCL_BYTES +
-                              (uint32_t)(((C::NMAT == 2 ? part : 0) * BMW + m) * 8);
+          // this row's 4 groups of scales and biases (bf16 pairs)
+          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * 8);
           asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(sc[0]), "=r"(sc[1]) : "r"(so));
           asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
                        : "=r"(bi[0]), "=r"(bi[1])
                        : "r"(so + C::SCL_BYTES / 2));
-          if (C::NMAT == 1 && part) {   // half 1: groups 2, 3
-            sc[0] = sc[1];
-            bi[0] = bi[1];
-          }
         }
-        if (C::Q4) {
-          // my row: 128 bytes = 8 chunks of 16 B (128-byte swizzle): chunk pair
-          // (2j, 2j+1) holds the 64 elements of A stage j (group 4kr + j).
-          // NMAT 2: this thread converts all 4 A stages of its matrix;
-          // NMAT 1: half `part` converts A stages 2*part and 2*part + 1.
-          const uint32_t rowa = rbase + (C::NMAT == 2 ? part * C::RAW_MAT : 0) + m * 128;
-          const int sw = m & 7;
-          constexpr int nst = C::NMAT == 2 ? 4 : 2;    // A stages this thread converts
-          const int cbase = C::NMAT == 2 ? 0 : 4 * part;  // its first 16-byte chunk
-          uint4 wv[2 * nst];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
 #pragma unroll
-          for (int c = 0; c < 2 * nst; ++c) wv[c] = lds128(rowa + (((cbase + c) ^ sw) << 4));
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
-#pragma unroll
-          for (int st = 0; st < nst; ++st) {
-            if (!ok) break;
-            const int j = (C::NMAT == 2 ? 0 : 2 * part) + st;   // A stage within the raw stage
-            const uint32_t sv = C::NMAT == 2 ? sc[st >> 1] : sc[0];
-            const uint32_t bv = C::NMAT == 2 ? bi[st >> 1] : bi[0];
+        for (int st = 0; st < C::A_PER_RAW; ++st) {
+          uint32_t vals[32];
+          if (C::Q4) {
+            // chunk pair (2st, 2st + 1) holds the 64 elements of group 4kr + st
+            const uint32_t sv = sc[st >> 1], bv = bi[st >> 1];
             const uint32_t s2 = f16x2_from_bf16((st & 1) ? (sv >> 16) : (sv & 0xFFFFu));
             const uint32_t b2 = f16x2_from_bf16((st & 1) ? (bv >> 16) : (bv & 0xFFFFu));
             const uint4 w0 = wv[2 * st], w1 = wv[2 * st + 1];
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) dequant_word(ws[i], s2, b2, vals + 4 * i);
-            const uint32_t stage = a_it + j;
-            const int as = stage % C::NS;
-            ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / C::NS) & 1) ^ 1, abort_flag,
-                                p.status);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t col = C::ACC_COLS + as * C::A_COLS + (C::NMAT == 2 ? part * (KA / 2) : 0);
-            tmem_st16(tl + col, vals);
-            tmem_st16(tl + col + 16, vals + 16);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(a_full + as));
-          }
-        } else {
-          // bf16 weights: my row is 128 bytes = 8 chunks of 16 B, 128-byte swizzle
-          const uint32_t rowa = rbase + (C::NMAT == 2 ? part * C::RAW_MAT : 0) + m * 128;
-          const int sw = m & 7;
-          const int c0 = C::NMAT == 2 ? 0 : 4 * part;
-          const int nc = C::NMAT == 2 ? 8 : 4;
-          for (int c = 0; c < nc; ++c) {
-            const uint4 v = lds128(rowa + (((c0 + c) ^ sw) << 4));
-            if (ROUTER) {
-              vals[4 * c + 0] = v.x;
-              vals[4 * c + 1] = v.y;
-              vals[4 * c + 2] = v.z;
-              vals[4 * c + 3] = v.w;
-            } else {
-              vals[4 * c + 0] = bf16x2_to_f16x2(v.x);
-              vals[4 * c + 1] = bf16x2_to_f16x2(v.y);
-              vals[4 * c + 2] = bf16x2_to_f16x2(v.z);
-              vals[4 * c + 3] = bf16x2_to_f16x2(v.w);
+          } else {
+            // bf16 weights: the 64 elements of the k-block; fp16 operands for
+            // the experts, bf16 kept as is for the router
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t w4[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) vals[4 * c + i] = ROUTER ? w4[i] : bf16x2_to_f16x2(w4[i]);
             }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
-          const uint32_t stage = a_it;
-          const int as = stage % C::NS;
-          ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / C::NS) & 1) ^ 1, abort_flag,
+          const uint32_t stage = a_it + st;
+          const uint32_t as = stage % NS;
+          ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / NS) & 1) ^ 1, abort_flag,
                               p.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t col = C::ACC_COLS + as * C::A_COLS +
-                               (C::NMAT == 2 ? part * (KA / 2) : part * 16);
+          const uint32_t col = C::ACC_COLS + as * C::A_COLS + q * (KA / 2);
           tmem_st16(tl + col, vals);
-          if (C::NMAT == 2) tmem_st16(tl + col + 16, vals + 16);
+          tmem_st16(tl + col + 16, vals + 16);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(a_full + as));
+          if (lane == 0) mbar_arrive(afull + as * 8);
         }
         ++raw_it;
         a_it += C::A_PER_RAW;
@@ -846,10 +796,51 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ i
   if (!__all_sync(0xffffffffu, ok) && (threadIdx.x & 31) == 0) report_status(status, MOE_ERR_RANGE);
 }
 
-template <int FMT, int EPI, bool GATHER, bool ROUTER>
+// bf16 rows gathered into fp16: out[r][:] = fp16(x[row_map[r]][:]), one
+// block per sorted row (8 values per thread); values that do not round to a
+// finite fp16 are reported as MOE_ERR_RANGE (they become +-inf).
+__global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict__ x,
+                                                         const uint32_t* __restrict__ row_map,
+                                                         int d8, uint4* __restrict__ out,
+                                                         int* status) {
+  pdl_wait();
+  pdl_launch();
+  const long long r = blockIdx.x;
+  const uint4* src = x + (size_t)__ldg(row_map + r) * d8;
+  uint4* dst = out + (size_t)r * d8;
+  bool ok = true;
+  for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+    const uint4 v = __ldg(src + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+      ok &= fabsf(a) < 65520.f && fabsf(b) < 65520.f;
+      uint32_t dd;
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(dd) : "f"(b), "f"(a));
+      o[j] = dd;
+    }
+    dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (!__all_sync(0xffffffffu, ok) && (threadIdx.x & 31) == 0) report_status(status, MOE_ERR_RANGE);
+}
+
+// The token-row maps of Params: [rows][K] 16-bit elements, one map per tile
+// height (16, 32, ..., 128 rows), 64 elements (128 bytes) wide.
+static bool token_maps(Params& p, const void* src, bool bf16, long long rows, int K) {
+  for (int i = 0; i < NBOX; ++i)
+    if (!make_map(&p.tmB[i], bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  src, (uint64_t)K, (uint64_t)rows, (uint64_t)K * 2, KA, 16 * (i + 1),
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  return true;
+}
+
+template <int FMT, int EPI, bool ROUTER>
 static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub, cudaStream_t s) {
-  using C = Cfg<FMT, EPI>;
-  auto kern = grouped_tc_kernel<FMT, EPI, GATHER, ROUTER>;
+  using C = Cfg<FMT>;
+  auto kern = grouped_tc_kernel<FMT, EPI, ROUTER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const long long grid = units_ub < num_sms() ? units_ub : num_sms();
@@ -858,10 +849,12 @@ static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub
   return cudaGetLastError();
 }
 
-// the kernels tile d and F by 128 rows; q4 raw stages span 256 elements of K
+// Shapes the kernels tile: gate|up units are 128 features (F % 128), down
+// units 256 output rows (d % 256); K (d or F) a multiple of 128 for the
+// k-block pairs, and of 256 for q4 raw stages.
 static bool tc_shape_ok(const moe_experts& ex) {
-  if (ex.d % 128 || ex.F % 128) return false;
-  if (ex.fmt == MOE_W_Q4G64) return ex.d % 256 == 0 && ex.F % 256 == 0;
+  if (ex.d % 256 || ex.F % 128) return false;
+  if (ex.fmt == MOE_W_Q4G64) return ex.F % 256 == 0;
   return ex.fmt == MOE_W_BF16;
 }
 
@@ -869,71 +862,88 @@ static bool tc_shape_ok(const moe_experts& ex) {
 
 int tc_block_m() { return tc::BN; }
 
+bool tc_shape_supported(int d, int F, int fmt) {
+  moe_experts ex{};
+  ex.d = d;
+  ex.F = F;
+  ex.fmt = (moe_wfmt)fmt;
+  return tc::tc_shape_ok(ex);
+}
+
 cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cudaStream_t s) {
   const long long n8 = n / 8;
   if (n8 <= 0) return cudaSuccess;
-  launch_pdl(tc::to_f16_kernel, (unsigned)((n8 + 255) / 256), 256, 0, s, (const uint4*)x, (uint4*)x16, n8,
-                                                                 status);
+  launch_pdl(tc::to_f16_kernel, (unsigned)((n8 + 255) / 256), 256, 0, s, (const uint4*)x,
+             (uint4*)x16, n8, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
-                             void* x16, int* status, cudaStream_t s) {
+                             void* xs16, int* status, cudaStream_t s) {
   using namespace tc;
   if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
-  // the expert GEMMs take fp16 operands: x is converted once into x16 [T][d]
-  cudaError_t e = launch_to_f16(x, (long long)T * ex.d, x16, status, s);
+  (void)T;
+  if (R <= 0) return cudaSuccess;
+  // the expert GEMMs take fp16 operands in row-sorted order: x gathered
+  // through row_map and converted once into xs16 [R][d]
+  launch_pdl(gather_f16_kernel, (unsigned)R, 256, 0, s, (const uint4*)x, row_map, ex.d / 8,
+             (uint4*)xs16, status);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap ta;
   if (!weight_map(&ta, ex.fmt, ex.w_gu, (long long)ex.E * 2 * ex.F, ex.d)) return cudaErrorInvalidValue;
   Params p{};
+  if (!token_maps(p, xs16, false, R, ex.d)) return cudaErrorInvalidValue;
   p.row_off = row_off;
   p.tile_off = tile_off;
   p.E = ex.E;
-  p.n_mb = ex.F / BMW;
+  p.n_units = ex.F / BMW;
+  p.unit_rows = BMW;
+  p.mat_off = ex.F;
   p.K = ex.d;
   p.rows_per_group = 2 * ex.F;
-  p.up_off = ex.F;
   p.G = ex.d / 64;
+  p.w_rows = (long long)ex.E * 2 * ex.F;
   p.scales = (const uint16_t*)ex.s_gu;
   p.biases = (const uint16_t*)ex.b_gu;
-  p.row_map = row_map;
-  p.b_src = x16;
   p.out = h;
   p.out_ld = ex.F;
   p.m_limit = ex.F;
   p.status = status;
-  const long long ub = max_tiles(R, ex.E, BN) * p.n_mb;
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_SWIGLU, true, false>(p, ta, ub, s);
-  return run<MOE_W_BF16, EPI_SWIGLU, true, false>(p, ta, ub, s);
+  const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
+  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_SWIGLU, false>(p, ta, ub, s);
+  return run<MOE_W_BF16, EPI_SWIGLU, false>(p, ta, ub, s);
 }
 
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
                            const moe_experts& ex, void* ys, int* status, cudaStream_t s) {
   using namespace tc;
   if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
+  if (R <= 0) return cudaSuccess;
   CUtensorMap ta;
   if (!weight_map(&ta, ex.fmt, ex.w_dn, (long long)ex.E * ex.d, ex.F)) return cudaErrorInvalidValue;
   Params p{};
+  if (!token_maps(p, h, false, R, ex.F)) return cudaErrorInvalidValue;
   p.row_off = row_off;
   p.tile_off = tile_off;
   p.E = ex.E;
-  p.n_mb = ex.d / BMW;
+  p.n_units = ex.d / (2 * BMW);
+  p.unit_rows = 2 * BMW;
+  p.mat_off = BMW;
   p.K = ex.F;
   p.rows_per_group = ex.d;
-  p.up_off = 0;
   p.G = ex.F / 64;
+  p.w_rows = (long long)ex.E * ex.d;
   p.scales = (const uint16_t*)ex.s_dn;
   p.biases = (const uint16_t*)ex.b_dn;
-  p.b_src = h;
   p.out = ys;
   p.out_ld = ex.d;
   p.m_limit = ex.d;
   p.status = status;
-  const long long ub = max_tiles(R, ex.E, BN) * p.n_mb;
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE_F32, false, false>(p, ta, ub, s);
-  return run<MOE_W_BF16, EPI_STORE_F32, false, false>(p, ta, ub, s);
+  const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
+  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE_F32, false>(p, ta, ub, s);
+  return run<MOE_W_BF16, EPI_STORE_F32, false>(p, ta, ub, s);
 }
 
 cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const float* bias, int T,
@@ -944,18 +954,23 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
   CUtensorMap ta;
   if (!weight_map(&ta, MOE_W_BF16, w_router, E, d)) return cudaErrorInvalidValue;
   Params p{};
+  if (!token_maps(p, x, true, T, d)) return cudaErrorInvalidValue;
   p.E = 1;
   p.n_rows = T;
-  p.n_mb = (E + BMW - 1) / BMW;
+  // units of two 128-row blocks of experts; rows past E are zero-filled by
+  // the TMA and never stored
+  p.n_units = (E + 2 * BMW - 1) / (2 * BMW);
+  p.unit_rows = 2 * BMW;
+  p.mat_off = BMW;
   p.K = d;
+  p.w_rows = E;
   p.out = logits;
   p.out_ld = E;
   p.m_limit = E;
   p.bias = bias;
-  p.b_src = x;
   p.status = status;
-  const long long ub = (long long)((T + BN - 1) / BN) * p.n_mb;
-  return run<MOE_W_BF16, EPI_STORE_F32, false, true>(p, ta, ub, s);
+  const long long ub = (long long)((T + BN - 1) / BN) * p.n_units;
+  return run<MOE_W_BF16, EPI_STORE_F32, true>(p, ta, ub, s);
 }
 
 }  // namespace moe

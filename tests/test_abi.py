@@ -102,8 +102,12 @@ def test_stage_calls_reject_bad_arguments(moe):
     assert L.moe_grouped_swiglu(fake, moe.BF16, P, fake, fake, 8, 4, 2, ctypes.byref(ex), fake, fake, 1 << 20, 0, P) == moe.ERR_INVALID_ARG
     assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 0, 4, 2, ctypes.byref(ex), fake, fake, 1 << 20, 0, P) == moe.ERR_INVALID_ARG
     # the tensor-core regime needs its fp16 staging workspace
-    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 128, 4, 2, ctypes.byref(ex), fake, P, 0, 2, P) == moe.ERR_WORKSPACE
-    assert L.moe_grouped_swiglu_workspace(4, 128, moe.BF16) >= 4 * 128 * 2
+    ex256 = _ex(moe, d=256)
+    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 128, 4, 2, ctypes.byref(ex256), fake, P, 0, 2, P) == moe.ERR_WORKSPACE
+    # ... and tiles d by 256: d = 128 is not a shape it takes
+    assert L.moe_grouped_swiglu(fake, moe.BF16, fake, fake, fake, 128, 4, 2, ctypes.byref(ex), fake, fake, 1 << 20, 2, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_grouped_down(fake, moe.BF16, fake, fake, 128, 4, 2, ctypes.byref(ex), fake, 2, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_grouped_swiglu_workspace(4, 2, 128, moe.BF16) >= 4 * 2 * 128 * 2
     assert L.moe_grouped_down(fake, moe.BF16, fake, fake, 8, 4, 2, P, fake, 0, P) == moe.ERR_INVALID_ARG
     # the tensor-core regime takes bf16 activations only
     exf = _ex(moe, fmt=0)
@@ -120,7 +124,8 @@ def test_forward_layout_is_consistent(moe):
                 L.row_off, L.tile_off, L.sort_ws, L.h, L.ys, L.x16]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert L.ys + T * k * d * 4 <= L.x16
-        assert L.x16 + T * d * 2 <= L.total
+        # fp16 token rows: T of them, or all T*k rows in sorted order (tensor cores)
+        assert L.x16 + (T * k if L.regime == moe.REGIME_TC else T) * d * 2 <= L.total
         assert L.h + T * k * F * 2 <= L.ys
         assert L.BM >= 1 and L.regime in (moe.REGIME_GEMV, moe.REGIME_TC)
         assert moe.lib.moe_forward_workspace(T, d, E, k, F, moe.BF16, 0) == L.total
