@@ -588,43 +588,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
       const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
+      // 16 columns at a time; the next chunk's TMEM loads are in flight
+      // while this one is computed and stored
+      uint32_t a0[16], a1[16];
+      tmem_ld16(c0, a0);
+      tmem_ld16(c1, a1);
       if (EPI == EPI_SWIGLU) {
         const int orow = unit * p.unit_rows + m;          // feature of this thread
-        __half* h = reinterpret_cast<__half*>(p.out);
+        __half* hp = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + orow;
         for (int n0 = 0; n0 < nv; n0 += 16) {
-          uint32_t g[16], uu[16];
-          tmem_ld16(c0 + n0, g);
-          tmem_ld16(c1 + n0, uu);
           tmem_ld_wait();
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = swiglu(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
+          if (n0 + 16 < nv) {
+            tmem_ld16(c0 + n0 + 16, a0);
+            tmem_ld16(c1 + n0 + 16, a1);
+          }
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = n0 + j;
-            if (n < nv) {
-              const float v = swiglu(__uint_as_float(g[j]), __uint_as_float(uu[j]));
-              range_ok &= fabsf(v) < 65520.f;    // rounds to a finite fp16
-              h[(size_t)(r0 + n) * p.out_ld + orow] = __float2half_rn(v);
+            if (n0 + j < nv) {
+              range_ok &= fabsf(v[j]) < 65520.f;    // rounds to a finite fp16
+              hp[(size_t)(n0 + j) * p.out_ld] = __float2half_rn(v[j]);
             }
           }
         }
       } else {
-        float* o = reinterpret_cast<float*>(p.out);
         const int orow0 = unit * p.unit_rows + m;
         const int orow1 = orow0 + BMW;
         const bool ok0 = orow0 < p.m_limit, ok1 = orow1 < p.m_limit;
         const float bv0 = (ok0 && p.bias) ? __ldg(p.bias + orow0) : 0.f;
         const float bv1 = (ok1 && p.bias) ? __ldg(p.bias + orow1) : 0.f;
+        float* op = reinterpret_cast<float*>(p.out) + (size_t)r0 * p.out_ld + orow0;
         for (int n0 = 0; n0 < nv; n0 += 16) {
-          uint32_t g0[16], g1[16];
-          tmem_ld16(c0 + n0, g0);
-          tmem_ld16(c1 + n0, g1);
           tmem_ld_wait();
+          float v0[16], v1[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = n0 + j;
-            if (n < nv) {
-              float* orow = o + (size_t)(r0 + n) * p.out_ld;
-              if (ok0) orow[orow0] = __uint_as_float(g0[j]) + bv0;
-              if (ok1) orow[orow1] = __uint_as_float(g1[j]) + bv1;
+            v0[j] = __uint_as_float(a0[j]) + bv0;
+            v1[j] = __uint_as_float(a1[j]) + bv1;
+          }
+          if (n0 + 16 < nv) {
+            tmem_ld16(c0 + n0 + 16, a0);
+            tmem_ld16(c1 + n0 + 16, a1);
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (n0 + j < nv) {
+              float* o = op + (size_t)(n0 + j) * p.out_ld;
+              if (ok0) o[0] = v0[j];
+              if (ok1) o[BMW] = v1[j];
             }
           }
         }
