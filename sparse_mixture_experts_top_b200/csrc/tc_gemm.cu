@@ -7,7 +7,7 @@
 // already sorted by expert. mlx-lm PR #2044, "What": each expert's weights are
 // read and dequantised once per tile instead of once per (token, slot).
 //
-// B200 design (one persistent CTA per SM, 16 warps). A unit of work is one
+// B200 design (one persistent CTA per SM, 24 warps). A unit of work is one
 // token tile x two 128-row weight matrices: gate and up rows of the same
 // features (gate|up), or two adjacent 128-row blocks (down, router).
 //   * swap-AB: the MMA's M = 128 weight rows, N = the tile's token rows
@@ -17,10 +17,12 @@
 //   * warp 2: one TMA per k-block of the tile's token rows, from a row-sorted
 //     16-bit copy (x gathered through row_map, or h, or x for the router),
 //     with one tensor map per tile height (16, 32, ..., 128 rows);
-//   * warps 8..15 (dequant, 4 per matrix): each thread owns one weight row
-//     (one TMEM lane), dequantises w = s*q + b to fp16 and writes it into
-//     TMEM with tcgen05.st, where the MMA takes it as its A operand -- the
-//     dequantised tile never goes back through shared memory;
+//   * warps 8..23 (dequant, 8 per matrix): each thread owns one weight row
+//     (one TMEM lane) and half of every raw stage, dequantises w = s*q + b
+//     to fp16 and writes it into TMEM with tcgen05.st, where the MMA takes it
+//     as its A operand -- the dequantised tile never goes back through shared
+//     memory. Two warps per row keep the conversion, which is bound by the
+//     latency of its integer and fp16 chains, off the critical path;
 //   * warps 1 and 3 (MMA): one thread each issues the tcgen05.mma of one
 //     matrix (A from TMEM, B from shared memory) into its own fp32
 //     accumulator. Two issuers, because at small N one thread cannot issue
@@ -56,7 +58,7 @@ constexpr int NS = 4;          // k-block stages of A in TMEM, released in pairs
 constexpr int NB = 6;          // token-row (B) stages in shared memory
 constexpr int NBOX = BN / 16;  // token-row tensor maps: tile heights 16, 32, ..., 128
 constexpr int kMaxE = 1024;    // tile / row tables cached in shared memory
-constexpr int kThreads = 512;
+constexpr int kThreads = 768;   // 24 warps
 constexpr int kEpiWarp0 = 4;
 constexpr int kDqWarp0 = 8;
 constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at the B200's clocks
@@ -230,29 +232,50 @@ __device__ __forceinline__ uint32_t idesc_mma(int n, bool f16) {
          ((uint32_t)(BMW >> 4) << 24);
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+// 16 columns of this warp's 32 lanes from each of two TMEM addresses, and the
+// wait for them, in one statement: the destination registers of tcgen05.ld
+// are written asynchronously until tcgen05.wait::ld, so the load and its wait
+// must not be separated where the compiler could spill or move them.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, uint32_t (&a)[16],
+                                            uint32_t (&b)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
+        "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]),
+        "=r"(a[14]), "=r"(a[15]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]),
+        "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]),
+        "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+// 16 (or 2 x 16) columns of this warp's 32 lanes stored and waited for in one
+// statement, so no source register is reused while the store is in flight.
+__device__ __forceinline__ void tmem_st16_sync(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
       "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
       "r"(v[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+__device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 
 // ------------------------------------------------------------------ dequant
@@ -377,9 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < C::NR; ++i) {
       // q4: the TMA arrive + the 32 lanes' cp.async arrivals for the scales
       mbar_init(smem_u32(raw_full + i), C::Q4 ? 33 : 1);
-      mbar_init(smem_u32(raw_empty + i), 8);   // the 8 dequant warps
+      mbar_init(smem_u32(raw_empty + i), 16);   // the 16 dequant warps
     }
-    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), 4);   // a matrix's 4 warps
+    // a matrix's stage is written by 4 warps (q4: one half) or 8 (bf16: both halves)
+    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::Q4 ? 4 : 8);
     for (int i = 0; i < NB; ++i) mbar_init(smem_u32(b_full + i), 1);
     for (int i = 0; i < NS / 2; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
     for (int i = 0; i < 2; ++i) {
@@ -588,28 +612,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
       const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
-      // 16 columns at a time; the next chunk's TMEM loads are in flight
-      // while this one is computed and stored
-      uint32_t a0[16], a1[16];
-      tmem_ld16(c0, a0);
-      tmem_ld16(c1, a1);
+      // 16 columns of both accumulators at a time
       if (EPI == EPI_SWIGLU) {
         const int orow = unit * p.unit_rows + m;          // feature of this thread
         __half* hp = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + orow;
         for (int n0 = 0; n0 < nv; n0 += 16) {
-          tmem_ld_wait();
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = swiglu(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
-          if (n0 + 16 < nv) {
-            tmem_ld16(c0 + n0 + 16, a0);
-            tmem_ld16(c1 + n0 + 16, a1);
-          }
+          uint32_t a0[16], a1[16];
+          tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (n0 + j < nv) {
-              range_ok &= fabsf(v[j]) < 65520.f;    // rounds to a finite fp16
-              hp[(size_t)(n0 + j) * p.out_ld] = __float2half_rn(v[j]);
+              const float v = swiglu(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
+              range_ok &= fabsf(v) < 65520.f;    // rounds to a finite fp16
+              hp[(size_t)(n0 + j) * p.out_ld] = __float2half_rn(v);
             }
           }
         }
@@ -621,23 +636,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float bv1 = (ok1 && p.bias) ? __ldg(p.bias + orow1) : 0.f;
         float* op = reinterpret_cast<float*>(p.out) + (size_t)r0 * p.out_ld + orow0;
         for (int n0 = 0; n0 < nv; n0 += 16) {
-          tmem_ld_wait();
-          float v0[16], v1[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            v0[j] = __uint_as_float(a0[j]) + bv0;
-            v1[j] = __uint_as_float(a1[j]) + bv1;
-          }
-          if (n0 + 16 < nv) {
-            tmem_ld16(c0 + n0 + 16, a0);
-            tmem_ld16(c1 + n0 + 16, a1);
-          }
+          uint32_t a0[16], a1[16];
+          tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (n0 + j < nv) {
               float* o = op + (size_t)(n0 + j) * p.out_ld;
-              if (ok0) o[0] = v0[j];
-              if (ok1) o[BMW] = v1[j];
+              if (ok0) o[0] = __uint_as_float(a0[j]) + bv0;
+              if (ok1) o[BMW] = __uint_as_float(a1[j]) + bv1;
             }
           }
         }
@@ -655,12 +661,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!__all_sync(0xffffffffu, range_ok) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------ dequant
-    const int dw = warp - kDqWarp0;                   // 0..7
-    const int q = dw >> 2;                            // matrix
+    // 16 warps: (matrix q, lane quadrant qd, half hf). q4: half hf converts
+    // A stages 2hf and 2hf + 1 of every raw stage (chunks 4hf .. 4hf + 3 of
+    // the row); bf16: half hf converts K elements 32hf .. 32hf + 31 of the
+    // raw stage's single A stage.
+    const int dw = warp - kDqWarp0;                   // 0..15
+    const int q = (dw >> 2) & 1;                      // matrix
+    const int hf = dw >> 3;                           // half of the raw stage
     const int qd = warp & 3;                          // TMEM lane quadrant
     const int m = qd * 32 + lane;                     // weight row of this thread
     const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
     const uint32_t afull = smem_u32(a_full + q * NS);
+    constexpr int NST = C::Q4 ? 2 : 1;                // A stages per raw stage of this warp
     uint32_t raw_it = 0, a_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
@@ -668,55 +680,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status);
         if (!ok) break;
-        // my row: 128 bytes = 8 chunks of 16 B in the 128-byte swizzle
+        // my half row: 4 chunks of 16 B in the 128-byte swizzle
         const uint32_t rowa = raw_base + rs * C::RAW_BYTES + q * C::RAW_MAT + m * 128;
         const int sw = m & 7;
-        uint4 wv[8];
+        uint4 wv[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) wv[c] = lds128(rowa + ((c ^ sw) << 4));
-        uint32_t sc[2] = {0, 0}, bi[2] = {0, 0};
+        for (int c = 0; c < 4; ++c) wv[c] = lds128(rowa + (((4 * hf + c) ^ sw) << 4));
+        uint32_t sc = 0, bi = 0;
         if (C::Q4) {
-          // this row's 4 groups of scales and biases (bf16 pairs)
-          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * 8);
-          asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(sc[0]), "=r"(sc[1]) : "r"(so));
-          asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
-                       : "=r"(bi[0]), "=r"(bi[1])
-                       : "r"(so + C::SCL_BYTES / 2));
+          // this row's scales and biases of groups 2hf, 2hf + 1 (bf16 pairs)
+          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * 8 + hf * 4);
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc) : "r"(so));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bi) : "r"(so + C::SCL_BYTES / 2));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
 #pragma unroll
-        for (int st = 0; st < C::A_PER_RAW; ++st) {
+        for (int j = 0; j < NST; ++j) {
           uint32_t vals[32];
           if (C::Q4) {
-            // chunk pair (2st, 2st + 1) holds the 64 elements of group 4kr + st
-            const uint32_t sv = sc[st >> 1], bv = bi[st >> 1];
-            const uint32_t s2 = f16x2_from_bf16((st & 1) ? (sv >> 16) : (sv & 0xFFFFu));
-            const uint32_t b2 = f16x2_from_bf16((st & 1) ? (bv >> 16) : (bv & 0xFFFFu));
-            const uint4 w0 = wv[2 * st], w1 = wv[2 * st + 1];
+            // chunk pair (2j, 2j + 1) of my half holds the 64 elements of
+            // group 4kr + 2hf + j
+            const uint32_t s2 = f16x2_from_bf16(j ? (sc >> 16) : (sc & 0xFFFFu));
+            const uint32_t b2 = f16x2_from_bf16(j ? (bi >> 16) : (bi & 0xFFFFu));
+            const uint4 w0 = wv[2 * j], w1 = wv[2 * j + 1];
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) dequant_word(ws[i], s2, b2, vals + 4 * i);
           } else {
-            // bf16 weights: the 64 elements of the k-block; fp16 operands for
+            // bf16 weights: 32 elements of the k-block; fp16 operands for
             // the experts, bf16 kept as is for the router
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
               const uint32_t w4[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) vals[4 * c + i] = ROUTER ? w4[i] : bf16x2_to_f16x2(w4[i]);
             }
           }
-          const uint32_t stage = a_it + st;
+          const uint32_t stage = a_it + (C::Q4 ? 2 * hf + j : 0);
           const uint32_t as = stage % NS;
           ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / NS) & 1) ^ 1, abort_flag,
                               p.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t col = C::ACC_COLS + as * C::A_COLS + q * (KA / 2);
-          tmem_st16(tl + col, vals);
-          tmem_st16(tl + col + 16, vals + 16);
-          tmem_st_wait();
+          const uint32_t col = C::ACC_COLS + as * C::A_COLS + q * (KA / 2) + (C::Q4 ? 0 : hf * 16);
+          if (C::Q4) tmem_st32_sync(tl + col, vals);
+          else tmem_st16_sync(tl + col, vals);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(afull + as * 8);
