@@ -56,6 +56,13 @@ constexpr int BMW = 128;       // weight rows per matrix (MMA M)
 constexpr int KA = 64;         // K elements per k-block (one q4 group)
 constexpr int NS = 4;          // k-block stages of A in TMEM, released in pairs
 constexpr int NB = 6;          // token-row (B) stages in shared memory
+// Release barriers: k-blocks 2P and 2P + 1 (pair P, counted over the CTA's
+// whole k-block sequence) are released on barrier P % NP, its completion
+// P / NP. A waiter may lag the barrier by less than one phase only: the
+// next completion of the same barrier covers k-blocks 2NP later, so a ring
+// reused at distance D needs D <= 2 NP (the TMEM stages: NS; the B stages:
+// NB). A parity wait on a barrier two phases ahead would never succeed.
+constexpr int NP = 4;
 constexpr int NBOX = BN / 16;  // token-row tensor maps: tile heights 16, 32, ..., 128
 constexpr int kMaxE = 1024;    // tile / row tables cached in shared memory
 constexpr int kThreads = 768;   // 24 warps
@@ -82,6 +89,7 @@ struct Cfg {
   static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
   static_assert(ACC_COLS + NS * A_COLS <= 512, "accumulators and A stages must fit TMEM");
   static_assert(NS % 2 == 0, "A stages are released in pairs");
+  static_assert(NS <= 2 * NP && NB <= 2 * NP, "a ring may not outrun its release barriers");
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
@@ -156,8 +164,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Every lane waits; the result is the same in all lanes, so the warp stays
 // converged for the .sync.aligned tcgen05 instructions that follow.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, int* status) {
-  const bool r = mbar_wait(bar, parity, abort_flag, status);
+                                               volatile int* abort_flag, int* status,
+                                               bool honor_abort = true) {
+  const bool r = mbar_wait(bar, parity, abort_flag, status, honor_abort);
   return __all_sync(0xffffffffu, r);
 }
 
@@ -181,35 +190,39 @@ __device__ __forceinline__ void tc_fence_after() {
 // in a single statement: D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (fp16 or
 // bf16 operands, fp32 accumulation). A columns advance 8 per K-step, the B
 // descriptor's start address 32 bytes (+2 in 16-byte units) inside the
-// 128-byte swizzle atom; accumulate unless `first`. The issuing thread is
-// on the critical path: at small N a tcgen05.mma from one thread is accepted
-// only every ~50-80 cycles and nothing queues behind it, so every other
-// instruction it executes adds to the tile's time.
-__device__ __forceinline__ void mma_kblock1(uint32_t d0, uint32_t a0, uint32_t blo, uint32_t bhi,
-                                            uint32_t idesc, uint32_t first) {
+// 128-byte swizzle atom; accumulate unless `first`. The whole warp executes
+// it with warp-uniform operands and one elected lane issues: issued from a
+// single active lane, a tcgen05.mma is accepted only every ~50 cycles; from
+// an elected lane of a converged warp the tensor core is the limit (~24
+// cycles at N = 48).
+__device__ __forceinline__ void mma_kblock(uint32_t d0, uint32_t a0, uint32_t blo, uint32_t bhi,
+                                           uint32_t idesc, uint32_t first) {
   asm volatile(
-      "{\n\t.reg .pred pf, pt;\n\t.reg .b64 b0, b1, b2, b3;\n\t"
+      "{\n\t.reg .pred pf, pt, e;\n\t.reg .b64 b0, b1, b2, b3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.eq.b32 pf, %5, 0;\n\t"
       "setp.ne.b32 pt, %4, 0;\n\t"
       "mov.b64 b0, {%2, %3};\n\t"
       "add.u32 %2, %2, 2;\n\tmov.b64 b1, {%2, %3};\n\t"
       "add.u32 %2, %2, 2;\n\tmov.b64 b2, {%2, %3};\n\t"
       "add.u32 %2, %2, 2;\n\tmov.b64 b3, {%2, %3};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b0, %4, pf;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b0, %4, pf;\n\t"
       "add.u32 %1, %1, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b1, %4, pt;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b1, %4, pt;\n\t"
       "add.u32 %1, %1, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b2, %4, pt;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b2, %4, pt;\n\t"
       "add.u32 %1, %1, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b3, %4, pt;\n\t}\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b3, %4, pt;\n\t}\n"
       : "+r"(d0), "+r"(a0), "+r"(blo), "+r"(bhi)
       : "r"(idesc), "r"(first)
       : "memory");
 }
 
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
+// tcgen05.commit from one elected lane of a converged warp
+__device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar)
       : "memory");
 }
 
@@ -382,8 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* raw_empty = raw_full + C::NR;                        // [NR]
   uint64_t* a_full = raw_empty + C::NR;                          // [2 matrices][NS]
   uint64_t* b_full = a_full + 2 * NS;                            // [NB]
-  uint64_t* s_empty = b_full + NB;                               // [NS / 2] stage pairs
-  uint64_t* acc_full = s_empty + NS / 2;                         // [2] accumulator buffers
+  uint64_t* s_empty = b_full + NB;                               // [NP] k-block pair releases
+  uint64_t* acc_full = s_empty + NP;                             // [2] accumulator buffers
   uint64_t* acc_empty = acc_full + 2;                            // [2]
   uint64_t* drain = acc_empty + 2;                               // [2] one per issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
@@ -405,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a matrix's stage is written by 4 warps (q4: one half) or 8 (bf16: both halves)
     for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::Q4 ? 4 : 8);
     for (int i = 0; i < NB; ++i) mbar_init(smem_u32(b_full + i), 1);
-    for (int i = 0; i < NS / 2; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
+    for (int i = 0; i < NP; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(acc_full + i), 2);    // both issuers
       mbar_init(smem_u32(acc_empty + i), 4);   // the 4 epilogue warps
@@ -509,8 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the row-sorted 16-bit operand, 64 elements (128 bytes) each, landing in
     // the 128B-swizzled K-major layout the MMA reads. Rows past the tile
     // belong to the next tile (their columns are never stored) or lie past
-    // the end (zero fill). B stage j is reused by k-block j + NB once the A
-    // stage pair that holds k-block j has been released by both issuers.
+    // the end (zero fill). B stage j is reused by k-block j + NB once the
+    // k-block pair that holds k-block j has been released by both issuers.
     if (lane == 0) {
       uint32_t j = 0;
       bool ok = true;
@@ -522,9 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < nka && ok; ++kb) {
           const int bs = j % NB;
           if (j >= (uint32_t)NB) {
-            const uint32_t jj = j - NB;
-            ok = mbar_wait(smem_u32(s_empty + ((jj % NS) >> 1)), (jj / NS) & 1, abort_flag,
-                           p.status);
+            const uint32_t pr = (j - NB) >> 1;
+            ok = mbar_wait(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status);
             if (!ok) break;
           }
           const uint32_t bar = smem_u32(b_full + bs);
@@ -541,59 +553,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
-    // warp 1 issues matrix 0, warp 3 matrix 1, each into its own accumulator
-    if (lane == 0) {
-      const int q = warp >> 1;
-      uint32_t ss = 0, sph = 0, bs = 0, bph = 0;      // A and B stage slots and phases
-      uint32_t nb = 0, uses0 = 0, uses1 = 0;          // accumulator buffers
-      bool ok = true;
-      // descriptor of B stage 0 (low word: start address / 16 and the
-      // leading offset; high word: stride offset, version, swizzle)
-      const uint64_t d0 = desc_sw128(b_base);
-      const uint32_t blo0 = (uint32_t)d0, bhi = (uint32_t)(d0 >> 32);
-      const uint32_t a_col0 = tmem + C::ACC_COLS + q * (KA / 2);
-      const uint32_t afull0 = smem_u32(a_full + q * NS);
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        int unit, r0, nv, e;
-        decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
-        const int n = mma_n(nv);
-        const uint32_t idesc = idesc_mma(n, !ROUTER);
-        // tiles of <= 64 rows alternate between the two 128-column buffers
-        // (matrix q at +64q); larger ones take both (matrix q at +128q)
-        const bool small = n <= 64;
-        const uint32_t b = small ? nb : 0u;
-        const bool use0 = !small || b == 0, use1 = !small || b == 1;
-        // the epilogue has drained the buffers' previous tiles
-        if (use0 && uses0 > 0)
-          ok = mbar_wait(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status);
-        if (ok && use1 && uses1 > 0)
-          ok = mbar_wait(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status);
+    // warp 1 issues matrix 0, warp 3 matrix 1, each into its own
+    // accumulator; the whole warp runs the loop (warp-uniform operands) and
+    // one elected lane issues
+    const int q = warp >> 1;
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    uint32_t ss = 0, sph = 0, bs = 0, bph = 0;        // A and B stage slots and phases
+    uint32_t kg = 0;                                  // k-blocks issued so far
+    uint32_t nb = 0, uses0 = 0, uses1 = 0;            // accumulator buffers
+    bool ok = true;
+    // descriptor of B stage 0 (low word: start address / 16 and the
+    // leading offset; high word: stride offset, version, swizzle)
+    const uint64_t d0 = desc_sw128(b_base);
+    const uint32_t blo0 = (uint32_t)d0, bhi = (uint32_t)(d0 >> 32);
+    const uint32_t a_col0 = tm + C::ACC_COLS + q * (KA / 2);
+    const uint32_t afull0 = smem_u32(a_full + q * NS);
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int unit, r0, nv, e;
+      decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+      const int n = mma_n(nv);
+      const uint32_t idesc = idesc_mma(n, !ROUTER);
+      // tiles of <= 64 rows alternate between the two 128-column buffers
+      // (matrix q at +64q); larger ones take both (matrix q at +128q)
+      const bool small = n <= 64;
+      const uint32_t b = small ? nb : 0u;
+      const bool use0 = !small || b == 0, use1 = !small || b == 1;
+      // the epilogue has drained the buffers' previous tiles
+      if (use0 && uses0 > 0)
+        ok = mbar_wait_warp(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status);
+      if (ok && use1 && uses1 > 0)
+        ok = mbar_wait_warp(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t dcol = tm + (small ? b * 128u + q * 64u : q * 128u);
+      for (int kb = 0; kb < nka && ok; ++kb) {
+        ok = mbar_wait_warp(afull0 + ss * 8, sph, abort_flag, p.status) &&
+             mbar_wait_warp(smem_u32(b_full + bs), bph, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t dcol = tmem + (small ? b * 128u + q * 64u : q * 128u);
-        for (int kb = 0; kb < nka && ok; ++kb) {
-          ok = mbar_wait(afull0 + ss * 8, sph, abort_flag, p.status) &&
-               mbar_wait(smem_u32(b_full + bs), bph, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          mma_kblock1(dcol, a_col0 + ss * (uint32_t)C::A_COLS,
-                      blo0 + bs * (uint32_t)(C::B_BYTES >> 4), bhi, idesc, kb == 0);
-          // a unit has an even number of k-blocks, so the pairs never
-          // straddle units
-          if (ss & 1) mma_commit(smem_u32(s_empty + (ss >> 1)));
-          if (++ss == (uint32_t)NS) { ss = 0; sph ^= 1; }
-          if (++bs == (uint32_t)NB) { bs = 0; bph ^= 1; }
-        }
-        if (!ok) break;
-        if (use0) { mma_commit(smem_u32(acc_full + 0)); ++uses0; }
-        if (use1) { mma_commit(smem_u32(acc_full + 1)); ++uses1; }
-        if (small) nb ^= 1u;
+        mma_kblock(dcol, a_col0 + ss * (uint32_t)C::A_COLS, blo0 + bs * (uint32_t)(C::B_BYTES >> 4),
+                   bhi, idesc, kb == 0);
+        // release k-block pair kg / 2 (a unit has an even number of k-blocks)
+        if (kg & 1) mma_commit_warp(smem_u32(s_empty + (kg >> 1) % NP));
+        ++kg;
+        if (++ss == (uint32_t)NS) { ss = 0; sph ^= 1; }
+        if (++bs == (uint32_t)NB) { bs = 0; bph ^= 1; }
       }
-      // all MMAs issued by this thread complete before TMEM is released
-      mma_commit(smem_u32(drain + q));
-      mbar_wait(smem_u32(drain + q), 0, abort_flag, p.status, false);
+      if (!ok) break;
+      if (use0) { mma_commit_warp(smem_u32(acc_full + 0)); ++uses0; }
+      if (use1) { mma_commit_warp(smem_u32(acc_full + 1)); ++uses1; }
+      if (small) nb ^= 1u;
     }
-    __syncwarp();
+    // all MMAs issued by this warp complete before TMEM is released
+    mma_commit_warp(smem_u32(drain + q));
+    mbar_wait_warp(smem_u32(drain + q), 0, abort_flag, p.status, false);
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;
@@ -719,9 +732,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t stage = a_it + (C::Q4 ? 2 * hf + j : 0);
           const uint32_t as = stage % NS;
-          ok = mbar_wait_warp(smem_u32(s_empty + (as >> 1)), ((stage / NS) & 1) ^ 1, abort_flag,
-                              p.status);
-          if (!ok) break;
+          if (stage >= (uint32_t)NS) {      // the slot's previous k-block is released
+            const uint32_t pr = (stage - NS) >> 1;
+            ok = mbar_wait_warp(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status);
+            if (!ok) break;
+          }
           tc_fence_after();
           const uint32_t col = C::ACC_COLS + as * C::A_COLS + q * (KA / 2) + (C::Q4 ? 0 : hf * 16);
           if (C::Q4) tmem_st32_sync(tl + col, vals);
