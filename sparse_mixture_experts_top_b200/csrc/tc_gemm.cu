@@ -90,6 +90,7 @@ struct Cfg {
   static_assert(ACC_COLS + NS * A_COLS <= 512, "accumulators and A stages must fit TMEM");
   static_assert(NS % 2 == 0, "A stages are released in pairs");
   static_assert(NS <= 2 * NP && NB <= 2 * NP, "a ring may not outrun its release barriers");
+  static_assert(NB % 2 == 0, "the MMA consumes B stages in pairs");
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
@@ -586,18 +587,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t dcol = tm + (small ? b * 128u + q * 64u : q * 128u);
-      for (int kb = 0; kb < nka && ok; ++kb) {
+      // k-blocks two at a time (a unit has an even number of them; NS and
+      // NB are even, so both stages of a pair share their phases): four
+      // waits, eight MMAs and one release per pair
+      for (int kb = 0; kb < nka && ok; kb += 2) {
         ok = mbar_wait_warp(afull0 + ss * 8, sph, abort_flag, p.status) &&
-             mbar_wait_warp(smem_u32(b_full + bs), bph, abort_flag, p.status);
+             mbar_wait_warp(smem_u32(b_full + bs), bph, abort_flag, p.status) &&
+             mbar_wait_warp(afull0 + (ss + 1) * 8, sph, abort_flag, p.status) &&
+             mbar_wait_warp(smem_u32(b_full + bs + 1), bph, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        mma_kblock(dcol, a_col0 + ss * (uint32_t)C::A_COLS, blo0 + bs * (uint32_t)(C::B_BYTES >> 4),
-                   bhi, idesc, kb == 0);
-        // release k-block pair kg / 2 (a unit has an even number of k-blocks)
-        if (kg & 1) mma_commit_warp(smem_u32(s_empty + (kg >> 1) % NP));
-        ++kg;
-        if (++ss == (uint32_t)NS) { ss = 0; sph ^= 1; }
-        if (++bs == (uint32_t)NB) { bs = 0; bph ^= 1; }
+        const uint32_t acol = a_col0 + ss * (uint32_t)C::A_COLS;
+        const uint32_t blo = blo0 + bs * (uint32_t)(C::B_BYTES >> 4);
+        mma_kblock(dcol, acol, blo, bhi, idesc, kb == 0);
+        mma_kblock(dcol, acol + C::A_COLS, blo + (C::B_BYTES >> 4), bhi, idesc, 0);
+        mma_commit_warp(smem_u32(s_empty + (kg >> 1) % NP));   // release k-block pair kg / 2
+        kg += 2;
+        if ((ss += 2) == (uint32_t)NS) { ss = 0; sph ^= 1; }
+        if ((bs += 2) == (uint32_t)NB) { bs = 0; bph ^= 1; }
       }
       if (!ok) break;
       if (use0) { mma_commit_warp(smem_u32(acc_full + 0)); ++uses0; }
