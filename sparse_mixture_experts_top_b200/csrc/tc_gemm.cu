@@ -143,21 +143,34 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes or about `ns` nanoseconds pass, instead of
+// spinning and taking issue slots from the warps that do the work
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of `parity` to complete. Returns false when the
 // kernel is aborting (another role timed out) or this wait ran out.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int* status, bool honor_abort = true) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (honor_abort && *abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *abort_flag = 1;
-        report_status(status, MOE_ERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_sleep(bar, parity, 20000u)) return true;
+    if (honor_abort && *abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      report_status(status, MOE_ERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -338,6 +351,25 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t b
   out[3] = f16x2_fma(f16x2_sub(__byte_perm(p1, M, 0x4342), c1024), s2, b2);
 }
 
+// The same for a permuted K order: out[c] holds elements (c, c + 4) of the
+// word. A nibble at bits 0..3 of a 16-bit half becomes the mantissa of
+// fp16 1024.0 (0x6400 | q = 1024 + q); one at bits 4..7 becomes mantissa
+// bits 4..7 of fp16 64.0, whose last place is 1/16 (0x5400 | 16q = 64 + q).
+// Each pair is then one AND-OR, half of the words are shifted once, the
+// magic number is subtracted exactly and one fused multiply-add applies the
+// scale and bias: 5 integer operations per word instead of 9. The other
+// operand must use the same order: within every 8 consecutive K elements,
+// position p holds element (0, 4, 1, 5, 2, 6, 3, 7)[p].
+__device__ __forceinline__ void dequant_word_perm(uint32_t w, uint32_t s2, uint32_t b2,
+                                                  uint32_t* out) {
+  const uint32_t w8 = w >> 8;
+  const uint32_t c1024 = 0x64006400u, c64 = 0x54005400u;
+  out[0] = f16x2_fma(f16x2_sub((w & 0x000F000Fu) | c1024, c1024), s2, b2);    // e0, e4
+  out[1] = f16x2_fma(f16x2_sub((w & 0x00F000F0u) | c64, c64), s2, b2);        // e1, e5
+  out[2] = f16x2_fma(f16x2_sub((w8 & 0x000F000Fu) | c1024, c1024), s2, b2);   // e2, e6
+  out[3] = f16x2_fma(f16x2_sub((w8 & 0x00F000F0u) | c64, c64), s2, b2);       // e3, e7
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -395,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(bar_area);   // [NR]
   uint64_t* raw_empty = raw_full + C::NR;                        // [NR]
   uint64_t* a_full = raw_empty + C::NR;                          // [2 matrices][NS]
-  uint64_t* b_full = a_full + 2 * NS;                            // [NB]
-  uint64_t* s_empty = b_full + NB;                               // [NP] k-block pair releases
+  uint64_t* b_full = a_full + 2 * NS;                            // [NB / 2] B stage pairs
+  uint64_t* s_empty = b_full + NB / 2;                           // [NP] k-block pair releases
   uint64_t* acc_full = s_empty + NP;                             // [2] accumulator buffers
   uint64_t* acc_empty = acc_full + 2;                            // [2]
   uint64_t* drain = acc_empty + 2;                               // [2] one per issuer
@@ -418,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // a matrix's stage is written by 4 warps (q4: one half) or 8 (bf16: both halves)
     for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::Q4 ? 4 : 8);
-    for (int i = 0; i < NB; ++i) mbar_init(smem_u32(b_full + i), 1);
+    for (int i = 0; i < NB / 2; ++i) mbar_init(smem_u32(b_full + i), 1);
     for (int i = 0; i < NP; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(acc_full + i), 2);    // both issuers
@@ -523,8 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the row-sorted 16-bit operand, 64 elements (128 bytes) each, landing in
     // the 128B-swizzled K-major layout the MMA reads. Rows past the tile
     // belong to the next tile (their columns are never stored) or lie past
-    // the end (zero fill). B stage j is reused by k-block j + NB once the
-    // k-block pair that holds k-block j has been released by both issuers.
+    // the end (zero fill). k-blocks go two at a time (one barrier for the
+    // pair); B stages j, j + 1 are reused by k-blocks j + NB, j + NB + 1 once
+    // their k-block pair has been released by both issuers.
     if (lane == 0) {
       uint32_t j = 0;
       bool ok = true;
@@ -533,22 +566,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
         const int n = mma_n(nv);
         const CUtensorMap* tm = &p.tmB[n / 16 - 1];
-        for (int kb = 0; kb < nka && ok; ++kb) {
+        for (int kb = 0; kb < nka && ok; kb += 2) {
           const int bs = j % NB;
           if (j >= (uint32_t)NB) {
             const uint32_t pr = (j - NB) >> 1;
             ok = mbar_wait(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status);
             if (!ok) break;
           }
-          const uint32_t bar = smem_u32(b_full + bs);
-          mbar_arrive_tx(bar, (uint32_t)n * 128u);
+          const uint32_t bar = smem_u32(b_full + bs / 2);
+          mbar_arrive_tx(bar, (uint32_t)n * 256u);
           tma_load_2d(b_base + bs * C::B_BYTES, tm, kb * KA, r0, bar);
-          ++j;
+          tma_load_2d(b_base + (bs + 1) * C::B_BYTES, tm, (kb + 1) * KA, r0, bar);
+          j += 2;
         }
       }
-      for (uint32_t i = 0; i < (uint32_t)NB && i < j; ++i) {
-        const uint32_t last = j - 1 - i;
-        mbar_wait(smem_u32(b_full + last % NB), (last / NB) & 1, abort_flag, p.status, false);
+      for (uint32_t i = 0; i < (uint32_t)NB && i < j; i += 2) {
+        const uint32_t last = (j - 2 - i) / 2;      // pair index
+        mbar_wait(smem_u32(b_full + last % (NB / 2)), (last / (NB / 2)) & 1, abort_flag, p.status,
+                  false);
       }
     }
     __syncwarp();
@@ -588,13 +623,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t dcol = tm + (small ? b * 128u + q * 64u : q * 128u);
       // k-blocks two at a time (a unit has an even number of them; NS and
-      // NB are even, so both stages of a pair share their phases): four
-      // waits, eight MMAs and one release per pair
+      // NB are even, so both stages of a pair share their phases): two
+      // waits, eight MMAs and one release per pair. Every dequant warp
+      // signals the pair's two A stages in order, so the second one being
+      // complete means the first one is; both B stages share one barrier.
       for (int kb = 0; kb < nka && ok; kb += 2) {
-        ok = mbar_wait_warp(afull0 + ss * 8, sph, abort_flag, p.status) &&
-             mbar_wait_warp(smem_u32(b_full + bs), bph, abort_flag, p.status) &&
-             mbar_wait_warp(afull0 + (ss + 1) * 8, sph, abort_flag, p.status) &&
-             mbar_wait_warp(smem_u32(b_full + bs + 1), bph, abort_flag, p.status);
+        ok = mbar_wait_warp(afull0 + (ss + 1) * 8, sph, abort_flag, p.status) &&
+             mbar_wait_warp(smem_u32(b_full + bs / 2), bph, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t acol = a_col0 + ss * (uint32_t)C::A_COLS;
@@ -726,7 +761,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4 w0 = wv[2 * j], w1 = wv[2 * j + 1];
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dequant_word(ws[i], s2, b2, vals + 4 * i);
+            for (int i = 0; i < 8; ++i) {
+              // gate|up reads token rows the gather wrote in permuted order
+              if (EPI == EPI_SWIGLU) dequant_word_perm(ws[i], s2, b2, vals + 4 * i);
+              else dequant_word(ws[i], s2, b2, vals + 4 * i);
+            }
           } else {
             // bf16 weights: 32 elements of the k-block; fp16 operands for
             // the experts, bf16 kept as is for the router
@@ -842,7 +881,10 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ i
 
 // bf16 rows gathered into fp16: out[r][:] = fp16(x[row_map[r]][:]), one
 // block per sorted row (8 values per thread); values that do not round to a
-// finite fp16 are reported as MOE_ERR_RANGE (they become +-inf).
+// finite fp16 are reported as MOE_ERR_RANGE (they become +-inf). PERM stores
+// every 8 consecutive elements in the order (0, 4, 1, 5, 2, 6, 3, 7), the K
+// order of dequant_word_perm.
+template <bool PERM>
 __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict__ x,
                                                          const uint32_t* __restrict__ row_map,
                                                          int d8, uint4* __restrict__ out,
@@ -856,13 +898,19 @@ __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict
   for (int c = threadIdx.x; c < d8; c += blockDim.x) {
     const uint4 v = __ldg(src + c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[2 * j] = __uint_as_float(w[j] << 16);
+      f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
-      ok &= fabsf(a) < 65520.f && fabsf(b) < 65520.f;
+      const float lo = PERM ? f[j] : f[2 * j], hi = PERM ? f[j + 4] : f[2 * j + 1];
+      ok &= fabsf(lo) < 65520.f && fabsf(hi) < 65520.f;
       uint32_t dd;
-      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(dd) : "f"(b), "f"(a));
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(dd) : "f"(hi), "f"(lo));
       o[j] = dd;
     }
     dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -931,8 +979,13 @@ cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, cons
   if (R <= 0) return cudaSuccess;
   // the expert GEMMs take fp16 operands in row-sorted order: x gathered
   // through row_map and converted once into xs16 [R][d]
-  launch_pdl(gather_f16_kernel, (unsigned)R, 256, 0, s, (const uint4*)x, row_map, ex.d / 8,
-             (uint4*)xs16, status);
+  // q4 weights are dequantised in a permuted K order, so are the token rows
+  if (ex.fmt == MOE_W_Q4G64)
+    launch_pdl(gather_f16_kernel<true>, (unsigned)R, 256, 0, s, (const uint4*)x, row_map, ex.d / 8,
+               (uint4*)xs16, status);
+  else
+    launch_pdl(gather_f16_kernel<false>, (unsigned)R, 256, 0, s, (const uint4*)x, row_map, ex.d / 8,
+               (uint4*)xs16, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap ta;
