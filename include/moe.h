@@ -207,9 +207,11 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
  * issue #112, switch_linear with sorted indices).
  *   h        (device) [T*k][F]: fp16 for bf16 activations (dt = MOE_BF16),
  *            fp32 for fp32 -- as moe_grouped_swiglu writes it
- *   ys       (device, out) [T*k][d] fp32: ys[i][o] = h[i] . w_dn[e][o]
- *            (kept in fp32 so the only rounding after the expert matmuls is
- *            the final one of y) */
+ *   ys       (device, out) [T*k][d]: ys[i][o] = h[i] . w_dn[e][o], fp32
+ *            accumulation, stored in fp16 for bf16 activations (its 11-bit
+ *            rounding is far below the final bf16 rounding of y; values
+ *            outside fp16 range are reported as MOE_ERR_RANGE in the device
+ *            status) and in fp32 for fp32 activations */
 moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
                             const int32_t* tile_off, int BM, int T, int k,
                             const moe_experts* experts, void* ys, moe_regime regime,
@@ -219,7 +221,9 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
  * #112, _scatter_unsort; "5.5 real sparse MoE kernels (Metal)", scatter_add
  * equivalent): y[t][o] = sum_{j=0..k-1} w[t][j] * ys[inv_order[t*k+j]][o],
  * summed in fp32 in j order, rounded once to dt.
- *   ys (device) [T*k][d] fp32, inv_order (device) [T*k], topk_w (device) [T][k]
+ *   ys (device) [T*k][d]: fp16 for dt = MOE_BF16, fp32 for MOE_F32 (as
+ *      moe_grouped_down writes it); inv_order (device) [T*k];
+ *      topk_w (device) [T][k] fp32
  *   y  (device, out) [T][d], dtype dt */
 moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* topk_w, int T, int k,
                        int d, moe_dtype dt, void* y, moe_stream_t stream);

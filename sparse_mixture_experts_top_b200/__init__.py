@@ -208,12 +208,12 @@ def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, ws=Non
 
 
 def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, stream=None):
-    """-> ys [T*k, d] fp32"""
+    """-> ys [T*k, d]: fp16 for bf16 activations (fp16 h), fp32 for fp32"""
     _dev(h)
     ex = experts_struct(experts)
-    ys = torch.empty(T * k, experts.d, dtype=torch.float32, device=h.device)
-    # h is fp16 exactly when the activations are bf16
+    # h is fp16 exactly when the activations are bf16; ys has h's dtype
     adt = BF16 if h.dtype == torch.float16 else F32
+    ys = torch.empty(T * k, experts.d, dtype=h.dtype, device=h.device)
     _check(lib.moe_grouped_down(_ptr(h), adt, _ptr(tables.row_off), _ptr(tables.tile_off),
                                 tables.BM, T, k, ctypes.byref(ex), _ptr(ys), regime,
                                 _stream(stream)), "moe_grouped_down")
@@ -221,10 +221,11 @@ def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, strea
 
 
 def combine(ys, inv_order, topk_w, T, k, dtype=torch.bfloat16, stream=None):
-    """-> y [T, d] in `dtype` from fp32 ys [T*k, d]"""
+    """-> y [T, d] in `dtype` from ys [T*k, d] (fp16 for bf16 `dtype`, fp32 for fp32)"""
     _dev(ys, inv_order, topk_w)
-    if ys.dtype != torch.float32:
-        raise TypeError("ys must be float32")
+    want = torch.float16 if dtype == torch.bfloat16 else torch.float32
+    if ys.dtype != want:
+        raise TypeError(f"ys must be {want} for {dtype} outputs")
     d = ys.shape[1]
     y = torch.empty(T, d, dtype=dtype, device=ys.device)
     _check(lib.moe_combine(_ptr(ys), _ptr(inv_order), _ptr(topk_w), T, k, d,

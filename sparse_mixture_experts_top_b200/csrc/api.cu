@@ -101,7 +101,7 @@ static cudaError_t down_gemv(const void* h, int dt, const int32_t* roff, const i
                              int BM, int R, const moe_experts& ex, void* ys, int* stp,
                              cudaStream_t s) {
   if (gemv_q4_mma_ok(ex, dt, BM)) return launch_down_q4_mma(h, roff, toff, BM, R, ex, ys, stp, s);
-  return launch_down_gemv(h, dt, roff, toff, BM, R, ex, ys, s);
+  return launch_down_gemv(h, dt, roff, toff, BM, R, ex, ys, stp, s);
 }
 
 }  // namespace moe
@@ -306,7 +306,7 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.tile_off = take((size_t)(E + 1) * 4);
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
   L.h = take((size_t)R * F * a);      // fp16 (bf16 activations) or fp32
-  L.ys = take((size_t)R * d * 4);
+  L.ys = take((size_t)R * d * a);     // fp16 (bf16 activations) or fp32
   L.regime = resolve_regime(regime, R, E, dt, d, F);
   L.BM = block_m_for(L.regime, R, E);
   // fp16 token rows: x converted (weight-streaming) or gathered in sorted

@@ -11,10 +11,11 @@
 
 namespace moe {
 
-// One thread per 8 consecutive outputs of one token: k gathers of 32 bytes
-// of fp32 ys, fp32 fused multiply-adds in j order, one rounding to TA.
-template <typename TA>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ ys,
+// One thread per 8 consecutive outputs of one token: k gathers of 8 ys values
+// (fp16 for bf16 activations, fp32 for fp32), fp32 fused multiply-adds in j
+// order, one rounding to TA.
+template <typename TA, typename TY>
+__global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ ys,
                                                       const uint32_t* __restrict__ inv_order,
                                                       const float* __restrict__ w, int T, int k,
                                                       int d, TA* __restrict__ y) {
@@ -31,10 +32,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   for (int i = 0; i < V; ++i) acc[i] = 0.f;
   for (int j = 0; j < k; ++j) {
     const float wj = __ldg(w + (size_t)t * k + j);
-    const float* src = ys + (size_t)__ldg(inv_order + (size_t)t * k + j) * d + o;
-    const float4 a = *reinterpret_cast<const float4*>(src);
-    const float4 b = *reinterpret_cast<const float4*>(src + 4);
-    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const TY* src = ys + (size_t)__ldg(inv_order + (size_t)t * k + j) * d + o;
+    float v[8];
+    if constexpr (sizeof(TY) == 2) {
+      const uint4 a = *reinterpret_cast<const uint4*>(src);
+      const uint32_t u[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
+    } else {
+      const float4 a = *reinterpret_cast<const float4*>(src);
+      const float4 b = *reinterpret_cast<const float4*>(src + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
   }
@@ -58,11 +72,11 @@ cudaError_t launch_combine(const void* ys, const uint32_t* inv_order, const floa
   if (n == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (dt == MOE_BF16)
-    launch_pdl(combine_kernel<__nv_bfloat16>, blocks, 256, 0, s, (const float*)ys, inv_order, w, T, k, d,
-                                                         (__nv_bfloat16*)y);
+    launch_pdl(combine_kernel<__nv_bfloat16, __half>, blocks, 256, 0, s, (const __half*)ys,
+               inv_order, w, T, k, d, (__nv_bfloat16*)y);
   else
-    launch_pdl(combine_kernel<float>, blocks, 256, 0, s, (const float*)ys, inv_order, w, T, k, d,
-                                                 (float*)y);
+    launch_pdl(combine_kernel<float, float>, blocks, 256, 0, s, (const float*)ys, inv_order, w, T,
+               k, d, (float*)y);
   return cudaGetLastError();
 }
 

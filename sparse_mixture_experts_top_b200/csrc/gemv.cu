@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
     const typename HType<TA>::T* __restrict__ hin, const int32_t* __restrict__ row_off,
     const int32_t* __restrict__ tile_off, int BM, int E, int d, int F,
     const uint32_t* __restrict__ wdn, const uint16_t* __restrict__ sdn,
-    const uint16_t* __restrict__ bdn, float* __restrict__ ys) {
+    const uint16_t* __restrict__ bdn, typename HType<TA>::T* __restrict__ ys, int* status) {
   pdl_wait();
   pdl_launch();
   using D = WDecode<FMT>;
@@ -245,7 +245,15 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
 #pragma unroll
     for (int j = 0; j < kRowsPerPass; ++j) {
       const float v = warp_sum(acc[j]);
-      if (lane == 0 && j < nr) ys[(size_t)(rb + j) * d + o] = v;
+      if (lane == 0 && j < nr) {
+        if (sizeof(typename HType<TA>::T) == 2) {
+          // fp16 ys (bf16 activations): out-of-range values are reported
+          if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
+          reinterpret_cast<__half*>(ys)[(size_t)(rb + j) * d + o] = __float2half_rn(v);
+        } else {
+          reinterpret_cast<float*>(ys)[(size_t)(rb + j) * d + o] = v;
+        }
+      }
     }
   }
 }
@@ -276,7 +284,7 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
 
 cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
                              const int32_t* tile_off, int BM, int R, const moe_experts& ex,
-                             void* ys, cudaStream_t s) {
+                             void* ys, int* status, cudaStream_t s) {
   const long long tiles = max_tiles(R, ex.E, BM);
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 65535) return cudaErrorInvalidConfiguration;
@@ -287,7 +295,7 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
 #define MOE_DOWN(TA, FMT)                                                                    \
   launch_pdl(down_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const typename HType<TA>::T*)h, row_off,    \
                                                  tile_off, BM, ex.E, ex.d, ex.F, w, sc, bi,     \
-                                                 (float*)ys)
+                                                 (typename HType<TA>::T*)ys, status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_DOWN(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
@@ -487,9 +495,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
         if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
         reinterpret_cast<__half*>(out)[(size_t)(r0 + n) * F + blk * 8 + g] = __float2half_rn(v);
       } else {
-        float* ys = reinterpret_cast<float*>(out);
-        ys[(size_t)(r0 + n) * d + blk * 16 + g] = acc[t][j];
-        ys[(size_t)(r0 + n) * d + blk * 16 + 8 + g] = acc[t][2 + j];
+        // fp16 ys; out-of-range values are reported
+        const float v0 = acc[t][j], v1 = acc[t][2 + j];
+        if (!(fabsf(v0) < 65520.f && fabsf(v1) < 65520.f)) report_status(status, MOE_ERR_RANGE);
+        __half* ys = reinterpret_cast<__half*>(out);
+        ys[(size_t)(r0 + n) * d + blk * 16 + g] = __float2half_rn(v0);
+        ys[(size_t)(r0 + n) * d + blk * 16 + 8 + g] = __float2half_rn(v1);
       }
     }
   }

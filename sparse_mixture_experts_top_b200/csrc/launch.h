@@ -43,10 +43,10 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
                                const moe_experts& ex, void* h, int* status, cudaStream_t s);
 cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
                              const int32_t* tile_off, int BM, int R, const moe_experts& ex,
-                             void* ys, cudaStream_t s);
+                             void* ys, int* status, cudaStream_t s);
 
 // q4 weights with bf16 activations and at most 16 rows per tile: mma.sync
-// fp16 GEMV (x16: activations converted to fp16; h fp16 in, ys fp32 out).
+// fp16 GEMV (x16: activations converted to fp16; h fp16 in, ys fp16 out).
 bool gemv_q4_mma_ok(const moe_experts& ex, int dt, int BM);
 cudaError_t launch_swiglu_q4_mma(const void* x16, const uint32_t* row_map, const int32_t* row_off,
                                  const int32_t* tile_off, int BM, int R, const moe_experts& ex,

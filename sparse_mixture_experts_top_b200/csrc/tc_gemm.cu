@@ -70,7 +70,9 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kDqWarp0 = 8;
 constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at the B200's clocks
 
-enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };   // fp32 store adds p.bias when set
+// EPI_STORE: the router stores fp32 logits (+ p.bias when set), the down
+// projection fp16 ys
+enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
 
 template <int FMT>
 struct Cfg {
@@ -655,7 +657,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = qd * 32 + lane;                     // weight row of this thread
     const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
     uint32_t nb = 0, uses0 = 0, uses1 = 0;
-    bool range_ok = true;
+    // largest fp16 magnitude bits stored: 0x7C00 and above is inf or NaN,
+    // i.e. a value that did not round to a finite fp16
+    uint32_t hmax = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       int unit, r0, nv, e;
       decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
@@ -674,12 +678,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n0 = 0; n0 < nv; n0 += 16) {
           uint32_t a0[16], a1[16];
           tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
+          const int lim = nv - n0;        // columns of this chunk that are rows of the tile
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (n0 + j < nv) {
-              const float v = swiglu(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
-              range_ok &= fabsf(v) < 65520.f;    // rounds to a finite fp16
-              hp[(size_t)(n0 + j) * p.out_ld] = __float2half_rn(v);
+            const __half v = __float2half_rn(swiglu(__uint_as_float(a0[j]), __uint_as_float(a1[j])));
+            if (j < lim) {
+              hmax = max(hmax, (uint32_t)__half_as_ushort(v) & 0x7FFFu);
+              hp[(size_t)(n0 + j) * p.out_ld] = v;
             }
           }
         }
@@ -687,18 +692,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int orow0 = unit * p.unit_rows + m;
         const int orow1 = orow0 + BMW;
         const bool ok0 = orow0 < p.m_limit, ok1 = orow1 < p.m_limit;
-        const float bv0 = (ok0 && p.bias) ? __ldg(p.bias + orow0) : 0.f;
-        const float bv1 = (ok1 && p.bias) ? __ldg(p.bias + orow1) : 0.f;
-        float* op = reinterpret_cast<float*>(p.out) + (size_t)r0 * p.out_ld + orow0;
-        for (int n0 = 0; n0 < nv; n0 += 16) {
-          uint32_t a0[16], a1[16];
-          tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
+        if (ROUTER) {
+          const float bv0 = (ok0 && p.bias) ? __ldg(p.bias + orow0) : 0.f;
+          const float bv1 = (ok1 && p.bias) ? __ldg(p.bias + orow1) : 0.f;
+          float* op = reinterpret_cast<float*>(p.out) + (size_t)r0 * p.out_ld + orow0;
+          for (int n0 = 0; n0 < nv; n0 += 16) {
+            uint32_t a0[16], a1[16];
+            tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (n0 + j < nv) {
-              float* o = op + (size_t)(n0 + j) * p.out_ld;
-              if (ok0) o[0] = __uint_as_float(a0[j]) + bv0;
-              if (ok1) o[BMW] = __uint_as_float(a1[j]) + bv1;
+            for (int j = 0; j < 16; ++j) {
+              if (n0 + j < nv) {
+                float* o = op + (size_t)(n0 + j) * p.out_ld;
+                if (ok0) o[0] = __uint_as_float(a0[j]) + bv0;
+                if (ok1) o[BMW] = __uint_as_float(a1[j]) + bv1;
+              }
+            }
+          }
+        } else {
+          // the down projection's units are 256 whole rows of d (d % 256 == 0)
+          __half* op = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + orow0;
+          for (int n0 = 0; n0 < nv; n0 += 16) {
+            uint32_t a0[16], a1[16];
+            tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
+            const int lim = nv - n0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const __half v0 = __float2half_rn(__uint_as_float(a0[j]));
+              const __half v1 = __float2half_rn(__uint_as_float(a1[j]));
+              if (j < lim) {
+                hmax = max(hmax, max((uint32_t)__half_as_ushort(v0) & 0x7FFFu,
+                                     (uint32_t)__half_as_ushort(v1) & 0x7FFFu));
+                __half* o = op + (size_t)(n0 + j) * p.out_ld;
+                o[0] = v0;
+                o[BMW] = v1;
+              }
             }
           }
         }
@@ -713,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (use1) ++uses1;
       if (small) nb ^= 1u;
     }
-    if (!__all_sync(0xffffffffu, range_ok) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
+    if (!__all_sync(0xffffffffu, hmax < 0x7C00u) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------ dequant
     // 16 warps: (matrix q, lane quadrant qd, half hf). q4: half hf converts
@@ -879,23 +906,26 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ i
   if (!__all_sync(0xffffffffu, ok) && (threadIdx.x & 31) == 0) report_status(status, MOE_ERR_RANGE);
 }
 
-// bf16 rows gathered into fp16: out[r][:] = fp16(x[row_map[r]][:]), one
-// block per sorted row (8 values per thread); values that do not round to a
+// bf16 rows gathered into fp16: out[r][:] = fp16(x[row_map[r]][:]), four
+// sorted rows per block (8 values per thread per load); values that do not round to a
 // finite fp16 are reported as MOE_ERR_RANGE (they become +-inf). PERM stores
 // every 8 consecutive elements in the order (0, 4, 1, 5, 2, 6, 3, 7), the K
 // order of dequant_word_perm.
 template <bool PERM>
 __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict__ x,
                                                          const uint32_t* __restrict__ row_map,
-                                                         int d8, uint4* __restrict__ out,
-                                                         int* status) {
+                                                         long long R, int d8,
+                                                         uint4* __restrict__ out, int* status) {
   pdl_wait();
   pdl_launch();
-  const long long r = blockIdx.x;
+  // 4 rows per block, 64 threads per row, 4 loads in flight per thread
+  const long long r = (long long)blockIdx.x * 4 + (threadIdx.x >> 6);
+  if (r >= R) return;
   const uint4* src = x + (size_t)__ldg(row_map + r) * d8;
   uint4* dst = out + (size_t)r * d8;
   bool ok = true;
-  for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+#pragma unroll 4
+  for (int c = threadIdx.x & 63; c < d8; c += 64) {
     const uint4 v = __ldg(src + c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float f[8];
@@ -915,7 +945,7 @@ __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict
     }
     dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  if (!__all_sync(0xffffffffu, ok) && (threadIdx.x & 31) == 0) report_status(status, MOE_ERR_RANGE);
+  if (!ok) report_status(status, MOE_ERR_RANGE);
 }
 
 // The token-row maps of Params: [rows][K] 16-bit elements, one map per tile
@@ -980,12 +1010,13 @@ cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, cons
   // the expert GEMMs take fp16 operands in row-sorted order: x gathered
   // through row_map and converted once into xs16 [R][d]
   // q4 weights are dequantised in a permuted K order, so are the token rows
+  const unsigned gblocks = (unsigned)((R + 3) / 4);
   if (ex.fmt == MOE_W_Q4G64)
-    launch_pdl(gather_f16_kernel<true>, (unsigned)R, 256, 0, s, (const uint4*)x, row_map, ex.d / 8,
-               (uint4*)xs16, status);
+    launch_pdl(gather_f16_kernel<true>, gblocks, 256, 0, s, (const uint4*)x, row_map, (long long)R,
+               ex.d / 8, (uint4*)xs16, status);
   else
-    launch_pdl(gather_f16_kernel<false>, (unsigned)R, 256, 0, s, (const uint4*)x, row_map, ex.d / 8,
-               (uint4*)xs16, status);
+    launch_pdl(gather_f16_kernel<false>, gblocks, 256, 0, s, (const uint4*)x, row_map, (long long)R,
+               ex.d / 8, (uint4*)xs16, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap ta;
@@ -1039,8 +1070,8 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.m_limit = ex.d;
   p.status = status;
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE_F32, false>(p, ta, ub, s);
-  return run<MOE_W_BF16, EPI_STORE_F32, false>(p, ta, ub, s);
+  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE, false>(p, ta, ub, s);
+  return run<MOE_W_BF16, EPI_STORE, false>(p, ta, ub, s);
 }
 
 cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const float* bias, int T,
@@ -1067,7 +1098,7 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
   p.bias = bias;
   p.status = status;
   const long long ub = (long long)((T + BN - 1) / BN) * p.n_units;
-  return run<MOE_W_BF16, EPI_STORE_F32, true>(p, ta, ub, s);
+  return run<MOE_W_BF16, EPI_STORE, true>(p, ta, ub, s);
 }
 
 }  // namespace moe

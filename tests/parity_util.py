@@ -100,14 +100,18 @@ def assert_h_close(h_gpu, href, g, u, ga, ua, d, u_w, u_h, tol, what=""):
     return float(err.max()) / max(rms(href), 1e-300)
 
 
-def assert_ys_close(ys_gpu, yref, habs, u_w, tol, what=""):
-    """ys = h . W_d^T kept in fp32: weights rounded to the operand format
-    (unit roundoff u_w) add at most u_w * sum |h w|."""
+def assert_ys_close(ys_gpu, yref, habs, u_w, tol, what="", u_ys=0.0):
+    """ys = h . W_d^T accumulated in fp32: weights rounded to the operand
+    format (unit roundoff u_w) add at most u_w * sum |h w|; storing ys in a
+    format of unit roundoff u_ys adds u_ys * |ys| (+ half its smallest
+    subnormal step, 2^-25 for fp16)."""
     g = to_np(ys_gpu).astype(np.float64)
     assert g.shape == yref.shape and np.isfinite(g).all(), what
     if yref.size == 0:
         return 0.0
     bound = tol * rms(yref) + u_w * habs
+    if u_ys:
+        bound = bound + u_ys * np.abs(yref) + 2.0 ** -25
     err = np.abs(g - yref)
     i = int(np.argmax(err - bound))
     assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "

@@ -179,10 +179,12 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
     ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
     hx = _host(layer.experts)
     yref = orc.expert_down(hin.double().numpy(), ref_st.row_off, hx)
-    assert ys.dtype == torch.float32
+    # ys is stored in fp16 for bf16 activations, fp32 for fp32
+    assert ys.dtype == (torch.float16 if wl.act == "bf16" else torch.float32)
     habs = orc.expert_down_abs(hin.double().numpy(), ref_st.row_off, hx)
     u_w = U_F16 if wl.wfmt == "q4" else 0.0
-    assert_ys_close(ys, yref, habs, u_w, _tol(wl.act), f"ys[{name}]")
+    u_ys = U_F16 if wl.act == "bf16" else 0.0
+    assert_ys_close(ys, yref, habs, u_w, _tol(wl.act), f"ys[{name}]", u_ys=u_ys)
 
 
 @pytest.mark.parametrize("T,k,d,dt", [(1, 8, 2048, torch.bfloat16), (16, 2, 128, torch.float32),
@@ -191,7 +193,9 @@ def test_combine_parity(moe, orc, T, k, d, dt):
     E = max(k, 16)
     idx = mi.random_topk_idx(T, E, k, seed=31)
     st = orc.sort_rows(idx.numpy(), E, 8)
-    ys = mi.random_ys(T * k, d, seed=32, dtype=torch.float32)
+    # ys arrive in fp16 for bf16 outputs, fp32 for fp32
+    ys = mi.random_ys(T * k, d, seed=32,
+                      dtype=torch.float16 if dt == torch.bfloat16 else torch.float32)
     w = mi.random_weights(T, k, seed=33)
     inv = torch.from_numpy(st.inv_order.view(np.int32)).view(torch.uint32)
     y = moe.combine(ys.to(DEV), inv.to(DEV), w.to(DEV), T, k, dtype=dt)
