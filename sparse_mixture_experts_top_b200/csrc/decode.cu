@@ -228,8 +228,10 @@ __device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile
 // acc[0..1] row a for tokens 2c, 2c+1, acc[2..3] row b. Inside the 16-wide
 // K slice m of a 128-element step, fragment columns (2c, 2c+1, 2c+8, 2c+9)
 // are elements c*32 + 4m + (0..3) for A and B alike, so both come from
-// contiguous loads. The token rows come through L2 (another CTA may have
-// written them in this launch); PD steps of them are in flight at once.
+// contiguous loads. The token rows were written earlier in this launch (by
+// any CTA, before a grid barrier) and are not written again, so plain loads
+// may keep them in L1 -- every item of a token reads the same rows -- but
+// the read-only path may not; PD steps of them are in flight at once.
 template <int PD>
 __device__ __forceinline__ void warp_mma_rows16(const uint32_t* wa, const uint32_t* wb,
                                                 const uint16_t* sa, const uint16_t* ba,
@@ -249,8 +251,7 @@ __device__ __forceinline__ void warp_mma_rows16(const uint32_t* wa, const uint32
     const int k0 = st * 128 + c * 32;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      v[i] = xvalid ? __ldcg(reinterpret_cast<const uint4*>(xrow + k0 + i * 8))
-                    : make_uint4(0, 0, 0, 0);
+      v[i] = xvalid ? *reinterpret_cast<const uint4*>(xrow + k0 + i * 8) : make_uint4(0, 0, 0, 0);
   };
   auto step = [&](const uint4 (&v)[4], int st) {
     const int k0 = st * 128 + c * 32;
@@ -291,12 +292,11 @@ __device__ __forceinline__ void warp_mma_rows16(const uint32_t* wa, const uint32
   for (int j = 0; j < 4; ++j) acc[j] += (ch[0][j] + ch[1][j]) + (ch[2][j] + ch[3][j]);
 }
 
-// Top-k of tokens warp, warp + kCw, ... (at most kMaxT / kCw per warp, all
-// at once) from the logits in global memory; results into shared memory.
-template <int VPL>
+// Top-k of tokens warp, warp + kCw, ... (at most TPW per warp, all at once)
+// from the logits in global memory; results into shared memory.
+template <int VPL, int TPW>
 __device__ __forceinline__ void topk_tokens(const Params& p, int warp, int lane, int* s_idx,
                                             float* s_w) {
-  constexpr int TPW = kMaxT / kCw;
   const int E = p.E, k = p.k;
   unsigned long long key[TPW][VPL];
   int my_e[TPW];
@@ -451,8 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // the lowest index among equal logits; weights exp(L - Lmax) / sum. A warp
   // takes tokens w, w + 8, w + 16, w + 24 together (independent chains).
   if (ok && warp < kCw) {
-    if (E <= 128) topk_tokens<4>(p, warp, lane, s_idx, s_w);
-    else topk_tokens<kMaxE / 32>(p, warp, lane, s_idx, s_w);
+    if (T <= kCw) {
+      if (E <= 128) topk_tokens<4, 1>(p, warp, lane, s_idx, s_w);
+      else topk_tokens<kMaxE / 32, 1>(p, warp, lane, s_idx, s_w);
+    } else {
+      if (E <= 128) topk_tokens<4, kMaxT / kCw>(p, warp, lane, s_idx, s_w);
+      else topk_tokens<kMaxE / 32, kMaxT / kCw>(p, warp, lane, s_idx, s_w);
+    }
   }
   __syncthreads();
   // stable counting sort of the routed rows by expert (all CTAs alike), by
