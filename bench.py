@@ -119,11 +119,13 @@ def gate_up_bytes(ex) -> int:
     return tot
 
 
-def kernels_per_forward(T, k, regime_tc: bool) -> int:
+def kernels_per_forward(T, k, regime_tc: bool, fused_decode: bool = False) -> int:
+    if fused_decode:
+        return 1                      # the whole layer in one cooperative kernel
     R = T * k
     sort = 1 if R <= 1024 else 3
-    conv = 1 if regime_tc else 0   # x -> fp16 for the tensor-core expert GEMMs
-    return 2 + sort + conv + 2 + 1   # router + top-k, sort, [x16], gate|up, down, combine
+    conv = 1                          # x -> fp16 (gathered for the tensor cores)
+    return 2 + sort + conv + 2 + 1    # router + top-k, sort, x16, gate|up, down, combine
 
 
 # ------------------------------------------------------------------ timing
