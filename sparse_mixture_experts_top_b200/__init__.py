@@ -55,7 +55,7 @@ class WsLayout(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m sparse_mixture_experts_top_b200.build` (needs nvcc)")
+                          "`python sparse_mixture_experts_top_b200/build.py` (needs nvcc)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.moe_route.argtypes = [P, I, P, P, I, I, I, I, P, P, P, P]

@@ -19,8 +19,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def moe():
-    from sparse_mixture_experts_top_b200 import build as b
-    b.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import sparse_mixture_experts_top_b200 as m
     return m
 
