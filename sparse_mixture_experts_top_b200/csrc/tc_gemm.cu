@@ -436,6 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;                               // [2] one per issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // one scratch word per warp (see the dequant role)
+  const uint32_t sink = smem_u32(bar_area + 512);
   int* s_toff = reinterpret_cast<int*>(bar_area + 1024);
   int* s_roff = s_toff + kMaxE + 1;
   // q4 scale ring: raw stage rs holds scales [2][128][4] then biases [2][128][4]
@@ -775,6 +777,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc) : "r"(so));
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bi) : "r"(so + C::SCL_BYTES / 2));
         }
+        // A shared-memory load has read its data only once an instruction has
+        // consumed its destination registers; until then the next TMA into
+        // this stage can overwrite rows the load has not read yet (seen on
+        // the first rows the TMA writes). So the loaded words are folded into
+        // one value stored to a scratch word before the stage is released.
+        uint32_t fold = sc ^ bi;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) fold ^= wv[c].x ^ wv[c].y ^ wv[c].z ^ wv[c].w;
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(sink + 4u * (uint32_t)warp), "r"(fold)
+                     : "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
 #pragma unroll
