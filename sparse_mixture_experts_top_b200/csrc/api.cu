@@ -369,10 +369,10 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
 
   cudaError_t e = cudaErrorNotSupported;
   // few tokens: the whole layer in one cooperative launch (its grid barrier
-  // counter lives in the ys region, which that path does not use)
+  // counter lives in the sort scratch, which that path does not use)
   if (regime_run == MOE_REGIME_GEMV && decode_fused_ok(T, k, E, d, F, experts->fmt, dt)) {
     e = launch_decode_fused(x, w_router, router_bias, *experts, T, k, L.BM, logits, idx, w, order,
-                            inv, rmap, counts, roff, toff, x16, h, y, (unsigned*)ys, stp, s);
+                            inv, rmap, counts, roff, toff, x16, h, ys, y, (unsigned*)sws, stp, s);
     if (e != cudaErrorNotSupported) return launched(e);
   }
   if (dt == MOE_BF16) e = launch_router_logits_tc(x, w_router, router_bias, T, d, E, logits, stp, s);

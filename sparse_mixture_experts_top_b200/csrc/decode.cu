@@ -5,24 +5,31 @@
 // of launches; DS4Server issue #112 keeps the weight-streaming kernels for
 // T*k/E small. On the B200 one thread block cannot stream the selected
 // experts' weights fast enough, so this is one *cooperative* launch of one
-// CTA per SM with two grid-wide barriers:
+// CTA per SM with three grid-wide barriers:
 //
-//   phase A  router logits x . W_r^T + b (one expert per CTA, one warp per
-//            token) and x converted to fp16 (shared by all CTAs)
+//   phase A  router logits x . W_r^T + b (a warp per expert and token) and x
+//            converted to fp16 (shared by all CTAs)
 //   -- grid barrier --
-//   phase B  every CTA repeats the top-k of all tokens (warp max of
-//            orderable keys, lowest expert index first on ties) and the
-//            stable counting sort of the T*k routed rows in shared memory
-//            (CTA 0 writes the tables to the workspace); then gate|up + SwiGLU:
-//            a work item is 8 features of one active expert (its 8 gate and
-//            8 up weight rows), one warp per item, mma.sync m16n8k16 fp16
-//            with fp32 accumulation; h goes to global memory in fp16
+//   phase B  every CTA repeats the top-k of all tokens (one warp per token,
+//            two warp reductions per selected expert, lowest expert index
+//            first on ties) and the stable counting sort of the T*k routed
+//            rows in shared memory; then gate|up + SwiGLU: a work item is 8
+//            features of one active expert (its 8 gate and 8 up weight rows)
 //   -- grid barrier --
-//   phase C  down + combine: a work item is 16 output features; its warps
-//            take the active experts in turn, multiply their h rows by the
-//            16 weight rows and add w[t][j] * ys into per-warp partial sums
-//            in shared memory, which are then added in warp order: no
-//            atomics, deterministic
+//   phase C  down: a work item is 16 output features of one active expert,
+//            written to ys (fp16, sorted row order)
+//   -- grid barrier --
+//   phase D  combine: y[t] = sum over j of w[t][j] * ys[inv_order[t*k + j]]
+//            in j order, one thread per 8 outputs: no atomics, deterministic
+//
+// Each CTA takes a contiguous range of the gate|up items and of the down
+// items (expert-major), so consecutive items share an expert and its token or
+// h rows stay in L1. The compute warps form groups of four. A group takes one
+// work item at a time and splits its K range: warp i of the group multiplies
+// the 128-wide K steps i, i + 4, ... (mma.sync m16n8k16, fp16 operands, fp32
+// accumulation), so an item's latency is a quarter of one warp's, and every
+// warp of the SM has work even when the SM has only a few items. The four
+// partial accumulators are added in group order through shared memory.
 //
 // The weight rows of every item are streamed by a producer warp with 1-D bulk
 // copies (cp.async.bulk) into a ring of shared-memory slots, so each SM keeps
@@ -30,6 +37,10 @@
 // its CTA (it repeats the same computation) and prefetches phase C's weights
 // while phase B still runs. Every wait is bounded (~1 s): on expiry the status
 // word gets MOE_ERR_TIMEOUT and the kernel returns.
+//
+// The fp16 token rows (x16) and h are stored with every 8 consecutive elements
+// in the order (0,4,1,5,2,6,3,7): the K order in which the dequantisation
+// produces weight pairs. ys, y and the tables have their plain layouts.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -38,14 +49,21 @@
 namespace moe {
 namespace dec {
 
-constexpr int kCw = 8;                        // compute warps
+constexpr int kCw = 16;                       // compute warps
+constexpr int kGw = 4;                        // warps per group (K split)
+constexpr int kNg = kCw / kGw;                // groups
 constexpr int kThreads = (kCw + 1) * 32;      // + the producer warp
 constexpr int kMaxT = 32;                     // tokens
 constexpr int kMaxR = 256;                    // routed rows T*k
-constexpr int kMaxE = 256;                    // experts (top-k keeps E/32 keys per lane)
-constexpr int kSlots = 10;                    // weight ring slots (>= kCw)
+constexpr int kMaxE = 256;                    // experts (top-k keeps E/32 logits per lane)
+constexpr int kSlots = 10;                    // weight ring slots
 constexpr int kSlotBytes = 18 * 1024;         // gate|up item: 16 KB of words + 2 KB scales
+constexpr int kTg = 8;                        // tokens per router work unit (one W_r row read)
 constexpr long long kWaitCycles = 2000000000LL;
+
+// shared memory after the ring: the groups' partial accumulators (double
+// buffered per group)
+constexpr int kRedBytes = 2 * kNg * kGw * 32 * 4 * 4;
 
 struct Params {
   const __nv_bfloat16* x;                     // [T][d]
@@ -69,6 +87,7 @@ struct Params {
   int32_t* tile_off;                          // [E+1]
   __half* x16;                                // [T][d]
   __half* h;                                  // [R][F]
+  __half* ys;                                 // [R][d], sorted row order
   __nv_bfloat16* y;                           // [T][d]
   unsigned* sync;                             // grid barrier counter, zero before launch
   int* status;
@@ -101,8 +120,8 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // bounded wait; false when it ran out or (honor_abort) the kernel is aborting
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, bool honor_abort = true) {
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int* status, bool honor_abort = true) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
@@ -147,28 +166,24 @@ __device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-// a bf16 value (low 16 bits) as an fp16 pair holding it twice
-__device__ __forceinline__ uint32_t h2_from_bf16(uint32_t v16) {
-  const float f = __uint_as_float(v16 << 16);
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(f));
-  return d;
-}
-// 8 nibbles of one word -> fp16 pairs (e0,e1) (e2,e3) (e4,e5) (e6,e7) of
-// s*q + b, rounded once: q goes into the mantissa of fp16 1024.0 (exact),
-// 1024 is subtracted exactly, one fused multiply-add applies scale and bias
-__device__ __forceinline__ void q4_word_f16(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* o) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-  const uint32_t p0 = __byte_perm(lo, hi, 0x5140), p1 = __byte_perm(lo, hi, 0x7362);
-  const uint32_t M = 0x64646464u, c1024 = 0x64006400u;
-  o[0] = h2_fma(h2_sub(__byte_perm(p0, M, 0x4140), c1024), s2, b2);
-  o[1] = h2_fma(h2_sub(__byte_perm(p0, M, 0x4342), c1024), s2, b2);
-  o[2] = h2_fma(h2_sub(__byte_perm(p1, M, 0x4140), c1024), s2, b2);
-  o[3] = h2_fma(h2_sub(__byte_perm(p1, M, 0x4342), c1024), s2, b2);
+// 8 nibbles of one word -> fp16 pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7) of
+// s*q + b, rounded once. Nibbles 0 and 4 (bits 0-3, 16-19) are ORed into the
+// mantissa of fp16 1024.0, whose last place is 1; nibbles 1 and 5 (bits 4-7,
+// 20-23) into that of fp16 64.0, whose last place is 1/16, so both pairs
+// read magic + q; the word shifted by 8 gives nibbles 2, 6 and 3, 7 the same
+// way. The magic is subtracted exactly and one fused multiply-add applies
+// scale and bias: 5 integer and 8 fp16 operations per 8 weights.
+__device__ __forceinline__ void q4_word_perm(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* o) {
+  const uint32_t c1024 = 0x64006400u, c64 = 0x54005400u;
+  const uint32_t w8 = w >> 8;
+  o[0] = h2_fma(h2_sub((w & 0x000F000Fu) | c1024, c1024), s2, b2);
+  o[1] = h2_fma(h2_sub((w & 0x00F000F0u) | c64, c64), s2, b2);
+  o[2] = h2_fma(h2_sub((w8 & 0x000F000Fu) | c1024, c1024), s2, b2);
+  o[3] = h2_fma(h2_sub((w8 & 0x00F000F0u) | c64, c64), s2, b2);
 }
 
 // Orderable 32-bit image of a float: larger float -> larger key; -0 -> +0;
-// NaN -> 0 (below -inf)
+// NaN -> 0 (below -inf, whose key is 0x007FFFFF)
 __device__ __forceinline__ uint32_t order_key(float v) {
   if (v == 0.0f) v = 0.0f;
   const uint32_t u = __float_as_uint(v);
@@ -176,30 +191,38 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w > v ? w : v;
-  }
-  return v;
-}
-
 // named barrier of the compute warps (the producer warp keeps streaming)
 __device__ __forceinline__ void compute_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kCw * 32) : "memory");
+}
+// named barrier of one group's four warps, returning whether `ok` holds in
+// all of them (so a group leaves a loop together)
+__device__ __forceinline__ bool group_sync_and(int grp, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(2 + grp), "r"(kGw * 32)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void group_sync(int grp) {
+  asm volatile("bar.sync %0, %1;" ::"r"(2 + grp), "r"(kGw * 32) : "memory");
 }
 
 // Grid-wide barrier of the compute warps of all CTAs: a counter that only
 // grows (zeroed before the launch); barrier n waits for n * gridDim.x
 // arrivals. Bounded: on expiry the status gets MOE_ERR_TIMEOUT.
-__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile int* abort_flag,
-                                             int* status) {
+__device__ __noinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile int* abort_flag,
+                                          int* status) {
   compute_sync();
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1u);
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
     const unsigned target = n * gridDim.x;
     const long long t0 = clock64();
     int ok = 1;
@@ -214,155 +237,169 @@ __device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile
         break;
       }
     }
-    __threadfence();
     s_ok = ok;
   }
   compute_sync();
   return s_ok != 0;
 }
 
-// One warp, 16 weight rows in shared memory (rows g of group `a` and of
-// group `b` for lane (g, c): the m16 A rows g and g + 8), K elements, against
-// one group of 8 token rows read from global memory (this lane's row `xrow`,
-// zero when !xvalid). mma.sync m16n8k16 fp16, fp32 accumulation into acc:
-// acc[0..1] row a for tokens 2c, 2c+1, acc[2..3] row b. Inside the 16-wide
-// K slice m of a 128-element step, fragment columns (2c, 2c+1, 2c+8, 2c+9)
-// are elements c*32 + 4m + (0..3) for A and B alike, so both come from
-// contiguous loads. The token rows were written earlier in this launch (by
-// any CTA, before a grid barrier) and are not written again, so plain loads
-// may keep them in L1 -- every item of a token reads the same rows -- but
-// the read-only path may not; PD steps of them are in flight at once.
-template <int PD>
-__device__ __forceinline__ void warp_mma_rows16(const uint32_t* wa, const uint32_t* wb,
-                                                const uint16_t* sa, const uint16_t* ba,
-                                                const uint16_t* sb, const uint16_t* bb,
-                                                const __half* xrow, bool xvalid, int K, int c,
-                                                float* acc) {
-  const int nst = K / 128;
-  uint4 xq[PD][4];
-  // four independent accumulator chains (K slice m goes to chain m % 4),
-  // added at the end: one chain would serialise the 8 MMAs of a step
-  float ch[4][4];
+// One warp, 16 weight rows in shared memory (row g of matrix `a` and of
+// matrix `b` for lane (g, c): the m16 A rows g and g + 8), against one group
+// of 8 token rows read from global memory (this lane's row `xrow`, zero when
+// !xvalid), over the 128-wide K steps st0, st0 + kGw, ... < nst. mma.sync
+// m16n8k16 fp16, fp32 accumulation into acc: acc[0..1] row a for tokens 2c,
+// 2c+1, acc[2..3] row b.
+//
+// K order: lane c takes elements 32c .. 32c + 31 of a step, four q4 words
+// per row, whose scale and bias are those of group 2 st + c / 2. Word j gives
+// the fp16 pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7); K slice 2j of the step
+// takes the first two as fragment columns (2c, 2c+1) and (2c+8, 2c+9), slice
+// 2j + 1 the last two. The token rows are stored with every 8 consecutive
+// elements in the order (0,4,1,5,2,6,3,7), so one 16-byte load holds the
+// matching B fragments of one word. The token rows were written earlier in
+// this launch (by any CTA, before a grid barrier) and are not written again,
+// so plain loads may keep them in L1 -- the items of an expert read the same
+// rows -- but the read-only path may not. Two steps of them are in flight.
+__device__ __forceinline__ void warp_mma_steps(const uint8_t* wa, const uint8_t* wb,
+                                               const uint16_t* sa, const uint16_t* ba,
+                                               const uint16_t* sb, const uint16_t* bb,
+                                               const __half* xrow, bool xvalid, int st0, int nst,
+                                               int c, float* acc) {
+  float ch[2][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) ch[i][j] = 0.f;
+  uint4 xq[2][4];
   auto load = [&](uint4 (&v)[4], int st) {
-    const int k0 = st * 128 + c * 32;
+    const uint4* src = reinterpret_cast<const uint4*>(xrow + st * 128 + c * 32);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      v[i] = xvalid ? *reinterpret_cast<const uint4*>(xrow + k0 + i * 8) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 4; ++i) v[i] = xvalid ? src[i] : make_uint4(0, 0, 0, 0);
   };
   auto step = [&](const uint4 (&v)[4], int st) {
-    const int k0 = st * 128 + c * 32;
-    const uint4 wl = *reinterpret_cast<const uint4*>(wa + k0 / 8);
-    const uint4 wh = *reinterpret_cast<const uint4*>(wb + k0 / 8);
-    const int grp = k0 / 64;
-    const uint32_t sl = h2_from_bf16(sa[grp]), bl = h2_from_bf16(ba[grp]);
-    const uint32_t sh = h2_from_bf16(sb[grp]), bh = h2_from_bf16(bb[grp]);
-    const uint32_t wlw[4] = {wl.x, wl.y, wl.z, wl.w};
-    const uint32_t whw[4] = {wh.x, wh.y, wh.z, wh.w};
+    const uint4 wl = *reinterpret_cast<const uint4*>(wa + st * 64 + c * 16);
+    const uint4 wh = *reinterpret_cast<const uint4*>(wb + st * 64 + c * 16);
+    const int grp = 2 * st + (c >> 1);
+    // scales and biases of rows a and b as fp16 pairs (value, value)
+    uint32_t s2, b2;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+        : "=r"(s2)
+        : "f"(__uint_as_float((uint32_t)sb[grp] << 16)),
+          "f"(__uint_as_float((uint32_t)sa[grp] << 16)));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+        : "=r"(b2)
+        : "f"(__uint_as_float((uint32_t)bb[grp] << 16)),
+          "f"(__uint_as_float((uint32_t)ba[grp] << 16)));
+    const uint32_t sl = __byte_perm(s2, 0, 0x1010), sh = __byte_perm(s2, 0, 0x3232);
+    const uint32_t bl = __byte_perm(b2, 0, 0x1010), bh = __byte_perm(b2, 0, 0x3232);
+    const uint32_t wlw[4] = {wl.x, wl.y, wl.z, wl.w}, whw[4] = {wh.x, wh.y, wh.z, wh.w};
 #pragma unroll
-    for (int qw = 0; qw < 4; ++qw) {            // word qw: K slices m = 2qw, 2qw + 1
+    for (int j = 0; j < 4; ++j) {
       uint32_t dl[4], dh[4];
-      q4_word_f16(wlw[qw], sl, bl, dl);
-      q4_word_f16(whw[qw], sh, bh, dh);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t av[4] = {dl[2 * half], dh[2 * half], dl[2 * half + 1], dh[2 * half + 1]};
-        const uint4 x = v[qw];                  // slice m = 2qw + half: words 2m, 2m + 1
-        mma_16816(ch[(2 * qw + half) & 3], av, half ? x.z : x.x, half ? x.w : x.y);
-      }
+      q4_word_perm(wlw[j], sl, bl, dl);
+      q4_word_perm(whw[j], sh, bh, dh);
+      const uint32_t a0[4] = {dl[0], dh[0], dl[1], dh[1]};
+      const uint32_t a1[4] = {dl[2], dh[2], dl[3], dh[3]};
+      mma_16816(ch[0], a0, v[j].x, v[j].y);
+      mma_16816(ch[1], a1, v[j].z, v[j].w);
     }
   };
-#pragma unroll
-  for (int i = 0; i < PD; ++i)
-    if (i < nst) load(xq[i], i);
-  for (int st0 = 0; st0 < nst; st0 += PD) {
-#pragma unroll
-    for (int i = 0; i < PD; ++i) {
-      const int st = st0 + i;
-      if (st < nst) {
-        step(xq[i], st);
-        if (st + PD < nst) load(xq[i], st + PD);
-      }
+  int st = st0;
+  if (st < nst) load(xq[0], st);
+  if (st + kGw < nst) load(xq[1], st + kGw);
+#pragma unroll 1
+  for (; st < nst; st += 2 * kGw) {
+    step(xq[0], st);
+    if (st + 2 * kGw < nst) load(xq[0], st + 2 * kGw);
+    if (st + kGw < nst) {
+      step(xq[1], st + kGw);
+      if (st + 3 * kGw < nst) load(xq[1], st + 3 * kGw);
     }
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) acc[j] += (ch[0][j] + ch[1][j]) + (ch[2][j] + ch[3][j]);
+  for (int j = 0; j < 4; ++j) acc[j] = ch[0][j] + ch[1][j];
 }
 
-// Top-k of tokens warp, warp + kCw, ... (at most TPW per warp, all at once)
-// from the logits in global memory; results into shared memory.
-template <int VPL, int TPW>
-__device__ __forceinline__ void topk_tokens(const Params& p, int warp, int lane, int* s_idx,
-                                            float* s_w) {
-  const int E = p.E, k = p.k;
-  unsigned long long key[TPW][VPL];
-  int my_e[TPW];
+// Top-k of one token by one warp, from its logits row in global memory;
+// results into shared memory. Lane l holds the logits of experts l, l + 32,
+// ...; each of the k rounds takes the lane's best remaining expert (largest
+// key, the lowest index among equal keys), the warp maximum of those keys,
+// and the lowest expert index among the lanes that hold it. The weights are
+// exp(L_j - L_max) / sum over the selected, in the lane order of a warp sum.
+__device__ __noinline__ void topk_token(const float* row, int E, int k, int lane, int* idx_out,
+                                        float* w_out) {
+  constexpr int VPL = kMaxE / 32;
+  uint32_t key[VPL];
+  float val[VPL];
+  uint32_t avail = 0;
 #pragma unroll
-  for (int q = 0; q < TPW; ++q) {
-    const int t = warp + q * kCw;
-    const float* row = p.logits + (size_t)(t < p.T ? t : 0) * E;
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    val[i] = e < E ? __ldcg(row + e) : 0.f;
+    key[i] = order_key(val[i]);
+    if (e < E) avail |= 1u << i;
+  }
+  int my_e = 0;
+  float my_v = 0.f;
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0;
+    int bi = -1;
+    float bv = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
-      key[q][i] = (t < p.T && e < E) ? (((unsigned long long)order_key(__ldcg(row + e)) << 32) |
-                                        (0xFFFFFFFFu - (uint32_t)e))
-                                     : 0ull;
+      if (((avail >> i) & 1u) && (bi < 0 || key[i] > bk)) {
+        bk = key[i];
+        bi = i;
+        bv = val[i];
+      }
     }
-    my_e[q] = -1;
-  }
-  for (int j = 0; j < k; ++j) {
-#pragma unroll
-    for (int q = 0; q < TPW; ++q) {
-      unsigned long long best = 0ull;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) best = key[q][i] > best ? key[q][i] : best;
-      best = warp_max_u64(best);
-      const int e = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
-      if (lane == j) my_e[q] = e;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (lane + 32 * i == e) key[q][i] = 0ull;
+    const uint32_t M = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
+    const uint32_t ce = (bi >= 0 && bk == M) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
+    const uint32_t es = __reduce_min_sync(0xffffffffu, ce);
+    const float v = __shfl_sync(0xffffffffu, bv, (int)(es & 31u));
+    if ((int)(es & 31u) == lane) avail &= ~(1u << (es >> 5));
+    if (lane == j) {
+      my_e = (int)es;
+      my_v = v;
     }
   }
-#pragma unroll
-  for (int q = 0; q < TPW; ++q) {
-    const int t = warp + q * kCw;
-    if (t >= p.T) continue;
-    const float* row = p.logits + (size_t)t * E;
-    const float m = __ldcg(row + __shfl_sync(0xffffffffu, my_e[q], 0));
-    const float ex = lane < k ? __expf(__ldcg(row + my_e[q]) - m) : 0.f;
-    const float den = warp_sum(ex);
-    if (lane < k) {
-      s_idx[t * k + lane] = my_e[q];
-      s_w[t * k + lane] = ex / den;
-    }
+  const float m = __shfl_sync(0xffffffffu, my_v, 0);
+  const float ex = lane < k ? __expf(my_v - m) : 0.f;
+  const float den = warp_sum(ex);
+  if (lane < k) {
+    idx_out[lane] = my_e;
+    w_out[lane] = ex / den;
   }
 }
 
 // ------------------------------------------------------------------ kernel
 
-// Work items of this CTA, identical in every role: gate|up items gi = c,
-// c + G, ... < nA * F/8 (active expert gi / (F/8), features 8 * (gi % (F/8))),
-// then for each down item ob = c, c + G, ... < d/16 one sub-item per active
-// expert. The ring sequence number s counts them in that order.
+// Work items of this CTA, identical in every role. Gate|up items are numbered
+// gi = a * (F/8) + fb over the active experts a (features 8 fb .. 8 fb + 7);
+// down items di = a * (d/16) + ob (output features 16 ob .. 16 ob + 15). Each
+// CTA takes a contiguous range of each list, so consecutive items share an
+// expert and its token (or h) rows stay in L1. The ring sequence number s
+// counts the CTA's gate|up items, then its down items; item s is taken by
+// compute group s % kNg.
 struct Plan {
   int nA;       // active experts
-  int nB;       // gate|up items of this CTA
-  int nC;       // down items of this CTA
   int fpb;      // feature blocks per expert (F / 8)
+  int opb;      // output blocks per expert (d / 16)
+  int b0, nB;   // first gate|up item and count
+  int c0, nC;   // first down item and count
 };
 
-__device__ __forceinline__ Plan make_plan(const Params& p, int nA) {
+__device__ __forceinline__ Plan make_plan(int d, int F, int nA) {
   Plan pl;
   pl.nA = nA;
-  pl.fpb = p.F / 8;
-  const int G = gridDim.x, c = blockIdx.x;
-  const int totB = nA * pl.fpb, totC = p.d / 16;
-  pl.nB = c < totB ? (totB - c + G - 1) / G : 0;
-  pl.nC = c < totC ? (totC - c + G - 1) / G : 0;
+  pl.fpb = F / 8;
+  pl.opb = d / 16;
+  const long long G = gridDim.x, c = blockIdx.x;
+  const long long totB = (long long)nA * pl.fpb, totC = (long long)nA * pl.opb;
+  pl.b0 = (int)(c * totB / G);
+  pl.nB = (int)((c + 1) * totB / G) - pl.b0;
+  pl.c0 = (int)(c * totC / G);
+  pl.nC = (int)((c + 1) * totC / G) - pl.c0;
   return pl;
 }
 
@@ -370,14 +407,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~(uintptr_t)127);
+  float* red = reinterpret_cast<float*>(ring + kSlots * kSlotBytes);   // [2][kNg][kGw][32][4]
   __shared__ uint64_t full[kSlots], empty[kSlots];
   __shared__ int s_idx[kMaxR];          // expert of routed row t*k + j
   __shared__ float s_w[kMaxR];          // its weight
   __shared__ int s_roff[kMaxE + 1];     // rows of expert e: s_roff[e] .. s_roff[e+1]-1
-  __shared__ int s_rows[kMaxR];         // sorted row r -> routed row t*k + j
+  __shared__ int s_rows[kMaxR];         // sorted row -> routed row t*k + j
+  __shared__ int s_inv[kMaxR];          // routed row -> sorted row
+  __shared__ int s_tok[kMaxR];          // sorted row -> token
   __shared__ int s_act[kMaxE];          // active experts, increasing
   __shared__ int s_nact;
-  __shared__ float s_y[kCw][kMaxT][16]; // down: per-warp partial sums
   __shared__ volatile int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -388,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(smem_u32(full + i), 1);
-      mbar_init(smem_u32(empty + i), 1);
+      mbar_init(smem_u32(empty + i), kGw);
     }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -398,67 +437,75 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   __syncthreads();
 
   // ---------------------------------------------------------------- phase A
-  // x -> fp16 (8 values per thread, all CTAs share the rows)
-  {
+  if (warp < kCw) {
+    // x -> fp16 (8 values per thread, all CTAs share the rows)
     const int n8 = T * d / 8;
     const uint4* xs = reinterpret_cast<const uint4*>(p.x);
     uint4* xo = reinterpret_cast<uint4*>(p.x16);
-    for (int i = blockIdx.x * kThreads + threadIdx.x; i < n8; i += G * kThreads) {
+    for (int i = blockIdx.x * (kCw * 32) + threadIdx.x; i < n8; i += G * kCw * 32) {
       const uint4 v = xs[i];
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      // stored as the pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7), the K order of
+      // the weight dequantisation
+      float e[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        e[2 * j] = __uint_as_float(w4[j] << 16);
+        e[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+      }
       uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float a = __uint_as_float(w4[j] << 16), b = __uint_as_float(w4[j] & 0xFFFF0000u);
-        if (!(fabsf(a) < 65520.f && fabsf(b) < 65520.f)) report_status(p.status, MOE_ERR_RANGE);
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(b), "f"(a));
+        if (!(fabsf(e[j]) < 65520.f && fabsf(e[j + 4]) < 65520.f))
+          report_status(p.status, MOE_ERR_RANGE);
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(e[j + 4]), "f"(e[j]));
       }
       xo[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-  }
-  // router logits: expert e of this CTA, token t per compute warp, fp32 sums
-  // of exact bf16 products
-  if (warp < kCw) {
-    for (int e = blockIdx.x; e < E; e += G) {
+    // router logits: a warp per (expert e, token t); per lane the 8-element
+    // chunks lane, lane + 32, ... of the row in order, fp32 sums of exact
+    // bf16 products, then a warp sum. All of a lane's chunks are loaded
+    // before the first product.
+    constexpr int kMaxC = 2048 / 256;          // 16-byte chunks per lane at d = 2048
+    const int nc8 = d / 8;
+    for (int u = blockIdx.x + G * warp; u < E * T; u += G * kCw) {
+      const int e = u % E, t = u / E;
       const uint4* wrow = reinterpret_cast<const uint4*>(p.wr + (size_t)e * d);
-      for (int t = warp; t < T; t += kCw) {
-        const uint4* xrow = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
-        float acc = 0.f;
-        for (int c8 = lane; c8 < d / 8; c8 += 32) {
-          const uint4 a = __ldg(wrow + c8), b = xrow[c8];
-          const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+      const uint4* xrow = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
+      uint4 wv[kMaxC], xv[kMaxC];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 fa = bf16x2_to_f32x2(wa[j]), fb = bf16x2_to_f32x2(wb[j]);
-            acc = fmaf(fa.x, fb.x, acc);
-            acc = fmaf(fa.y, fb.y, acc);
+      for (int i = 0; i < kMaxC; ++i) {
+        const bool in = lane + 32 * i < nc8;
+        wv[i] = in ? __ldg(wrow + lane + 32 * i) : make_uint4(0, 0, 0, 0);
+        xv[i] = in ? xrow[lane + 32 * i] : make_uint4(0, 0, 0, 0);
+      }
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxC; ++i) {
+        if (lane + 32 * i < nc8) {
+          const uint32_t wa[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+          const uint32_t wb[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 fa = bf16x2_to_f32x2(wa[q]), fb = bf16x2_to_f32x2(wb[q]);
+            acc = fmaf(fb.x, fa.x, acc);
+            acc = fmaf(fb.y, fa.y, acc);
           }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) p.logits[(size_t)t * E + e] = acc + (p.rbias ? p.rbias[e] : 0.f);
       }
+      const float v = warp_sum(acc);
+      if (lane == 0) p.logits[(size_t)t * E + e] = v + (p.rbias ? p.rbias[e] : 0.f);
     }
   }
-  __syncthreads();
   bool ok = true;
   if (warp < kCw) ok = grid_barrier(p.sync, 1, &s_abort, p.status);
   __syncthreads();
   if (s_abort) ok = false;
 
   // ---------------------------------------------------------------- routing
-  // top-k of every token (all CTAs alike): lane l keeps keys of experts
-  // l, l + 32, ...; k rounds of a warp max pick the best remaining expert,
-  // the lowest index among equal logits; weights exp(L - Lmax) / sum. A warp
-  // takes tokens w, w + 8, w + 16, w + 24 together (independent chains).
-  if (ok && warp < kCw) {
-    if (T <= kCw) {
-      if (E <= 128) topk_tokens<4, 1>(p, warp, lane, s_idx, s_w);
-      else topk_tokens<kMaxE / 32, 1>(p, warp, lane, s_idx, s_w);
-    } else {
-      if (E <= 128) topk_tokens<4, kMaxT / kCw>(p, warp, lane, s_idx, s_w);
-      else topk_tokens<kMaxE / 32, kMaxT / kCw>(p, warp, lane, s_idx, s_w);
-    }
-  }
+  if (ok && warp < kCw)
+    for (int t = warp; t < T; t += kCw)
+      topk_token(p.logits + (size_t)t * E, E, k, lane, s_idx + t * k, s_w + t * k);
   __syncthreads();
   // stable counting sort of the routed rows by expert (all CTAs alike), by
   // warp 0: chunks of 32 rows in order; __match_any_sync groups the lanes of
@@ -515,29 +562,235 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   }
   __syncthreads();
   if (ok) {
-    int rk[(kMaxR + kThreads - 1) / kThreads];
-#pragma unroll
-    for (int q = 0; q * kThreads < kMaxR; ++q) {
-      const int i = q * kThreads + threadIdx.x;
-      rk[q] = i < R ? s_roff[s_idx[i]] + s_rows[i] : 0;
-    }
+    int rk = 0;
+    if (threadIdx.x < R) rk = s_roff[s_idx[threadIdx.x]] + s_rows[threadIdx.x];
     __syncthreads();
-#pragma unroll
-    for (int q = 0; q * kThreads < kMaxR; ++q) {
-      const int i = q * kThreads + threadIdx.x;
-      if (i < R) s_rows[rk[q]] = i;                         // sorted row -> routed row
+    if (threadIdx.x < R) {
+      s_rows[rk] = threadIdx.x;          // sorted row -> routed row
+      s_inv[threadIdx.x] = rk;           // routed row -> sorted row
+      s_tok[rk] = threadIdx.x / k;
     }
   }
   __syncthreads();
-  // the workspace tables, as moe_route and moe_sort_rows write them
-  if (ok && blockIdx.x == 0) {
+  const Plan pl = make_plan(d, F, s_nact);
+  const int nseq = pl.nB + pl.nC;        // ring sequence of this CTA
+
+  if (warp == kCw) {
+    // ------------------------------------------------------------ producer
+    // one thread streams every item's weight rows (and their scales and
+    // biases) into ring slot s % kSlots, after the item kSlots earlier in the
+    // sequence has released it
+    if (lane == 0 && ok) {
+      int s = 0;
+      for (; s < nseq; ++s) {
+        const int slot = s % kSlots;
+        if (s >= kSlots &&
+            !mbar_wait(smem_u32(empty + slot), ((s / kSlots) - 1) & 1, &s_abort, p.status))
+          break;
+        const uint32_t dst = smem_u32(ring + slot * kSlotBytes);
+        const uint32_t bar = smem_u32(full + slot);
+        // slot layout: 16 weight rows of K/2 bytes, then the 16 rows'
+        // scales, then their biases
+        if (s < pl.nB) {
+          const int gi = pl.b0 + s;
+          const int e = s_act[gi / pl.fpb], f0 = (gi % pl.fpb) * 8;
+          const size_t rg = (size_t)e * 2 * F + f0, ru = rg + F;   // first gate / up row
+          const uint32_t wb = 8u * (uint32_t)(d / 2), sb = 8u * (uint32_t)(d / 32);
+          mbar_expect_tx(bar, 2 * wb + 4 * sb);
+          bulk_g2s(dst, p.w_gu + rg * (d / 8), wb, bar);
+          bulk_g2s(dst + wb, p.w_gu + ru * (d / 8), wb, bar);
+          const uint32_t sc = dst + 2 * wb;
+          bulk_g2s(sc, p.s_gu + rg * (d / 64), sb, bar);
+          bulk_g2s(sc + sb, p.s_gu + ru * (d / 64), sb, bar);
+          bulk_g2s(sc + 2 * sb, p.b_gu + rg * (d / 64), sb, bar);
+          bulk_g2s(sc + 3 * sb, p.b_gu + ru * (d / 64), sb, bar);
+        } else {
+          const int di = pl.c0 + (s - pl.nB);
+          const int a = di / pl.opb, ob = di % pl.opb;
+          const size_t r = (size_t)s_act[a] * d + (size_t)ob * 16;     // first of 16 rows
+          const uint32_t wb = 16u * (uint32_t)(F / 2), sb = 16u * (uint32_t)(F / 32);
+          mbar_expect_tx(bar, wb + 2 * sb);
+          bulk_g2s(dst, p.w_dn + r * (F / 8), wb, bar);
+          const uint32_t sc = dst + wb;
+          bulk_g2s(sc, p.s_dn + r * (F / 64), sb, bar);
+          bulk_g2s(sc + sb, p.b_dn + r * (F / 64), sb, bar);
+        }
+      }
+      // copies in flight land before the CTA may exit (bounded, also when
+      // aborting)
+      for (int i = 0; i < kSlots && i < s; ++i) {
+        const int last = s - 1 - i;
+        mbar_wait(smem_u32(full + last % kSlots), (last / kSlots) & 1, &s_abort, p.status, false);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ compute warps
+    // Lane (g, c) holds A rows g and g + 8 (gate row g and up row g of the 8
+    // features, or output rows g and g + 8 of the 16) and token g of each
+    // group of 8 (B columns). Each warp of a group multiplies its K steps;
+    // the group adds the four partial sums in warp order (double-buffered
+    // scratch, one group barrier per 8 tokens) and warp 0 of the group
+    // stores the result.
+    const int g = lane >> 2, c = lane & 3;
+    const int grp = warp / kGw, gw = warp % kGw;
+    int buf = 0;
+    // sums the group's partials of this pass into a4 (warp 0 of the group)
+    auto reduce = [&](const float* acc, float* a4) {
+      float* rb = red + (((size_t)buf * kNg + grp) * kGw) * 128;
+      *reinterpret_cast<float4*>(rb + gw * 128 + lane * 4) = make_float4(acc[0], acc[1], acc[2],
+                                                                         acc[3]);
+      group_sync(grp);
+      a4[0] = a4[1] = a4[2] = a4[3] = 0.f;
+      if (gw == 0) {
+#pragma unroll
+        for (int w = 0; w < kGw; ++w) {
+          const float4 v = *reinterpret_cast<const float4*>(rb + w * 128 + lane * 4);
+          a4[0] += v.x;
+          a4[1] += v.y;
+          a4[2] += v.z;
+          a4[3] += v.w;
+        }
+      }
+      buf ^= 1;
+    };
+
+    // gate|up + SwiGLU -> h (fp16; every 8 features stored in the order
+    // (0,4,1,5,2,6,3,7), the K order of the down projection's dequantisation)
+    const int nstB = d / 128;
+    const int rsB = d / 2;
+    for (int s = grp; s < pl.nB; s += kNg) {
+      const int slot = s % kSlots;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(full + slot), (s / kSlots) & 1,
+                                                   &s_abort, p.status));
+      ok = group_sync_and(grp, ok);
+      if (!ok) break;
+      const uint8_t* sp = ring + slot * kSlotBytes;
+      const int gi = pl.b0 + s;
+      const int f0 = (gi % pl.fpb) * 8;
+      const int e = s_act[gi / pl.fpb];
+      const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
+      const uint16_t* scl = reinterpret_cast<const uint16_t*>(sp + 16 * rsB);
+      const uint16_t* sg = scl + g * (d / 64);
+      const uint16_t* su = scl + (8 + g) * (d / 64);
+      const uint16_t* bg = scl + (16 + g) * (d / 64);
+      const uint16_t* bu = scl + (24 + g) * (d / 64);
+      for (int q = 0; q * 8 < nv; ++q) {
+        const int n = q * 8 + g;
+        const bool xv = n < nv;
+        const __half* xr = p.x16 + (size_t)(xv ? s_tok[r0 + n] : 0) * d;
+        float acc[4], a4[4];
+        warp_mma_steps(sp + g * rsB, sp + (8 + g) * rsB, sg, bg, su, bu, xr, xv, gw, nstB, c, acc);
+        reduce(acc, a4);
+        // lane (g, c): gate (a4[0..1]) and up (a4[2..3]) of feature f0 + g
+        // for the expert's tokens q*8 + 2c, q*8 + 2c + 1
+        if (gw == 0) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int n2 = q * 8 + 2 * c + j;
+            if (n2 < nv) {
+              const float v = swiglu(a4[j], a4[2 + j]);
+              if (!(fabsf(v) < 65520.f)) report_status(p.status, MOE_ERR_RANGE);
+              p.h[(size_t)(r0 + n2) * F + f0 + (g & 3) * 2 + (g >> 2)] = __float2half_rn(v);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+    }
+    // all of h is written before any CTA reads it
+    if (!grid_barrier(p.sync, 2, &s_abort, p.status)) ok = false;
+
+    // down -> ys (fp16, sorted row order): rows 16 ob + g and 16 ob + 8 + g
+    // of active expert a against the expert's h rows
+    const int nstC = F / 128;
+    const int rsC = F / 2;
+    for (int s = pl.nB + (((grp - pl.nB) % kNg) + kNg) % kNg; s < nseq; s += kNg) {
+      const int slot = s % kSlots;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(full + slot), (s / kSlots) & 1,
+                                                   &s_abort, p.status));
+      ok = group_sync_and(grp, ok);
+      if (!ok) break;
+      const uint8_t* sp = ring + slot * kSlotBytes;
+      const int di = pl.c0 + (s - pl.nB);
+      const int a = di / pl.opb, o0 = (di % pl.opb) * 16;
+      const int e = s_act[a];
+      const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
+      const uint16_t* sc_ = reinterpret_cast<const uint16_t*>(sp + 16 * rsC);
+      const uint16_t* bi_ = sc_ + 16 * (F / 64);
+      for (int q = 0; q * 8 < nv; ++q) {
+        const int n = q * 8 + g;
+        const bool hvld = n < nv;
+        const __half* hr = p.h + (size_t)(hvld ? r0 + n : 0) * F;
+        float acc[4], a4[4];
+        warp_mma_steps(sp + g * rsC, sp + (g + 8) * rsC, sc_ + g * (F / 64), bi_ + g * (F / 64),
+                       sc_ + (g + 8) * (F / 64), bi_ + (g + 8) * (F / 64), hr, hvld, gw, nstC, c,
+                       acc);
+        reduce(acc, a4);
+        // lane (g, c): outputs o0 + g (a4[0..1]) and o0 + 8 + g (a4[2..3])
+        // of the expert's rows q*8 + 2c, q*8 + 2c + 1
+        if (gw == 0) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int n2 = q * 8 + 2 * c + j;
+            if (n2 < nv) {
+              if (!(fabsf(a4[j]) < 65520.f && fabsf(a4[2 + j]) < 65520.f))
+                report_status(p.status, MOE_ERR_RANGE);
+              __half* yr = p.ys + (size_t)(r0 + n2) * d + o0;
+              yr[g] = __float2half_rn(a4[j]);
+              yr[g + 8] = __float2half_rn(a4[2 + j]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+    }
+    // all of ys is written before any CTA reads it
+    if (!grid_barrier(p.sync, 3, &s_abort, p.status)) ok = false;
+
+    // combine: y[t][o .. o+7] = sum over j of w[t][j] * ys[inv[t*k + j]][o ..
+    // o+7], fp32 fused multiply-adds in j order, one rounding to bf16
+    if (ok) {
+      const int per_row = d / 8;
+      for (int i = blockIdx.x * (kCw * 32) + threadIdx.x; i < T * per_row; i += G * kCw * 32) {
+        const int t = i / per_row, o = (i % per_row) * 8;
+        float acc8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc8[q] = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const float wj = s_w[t * k + j];
+          const uint4 v = __ldcg(reinterpret_cast<const uint4*>(
+              p.ys + (size_t)s_inv[t * k + j] * d + o));
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[q]));
+            acc8[2 * q] = fmaf(wj, f.x, acc8[2 * q]);
+            acc8[2 * q + 1] = fmaf(wj, f.y, acc8[2 * q + 1]);
+          }
+        }
+        uint4 out;
+        out.x = pack_bf16x2(acc8[0], acc8[1]);
+        out.y = pack_bf16x2(acc8[2], acc8[3]);
+        out.z = pack_bf16x2(acc8[4], acc8[5]);
+        out.w = pack_bf16x2(acc8[6], acc8[7]);
+        *reinterpret_cast<uint4*>(p.y + (size_t)t * d + o) = out;
+      }
+    }
+  }
+
+  // the workspace tables, as moe_route and moe_sort_rows write them, by the
+  // last CTA once its own work is done: they are not needed inside this
+  // launch
+  if (!s_abort && blockIdx.x == G - 1) {
     for (int i = threadIdx.x; i < R; i += kThreads) {
       p.topk_idx[i] = s_idx[i];
       p.topk_w[i] = s_w[i];
-      const uint32_t slot = (uint32_t)s_rows[i];
-      p.order[i] = slot;
-      p.inv_order[slot] = (uint32_t)i;
-      p.row_map[i] = slot / (uint32_t)k;
+      p.order[i] = (uint32_t)s_rows[i];
+      p.inv_order[i] = (uint32_t)s_inv[i];
+      p.row_map[i] = (uint32_t)(s_rows[i] / k);
     }
     for (int e = threadIdx.x; e <= E; e += kThreads) {
       p.row_off[e] = s_roff[e];
@@ -559,166 +812,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
   }
-  __syncthreads();
-  const Plan pl = make_plan(p, s_nact);
-  const int nseq = pl.nB + pl.nC * pl.nA;      // ring sequence of this CTA
-
-  if (warp == kCw) {
-    // ------------------------------------------------------------ producer
-    // one thread streams every item's weight rows (and their scales and
-    // biases) into ring slot s % kSlots, after the item kSlots earlier in the
-    // sequence has released it
-    if (lane == 0 && ok) {
-      int s = 0;
-      for (; s < nseq; ++s) {
-        const int slot = s % kSlots;
-        if (s >= kSlots &&
-            !mbar_wait(smem_u32(empty + slot), ((s / kSlots) - 1) & 1, &s_abort, p.status))
-          break;
-        const uint32_t dst = smem_u32(ring + slot * kSlotBytes);
-        const uint32_t bar = smem_u32(full + slot);
-        if (s < pl.nB) {
-          const int gi = blockIdx.x + s * G;
-          const int e = s_act[gi / pl.fpb], f0 = (gi % pl.fpb) * 8;
-          const size_t rg = (size_t)e * 2 * F + f0, ru = rg + F;   // first gate / up row
-          const uint32_t wb = 8u * (uint32_t)(d / 2), sb = 8u * (uint32_t)(d / 32);
-          mbar_expect_tx(bar, 2 * wb + 4 * sb);
-          bulk_g2s(dst, p.w_gu + rg * (d / 8), wb, bar);
-          bulk_g2s(dst + wb, p.w_gu + ru * (d / 8), wb, bar);
-          bulk_g2s(dst + 2 * wb, p.s_gu + rg * (d / 64), sb, bar);
-          bulk_g2s(dst + 2 * wb + sb, p.s_gu + ru * (d / 64), sb, bar);
-          bulk_g2s(dst + 2 * wb + 2 * sb, p.b_gu + rg * (d / 64), sb, bar);
-          bulk_g2s(dst + 2 * wb + 3 * sb, p.b_gu + ru * (d / 64), sb, bar);
-        } else {
-          const int sc = s - pl.nB;
-          const int m = sc / pl.nA, a = sc - m * pl.nA;
-          const int ob = blockIdx.x + m * G;
-          const size_t r = (size_t)s_act[a] * d + (size_t)ob * 16;     // first of 16 rows
-          const uint32_t wb = 16u * (uint32_t)(F / 2), sb = 16u * (uint32_t)(F / 32);
-          mbar_expect_tx(bar, wb + 2 * sb);
-          bulk_g2s(dst, p.w_dn + r * (F / 8), wb, bar);
-          bulk_g2s(dst + wb, p.s_dn + r * (F / 64), sb, bar);
-          bulk_g2s(dst + wb + sb, p.b_dn + r * (F / 64), sb, bar);
-        }
-      }
-      // copies in flight land before the CTA may exit (bounded, also when
-      // aborting)
-      for (int i = 0; i < kSlots && i < s; ++i) {
-        const int last = s - 1 - i;
-        mbar_wait(smem_u32(full + last % kSlots), (last / kSlots) & 1, &s_abort, p.status, false);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ compute warps
-    const int g = lane >> 2, c = lane & 3;
-    // gate|up + SwiGLU: item s of this CTA, one warp per item. Lane (g, c)
-    // holds gate row g and up row g of the 8 features (the m16 A rows g and
-    // g + 8) and token g of each group of 8 (B columns); inside the 16-wide
-    // K slice m of a 128-element step, fragment columns (2c, 2c+1, 2c+8,
-    // 2c+9) are elements c*32 + 4m + (0..3) for A and B alike, so both come
-    // from contiguous loads.
-    for (int s = warp; s < pl.nB && ok; s += kCw) {
-      const int slot = s % kSlots;
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(full + slot), (s / kSlots) & 1, &s_abort,
-                                              p.status));
-      if (!ok) break;
-      const uint8_t* sp = ring + slot * kSlotBytes;
-      const int gi = blockIdx.x + s * G;
-      const int f0 = (gi % pl.fpb) * 8;
-      const int e = s_act[gi / pl.fpb];
-      const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
-      const uint32_t* wg = reinterpret_cast<const uint32_t*>(sp) + g * (d / 8);
-      const uint32_t* wu = reinterpret_cast<const uint32_t*>(sp + 4 * d) + g * (d / 8);
-      const uint16_t* sg = reinterpret_cast<const uint16_t*>(sp + 8 * d) + g * (d / 64);
-      const uint16_t* su = sg + 8 * (d / 64);
-      const uint16_t* bg = su + 8 * (d / 64);
-      const uint16_t* bu = bg + 8 * (d / 64);
-      // 8 token rows per pass; the weights stay in shared memory
-      for (int q = 0; q * 8 < nv; ++q) {
-        const int n = q * 8 + g;
-        const bool xv = n < nv;
-        const __half* xr = p.x16 + (size_t)(xv ? s_rows[r0 + n] / k : 0) * d;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        warp_mma_rows16<4>(wg, wu, sg, bg, su, bu, xr, xv, d, c, acc);
-        // lane (g, c): gate (acc[0..1]) and up (acc[2..3]) of feature f0 + g
-        // for the expert's tokens q*8 + 2c, q*8 + 2c + 1
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int n2 = q * 8 + 2 * c + j;
-          if (n2 < nv) {
-            const float v = swiglu(acc[j], acc[2 + j]);
-            if (!(fabsf(v) < 65520.f)) report_status(p.status, MOE_ERR_RANGE);
-            p.h[(size_t)(r0 + n2) * F + f0 + g] = __float2half_rn(v);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
-    }
-    // all of h is written before any CTA reads it
-    if (!grid_barrier(p.sync, 2, &s_abort, p.status)) ok = false;
-
-    // down + combine: item ob (16 output features); warp w takes active
-    // experts w, w + 8, ...: rows o0 + g and o0 + 8 + g (A rows g, g + 8)
-    // against the expert's h rows (B columns), then y[t][o] += w[t][j] * ys
-    // into this warp's partial sums
-    // (every compute warp runs every iteration: the named barriers inside
-    // need all of them, so a failed wait only skips the work)
-    for (int m = 0; m < pl.nC; ++m) {
-      const int ob = blockIdx.x + m * G;
-      for (int i = threadIdx.x; i < kCw * kMaxT * 16; i += kCw * 32) (&s_y[0][0][0])[i] = 0.f;
-      compute_sync();
-      for (int a = warp; a < pl.nA && ok; a += kCw) {
-        const int s = pl.nB + m * pl.nA + a;
-        const int slot = s % kSlots;
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(full + slot), (s / kSlots) & 1, &s_abort,
-                                                p.status));
-        if (!ok) break;
-        const uint8_t* sp = ring + slot * kSlotBytes;
-        const int e = s_act[a];
-        const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
-        const uint32_t* wl_ = reinterpret_cast<const uint32_t*>(sp) + g * (F / 8);
-        const uint32_t* wh_ = reinterpret_cast<const uint32_t*>(sp) + (g + 8) * (F / 8);
-        const uint16_t* sc_ = reinterpret_cast<const uint16_t*>(sp + 8 * F);
-        const uint16_t* bi_ = sc_ + 16 * (F / 64);
-        for (int q = 0; q * 8 < nv; ++q) {
-          const int n = q * 8 + g;
-          const bool hvld = n < nv;
-          const __half* hr = p.h + (size_t)(hvld ? r0 + n : 0) * F;
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          warp_mma_rows16<4>(wl_, wh_, sc_ + g * (F / 64), bi_ + g * (F / 64),
-                             sc_ + (g + 8) * (F / 64), bi_ + (g + 8) * (F / 64), hr, hvld, F, c,
-                             acc);
-          // lane (g, c): rows o0 + g (acc[0..1]) and o0 + 8 + g (acc[2..3])
-          // for the expert's tokens q*8 + 2c, q*8 + 2c + 1
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int n2 = q * 8 + 2 * c + j;
-            if (n2 < nv) {
-              const int i = s_rows[r0 + n2];
-              const int t = i / k;
-              const float wt = s_w[i];
-              s_y[warp][t][g] += wt * acc[j];
-              s_y[warp][t][g + 8] += wt * acc[2 + j];
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(empty + slot));
-      }
-      compute_sync();
-      if (s_abort) ok = false;
-      for (int i = threadIdx.x; i < T * 16 && !s_abort; i += kCw * 32) {
-        const int t = i >> 4, o = i & 15;
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kCw; ++w) v += s_y[w][t][o];
-        p.y[(size_t)t * d + ob * 16 + o] = __float2bfloat16_rn(v);
-      }
-      compute_sync();
-    }
-  }
 }
 
 // ------------------------------------------------------------------ host
@@ -738,14 +831,14 @@ bool decode_fused_ok(int T, int k, int E, int d, int F, int fmt, int dt) {
          E <= kMaxE && k <= 32 && d % 128 == 0 && F % 128 == 0 && d <= 2048 && F <= 2048;
 }
 
-size_t decode_smem_bytes() { return dec::kSlots * dec::kSlotBytes + 128; }
+size_t decode_smem_bytes() { return dec::kSlots * dec::kSlotBytes + dec::kRedBytes + 128; }
 
 cudaError_t launch_decode_fused(const void* x, const void* w_router, const float* bias,
                                 const moe_experts& ex, int T, int k, int BM, float* logits,
                                 int32_t* idx, float* w, uint32_t* order, uint32_t* inv_order,
                                 uint32_t* row_map, int32_t* counts, int32_t* row_off,
-                                int32_t* tile_off, void* x16, void* h, void* y, unsigned* sync,
-                                int* status, cudaStream_t s) {
+                                int32_t* tile_off, void* x16, void* h, void* ys, void* y,
+                                unsigned* sync, int* status, cudaStream_t s) {
   using namespace dec;
   if (!decode_fused_ok(T, k, ex.E, ex.d, ex.F, ex.fmt, MOE_BF16)) return cudaErrorNotSupported;
   const int G = sm_count();
@@ -777,6 +870,7 @@ cudaError_t launch_decode_fused(const void* x, const void* w_router, const float
   p.tile_off = tile_off;
   p.x16 = (__half*)x16;
   p.h = (__half*)h;
+  p.ys = (__half*)ys;
   p.y = (__nv_bfloat16*)y;
   p.sync = sync;
   p.status = status;

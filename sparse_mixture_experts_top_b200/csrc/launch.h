@@ -74,14 +74,15 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
 // The decode layer fused into one cooperative launch (q4 experts, bf16
 // activations, T <= 32, T*k <= 256, E <= 256, d and F multiples of 128 and at
 // most 2048). Writes the same workspace tables as the separate stages (logits,
-// top-k, sort tables, x16, h) and y; `sync` is a 4-byte scratch word.
+// top-k, sort tables, x16, h, ys in fp16) and y; `sync` is a 4-byte scratch
+// word.
 bool decode_fused_ok(int T, int k, int E, int d, int F, int fmt, int dt);
 cudaError_t launch_decode_fused(const void* x, const void* w_router, const float* bias,
                                 const moe_experts& ex, int T, int k, int BM, float* logits,
                                 int32_t* idx, float* w, uint32_t* order, uint32_t* inv_order,
                                 uint32_t* row_map, int32_t* counts, int32_t* row_off,
-                                int32_t* tile_off, void* x16, void* h, void* y, unsigned* sync,
-                                int* status, cudaStream_t s);
+                                int32_t* tile_off, void* x16, void* h, void* ys, void* y,
+                                unsigned* sync, int* status, cudaStream_t s);
 
 cudaError_t launch_combine(const void* ys, const uint32_t* inv_order, const float* w, int T, int k,
                            int d, int dt, void* y, cudaStream_t s);
