@@ -37,6 +37,10 @@ sys.path.insert(0, ROOT)
 import moe_inputs as mi  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one gate|up launch, from the ncu capture in
+# profiles/grouped_gate_up_q4_prefill_ncu.md (675.19 MB + 20.85 MB); to be
+# retaken whenever that kernel changes
+GATE_UP_TRAFFIC = {"prefill": 696040448}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -358,7 +362,8 @@ def main():
             "roofline": {"kernel": "grouped gate|up + SwiGLU (moe_grouped_swiglu)",
                          "bound": "hbm", "achieved": res["achieved_gbs"],
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": res["achieved_gbs"] / pk["hbm_gbs"], "traffic": None,
+                         "frac": res["achieved_gbs"] / pk["hbm_gbs"],
+                         "traffic": GATE_UP_TRAFFIC.get(args.workload),
                          "peak_source": res["pk_kind"],
                          "us_per_launch": res["ms_swiglu"] * 1e3,
                          "tensor_tflops": res["tflops_swiglu"],

@@ -5,11 +5,12 @@
 // trip; MOE_OPTIMIZATION_COMPLETE.md, "Mega Kernel Architecture": router
 // matmul, softmax and top-K on the GPU.
 //
-// Top-k runs one warp per token: every lane holds E/32 logits in registers as
-// 64-bit keys (orderable value bits << 32 | ~expert), so one warp max-reduce
-// gives the best remaining expert with the lowest index among equal values;
-// k rounds of that select the experts best first. -0.0 is mapped to +0.0 and
-// NaN to the lowest key, so the order is total and deterministic.
+// Top-k runs one warp per token: every lane holds E/32 logits in registers
+// with their orderable 32-bit keys; per round a warp max-reduce of the lanes'
+// best keys and a min-reduce of the expert indices holding that key give the
+// best remaining expert with the lowest index among equal values; k rounds of
+// that select the experts best first. -0.0 is mapped to +0.0 and NaN to the
+// lowest key, so the order is total and deterministic.
 #include "common.cuh"
 #include "launch.h"
 
@@ -146,16 +147,11 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w > v ? w : v;
-  }
-  return v;
-}
-
-// VPL = logits held per lane (E <= 32 * VPL).
+// VPL = logits held per lane (E <= 32 * VPL). Each of the k rounds takes the
+// lane's best remaining expert (largest key, the lowest index among equal
+// keys), the warp maximum of those keys and then the lowest expert index among
+// the lanes that hold it: two single-instruction warp reductions per selected
+// expert instead of a five-step 64-bit shuffle tree.
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
                                                    int k, int32_t* __restrict__ idx_out,
@@ -166,31 +162,43 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   const float* row = logits + (size_t)t * E;
-  unsigned long long key[VPL];
+  uint32_t key[VPL];
+  float val[VPL];
+  uint32_t avail = 0;                 // bit i: expert lane + 32 i exists and is not taken
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    int e = lane + 32 * i;
-    key[i] = (e < E) ? (((unsigned long long)order_key(row[e]) << 32) | (0xFFFFFFFFu - (uint32_t)e))
-                     : 0ull;   // absent experts rank below everything (k <= E)
+    const int e = lane + 32 * i;
+    val[i] = e < E ? row[e] : 0.f;
+    key[i] = order_key(val[i]);
+    if (e < E) avail |= 1u << i;
   }
-  int my_e = -1;   // lane j keeps the j-th selected expert
+  int my_e = 0;                       // lane j keeps the j-th selected expert and its logit
+  float my_v = 0.f;
   for (int j = 0; j < k; ++j) {
-    unsigned long long best = 0ull;
+    uint32_t bk = 0;
+    int bi = -1;
+    float bv = 0.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) best = key[i] > best ? key[i] : best;
-    best = warp_max_u64(best);
-    const int e = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
-    if (lane == j) my_e = e;
-    if ((e & 31) == lane) {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (lane + 32 * i == e) key[i] = 0ull;
+    for (int i = 0; i < VPL; ++i) {
+      if (((avail >> i) & 1u) && (bi < 0 || key[i] > bk)) {
+        bk = key[i];
+        bi = i;
+        bv = val[i];
+      }
+    }
+    const uint32_t M = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
+    const uint32_t ce = (bi >= 0 && bk == M) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
+    const uint32_t es = __reduce_min_sync(0xffffffffu, ce);
+    const float v = __shfl_sync(0xffffffffu, bv, (int)(es & 31u));
+    if ((int)(es & 31u) == lane) avail &= ~(1u << (es >> 5));
+    if (lane == j) {
+      my_e = (int)es;
+      my_v = v;
     }
   }
   // weights: exp(L_j - m) / sum over the selected, m = the best logit
-  const float m = row[__shfl_sync(0xffffffffu, my_e, 0)];
-  float ex = 0.f;
-  if (lane < k) ex = __expf(row[my_e] - m);
+  const float m = __shfl_sync(0xffffffffu, my_v, 0);
+  const float ex = lane < k ? __expf(my_v - m) : 0.f;
   const float den = warp_sum(ex);
   if (lane < k) {
     idx_out[(size_t)t * k + lane] = my_e;
