@@ -37,9 +37,9 @@ sys.path.insert(0, ROOT)
 import moe_inputs as mi  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one gate|up launch, from the ncu capture in
-# profiles/grouped_gate_up_q4_prefill_ncu.md (675.19 MB + 20.85 MB); to be
-# retaken whenever that kernel changes
+# DRAM bytes (read + write) of one gate|up launch on the prefill workload,
+# from an ncu capture of that kernel (675.19 MB read + 20.85 MB written); to
+# be retaken whenever that kernel changes
 GATE_UP_TRAFFIC = {"prefill": 696040448}
 L2_FLUSH_BYTES = 256 << 20
 
