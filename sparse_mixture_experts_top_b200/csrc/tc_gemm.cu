@@ -102,6 +102,7 @@ struct Params {
   const int32_t* tile_off;
   int E;               // groups (experts); 1 for the router
   int n_rows;          // router: tokens T
+  int row_tile;        // router: tokens per tile (16, 32, 64 or 128)
   int n_units;         // units (pairs of weight matrices) per token tile
   int unit_rows;       // weight rows from one unit to the next
   int mat_off;         // row offset of matrix 1 from matrix 0 inside a unit
@@ -391,8 +392,8 @@ __device__ __forceinline__ void decode_unit(const Params& p, const int* s_toff, 
   unit = u - tau * p.n_units;
   if (ROUTER) {
     e = 0;
-    r0 = tau * BN;
-    nv = min(BN, p.n_rows - r0);
+    r0 = tau * p.row_tile;
+    nv = min(p.row_tile, p.n_rows - r0);
   } else {
     int lo = 0, hi = p.E - 1;      // largest e with tile_off[e] <= tau
     while (lo < hi) {
@@ -407,7 +408,7 @@ __device__ __forceinline__ void decode_unit(const Params& p, const int* s_toff, 
 
 template <bool ROUTER>
 __device__ __forceinline__ int total_units(const Params& p, const int* s_toff) {
-  if (ROUTER) return ((p.n_rows + BN - 1) / BN) * p.n_units;
+  if (ROUTER) return ((p.n_rows + p.row_tile - 1) / p.row_tile) * p.n_units;
   return s_toff[p.E] * p.n_units;
 }
 
@@ -1109,7 +1110,13 @@ cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const f
   p.m_limit = E;
   p.bias = bias;
   p.status = status;
-  const long long ub = (long long)((T + BN - 1) / BN) * p.n_units;
+  // token tiles small enough that at least half of the SMs get a unit: every
+  // unit streams the same weight rows through one SM, so more, shorter
+  // units spread the router over the GPU (down to 16 rows, the MMA's least N)
+  int tile = BN;
+  while (tile > 16 && (long long)((T + tile - 1) / tile) * p.n_units < num_sms() / 2) tile /= 2;
+  p.row_tile = tile;
+  const long long ub = (long long)((T + tile - 1) / tile) * p.n_units;
   return run<MOE_W_BF16, EPI_STORE, true>(p, ta, ub, s);
 }
 
