@@ -453,8 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(raw_full + i), C::Q4 ? 33 : 1);
       mbar_init(smem_u32(raw_empty + i), 16);   // the 16 dequant warps
     }
-    // a matrix's stage is written by 4 warps (q4: one half) or 8 (bf16: both halves)
-    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::Q4 ? 4 : 8);
+    // one barrier per A stage pair of a matrix: q4, each stage of the pair is
+    // written by the 4 warps of one half (8 arrivals); bf16, each stage by
+    // the 8 warps of both halves (16 arrivals)
+    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::Q4 ? 8 : 16);
     for (int i = 0; i < NB / 2; ++i) mbar_init(smem_u32(b_full + i), 1);
     for (int i = 0; i < NP; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
     for (int i = 0; i < 2; ++i) {
@@ -629,11 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dcol = tm + (small ? b * 128u + q * 64u : q * 128u);
       // k-blocks two at a time (a unit has an even number of them; NS and
       // NB are even, so both stages of a pair share their phases): two
-      // waits, eight MMAs and one release per pair. Every dequant warp
-      // signals the pair's two A stages in order, so the second one being
-      // complete means the first one is; both B stages share one barrier.
+      // waits, eight MMAs and one release per pair. The pair's two A stages
+      // complete one barrier; both B stages share another.
       for (int kb = 0; kb < nka && ok; kb += 2) {
-        ok = mbar_wait_warp(afull0 + (ss + 1) * 8, sph, abort_flag, p.status) &&
+        ok = mbar_wait_warp(afull0 + (ss >> 1) * 8, sph, abort_flag, p.status) &&
              mbar_wait_warp(smem_u32(b_full + bs / 2), bph, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
@@ -747,9 +748,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------ dequant
     // 16 warps: (matrix q, lane quadrant qd, half hf). q4: half hf converts
-    // A stages 2hf and 2hf + 1 of every raw stage (chunks 4hf .. 4hf + 3 of
-    // the row); bf16: half hf converts K elements 32hf .. 32hf + 31 of the
-    // raw stage's single A stage.
+    // k-blocks hf and 2 + hf of every raw stage (chunks 2hf, 2hf + 1 and
+    // 4 + 2hf, 5 + 2hf of the row), so both halves fill a k-block pair
+    // together and the MMAs of one pair overlap the conversion of the next;
+    // bf16: half hf converts K elements 32hf .. 32hf + 31 of the raw stage's
+    // single A stage.
     const int dw = warp - kDqWarp0;                   // 0..15
     const int q = (dw >> 2) & 1;                      // matrix
     const int hf = dw >> 3;                           // half of the raw stage
@@ -770,13 +773,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sw = m & 7;
         uint4 wv[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) wv[c] = lds128(rowa + (((4 * hf + c) ^ sw) << 4));
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = C::Q4 ? 2 * hf + c + (c & 2) : 4 * hf + c;
+          wv[c] = lds128(rowa + (((uint32_t)chunk ^ (uint32_t)sw) << 4));
+        }
         uint32_t sc = 0, bi = 0;
         if (C::Q4) {
-          // this row's scales and biases of groups 2hf, 2hf + 1 (bf16 pairs)
-          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * 8 + hf * 4);
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc) : "r"(so));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bi) : "r"(so + C::SCL_BYTES / 2));
+          // this row's scales and biases of groups hf and 2 + hf (its two
+          // k-blocks), each a bf16 in the low half
+          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * 8);
+          uint32_t s01, s23, b01, b23;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s01), "=r"(s23) : "r"(so));
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                       : "=r"(b01), "=r"(b23)
+                       : "r"(so + C::SCL_BYTES / 2));
+          sc = hf ? ((s01 >> 16) | (s23 & 0xFFFF0000u)) : ((s01 & 0xFFFFu) | (s23 << 16));
+          bi = hf ? ((b01 >> 16) | (b23 & 0xFFFF0000u)) : ((b01 & 0xFFFFu) | (b23 << 16));
         }
         // A shared-memory load has read its data only once an instruction has
         // consumed its destination registers; until then the next TMA into
@@ -794,8 +806,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < NST; ++j) {
           uint32_t vals[32];
           if (C::Q4) {
-            // chunk pair (2j, 2j + 1) of my half holds the 64 elements of
-            // group 4kr + 2hf + j
+            // my chunks 2j, 2j + 1 hold the 64 elements of k-block hf + 2j of
+            // the raw stage, group 4kr + hf + 2j
             const uint32_t s2 = f16x2_from_bf16(j ? (sc >> 16) : (sc & 0xFFFFu));
             const uint32_t b2 = f16x2_from_bf16(j ? (bi >> 16) : (bi & 0xFFFFu));
             const uint4 w0 = wv[2 * j], w1 = wv[2 * j + 1];
@@ -816,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 4; ++i) vals[4 * c + i] = ROUTER ? w4[i] : bf16x2_to_f16x2(w4[i]);
             }
           }
-          const uint32_t stage = a_it + (C::Q4 ? 2 * hf + j : 0);
+          const uint32_t stage = a_it + (C::Q4 ? hf + 2 * j : 0);
           const uint32_t as = stage % NS;
           if (stage >= (uint32_t)NS) {      // the slot's previous k-block is released
             const uint32_t pr = (stage - NS) >> 1;
@@ -829,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           else tmem_st16_sync(tl + col, vals);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(afull + as * 8);
+          if (lane == 0) mbar_arrive(afull + (as >> 1) * 8);
         }
         ++raw_it;
         a_it += C::A_PER_RAW;
