@@ -246,7 +246,7 @@ __device__ __noinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile in
 // One warp, 16 weight rows in shared memory (row g of matrix `a` and of
 // matrix `b` for lane (g, c): the m16 A rows g and g + 8), against one group
 // of 8 token rows read from global memory (this lane's row `xrow`, zero when
-// !xvalid), over the 128-wide K steps st0, st0 + kGw, ... < nst. mma.sync
+// !xvalid), over the 128-wide K steps st0, st0 + sstride, ... < nst. mma.sync
 // m16n8k16 fp16, fp32 accumulation into acc: acc[0..1] row a for tokens 2c,
 // 2c+1, acc[2..3] row b.
 //
@@ -264,7 +264,7 @@ __device__ __forceinline__ void warp_mma_steps(const uint8_t* wa, const uint8_t*
                                                const uint16_t* sa, const uint16_t* ba,
                                                const uint16_t* sb, const uint16_t* bb,
                                                const __half* xrow, bool xvalid, int st0, int nst,
-                                               int c, float* acc) {
+                                               int sstride, int c, float* acc) {
   float ch[2][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -306,14 +306,14 @@ __device__ __forceinline__ void warp_mma_steps(const uint8_t* wa, const uint8_t*
   };
   int st = st0;
   if (st < nst) load(xq[0], st);
-  if (st + kGw < nst) load(xq[1], st + kGw);
+  if (st + sstride < nst) load(xq[1], st + sstride);
 #pragma unroll 1
-  for (; st < nst; st += 2 * kGw) {
+  for (; st < nst; st += 2 * sstride) {
     step(xq[0], st);
-    if (st + 2 * kGw < nst) load(xq[0], st + 2 * kGw);
-    if (st + kGw < nst) {
-      step(xq[1], st + kGw);
-      if (st + 3 * kGw < nst) load(xq[1], st + 3 * kGw);
+    if (st + 2 * sstride < nst) load(xq[0], st + 2 * sstride);
+    if (st + sstride < nst) {
+      step(xq[1], st + sstride);
+      if (st + 3 * sstride < nst) load(xq[1], st + 3 * sstride);
     }
   }
 #pragma unroll
@@ -384,7 +384,8 @@ __device__ __noinline__ void topk_token(const float* row, int E, int k, int lane
 struct Plan {
   int nA;       // active experts
   int fpb;      // feature blocks per expert (F / 8)
-  int opb;      // output blocks per expert (d / 16)
+  int dr;       // output rows per down item (16 or 32)
+  int opb;      // output blocks per expert (d / dr)
   int b0, nB;   // first gate|up item and count
   int c0, nC;   // first down item and count
 };
@@ -393,7 +394,10 @@ __device__ __forceinline__ Plan make_plan(int d, int F, int nA) {
   Plan pl;
   pl.nA = nA;
   pl.fpb = F / 8;
-  pl.opb = d / 16;
+  // 32 rows when they fit a ring slot (their K = F words, scales and biases:
+  // 18 F bytes), so the four warps of a group split an item evenly
+  pl.dr = 18 * F <= kSlotBytes ? 32 : 16;
+  pl.opb = d / pl.dr;
   const long long G = gridDim.x, c = blockIdx.x;
   const long long totB = (long long)nA * pl.fpb, totC = (long long)nA * pl.opb;
   pl.b0 = (int)(c * totB / G);
@@ -607,8 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         } else {
           const int di = pl.c0 + (s - pl.nB);
           const int a = di / pl.opb, ob = di % pl.opb;
-          const size_t r = (size_t)s_act[a] * d + (size_t)ob * 16;     // first of 16 rows
-          const uint32_t wb = 16u * (uint32_t)(F / 2), sb = 16u * (uint32_t)(F / 32);
+          const size_t r = (size_t)s_act[a] * d + (size_t)ob * pl.dr;  // first of dr rows
+          const uint32_t wb = (uint32_t)pl.dr * (uint32_t)(F / 2);
+          const uint32_t sb = (uint32_t)pl.dr * (uint32_t)(F / 32);
           mbar_expect_tx(bar, wb + 2 * sb);
           bulk_g2s(dst, p.w_dn + r * (F / 8), wb, bar);
           const uint32_t sc = dst + wb;
@@ -635,16 +640,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int g = lane >> 2, c = lane & 3;
     const int grp = warp / kGw, gw = warp % kGw;
     int buf = 0;
-    // sums the group's partials of this pass into a4 (warp 0 of the group)
-    auto reduce = [&](const float* acc, float* a4) {
+    // sums the partials of warps gw .. gw + ks - 1 of the group into a4 (in
+    // the first of them, gw % ks == 0)
+    auto reduce = [&](const float* acc, float* a4, int ks) {
       float* rb = red + (((size_t)buf * kNg + grp) * kGw) * 128;
       *reinterpret_cast<float4*>(rb + gw * 128 + lane * 4) = make_float4(acc[0], acc[1], acc[2],
                                                                          acc[3]);
       group_sync(grp);
       a4[0] = a4[1] = a4[2] = a4[3] = 0.f;
-      if (gw == 0) {
-#pragma unroll
-        for (int w = 0; w < kGw; ++w) {
+      if (gw % ks == 0) {
+        for (int w = gw; w < gw + ks; ++w) {
           const float4 v = *reinterpret_cast<const float4*>(rb + w * 128 + lane * 4);
           a4[0] += v.x;
           a4[1] += v.y;
@@ -680,8 +685,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const bool xv = n < nv;
         const __half* xr = p.x16 + (size_t)(xv ? s_tok[r0 + n] : 0) * d;
         float acc[4], a4[4];
-        warp_mma_steps(sp + g * rsB, sp + (8 + g) * rsB, sg, bg, su, bu, xr, xv, gw, nstB, c, acc);
-        reduce(acc, a4);
+        warp_mma_steps(sp + g * rsB, sp + (8 + g) * rsB, sg, bg, su, bu, xr, xv, gw, nstB, kGw, c,
+                       acc);
+        reduce(acc, a4, kGw);
         // lane (g, c): gate (a4[0..1]) and up (a4[2..3]) of feature f0 + g
         // for the expert's tokens q*8 + 2c, q*8 + 2c + 1
         if (gw == 0) {
@@ -702,10 +708,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // all of h is written before any CTA reads it
     if (!grid_barrier(p.sync, 2, &s_abort, p.status)) ok = false;
 
-    // down -> ys (fp16, sorted row order): rows 16 ob + g and 16 ob + 8 + g
-    // of active expert a against the expert's h rows
+    // down -> ys (fp16, sorted row order): an item is dr output rows of active
+    // expert a against the expert's h rows; with 32 rows, warps 0-1 of the
+    // group take rows 0-15 and warps 2-3 rows 16-31, each pair splitting K
     const int nstC = F / 128;
     const int rsC = F / 2;
+    const int ksC = kGw / (pl.dr / 16);           // warps per 16 rows
+    const int rbC = (gw / ksC) * 16;              // this warp's first row of the item
     for (int s = pl.nB + (((grp - pl.nB) % kNg) + kNg) % kNg; s < nseq; s += kNg) {
       const int slot = s % kSlots;
       ok = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(full + slot), (s / kSlots) & 1,
@@ -714,23 +723,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (!ok) break;
       const uint8_t* sp = ring + slot * kSlotBytes;
       const int di = pl.c0 + (s - pl.nB);
-      const int a = di / pl.opb, o0 = (di % pl.opb) * 16;
+      const int a = di / pl.opb, o0 = (di % pl.opb) * pl.dr + rbC;
       const int e = s_act[a];
       const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
-      const uint16_t* sc_ = reinterpret_cast<const uint16_t*>(sp + 16 * rsC);
-      const uint16_t* bi_ = sc_ + 16 * (F / 64);
+      const uint16_t* sc_ = reinterpret_cast<const uint16_t*>(sp + pl.dr * rsC);
+      const uint16_t* bi_ = sc_ + pl.dr * (F / 64);
+      const int ra = rbC + g, rb_ = rbC + 8 + g;     // A rows g and g + 8 of this warp
       for (int q = 0; q * 8 < nv; ++q) {
         const int n = q * 8 + g;
         const bool hvld = n < nv;
         const __half* hr = p.h + (size_t)(hvld ? r0 + n : 0) * F;
         float acc[4], a4[4];
-        warp_mma_steps(sp + g * rsC, sp + (g + 8) * rsC, sc_ + g * (F / 64), bi_ + g * (F / 64),
-                       sc_ + (g + 8) * (F / 64), bi_ + (g + 8) * (F / 64), hr, hvld, gw, nstC, c,
-                       acc);
-        reduce(acc, a4);
+        warp_mma_steps(sp + ra * rsC, sp + rb_ * rsC, sc_ + ra * (F / 64), bi_ + ra * (F / 64),
+                       sc_ + rb_ * (F / 64), bi_ + rb_ * (F / 64), hr, hvld, gw % ksC, nstC, ksC,
+                       c, acc);
+        reduce(acc, a4, ksC);
         // lane (g, c): outputs o0 + g (a4[0..1]) and o0 + 8 + g (a4[2..3])
         // of the expert's rows q*8 + 2c, q*8 + 2c + 1
-        if (gw == 0) {
+        if (gw % ksC == 0) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int n2 = q * 8 + 2 * c + j;
