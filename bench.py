@@ -257,10 +257,34 @@ def run_ours(args, rank, world, local_rank):
                             "hbm_frac": dbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"]}
             del dl, dws, g2
 
+    # sparse (top-k) against dense soft routing (k = E: every expert, full
+    # softmax weights) at the PRD's acceptance shape, through the same call
+    dense = {}
+    if not args.no_dense:
+        al = mi.make_layer("acceptance", seed=args.seed + 1000 * rank, device=dev)
+        times = {}
+        for kk in (al.wl.k, al.wl.E):
+            aws = moe.forward_workspace(al.x, al.experts, kk)
+            ay = torch.empty(al.wl.T, al.wl.d, dtype=al.x.dtype, device=dev)
+            f3 = lambda: moe.forward(al.x, al.w_router, None, al.experts, kk, ws=aws, out=ay)
+            f3()
+            g3 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g3):
+                f3()
+            torch.cuda.synchronize()
+            times[kk] = statistics.mean(time_device(g3.replay, max(args.steps, 20), args.warmup,
+                                                    flush))
+            del g3, aws
+        wlA = al.wl
+        dense = {"workload": f"acceptance: T={wlA.T} d={wlA.d} E={wlA.E} F={wlA.F} bf16 experts",
+                 "sparse_k": wlA.k, "sparse_ms": times[wlA.k], "dense_ms": times[wlA.E],
+                 "speedup": times[wlA.E] / times[wlA.k], "target": 1.5}
+        del al
+
     step_ms = statistics.mean(ms)
     res = {"ms": step_ms, "ms_eager": statistics.mean(ms_eager), "ms_e2e": statistics.mean(ms_e2e),
            "ms_swiglu": statistics.mean(ms_swiglu), "achieved_gbs": achieved_gbs,
-           "tflops_swiglu": tflops, "gu_bytes": gu_bytes, "clocks": clocks, "decode": decode,
+           "tflops_swiglu": tflops, "gu_bytes": gu_bytes, "clocks": clocks, "decode": decode, "sparse_vs_dense": dense,
            "active": active, "regime": regime, "BM": L.BM, "pk": pk, "pk_kind": pk_kind,
            "layer_bytes": active * expert_bytes(ex) + 2 * T * wl.d * 2,
            "layer_flops": 6.0 * T * k * wl.d * wl.F}
@@ -307,6 +331,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -378,6 +403,7 @@ def main():
             "gpu_launches": kernels_per_forward(wl.T, wl.k, res["regime"] == 2) * args.steps,
             "clocks": res["clocks"],
             "decode": res["decode"],
+            "sparse_vs_dense": res["sparse_vs_dense"],
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(layer)

@@ -255,6 +255,20 @@ def test_forward_parity_prefill_sampled(moe, orc, regime):
     assert moe.device_status() == moe.OK
 
 
+def test_forward_parity_dense_soft_routing(moe, orc):
+    """k = E selects every expert and the renormalised weights are the full
+    softmax: the layer is then dense soft routing, the baseline of the PRD's
+    acceptance test ("5.5 real sparse MoE kernels (Metal)", Acceptance)."""
+    layer = mi.make_layer("acceptance", seed=0, device=DEV)
+    E = layer.wl.E
+    y = moe.forward(layer.x, layer.w_router, None, layer.experts, E)
+    torch.cuda.synchronize()
+    rows = np.arange(0, layer.wl.T, 32)
+    r = orc.forward(layer.x.cpu()[rows], layer.w_router.cpu(), None, _host(layer.experts), E)
+    assert_close_rms(to_np(y)[rows], r.y, TOL_BF16, "y[acceptance, k = E]")
+    assert moe.device_status() == moe.OK
+
+
 def test_forward_parity_decode_t32_tensor_core(moe, orc):
     layer = mi.make_layer("decode_t32", seed=1, device=DEV)
     _forward_and_compare(moe, orc, layer, regime=2)
