@@ -93,6 +93,12 @@ typedef enum { MOE_W_F32 = 0, MOE_W_BF16 = 1, MOE_W_Q4G64 = 2 } moe_wfmt;
 
 typedef enum { MOE_REGIME_AUTO = 0, MOE_REGIME_GEMV = 1, MOE_REGIME_TC = 2 } moe_regime;
 
+/* The GLU's gate activation (mlx-lm PR #2044, "When it applies": SwiGLU or
+ * tanh-GELU GLU): h = act(gate) * up with
+ *   MOE_ACT_SWIGLU:     act(g) = silu(g) = g / (1 + exp(-g))
+ *   MOE_ACT_GEGLU_TANH: act(g) = 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))) */
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GEGLU_TANH = 1 } moe_act;
+
 /* Expert weights (all device, read-only, caller-owned).
  *   MOE_W_F32 / MOE_W_BF16:
  *     w_gu [E][2F][d]  rows 0..F-1 gate, rows F..2F-1 up (fused [gate|up])
@@ -103,7 +109,9 @@ typedef enum { MOE_REGIME_AUTO = 0, MOE_REGIME_GEMV = 1, MOE_REGIME_TC = 2 } moe
  *     w_gu uint32 [E][2F][d/8], s_gu, b_gu bf16 [E][2F][d/64]
  *     w_dn uint32 [E][d][F/8],  s_dn, b_dn bf16 [E][d][F/64]
  *     element j of a word sits in bits [4j, 4j+3] (low nibble first);
- *     value = scale[group] * q + bias[group]. */
+ *     value = scale[group] * q + bias[group].
+ *   act: moe_act, the gate activation of every expert (0, SwiGLU, when the
+ *     struct is zero-initialised); other values: MOE_ERR_INVALID_ARG. */
 typedef struct {
   int32_t fmt; /* moe_wfmt */
   int32_t E, d, F;
@@ -113,6 +121,7 @@ typedef struct {
   const void* w_dn;
   const void* s_dn;
   const void* b_dn;
+  int32_t act; /* moe_act */
 } moe_experts;
 
 /* Router: logits, softmax, top-k, renormalised weights.
@@ -187,7 +196,8 @@ moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, i
  *   row_map, row_off, tile_off: as written by moe_sort_rows with the same BM
  *            (the tensor-core regime needs BM = 128)
  *   h        (device, out) [T*k][F]: fp16 for bf16 activations, fp32 for fp32:
- *            h[i][f] = silu(g) * u, g = x[row_map[i]] . w_gu[e][f],
+ *            h[i][f] = act(g) * u (experts->act: silu or tanh-GELU),
+ *            g = x[row_map[i]] . w_gu[e][f],
  *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
  *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, k, d, dt)
  *            bytes (the token rows in fp16: x converted, or, in the

@@ -147,18 +147,24 @@ class Experts:
     b_gu: torch.Tensor | None = None
     s_dn: torch.Tensor | None = None
     b_dn: torch.Tensor | None = None
+    act: str = "swiglu"       # the GLU's gate activation: "swiglu" or "geglu"
 
     def to(self, device) -> "Experts":
         mv = lambda t: None if t is None else t.to(device)
         return Experts(self.fmt, self.E, self.d, self.F, mv(self.w_gu), mv(self.w_dn),
-                       mv(self.s_gu), mv(self.b_gu), mv(self.s_dn), mv(self.b_dn))
+                       mv(self.s_gu), mv(self.b_gu), mv(self.s_dn), mv(self.b_dn), self.act)
+
+    def with_act(self, act: str) -> "Experts":
+        """The same weights with another GLU activation."""
+        return Experts(self.fmt, self.E, self.d, self.F, self.w_gu, self.w_dn, self.s_gu,
+                       self.b_gu, self.s_dn, self.b_dn, act)
 
     def select(self, experts) -> "Experts":
         """Copy of the listed experts only (for sampled checks on the host)."""
         ix = torch.as_tensor(experts, dtype=torch.long, device=self.w_gu.device)
         sl = lambda t: None if t is None else t.index_select(0, ix)
         return Experts(self.fmt, len(ix), self.d, self.F, sl(self.w_gu), sl(self.w_dn),
-                       sl(self.s_gu), sl(self.b_gu), sl(self.s_dn), sl(self.b_dn))
+                       sl(self.s_gu), sl(self.b_gu), sl(self.s_dn), sl(self.b_dn), self.act)
 
     def nbytes_per_expert(self) -> int:
         tot = 0

@@ -61,11 +61,11 @@ def lib():
         L.orc_topk.argtypes = [P, I, I, I, P, P]
         L.orc_topk_weights_full_softmax.argtypes = [P, P, I, I, I, P]
         L.orc_sort_rows.argtypes = [P, I, I, I, I, P, P, P, P, P, P]
-        L.orc_expert_swiglu.argtypes = [P, I, P, P, I, I, I, I, P, P, P, P, I]
+        L.orc_expert_swiglu.argtypes = [P, I, P, P, I, I, I, I, P, P, P, P, I, I]
         L.orc_expert_down.argtypes = [P, P, I, I, I, I, P, P, P, P, I]
         L.orc_combine.argtypes = [P, P, P, I, I, I, P]
         L.orc_forward.argtypes = [P, I, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P,
-                                  P, P, P, P, P, P, I]
+                                  P, P, P, P, P, P, I, I]
         L.orc_expert_gate_up.argtypes = [P, I, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
         L.orc_expert_down_abs.argtypes = [P, P, I, I, I, I, P, P, P, P, I]
         L.orc_weight_value.argtypes = [I, P, P, P, I, I, I, I, I]
@@ -197,6 +197,14 @@ def _wargs(experts, which):
     return wa, _np(s), _np(b)
 
 
+# the gate's activation of the GLU: SwiGLU (silu) or GeGLU (tanh-form GELU)
+ACTS = {"swiglu": 0, "geglu": 1}
+
+
+def act_code(experts) -> int:
+    return ACTS[getattr(experts, "act", "swiglu")]
+
+
 def expert_swiglu(x, row_map, row_off, experts, nthreads=None):
     xa = _np(x)
     rm = _np(row_map, np.uint32)
@@ -206,7 +214,8 @@ def expert_swiglu(x, row_map, row_off, experts, nthreads=None):
     h = np.empty((R, experts.F), np.float64)
     _check(lib().orc_expert_swiglu(_p(xa), _act_code(xa), _p(rm), _p(ro), experts.E, experts.d,
                                    experts.F, WFMT[experts.fmt], _p(w), _p(s), _p(b), _p(h),
-                                   nthreads or default_threads()), "expert_swiglu")
+                                   act_code(experts), nthreads or default_threads()),
+           "expert_swiglu")
     return h
 
 
@@ -286,7 +295,7 @@ def forward(x, w_router, bias, experts, k, BM=1, keep_intermediates=False, nthre
     _check(lib().orc_forward(_p(xa), _act_code(xa), _p(wra), _p(ba), T, d, E, k, F, BM,
                              WFMT[experts.fmt], _p(wg), _p(sg), _p(bg), _p(wd), _p(sd), _p(bd),
                              _p(y), _p(L), _p(idx), _p(w), _p(h), _p(ys),
-                             nthreads or default_threads()), "forward")
+                             act_code(experts), nthreads or default_threads()), "forward")
     return ForwardResult(y, L, idx, w, h, ys)
 
 

@@ -19,7 +19,8 @@
  *      argsort(order), row_map = order // k, per-expert counts and the row and
  *      tile prefix tables (DS4Server issue #112, "Current upstream route",
  *      sort_rows; "Kernel contract", _schedule)
- *   4. gate|up projection with the SwiGLU epilogue silu(gate) * up over the
+ *   4. gate|up projection with the GLU epilogue act(gate) * up, act = silu
+ *      (SwiGLU) or the tanh form of GELU (GeGLU), over the
  *      sorted rows, reading token rows through row_map (issue #112,
  *      swiglu_rows; mlxcel PR #275, "What it does")
  *   5. down projection of the sorted rows (issue #112, switch_linear with
@@ -258,8 +259,20 @@ int orc_sort_rows(const int32_t* idx, int T, int k, int E, int BM,
 
 typedef struct {
     const void* x; int xdt; const uint32_t* row_map; const int32_t* row_off;
-    orc_wmat gu; int d, F; double* h;
+    orc_wmat gu; int d, F; double* h; int act;
 } swiglu_ctx;
+
+/* The gate's activation of the GLU. act 0: silu(g) = g * sigmoid(g) =
+ * g / (1 + exp(-g)) (SwiGLU). act 1: the tanh form of GELU (Hendrycks and
+ * Gimpel), 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))) -- the
+ * "tanh-GELU GLU" of mlx-lm PR #2044, "When it applies" (Gemma-4's GeGLU). */
+static double glu_gate(double g, int act) {
+    if (act == 1) {
+        const double c = sqrt(2.0 / (4.0 * atan(1.0)));   /* sqrt(2 / pi) */
+        return 0.5 * g * (1.0 + tanh(c * (g + 0.044715 * g * g * g)));
+    }
+    return g / (1.0 + exp(-g));
+}
 
 static void swiglu_range(void* p, int lo, int hi) {
     swiglu_ctx* c = (swiglu_ctx*)p;
@@ -279,8 +292,7 @@ static void swiglu_range(void* p, int lo, int hi) {
                     g += xv * wg[a];
                     u += xv * wu[a];
                 }
-                /* silu(g) * u with silu(g) = g * sigmoid(g) = g / (1 + exp(-g)) */
-                c->h[(size_t)i * c->F + f] = g / (1.0 + exp(-g)) * u;
+                c->h[(size_t)i * c->F + f] = glu_gate(g, c->act) * u;
             }
         }
     }
@@ -293,8 +305,9 @@ static void swiglu_range(void* p, int lo, int hi) {
  * 0..F-1, up rows F..2F-1). */
 int orc_expert_swiglu(const void* x, int xdt, const uint32_t* row_map, const int32_t* row_off,
                       int E, int d, int F, int wfmt, const void* w_gu, const uint16_t* s_gu,
-                      const uint16_t* b_gu, double* h, int nthreads) {
-    swiglu_ctx c = {x, xdt, row_map, row_off, {wfmt, w_gu, s_gu, b_gu, 2 * F, d}, d, F, h};
+                      const uint16_t* b_gu, double* h, int act, int nthreads) {
+    if (act != 0 && act != 1) return 1;
+    swiglu_ctx c = {x, xdt, row_map, row_off, {wfmt, w_gu, s_gu, b_gu, 2 * F, d}, d, F, h, act};
     orc_parallel(swiglu_range, &c, E, nthreads);
     return 0;
 }
@@ -438,7 +451,7 @@ int orc_forward(const void* x, int xdt, const void* w_router, const float* bias,
                 int wfmt, const void* w_gu, const uint16_t* s_gu, const uint16_t* b_gu,
                 const void* w_dn, const uint16_t* s_dn, const uint16_t* b_dn,
                 double* y, double* logits64, int32_t* idx_out, double* w_out,
-                double* h_out, double* ys_out, int nthreads) {
+                double* h_out, double* ys_out, int act, int nthreads) {
     if (k < 1 || k > E || T < 0) return 1;
     size_t R = (size_t)T * k;
     double* L = (double*)malloc(sizeof(double) * ((size_t)T * E + 1));
@@ -457,7 +470,7 @@ int orc_forward(const void* x, int xdt, const void* w_router, const float* bias,
     for (size_t i = 0; rc == 0 && i < (size_t)T * E; ++i) L[i] = (double)(float)L[i];
     if (rc == 0) rc = orc_topk(L, T, E, k, idx, w);
     if (rc == 0) rc = orc_sort_rows(idx, T, k, E, BM, order, inv, rmap, counts, roff, toff);
-    if (rc == 0) rc = orc_expert_swiglu(x, xdt, rmap, roff, E, d, F, wfmt, w_gu, s_gu, b_gu, h, nthreads);
+    if (rc == 0) rc = orc_expert_swiglu(x, xdt, rmap, roff, E, d, F, wfmt, w_gu, s_gu, b_gu, h, act, nthreads);
     if (rc == 0) rc = orc_expert_down(h, roff, E, d, F, wfmt, w_dn, s_dn, b_dn, ys, nthreads);
     if (rc == 0) rc = orc_combine(ys, inv, w, T, k, d, y);
     if (rc == 0) {

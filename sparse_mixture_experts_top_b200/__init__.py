@@ -42,7 +42,7 @@ class Experts(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("F", ctypes.c_int32), ("w_gu", ctypes.c_void_p), ("s_gu", ctypes.c_void_p),
                 ("b_gu", ctypes.c_void_p), ("w_dn", ctypes.c_void_p), ("s_dn", ctypes.c_void_p),
-                ("b_dn", ctypes.c_void_p)]
+                ("b_dn", ctypes.c_void_p), ("act", ctypes.c_int32)]
 
 
 class WsLayout(ctypes.Structure):
@@ -125,15 +125,20 @@ def _dev(*ts):
 
 
 _FMT = {"f32": W_F32, "bf16": W_BF16, "q4": W_Q4G64}
+ACT_SWIGLU, ACT_GEGLU_TANH = 0, 1
+_ACT = {"swiglu": ACT_SWIGLU, "geglu": ACT_GEGLU_TANH}
 
 
 def experts_struct(ex) -> Experts:
     """C view of an expert-weight set (any object with fmt, E, d, F, w_gu,
-    s_gu, b_gu, w_dn, s_dn, b_dn, tensors on the device)."""
+    s_gu, b_gu, w_dn, s_dn, b_dn, tensors on the device; act, "swiglu" or
+    "geglu", defaults to "swiglu")."""
     _dev(ex.w_gu, ex.w_dn, ex.s_gu, ex.b_gu, ex.s_dn, ex.b_dn)
     fmt = _FMT[ex.fmt] if isinstance(ex.fmt, str) else int(ex.fmt)
+    act = getattr(ex, "act", "swiglu")
+    act = _ACT[act] if isinstance(act, str) else int(act)
     return Experts(fmt, ex.E, ex.d, ex.F, _ptr(ex.w_gu), _ptr(ex.s_gu), _ptr(ex.b_gu),
-                   _ptr(ex.w_dn), _ptr(ex.s_dn), _ptr(ex.b_dn))
+                   _ptr(ex.w_dn), _ptr(ex.s_dn), _ptr(ex.b_dn), act)
 
 
 # ------------------------------------------------------------------ stages

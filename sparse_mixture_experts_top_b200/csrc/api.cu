@@ -47,6 +47,7 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
   if (ex->d % 64 || ex->F % 64) return MOE_ERR_UNSUPPORTED;
   if (!ex->w_gu || !ex->w_dn) return MOE_ERR_INVALID_ARG;
   if (!aligned16(ex->w_gu) || !aligned16(ex->w_dn)) return MOE_ERR_INVALID_ARG;
+  if (ex->act != MOE_ACT_SWIGLU && ex->act != MOE_ACT_GEGLU_TANH) return MOE_ERR_INVALID_ARG;
   switch (ex->fmt) {
     case MOE_W_F32:
       if (dt != MOE_F32) return MOE_ERR_UNSUPPORTED;

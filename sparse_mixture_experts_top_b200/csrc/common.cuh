@@ -52,6 +52,16 @@ __device__ __forceinline__ float swiglu(float g, float u) {
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
+// act(g) * u for the GLU's gate activation (moe_act): silu, or the tanh form
+// of GELU, 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))
+__device__ __forceinline__ float glu(int act, float g, float u) {
+  if (act == MOE_ACT_GEGLU_TANH) {
+    const float z = 0.7978845608028654f * fmaf(0.044715f * g, g * g, g);
+    return 0.5f * g * (1.0f + tanhf(z)) * u;
+  }
+  return swiglu(g, u);
+}
+
 // ---------------------------------------------------------------- warps
 
 __device__ __forceinline__ float warp_sum(float v) {

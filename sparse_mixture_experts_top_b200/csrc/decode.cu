@@ -76,6 +76,7 @@ struct Params {
   const uint16_t* s_dn;                       // [E][d][F/64]
   const uint16_t* b_dn;
   int T, d, E, k, F, BM;
+  int act;                                    // the GLU's gate activation (moe_act)
   float* logits;                              // [T][E]
   int32_t* topk_idx;                          // [T][k]
   float* topk_w;                              // [T][k]
@@ -695,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           for (int j = 0; j < 2; ++j) {
             const int n2 = q * 8 + 2 * c + j;
             if (n2 < nv) {
-              const float v = swiglu(a4[j], a4[2 + j]);
+              const float v = glu(p.act, a4[j], a4[2 + j]);
               if (!(fabsf(v) < 65520.f)) report_status(p.status, MOE_ERR_RANGE);
               p.h[(size_t)(r0 + n2) * F + f0 + (g & 3) * 2 + (g >> 2)] = __float2half_rn(v);
             }
@@ -869,6 +870,7 @@ cudaError_t launch_decode_fused(const void* x, const void* w_router, const float
   p.k = k;
   p.F = ex.F;
   p.BM = BM;
+  p.act = ex.act;
   p.logits = logits;
   p.topk_idx = idx;
   p.topk_w = w;

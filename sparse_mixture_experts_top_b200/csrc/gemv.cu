@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
     const TA* __restrict__ x, const uint32_t* __restrict__ row_map,
     const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E, int d,
     int F, const uint32_t* __restrict__ wgu, const uint16_t* __restrict__ sgu,
-    const uint16_t* __restrict__ bgu, typename HType<TA>::T* __restrict__ h, int* status) {
+    const uint16_t* __restrict__ bgu, typename HType<TA>::T* __restrict__ h, int act,
+    int* status) {
   pdl_wait();
   pdl_launch();
   using TH = typename HType<TA>::T;
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
       const float g = warp_sum(ag[j]);
       const float u = warp_sum(au[j]);
       if (lane == 0 && j < nr) {
-        const float v = swiglu(g, u);
+        const float v = glu(act, g, u);
         if constexpr (std::is_same<TH, __half>::value) {
           if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
           h[(size_t)(rb + j) * F + f] = __float2half_rn(v);
@@ -273,7 +274,7 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
 #define MOE_SWIGLU(TA, FMT)                                                                    \
   launch_pdl(swiglu_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const TA*)x, row_map, row_off, tile_off, BM, \
                                                    ex.E, ex.d, ex.F, w, sc, bi,                  \
-                                                   (typename HType<TA>::T*)h, status)
+                                                   (typename HType<TA>::T*)h, ex.act, status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_SWIGLU(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_SWIGLU(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q4G64);
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
     const __half* __restrict__ x16, const uint32_t* __restrict__ row_map,
     const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E,
     int d, int F, const uint32_t* __restrict__ w, const uint16_t* __restrict__ sc,
-    const uint16_t* __restrict__ bi, void* __restrict__ out, int* status) {
+    const uint16_t* __restrict__ bi, void* __restrict__ out, int act, int* status) {
   pdl_wait();
   pdl_launch();
   __shared__ float red[kMmaWarps - 1][32][8];
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
       const int n = t * 8 + 2 * c + j;
       if (n >= nv) continue;
       if (SWIGLU) {
-        const float v = swiglu(acc[t][j], acc[t][2 + j]);
+        const float v = glu(act, acc[t][j], acc[t][2 + j]);
         if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
         reinterpret_cast<__half*>(out)[(size_t)(r0 + n) * F + blk * 8 + g] = __float2half_rn(v);
       } else {
@@ -520,7 +521,8 @@ cudaError_t launch_swiglu_q4_mma(const void* x16, const uint32_t* row_map, const
   dim3 grid(ex.F / 8, (unsigned)tiles);
   launch_pdl(gemv_q4_mma_kernel<true>, grid, kMmaWarps * 32, 0, s, 
       (const __half*)x16, row_map, row_off, tile_off, BM, ex.E, ex.d, ex.F,
-      (const uint32_t*)ex.w_gu, (const uint16_t*)ex.s_gu, (const uint16_t*)ex.b_gu, h, status);
+      (const uint32_t*)ex.w_gu, (const uint16_t*)ex.s_gu, (const uint16_t*)ex.b_gu, h, ex.act,
+      status);
   return cudaGetLastError();
 }
 
@@ -533,7 +535,8 @@ cudaError_t launch_down_q4_mma(const void* h, const int32_t* row_off, const int3
   dim3 grid(ex.d / 16, (unsigned)tiles);
   launch_pdl(gemv_q4_mma_kernel<false>, grid, kMmaWarps * 32, 0, s, 
       (const __half*)h, nullptr, row_off, tile_off, BM, ex.E, ex.d, ex.F,
-      (const uint32_t*)ex.w_dn, (const uint16_t*)ex.s_dn, (const uint16_t*)ex.b_dn, ys, status);
+      (const uint32_t*)ex.w_dn, (const uint16_t*)ex.s_dn, (const uint16_t*)ex.b_dn, ys,
+      MOE_ACT_SWIGLU, status);
   return cudaGetLastError();
 }
 

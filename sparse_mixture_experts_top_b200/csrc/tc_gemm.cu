@@ -115,6 +115,7 @@ struct Params {
   void* out;
   int out_ld;          // elements per output row
   int m_limit;         // valid weight rows per group (router: E)
+  int act;             // gate|up: the GLU's gate activation (moe_act)
   const float* bias;   // router bias or null
   int* status;
 };
@@ -685,7 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int lim = nv - n0;        // columns of this chunk that are rows of the tile
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const __half v = __float2half_rn(swiglu(__uint_as_float(a0[j]), __uint_as_float(a1[j])));
+            const __half v =
+                __float2half_rn(glu(p.act, __uint_as_float(a0[j]), __uint_as_float(a1[j])));
             if (j < lim) {
               hmax = max(hmax, (uint32_t)__half_as_ushort(v) & 0x7FFFu);
               hp[(size_t)(n0 + j) * p.out_ld] = v;
@@ -1063,6 +1065,7 @@ cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, cons
   p.out = h;
   p.out_ld = ex.F;
   p.m_limit = ex.F;
+  p.act = ex.act;
   p.status = status;
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
   if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_SWIGLU, false>(p, ta, ub, s);

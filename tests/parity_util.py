@@ -75,13 +75,26 @@ def kth_gap(logits_np, k):
     return (s[:, : m - 1] - s[:, 1:m]).min(axis=1)
 
 
-def assert_h_close(h_gpu, href, g, u, ga, ua, d, u_w, u_h, tol, what=""):
-    """h = silu(g) * u as the kernels compute it: weights rounded to the
+def _act_and_slope(g, act):
+    """The gate activation and its derivative: silu, or the tanh form of GELU
+    (0.5 g (1 + tanh(z)), z = sqrt(2/pi) (g + 0.044715 g^3))."""
+    if act == "geglu":
+        c = np.sqrt(2.0 / np.pi)
+        th = np.tanh(c * (g + 0.044715 * g ** 3))
+        a = 0.5 * g * (1.0 + th)
+        da = 0.5 * (1.0 + th) + 0.5 * g * (1.0 - th * th) * c * (1.0 + 3 * 0.044715 * g * g)
+        return a, da
+    sig = 1.0 / (1.0 + np.exp(-g))
+    return g * sig, sig * (1.0 + g * (1.0 - sig))
+
+
+def assert_h_close(h_gpu, href, g, u, ga, ua, d, u_w, u_h, tol, what="", act="swiglu"):
+    """h = act(g) * u as the kernels compute it: weights rounded to the
     operand format before the products (unit roundoff u_w, so |dg| <= u_w *
     sum |x w|; 0 when the weights are exact in it), products accumulated in
     fp32 (2 d 2^-24 * sum |x w| with margin), h rounded once to its storage
     format (u_h |h|). The first-order bound per element is
-        tol * RMS(h) + u_h |h| + |u silu'(g)| dg + |silu(g)| du."""
+        tol * RMS(h) + u_h |h| + |u act'(g)| dg + |act(g)| du."""
     gh = to_np(h_gpu).astype(np.float64)
     assert gh.shape == href.shape, (what, gh.shape, href.shape)
     assert np.isfinite(gh).all(), f"{what}: non-finite GPU output"
@@ -90,9 +103,8 @@ def assert_h_close(h_gpu, href, g, u, ga, ua, d, u_w, u_h, tol, what=""):
     acc = 2.0 * d * 2.0 ** -24
     dg = (u_w + acc) * ga
     du = (u_w + acc) * ua
-    sig = 1.0 / (1.0 + np.exp(-g))
-    bound = (tol * rms(href) + u_h * np.abs(href)
-             + np.abs(u * sig * (1.0 + g * (1.0 - sig))) * dg + np.abs(g * sig) * du)
+    a, da = _act_and_slope(g, act)
+    bound = tol * rms(href) + u_h * np.abs(href) + np.abs(u * da) * dg + np.abs(a) * du
     err = np.abs(gh - href)
     i = int(np.argmax(err - bound))
     assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "

@@ -75,6 +75,10 @@ def test_forward_rejects_bad_arguments_without_launching(moe):
     # unknown weight format
     bad = _ex(moe, fmt=7)
     assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(bad), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
+    # unknown gate activation
+    bad = _ex(moe)
+    bad.act = 7
+    assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(bad), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
     # workspace too small / missing
     assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 16, 0, P) == moe.ERR_WORKSPACE
     assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(ex), 4, 2, fake, P, 1 << 30, 0, P) == moe.ERR_WORKSPACE

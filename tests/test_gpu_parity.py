@@ -281,6 +281,41 @@ def test_forward_parity_skewed_sampled(moe, orc):
     _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(4096, 24, replace=False)))
 
 
+# ------------------------------------------------------------------ GeGLU
+
+@pytest.mark.parametrize("name,T,regime,BM", [("decode_t32", 32, 1, 8), ("prefill", 200, 2, 128),
+                                              ("acceptance", 300, 2, 128)])
+def test_grouped_geglu_parity(moe, orc, name, T, regime, BM):
+    """The tanh-GELU GLU (mlx-lm PR #2044, "When it applies") through the
+    weight-streaming and tensor-core gate|up kernels."""
+    wl = mi.workload(name, T=T)
+    layer, idx = _stage_setup(wl, T, 23, 0.0)
+    ex = layer.experts.with_act("geglu")
+    st = moe.sort_rows(idx.to(DEV), wl.E, BM)
+    h = moe.grouped_swiglu(layer.x, st, wl.k, ex, regime=regime)
+    ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
+    hx = _host(ex)
+    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    u_w = U_F16 if wl.wfmt == "q4" else 0.0
+    assert_h_close(h, href, g, u, ga, ua, wl.d, u_w, U_F16, TOL_BF16, f"h[{name}, GeGLU]",
+                   act="geglu")
+
+
+@pytest.mark.parametrize("name", ["decode_t1", "decode_t32"])
+def test_forward_geglu_fused_decode(moe, orc, name):
+    layer = mi.make_layer(name, seed=5, device=DEV)
+    layer.experts = layer.experts.with_act("geglu")
+    _forward_and_compare(moe, orc, layer)
+
+
+def test_forward_geglu_prefill_sampled(moe, orc):
+    layer = mi.make_layer("prefill", seed=1, device=DEV)
+    layer.experts = layer.experts.with_act("geglu")
+    rng = np.random.default_rng(2)
+    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(2048, 48, replace=False)))
+
+
 def test_forward_deterministic(moe):
     layer = mi.make_layer("decode_t32", seed=3, device=DEV)
     a = moe.forward(layer.x, layer.w_router, None, layer.experts, layer.wl.k)

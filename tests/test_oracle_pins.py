@@ -233,6 +233,28 @@ def test_single_expert_is_dense_swiglu_ffn(orc):
     np.testing.assert_allclose(r.y, y.numpy(), rtol=1e-11, atol=1e-12)
 
 
+def test_single_expert_is_dense_geglu_ffn(orc):
+    """E = 1, k = 1 with the tanh-GELU GLU (mlx-lm PR #2044, "When it
+    applies"): a plain GeGLU FFN, checked against torch's own tanh-form GELU
+    on fp64 matmuls. A wrong constant or a dropped cubic term in the oracle's
+    GELU fails this."""
+    wl = mi.workload("tiny", T=9, d=64, E=1, k=1, F=128)
+    L = mi.make_layer(wl, seed=4)
+    ex = L.experts.with_act("geglu")
+    r = orc.forward(L.x, L.w_router, None, ex, 1, keep_intermediates=True)
+    x = L.x.double()
+    wgu, wdn = ex.w_gu[0].double(), ex.w_dn[0].double()
+    F = wl.F
+    g, u = x @ wgu[:F].T, x @ wgu[F:].T
+    h = torch.nn.functional.gelu(g, approximate="tanh") * u
+    y = h @ wdn.T
+    np.testing.assert_allclose(r.h, h.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(r.y, y.numpy(), rtol=1e-11, atol=1e-12)
+    # and it is not the SwiGLU result
+    rs = orc.forward(L.x, L.w_router, None, L.experts, 1)
+    assert np.abs(rs.y - r.y).max() > 1e-3 * np.abs(r.y).max()
+
+
 @pytest.mark.parametrize("wfmt,act", [("f32", "f32"), ("bf16", "bf16")])
 def test_dense_soft_routing_restricted_to_topk(orc, wfmt, act):
     """The sorted, grouped oracle equals a dense reference that runs every
