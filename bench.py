@@ -132,6 +132,24 @@ def kernels_per_forward(T, k, regime_tc: bool, fused_decode: bool = False) -> in
     return 2 + sort + conv + 2 + 1    # router + top-k, sort, x16, gate|up, down, combine
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(vals, device):
+    """Each value's maximum over all ranks (the slowest rank's time) when a
+    process group is up; the values unchanged in a single process."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def replicas_tokens_per_s(world: int, T: int, ms: float) -> float:
+    """Whole-job throughput of `world` independent replicas of T tokens each,
+    timed by the slowest rank: every rank's tokens over that time."""
+    return world * T / (ms * 1e-3)
+
+
 # ------------------------------------------------------------------ timing
 
 def time_device(fn, steps, warmup, flush):
@@ -370,14 +388,12 @@ def main():
     ms = res["ms"]
     ms_e2e = res["ms_e2e"]
     if world > 1:
-        t = torch.tensor([ms, ms_e2e], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
+        ms, ms_e2e = max_over_ranks([ms, ms_e2e], torch.device("cuda", local_rank))
     if rank == 0:
         pk = res["pk"]
         sw_s = res["ms_swiglu"] * 1e-3
         line = {
-            "metric": metric, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
+            "metric": metric, "value": replicas_tokens_per_s(world, wl.T, ms), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; shapes and distributions of the workload)",
@@ -398,7 +414,7 @@ def main():
                 "hbm_frac": res["layer_bytes"] / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "tensor_frac": res["layer_flops"] / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
             "ms_per_step_eager": res["ms_eager"],
-            "e2e": {"value": world * wl.T / (ms_e2e * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": replicas_tokens_per_s(world, wl.T, ms_e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": wl.T * wl.d * 2, "d2h_bytes_per_step": wl.T * wl.d * 2},
             "gpu_launches": kernels_per_forward(wl.T, wl.k, res["regime"] == 2) * args.steps,
             "clocks": res["clocks"],
