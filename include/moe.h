@@ -265,6 +265,22 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
  * the last read) and reset it. Synchronises the current device. */
 moe_status moe_device_status(void);
 
+/* Pack separate gate and up projections into the fused [gate|up] layout the
+ * kernels read (w_gu rows 0..F-1 gate, F..2F-1 up of every expert).
+ * DS4Server issue #112, "Kernel contract", takes both the fused [gate | up]
+ * weight and separate gate/up weights; here separate weights are packed once,
+ * at load time, rather than streamed as two tensors in every kernel.
+ *   fmt            moe_wfmt of all six tensors
+ *   w_g, w_u       (device) [E][F][d] (f32/bf16) or uint32 [E][F][d/8] (q4)
+ *   s_g, b_g, s_u, b_u (device) q4 only: bf16 [E][F][d/64]; else ignored
+ *   w_gu, s_gu, b_gu   (device, out) the fused tensors, [E][2F][...]
+ * One strided device-to-device copy per tensor on `stream`; nothing is
+ * allocated. d and F are multiples of 64; E, d, F > 0; the outputs must not
+ * overlap the inputs. */
+moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const void* s_g,
+                            const void* b_g, const void* w_u, const void* s_u, const void* b_u,
+                            void* w_gu, void* s_gu, void* b_gu, moe_stream_t stream);
+
 const char* moe_status_str(moe_status s);
 const char* moe_version(void);
 

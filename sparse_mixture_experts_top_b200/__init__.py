@@ -27,7 +27,7 @@ REGIME_AUTO, REGIME_GEMV, REGIME_TC = 0, 1, 2
 EXPORTS = ("moe_route", "moe_topk", "moe_sort_rows_workspace", "moe_sort_rows",
            "moe_sort_rows_noalloc",
            "moe_grouped_swiglu_workspace", "moe_grouped_swiglu", "moe_grouped_down",
-           "moe_combine", "moe_forward_workspace",
+           "moe_combine", "moe_forward_workspace", "moe_pack_gate_up",
            "moe_forward", "moe_forward_layout", "moe_device_status", "moe_status_str",
            "moe_version")
 
@@ -73,6 +73,8 @@ def _load():
     L.moe_forward_workspace.restype = S
     L.moe_forward.argtypes = [P, I, P, P, ctypes.POINTER(Experts), I, I, P, P, S, I, P]
     L.moe_forward_layout.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(WsLayout)]
+    L.moe_pack_gate_up.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, P, P]
+    L.moe_pack_gate_up.restype = ctypes.c_int
     L.moe_device_status.argtypes = []
     L.moe_status_str.argtypes = [I]
     L.moe_status_str.restype = ctypes.c_char_p
@@ -267,6 +269,24 @@ def forward(x, w_router, router_bias, experts, k, regime=REGIME_AUTO, ws=None, o
                            T, k, _ptr(y), _ptr(ws), ws.numel(), regime, _stream(stream)),
            "moe_forward")
     return y
+
+
+def pack_gate_up(fmt, w_g, w_u, s_g=None, b_g=None, s_u=None, b_u=None, stream=None):
+    """Fused [gate|up] tensors (w_gu, s_gu, b_gu) from separate gate and up
+    projections [E][F][...] on the device; s_gu, b_gu are None unless q4."""
+    _dev(w_g, w_u, s_g, b_g, s_u, b_u)
+    E, F = w_g.shape[0], w_g.shape[1]
+    fmt_c = _FMT[fmt] if isinstance(fmt, str) else int(fmt)
+    d = {W_F32: w_g.shape[2], W_BF16: w_g.shape[2], W_Q4G64: w_g.shape[2] * 8}[fmt_c]
+    w_gu = torch.empty((E, 2 * F) + tuple(w_g.shape[2:]), dtype=w_g.dtype, device=w_g.device)
+    s_gu = b_gu = None
+    if fmt_c == W_Q4G64:
+        s_gu = torch.empty((E, 2 * F, d // 64), dtype=s_g.dtype, device=s_g.device)
+        b_gu = torch.empty_like(s_gu)
+    _check(lib.moe_pack_gate_up(fmt_c, E, d, F, _ptr(w_g), _ptr(s_g), _ptr(b_g), _ptr(w_u),
+                                _ptr(s_u), _ptr(b_u), _ptr(w_gu), _ptr(s_gu), _ptr(b_gu),
+                                _stream(stream)), "moe_pack_gate_up")
+    return w_gu, s_gu, b_gu
 
 
 def device_status() -> int:

@@ -278,6 +278,42 @@ moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* t
   return launched(launch_combine(ys, inv_order, topk_w, T, k, d, dt, y, (cudaStream_t)stream));
 }
 
+moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const void* s_g,
+                            const void* b_g, const void* w_u, const void* s_u, const void* b_u,
+                            void* w_gu, void* s_gu, void* b_gu, moe_stream_t stream) {
+  if (E <= 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 64 || F % 64) return MOE_ERR_UNSUPPORTED;
+  if (!w_g || !w_u || !w_gu) return MOE_ERR_INVALID_ARG;
+  size_t row_bytes = 0;          // bytes of one weight row of d inputs
+  switch (fmt) {
+    case MOE_W_F32: row_bytes = (size_t)d * 4; break;
+    case MOE_W_BF16: row_bytes = (size_t)d * 2; break;
+    case MOE_W_Q4G64:
+      row_bytes = (size_t)d / 2;
+      if (!s_g || !b_g || !s_u || !b_u || !s_gu || !b_gu) return MOE_ERR_INVALID_ARG;
+      break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  // expert e's F gate rows go to rows 0..F-1 of its 2F-row block, its F up
+  // rows to rows F..2F-1: a 2-D copy of E blocks of F rows each
+  auto pack = [&](const void* g, const void* u, void* out, size_t rb) -> cudaError_t {
+    const size_t blk = (size_t)F * rb;
+    cudaError_t e = cudaMemcpy2DAsync(out, 2 * blk, g, blk, blk, (size_t)E,
+                                      cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return e;
+    return cudaMemcpy2DAsync(static_cast<char*>(out) + blk, 2 * blk, u, blk, blk, (size_t)E,
+                             cudaMemcpyDeviceToDevice, s);
+  };
+  cudaError_t e = pack(w_g, w_u, w_gu, row_bytes);
+  if (e == cudaSuccess && fmt == MOE_W_Q4G64) {
+    const size_t srb = (size_t)(d / 64) * 2;     // one row's bf16 scales (or biases)
+    e = pack(s_g, s_u, s_gu, srb);
+    if (e == cudaSuccess) e = pack(b_g, b_u, b_gu, srb);
+  }
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime,
                               moe_ws_layout* out) {
   if (!out) return MOE_ERR_INVALID_ARG;

@@ -121,6 +121,16 @@ def test_stage_calls_reject_bad_arguments(moe):
     assert L.moe_combine(fake, fake, fake, 0, 2, 128, moe.BF16, fake, P) == moe.OK
 
 
+def test_pack_gate_up_rejects_bad_arguments(moe):
+    L = moe.lib
+    fake = ctypes.c_void_p(0x10000)
+    # unknown format, zero sizes, d not a multiple of 64, missing q4 scales
+    assert L.moe_pack_gate_up(7, 2, 64, 64, fake, fake, fake, fake, fake, fake, fake, fake, fake, P) == moe.ERR_INVALID_ARG
+    assert L.moe_pack_gate_up(moe.W_BF16, 0, 64, 64, fake, P, P, fake, P, P, fake, P, P, P) == moe.ERR_INVALID_ARG
+    assert L.moe_pack_gate_up(moe.W_BF16, 2, 96, 64, fake, P, P, fake, P, P, fake, P, P, P) == moe.ERR_UNSUPPORTED
+    assert L.moe_pack_gate_up(moe.W_Q4G64, 2, 64, 64, fake, P, fake, fake, fake, fake, fake, fake, fake, P) == moe.ERR_INVALID_ARG
+
+
 def test_forward_layout_is_consistent(moe):
     for (T, d, E, k, F) in [(1, 2048, 128, 8, 768), (2048, 2048, 512, 10, 512), (16, 128, 8, 2, 256)]:
         L = moe.forward_layout(T, d, E, k, F, __import__("torch").bfloat16)

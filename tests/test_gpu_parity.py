@@ -316,6 +316,33 @@ def test_forward_geglu_prefill_sampled(moe, orc):
     _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(2048, 48, replace=False)))
 
 
+# ------------------------------------------------------------------ packing
+
+@pytest.mark.parametrize("name", ["tiny", "acceptance", "decode_t32"])
+def test_pack_separate_gate_up(moe, name):
+    """Separate gate and up projections packed into the fused [gate|up]
+    layout (DS4Server issue #112, "Kernel contract": fused or separate
+    gate/up weights) give the fused tensors byte for byte, and so the same
+    forward."""
+    layer = mi.make_layer(mi.workload(name, T=8), seed=7, device=DEV)
+    ex = layer.experts
+    F = ex.F
+    split = lambda t: (None, None) if t is None else (t[:, :F].contiguous(), t[:, F:].contiguous())
+    wg, wu = split(ex.w_gu)
+    sg, su = split(ex.s_gu)
+    bg, bu = split(ex.b_gu)
+    w_gu, s_gu, b_gu = moe.pack_gate_up(ex.fmt, wg, wu, sg, bg, su, bu)
+    torch.cuda.synchronize()
+    assert torch.equal(w_gu, ex.w_gu)
+    if ex.fmt == "q4":
+        assert torch.equal(s_gu, ex.s_gu) and torch.equal(b_gu, ex.b_gu)
+    packed = mi.Experts(ex.fmt, ex.E, ex.d, F, w_gu, ex.w_dn, s_gu, b_gu, ex.s_dn, ex.b_dn)
+    a = moe.forward(layer.x, layer.w_router, layer.router_bias, ex, layer.wl.k)
+    b = moe.forward(layer.x, layer.w_router, layer.router_bias, packed, layer.wl.k)
+    assert torch.equal(a.view(torch.int16) if a.dtype != torch.float32 else a,
+                       b.view(torch.int16) if b.dtype != torch.float32 else b)
+
+
 def test_forward_deterministic(moe):
     layer = mi.make_layer("decode_t32", seed=3, device=DEV)
     a = moe.forward(layer.x, layer.w_router, None, layer.experts, layer.wl.k)
