@@ -89,7 +89,13 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype; /* activations */
 
-typedef enum { MOE_W_F32 = 0, MOE_W_BF16 = 1, MOE_W_Q4G64 = 2 } moe_wfmt;
+typedef enum {
+  MOE_W_F32 = 0,
+  MOE_W_BF16 = 1,
+  MOE_W_Q4G64 = 2,
+  MOE_W_Q4G32 = 3,   /* as MOE_W_Q4G64 with one scale and bias per 32 elements */
+  MOE_W_Q4G128 = 4   /* ... per 128 elements */
+} moe_wfmt;
 
 typedef enum { MOE_REGIME_AUTO = 0, MOE_REGIME_GEMV = 1, MOE_REGIME_TC = 2 } moe_regime;
 
@@ -110,6 +116,11 @@ typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GEGLU_TANH = 1 } moe_act;
  *     w_dn uint32 [E][d][F/8],  s_dn, b_dn bf16 [E][d][F/64]
  *     element j of a word sits in bits [4j, 4j+3] (low nibble first);
  *     value = scale[group] * q + bias[group].
+ *   MOE_W_Q4G32 / MOE_W_Q4G128: the same with groups of 32 or 128 (DS4Server
+ *     issue #112, "Kernel contract": group 32/64/128); s_* and b_* are
+ *     [E][rows][cols/32] or [E][rows][cols/128]. They run on the
+ *     weight-streaming and fused-decode kernels; the tensor-core kernels take
+ *     group 64, so a forward that would use them runs weight-streaming.
  *   act: moe_act, the gate activation of every expert (0, SwiGLU, when the
  *     struct is zero-initialised); other values: MOE_ERR_INVALID_ARG. */
 typedef struct {

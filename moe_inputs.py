@@ -58,7 +58,7 @@ class Workload:
     k: int
     F: int
     act: str          # "f32" | "bf16"
-    wfmt: str         # "f32" | "bf16" | "q4"
+    wfmt: str         # "f32" | "bf16" | "q4" (group 64) | "q4g32" | "q4g128"
     bias: str = "none"  # "none" | "normal0.5" | "zipf1.1"
     note: str = ""
 
@@ -99,17 +99,22 @@ def _act_dtype(act: str) -> torch.dtype:
     return {"f32": torch.float32, "bf16": torch.bfloat16}[act]
 
 
-def quantize_q4g64(w: torch.Tensor):
+def q4_group(wfmt: str) -> int:
+    """Group size of a 4-bit format name ("q4" is group 64), 0 otherwise."""
+    return {"q4": 64, "q4g32": 32, "q4g128": 128}.get(wfmt, 0)
+
+
+def quantize_q4g64(w: torch.Tensor, group: int = GROUP):
     """Encode fp32 weights [..., n, K] into the packed 4-bit affine format.
 
-    Data generation only: per group of 64 consecutive input elements take
-    min and max, scale = bf16((max - min) / 15), bias = bf16(min), and
+    Data generation only: per group of `group` consecutive input elements
+    take min and max, scale = bf16((max - min) / 15), bias = bf16(min), and
     q = clamp(round_half_even((w - bias) / scale), 0, 15). Returns
-    (packed uint32 [..., n, K/8], scales bf16 [..., n, K/64], biases bf16).
+    (packed uint32 [..., n, K/8], scales bf16 [..., n, K/group], biases bf16).
     """
     *lead, K = w.shape
-    assert K % GROUP == 0
-    wg = w.float().reshape(*lead, K // GROUP, GROUP)
+    assert K % group == 0
+    wg = w.float().reshape(*lead, K // group, group)
     mn = wg.amin(dim=-1)
     mx = wg.amax(dim=-1)
     scale = ((mx - mn) / 15.0).clamp_min(1e-8).to(torch.bfloat16)
@@ -199,10 +204,10 @@ def make_experts(wl: Workload, seed: int, device="cpu") -> Experts:
         elif wl.wfmt == "bf16":
             gu.append(wgu.to(torch.bfloat16))
             dn.append(wdn.to(torch.bfloat16))
-        elif wl.wfmt == "q4":
-            p, s, b = quantize_q4g64(wgu)
+        elif q4_group(wl.wfmt):
+            p, s, b = quantize_q4g64(wgu, q4_group(wl.wfmt))
             gu.append(p); sgu.append(s); bgu.append(b)
-            p, s, b = quantize_q4g64(wdn)
+            p, s, b = quantize_q4g64(wdn, q4_group(wl.wfmt))
             dn.append(p); sdn.append(s); bdn.append(b)
         else:
             raise ValueError(wl.wfmt)

@@ -58,7 +58,13 @@
 #include <string.h>
 
 enum { ORC_F32 = 0, ORC_BF16 = 1 };             /* activation / dense dtypes */
-enum { ORC_W_F32 = 0, ORC_W_BF16 = 1, ORC_W_Q4 = 2 };
+/* 4-bit affine with group 64 (ORC_W_Q4), 32 or 128 input elements per
+ * scale and bias (the group sizes of DS4Server issue #112, "Kernel contract") */
+enum { ORC_W_F32 = 0, ORC_W_BF16 = 1, ORC_W_Q4 = 2, ORC_W_Q4G32 = 3, ORC_W_Q4G128 = 4 };
+
+static int q4_group(int fmt) {
+    return fmt == ORC_W_Q4 ? 64 : fmt == ORC_W_Q4G32 ? 32 : fmt == ORC_W_Q4G128 ? 128 : 0;
+}
 
 /* a bf16 value is the upper 16 bits of the fp32 with the same bits */
 static double bf16_value(uint16_t h) {
@@ -77,8 +83,8 @@ static double act_value(const void* p, int dt, size_t i) {
 typedef struct {
     int fmt;                 /* ORC_W_* */
     const void* w;           /* f32/bf16: [E][rows][cols]; q4: u32 [E][rows][cols/8] */
-    const uint16_t* s;       /* q4 only: bf16 [E][rows][cols/64] */
-    const uint16_t* b;       /* q4 only: bf16 [E][rows][cols/64] */
+    const uint16_t* s;       /* q4 only: bf16 [E][rows][cols/group] */
+    const uint16_t* b;       /* q4 only: bf16 [E][rows][cols/group] */
     int rows, cols;
 } orc_wmat;
 
@@ -89,7 +95,8 @@ static double weight_value(const orc_wmat* m, int e, int r, int c) {
     if (m->fmt == ORC_W_BF16) return bf16_value(((const uint16_t*)m->w)[row * m->cols + c]);
     uint32_t word = ((const uint32_t*)m->w)[row * (m->cols / 8) + c / 8];
     int q = (int)((word >> (4 * (c % 8))) & 0xFu);
-    size_t g = row * (m->cols / 64) + c / 64;
+    const int gs = q4_group(m->fmt);
+    size_t g = row * (m->cols / gs) + c / gs;
     return bf16_value(m->s[g]) * (double)q + bf16_value(m->b[g]);
 }
 

@@ -126,7 +126,8 @@ def _dev(*ts):
             raise ValueError("inputs must be contiguous CUDA tensors")
 
 
-_FMT = {"f32": W_F32, "bf16": W_BF16, "q4": W_Q4G64}
+W_Q4G32, W_Q4G128 = 3, 4
+_FMT = {"f32": W_F32, "bf16": W_BF16, "q4": W_Q4G64, "q4g32": W_Q4G32, "q4g128": W_Q4G128}
 ACT_SWIGLU, ACT_GEGLU_TANH = 0, 1
 _ACT = {"swiglu": ACT_SWIGLU, "geglu": ACT_GEGLU_TANH}
 

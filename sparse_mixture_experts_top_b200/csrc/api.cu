@@ -56,8 +56,11 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
       if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
       break;
     case MOE_W_Q4G64:
+    case MOE_W_Q4G32:
+    case MOE_W_Q4G128:
       if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
       if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
+      if (ex->d % q4_group(ex->fmt) || ex->F % q4_group(ex->fmt)) return MOE_ERR_UNSUPPORTED;
       break;
     default:
       return MOE_ERR_INVALID_ARG;
@@ -289,7 +292,10 @@ moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const
     case MOE_W_F32: row_bytes = (size_t)d * 4; break;
     case MOE_W_BF16: row_bytes = (size_t)d * 2; break;
     case MOE_W_Q4G64:
+    case MOE_W_Q4G32:
+    case MOE_W_Q4G128:
       row_bytes = (size_t)d / 2;
+      if (d % q4_group(fmt)) return MOE_ERR_UNSUPPORTED;
       if (!s_g || !b_g || !s_u || !b_u || !s_gu || !b_gu) return MOE_ERR_INVALID_ARG;
       break;
     default: return MOE_ERR_INVALID_ARG;
@@ -306,8 +312,8 @@ moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const
                              cudaMemcpyDeviceToDevice, s);
   };
   cudaError_t e = pack(w_g, w_u, w_gu, row_bytes);
-  if (e == cudaSuccess && fmt == MOE_W_Q4G64) {
-    const size_t srb = (size_t)(d / 64) * 2;     // one row's bf16 scales (or biases)
+  if (e == cudaSuccess && q4_group(fmt)) {
+    const size_t srb = (size_t)(d / q4_group(fmt)) * 2;   // one row's bf16 scales (or biases)
     e = pack(s_g, s_u, s_gu, srb);
     if (e == cudaSuccess) e = pack(b_g, b_u, b_gu, srb);
   }

@@ -62,6 +62,11 @@ __device__ __forceinline__ float glu(int act, float g, float u) {
   return swiglu(g, u);
 }
 
+// Elements per scale and bias of a 4-bit format (moe_wfmt), 0 for the others
+__host__ __device__ __forceinline__ int q4_group(int fmt) {
+  return fmt == MOE_W_Q4G64 ? 64 : fmt == MOE_W_Q4G32 ? 32 : fmt == MOE_W_Q4G128 ? 128 : 0;
+}
+
 // ---------------------------------------------------------------- warps
 
 __device__ __forceinline__ float warp_sum(float v) {

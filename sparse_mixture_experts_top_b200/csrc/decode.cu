@@ -57,7 +57,9 @@ constexpr int kMaxT = 32;                     // tokens
 constexpr int kMaxR = 256;                    // routed rows T*k
 constexpr int kMaxE = 256;                    // experts (top-k keeps E/32 logits per lane)
 constexpr int kSlots = 10;                    // weight ring slots
-constexpr int kSlotBytes = 18 * 1024;         // gate|up item: 16 KB of words + 2 KB scales
+// gate|up item at d = 2048: 16 KB of words + up to 4 KB of scales and biases
+// (group 32)
+constexpr int kSlotBytes = 20 * 1024;
 constexpr int kTg = 8;                        // tokens per router work unit (one W_r row read)
 constexpr long long kWaitCycles = 2000000000LL;
 
@@ -70,13 +72,14 @@ struct Params {
   const __nv_bfloat16* wr;                    // [E][d]
   const float* rbias;                         // [E] or null
   const uint32_t* w_gu;                       // [E][2F][d/8] q4 words
-  const uint16_t* s_gu;                       // [E][2F][d/64] bf16
+  const uint16_t* s_gu;                       // [E][2F][d/gs] bf16
   const uint16_t* b_gu;
   const uint32_t* w_dn;                       // [E][d][F/8]
-  const uint16_t* s_dn;                       // [E][d][F/64]
+  const uint16_t* s_dn;                       // [E][d][F/gs]
   const uint16_t* b_dn;
   int T, d, E, k, F, BM;
   int act;                                    // the GLU's gate activation (moe_act)
+  int gs, gshift;                             // elements per q4 scale (32, 64, 128), log2
   float* logits;                              // [T][E]
   int32_t* topk_idx;                          // [T][k]
   float* topk_w;                              // [T][k]
@@ -252,7 +255,8 @@ __device__ __noinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile in
 // 2c+1, acc[2..3] row b.
 //
 // K order: lane c takes elements 32c .. 32c + 31 of a step, four q4 words
-// per row, whose scale and bias are those of group 2 st + c / 2. Word j gives
+// per row, which share one scale and bias (groups of 32, 64 or 128 elements,
+// 1 << gshift). Word j gives
 // the fp16 pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7); K slice 2j of the step
 // takes the first two as fragment columns (2c, 2c+1) and (2c+8, 2c+9), slice
 // 2j + 1 the last two. The token rows are stored with every 8 consecutive
@@ -265,7 +269,7 @@ __device__ __forceinline__ void warp_mma_steps(const uint8_t* wa, const uint8_t*
                                                const uint16_t* sa, const uint16_t* ba,
                                                const uint16_t* sb, const uint16_t* bb,
                                                const __half* xrow, bool xvalid, int st0, int nst,
-                                               int sstride, int c, float* acc) {
+                                               int sstride, int gshift, int c, float* acc) {
   float ch[2][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -280,7 +284,7 @@ __device__ __forceinline__ void warp_mma_steps(const uint8_t* wa, const uint8_t*
   auto step = [&](const uint4 (&v)[4], int st) {
     const uint4 wl = *reinterpret_cast<const uint4*>(wa + st * 64 + c * 16);
     const uint4 wh = *reinterpret_cast<const uint4*>(wb + st * 64 + c * 16);
-    const int grp = 2 * st + (c >> 1);
+    const int grp = (st * 128 + c * 32) >> gshift;
     // scales and biases of rows a and b as fp16 pairs (value, value)
     uint32_t s2, b2;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;"
@@ -391,13 +395,14 @@ struct Plan {
   int c0, nC;   // first down item and count
 };
 
-__device__ __forceinline__ Plan make_plan(int d, int F, int nA) {
+__device__ __forceinline__ Plan make_plan(int d, int F, int gshift, int nA) {
   Plan pl;
   pl.nA = nA;
   pl.fpb = F / 8;
-  // 32 rows when they fit a ring slot (their K = F words, scales and biases:
-  // 18 F bytes), so the four warps of a group split an item evenly
-  pl.dr = 18 * F <= kSlotBytes ? 32 : 16;
+  // 32 rows when they fit a ring slot (their F / 2 bytes of words and 2 F / gs
+  // of scales and biases each), so the four warps of a group split an item
+  // evenly
+  pl.dr = 32 * (F / 2 + 4 * (F >> gshift)) <= kSlotBytes ? 32 : 16;
   pl.opb = d / pl.dr;
   const long long G = gridDim.x, c = blockIdx.x;
   const long long totB = (long long)nA * pl.fpb, totC = (long long)nA * pl.opb;
@@ -577,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
   }
   __syncthreads();
-  const Plan pl = make_plan(d, F, s_nact);
+  const Plan pl = make_plan(d, F, p.gshift, s_nact);
   const int nseq = pl.nB + pl.nC;        // ring sequence of this CTA
 
   if (warp == kCw) {
@@ -600,26 +605,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const int gi = pl.b0 + s;
           const int e = s_act[gi / pl.fpb], f0 = (gi % pl.fpb) * 8;
           const size_t rg = (size_t)e * 2 * F + f0, ru = rg + F;   // first gate / up row
-          const uint32_t wb = 8u * (uint32_t)(d / 2), sb = 8u * (uint32_t)(d / 32);
+          const uint32_t wb = 8u * (uint32_t)(d / 2), sb = 8u * 2u * (uint32_t)(d >> p.gshift);
           mbar_expect_tx(bar, 2 * wb + 4 * sb);
           bulk_g2s(dst, p.w_gu + rg * (d / 8), wb, bar);
           bulk_g2s(dst + wb, p.w_gu + ru * (d / 8), wb, bar);
           const uint32_t sc = dst + 2 * wb;
-          bulk_g2s(sc, p.s_gu + rg * (d / 64), sb, bar);
-          bulk_g2s(sc + sb, p.s_gu + ru * (d / 64), sb, bar);
-          bulk_g2s(sc + 2 * sb, p.b_gu + rg * (d / 64), sb, bar);
-          bulk_g2s(sc + 3 * sb, p.b_gu + ru * (d / 64), sb, bar);
+          const size_t gr = (size_t)(d >> p.gshift);          // groups per row
+          bulk_g2s(sc, p.s_gu + rg * gr, sb, bar);
+          bulk_g2s(sc + sb, p.s_gu + ru * gr, sb, bar);
+          bulk_g2s(sc + 2 * sb, p.b_gu + rg * gr, sb, bar);
+          bulk_g2s(sc + 3 * sb, p.b_gu + ru * gr, sb, bar);
         } else {
           const int di = pl.c0 + (s - pl.nB);
           const int a = di / pl.opb, ob = di % pl.opb;
           const size_t r = (size_t)s_act[a] * d + (size_t)ob * pl.dr;  // first of dr rows
           const uint32_t wb = (uint32_t)pl.dr * (uint32_t)(F / 2);
-          const uint32_t sb = (uint32_t)pl.dr * (uint32_t)(F / 32);
+          const uint32_t sb = (uint32_t)pl.dr * 2u * (uint32_t)(F >> p.gshift);
           mbar_expect_tx(bar, wb + 2 * sb);
           bulk_g2s(dst, p.w_dn + r * (F / 8), wb, bar);
           const uint32_t sc = dst + wb;
-          bulk_g2s(sc, p.s_dn + r * (F / 64), sb, bar);
-          bulk_g2s(sc + sb, p.b_dn + r * (F / 64), sb, bar);
+          bulk_g2s(sc, p.s_dn + r * (size_t)(F >> p.gshift), sb, bar);
+          bulk_g2s(sc + sb, p.b_dn + r * (size_t)(F >> p.gshift), sb, bar);
         }
       }
       // copies in flight land before the CTA may exit (bounded, also when
@@ -677,17 +683,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const int e = s_act[gi / pl.fpb];
       const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
       const uint16_t* scl = reinterpret_cast<const uint16_t*>(sp + 16 * rsB);
-      const uint16_t* sg = scl + g * (d / 64);
-      const uint16_t* su = scl + (8 + g) * (d / 64);
-      const uint16_t* bg = scl + (16 + g) * (d / 64);
-      const uint16_t* bu = scl + (24 + g) * (d / 64);
+      const int gB = d >> p.gshift;                // groups per row
+      const uint16_t* sg = scl + g * gB;
+      const uint16_t* su = scl + (8 + g) * gB;
+      const uint16_t* bg = scl + (16 + g) * gB;
+      const uint16_t* bu = scl + (24 + g) * gB;
       for (int q = 0; q * 8 < nv; ++q) {
         const int n = q * 8 + g;
         const bool xv = n < nv;
         const __half* xr = p.x16 + (size_t)(xv ? s_tok[r0 + n] : 0) * d;
         float acc[4], a4[4];
-        warp_mma_steps(sp + g * rsB, sp + (8 + g) * rsB, sg, bg, su, bu, xr, xv, gw, nstB, kGw, c,
-                       acc);
+        warp_mma_steps(sp + g * rsB, sp + (8 + g) * rsB, sg, bg, su, bu, xr, xv, gw, nstB, kGw,
+                       p.gshift, c, acc);
         reduce(acc, a4, kGw);
         // lane (g, c): gate (a4[0..1]) and up (a4[2..3]) of feature f0 + g
         // for the expert's tokens q*8 + 2c, q*8 + 2c + 1
@@ -728,16 +735,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const int e = s_act[a];
       const int r0 = s_roff[e], nv = s_roff[e + 1] - r0;
       const uint16_t* sc_ = reinterpret_cast<const uint16_t*>(sp + pl.dr * rsC);
-      const uint16_t* bi_ = sc_ + pl.dr * (F / 64);
+      const int gC = F >> p.gshift;                // groups per row
+      const uint16_t* bi_ = sc_ + pl.dr * gC;
       const int ra = rbC + g, rb_ = rbC + 8 + g;     // A rows g and g + 8 of this warp
       for (int q = 0; q * 8 < nv; ++q) {
         const int n = q * 8 + g;
         const bool hvld = n < nv;
         const __half* hr = p.h + (size_t)(hvld ? r0 + n : 0) * F;
         float acc[4], a4[4];
-        warp_mma_steps(sp + ra * rsC, sp + rb_ * rsC, sc_ + ra * (F / 64), bi_ + ra * (F / 64),
-                       sc_ + rb_ * (F / 64), bi_ + rb_ * (F / 64), hr, hvld, gw % ksC, nstC, ksC,
-                       c, acc);
+        warp_mma_steps(sp + ra * rsC, sp + rb_ * rsC, sc_ + ra * gC, bi_ + ra * gC, sc_ + rb_ * gC,
+                       bi_ + rb_ * gC, hr, hvld, gw % ksC, nstC, ksC, p.gshift, c, acc);
         reduce(acc, a4, ksC);
         // lane (g, c): outputs o0 + g (a4[0..1]) and o0 + 8 + g (a4[2..3])
         // of the expert's rows q*8 + 2c, q*8 + 2c + 1
@@ -838,7 +845,7 @@ static int sm_count() {
 
 bool decode_fused_ok(int T, int k, int E, int d, int F, int fmt, int dt) {
   using namespace dec;
-  return fmt == MOE_W_Q4G64 && dt == MOE_BF16 && T >= 1 && T <= kMaxT && T * k <= kMaxR &&
+  return q4_group(fmt) != 0 && dt == MOE_BF16 && T >= 1 && T <= kMaxT && T * k <= kMaxR &&
          E <= kMaxE && k <= 32 && d % 128 == 0 && F % 128 == 0 && d <= 2048 && F <= 2048;
 }
 
@@ -871,6 +878,8 @@ cudaError_t launch_decode_fused(const void* x, const void* w_router, const float
   p.F = ex.F;
   p.BM = BM;
   p.act = ex.act;
+  p.gs = q4_group(ex.fmt);
+  p.gshift = p.gs == 32 ? 5 : p.gs == 64 ? 6 : 7;
   p.logits = logits;
   p.topk_idx = idx;
   p.topk_w = w;

@@ -93,12 +93,13 @@ __device__ __forceinline__ void load_act(const TA* p, float* out) {
 }
 
 // Elements of the weight row covered by 32-bit word `wi` start at wi*EPW.
-// q4 scales/biases: one per 64 elements.
+// q4 scales/biases: one per gs (32, 64 or 128) elements; every 4-bit format
+// runs the MOE_W_Q4G64 instantiation with its own gs.
 template <int FMT>
 __device__ __forceinline__ void scale_bias(const uint16_t* s, const uint16_t* b, size_t row,
-                                           int K, int elem, float& sv, float& bv) {
+                                           int K, int elem, int gs, float& sv, float& bv) {
   if constexpr (FMT == MOE_W_Q4G64) {
-    size_t g = row * (size_t)(K / 64) + elem / 64;
+    size_t g = row * (size_t)(K / gs) + elem / gs;
     sv = bf16_bits_to_f32(__ldg(s + g));
     bv = bf16_bits_to_f32(__ldg(b + g));
   } else {
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
     const TA* __restrict__ x, const uint32_t* __restrict__ row_map,
     const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E, int d,
     int F, const uint32_t* __restrict__ wgu, const uint16_t* __restrict__ sgu,
-    const uint16_t* __restrict__ bgu, typename HType<TA>::T* __restrict__ h, int act,
+    const uint16_t* __restrict__ bgu, typename HType<TA>::T* __restrict__ h, int act, int qg,
     int* status) {
   pdl_wait();
   pdl_launch();
@@ -157,8 +158,8 @@ __global__ void __launch_bounds__(256) swiglu_gemv_kernel(
       for (int q = 0; q < 4; ++q) {
         const int elem = (c * 4 + q) * EPW;
         float gs, gb, us, ub;
-        scale_bias<FMT>(sgu, bgu, grow, d, elem, gs, gb);
-        scale_bias<FMT>(sgu, bgu, urow, d, elem, us, ub);
+        scale_bias<FMT>(sgu, bgu, grow, d, elem, qg, gs, gb);
+        scale_bias<FMT>(sgu, bgu, urow, d, elem, qg, us, ub);
         float gv[EPW], uv[EPW];
         D::run(gws[q], gs, gb, gv);
         D::run(uws[q], us, ub, uv);
@@ -200,7 +201,8 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
     const typename HType<TA>::T* __restrict__ hin, const int32_t* __restrict__ row_off,
     const int32_t* __restrict__ tile_off, int BM, int E, int d, int F,
     const uint32_t* __restrict__ wdn, const uint16_t* __restrict__ sdn,
-    const uint16_t* __restrict__ bdn, typename HType<TA>::T* __restrict__ ys, int* status) {
+    const uint16_t* __restrict__ bdn, typename HType<TA>::T* __restrict__ ys, int qg,
+    int* status) {
   pdl_wait();
   pdl_launch();
   using D = WDecode<FMT>;
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
       for (int q = 0; q < 4; ++q) {
         const int elem = (c * 4 + q) * EPW;
         float s, b;
-        scale_bias<FMT>(sdn, bdn, wrow, F, elem, s, b);
+        scale_bias<FMT>(sdn, bdn, wrow, F, elem, qg, s, b);
         float wv[EPW];
         D::run(wws[q], s, b, wv);
 #pragma unroll
@@ -274,10 +276,11 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
 #define MOE_SWIGLU(TA, FMT)                                                                    \
   launch_pdl(swiglu_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const TA*)x, row_map, row_off, tile_off, BM, \
                                                    ex.E, ex.d, ex.F, w, sc, bi,                  \
-                                                   (typename HType<TA>::T*)h, ex.act, status)
+                                                   (typename HType<TA>::T*)h, ex.act,          \
+                                                   q4_group(ex.fmt), status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_SWIGLU(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_SWIGLU(__nv_bfloat16, MOE_W_BF16);
-  else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q4G64);
+  else if (dt == MOE_BF16 && q4_group(ex.fmt)) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q4G64);
   else return cudaErrorInvalidValue;
 #undef MOE_SWIGLU
   return cudaGetLastError();
@@ -296,10 +299,11 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
 #define MOE_DOWN(TA, FMT)                                                                    \
   launch_pdl(down_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const typename HType<TA>::T*)h, row_off,    \
                                                  tile_off, BM, ex.E, ex.d, ex.F, w, sc, bi,     \
-                                                 (typename HType<TA>::T*)ys, status)
+                                                 (typename HType<TA>::T*)ys,                \
+                                                 q4_group(ex.fmt), status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_DOWN(__nv_bfloat16, MOE_W_BF16);
-  else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q4G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
+  else if (dt == MOE_BF16 && q4_group(ex.fmt)) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
   else return cudaErrorInvalidValue;
 #undef MOE_DOWN
   return cudaGetLastError();
@@ -373,7 +377,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
     const __half* __restrict__ x16, const uint32_t* __restrict__ row_map,
     const int32_t* __restrict__ row_off, const int32_t* __restrict__ tile_off, int BM, int E,
     int d, int F, const uint32_t* __restrict__ w, const uint16_t* __restrict__ sc,
-    const uint16_t* __restrict__ bi, void* __restrict__ out, int act, int* status) {
+    const uint16_t* __restrict__ bi, void* __restrict__ out, int act, int gs, int* status) {
   pdl_wait();
   pdl_launch();
   __shared__ float red[kMmaWarps - 1][32][8];
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
   const int blk = blockIdx.x;                   // block of 16 weight rows
   const size_t row_lo = (size_t)e * rows_e + (SWIGLU ? blk * 8 + g : blk * 16 + g);
   const size_t row_hi = SWIGLU ? row_lo + F : row_lo + 8;
-  const int words = K / 8, G = K / 64;
+  const int words = K / 8, G = K / gs;         // gs: elements per scale (32, 64 or 128)
   const uint32_t* wlo = w + row_lo * words;
   const uint32_t* whi = w + row_hi * words;
   // token rows of this lane's B fragment: tokens g (group 0) and 8+g (group 1)
@@ -417,7 +421,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
     const int k0 = st * 128 + c * 32;
     S.wl = ldg_nc_v4(wlo + k0 / 8);
     S.wh = ldg_nc_v4(whi + k0 / 8);
-    const int grp = k0 / 64;
+    const int grp = k0 / gs;                    // a lane's 32 elements share one group
     S.sl = __ldg(sc + row_lo * G + grp);
     S.bl = __ldg(bi + row_lo * G + grp);
     S.sh = __ldg(sc + row_hi * G + grp);
@@ -508,7 +512,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
 }
 
 bool gemv_q4_mma_ok(const moe_experts& ex, int dt, int BM) {
-  return ex.fmt == MOE_W_Q4G64 && dt == MOE_BF16 && BM <= kMmaMaxRows && ex.d % 128 == 0 &&
+  return q4_group(ex.fmt) != 0 && dt == MOE_BF16 && BM <= kMmaMaxRows && ex.d % 128 == 0 &&
          ex.F % 128 == 0;
 }
 
@@ -522,7 +526,7 @@ cudaError_t launch_swiglu_q4_mma(const void* x16, const uint32_t* row_map, const
   launch_pdl(gemv_q4_mma_kernel<true>, grid, kMmaWarps * 32, 0, s, 
       (const __half*)x16, row_map, row_off, tile_off, BM, ex.E, ex.d, ex.F,
       (const uint32_t*)ex.w_gu, (const uint16_t*)ex.s_gu, (const uint16_t*)ex.b_gu, h, ex.act,
-      status);
+      q4_group(ex.fmt), status);
   return cudaGetLastError();
 }
 
@@ -536,7 +540,7 @@ cudaError_t launch_down_q4_mma(const void* h, const int32_t* row_off, const int3
   launch_pdl(gemv_q4_mma_kernel<false>, grid, kMmaWarps * 32, 0, s, 
       (const __half*)h, nullptr, row_off, tile_off, BM, ex.E, ex.d, ex.F,
       (const uint32_t*)ex.w_dn, (const uint16_t*)ex.s_dn, (const uint16_t*)ex.b_dn, ys,
-      MOE_ACT_SWIGLU, status);
+      MOE_ACT_SWIGLU, q4_group(ex.fmt), status);
   return cudaGetLastError();
 }
 

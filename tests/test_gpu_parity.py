@@ -164,7 +164,7 @@ def test_grouped_swiglu_parity(moe, orc, name, T, regime, BM, skew):
         assert h.dtype == torch.float16
         g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
         # q4 weights are dequantised to fp16 (bf16 weights are exact in fp16)
-        u_w = U_F16 if wl.wfmt == "q4" else 0.0
+        u_w = U_F16 if mi.q4_group(wl.wfmt) else 0.0
         assert_h_close(h, href, g, u, ga, ua, wl.d, u_w, U_F16, TOL_BF16, f"h[{name}]")
 
 
@@ -182,7 +182,7 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
     # ys is stored in fp16 for bf16 activations, fp32 for fp32
     assert ys.dtype == (torch.float16 if wl.act == "bf16" else torch.float32)
     habs = orc.expert_down_abs(hin.double().numpy(), ref_st.row_off, hx)
-    u_w = U_F16 if wl.wfmt == "q4" else 0.0
+    u_w = U_F16 if mi.q4_group(wl.wfmt) else 0.0
     u_ys = U_F16 if wl.act == "bf16" else 0.0
     assert_ys_close(ys, yref, habs, u_w, _tol(wl.act), f"ys[{name}]", u_ys=u_ys)
 
@@ -297,7 +297,7 @@ def test_grouped_geglu_parity(moe, orc, name, T, regime, BM):
     hx = _host(ex)
     href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
     g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
-    u_w = U_F16 if wl.wfmt == "q4" else 0.0
+    u_w = U_F16 if mi.q4_group(wl.wfmt) else 0.0
     assert_h_close(h, href, g, u, ga, ua, wl.d, u_w, U_F16, TOL_BF16, f"h[{name}, GeGLU]",
                    act="geglu")
 
@@ -334,13 +334,53 @@ def test_pack_separate_gate_up(moe, name):
     w_gu, s_gu, b_gu = moe.pack_gate_up(ex.fmt, wg, wu, sg, bg, su, bu)
     torch.cuda.synchronize()
     assert torch.equal(w_gu, ex.w_gu)
-    if ex.fmt == "q4":
+    if mi.q4_group(ex.fmt):
         assert torch.equal(s_gu, ex.s_gu) and torch.equal(b_gu, ex.b_gu)
     packed = mi.Experts(ex.fmt, ex.E, ex.d, F, w_gu, ex.w_dn, s_gu, b_gu, ex.s_dn, ex.b_dn)
     a = moe.forward(layer.x, layer.w_router, layer.router_bias, ex, layer.wl.k)
     b = moe.forward(layer.x, layer.w_router, layer.router_bias, packed, layer.wl.k)
     assert torch.equal(a.view(torch.int16) if a.dtype != torch.float32 else a,
                        b.view(torch.int16) if b.dtype != torch.float32 else b)
+
+
+# ------------------------------------------------------------------ q4 groups 32 / 128
+
+@pytest.mark.parametrize("wfmt", ["q4g32", "q4g128"])
+@pytest.mark.parametrize("name,T", [("decode_t1", 1), ("decode_t32", 32)])
+def test_forward_q4_group_sizes_fused_decode(moe, orc, wfmt, name, T):
+    """4-bit weights with groups of 32 and 128 (DS4Server issue #112, "Kernel
+    contract") through the fused decode kernel."""
+    layer = mi.make_layer(mi.workload(name, T=T, wfmt=wfmt), seed=6, device=DEV)
+    _forward_and_compare(moe, orc, layer)
+
+
+@pytest.mark.parametrize("wfmt", ["q4g32", "q4g128"])
+def test_grouped_stages_q4_group_sizes(moe, orc, wfmt):
+    """The weight-streaming gate|up and down kernels with groups of 32 / 128."""
+    wl = mi.workload("decode_t32", T=32, wfmt=wfmt)
+    layer, idx = _stage_setup(wl, 32, 29, 0.0)
+    st = moe.sort_rows(idx.to(DEV), wl.E, 8)
+    h = moe.grouped_swiglu(layer.x, st, wl.k, layer.experts, regime=1)
+    ref_st = orc.sort_rows(idx.numpy(), wl.E, 8)
+    hx = _host(layer.experts)
+    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    assert_h_close(h, href, g, u, ga, ua, wl.d, U_F16, U_F16, TOL_BF16, f"h[{wfmt}]")
+    ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1)
+    yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    assert_ys_close(ys, yref, habs, U_F16, TOL_BF16, f"ys[{wfmt}]", u_ys=U_F16)
+
+
+@pytest.mark.parametrize("wfmt,T", [("q4g128", 300), ("q4g32", 1024)])
+def test_forward_q4_group_sizes_prefill_shape(moe, orc, wfmt, T):
+    """Prefill shapes: 300 tokens run the weight-streaming tensor-core GEMV;
+    1,024 tokens would take the tcgen05 kernels, which take group 64 only,
+    so the forward runs the weight-streaming kernels with 128-row tiles."""
+    layer = mi.make_layer(mi.workload("prefill", T=T, wfmt=wfmt), seed=8, device=DEV)
+    rng = np.random.default_rng(3)
+    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(T, 32, replace=False)))
+    assert moe.device_status() == moe.OK
 
 
 def test_forward_deterministic(moe):

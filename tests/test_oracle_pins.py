@@ -85,6 +85,28 @@ def test_q4_forward_equals_dense_forward_on_same_values(orc):
     np.testing.assert_allclose(a.y, b.y, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("fmt", ["q4g32", "q4g128"])
+def test_q4_other_group_sizes_dequantise_to_the_encoded_weights(orc, fmt):
+    """Groups of 32 and 128 (DS4Server issue #112, "Kernel contract"): the
+    oracle's value of every element is within half a quantisation step of the
+    fp32 weight the generator encoded. A wrong group index takes another
+    group's scale and bias and misses by far more than that (the groups are
+    given very different ranges)."""
+    G = mi.q4_group(fmt)
+    K = 256
+    torch.manual_seed(1)
+    # group j spans [-(j + 1), j + 1] / 4: every group's scale and bias differ
+    spread = (torch.arange(K // G, dtype=torch.float32) + 1.0).repeat_interleave(G) / 4
+    w = (torch.rand(1, 3, K) * 2 - 1) * spread
+    p, s, b = mi.quantize_q4g64(w, G)
+    ex = mi.Experts(fmt, 1, K, 2, p, torch.zeros(1, K, 1, dtype=torch.uint32), s, b)
+    for r in range(3):
+        for c in range(K):
+            step = float(s[0, r, c // G].float())
+            got = orc.weight_value(ex, "gu", 0, r, c)
+            assert abs(got - float(w[0, r, c])) <= 0.5 * step * (1 + 1e-2) + 1e-6, (r, c)
+
+
 def test_q4_encoder_roundtrip_is_close(orc):
     """Generator sanity (not a pin of the oracle): dequantised weights stay
     within half a quantisation step of the fp32 weights they encode."""
