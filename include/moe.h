@@ -94,7 +94,8 @@ typedef enum {
   MOE_W_BF16 = 1,
   MOE_W_Q4G64 = 2,
   MOE_W_Q4G32 = 3,   /* as MOE_W_Q4G64 with one scale and bias per 32 elements */
-  MOE_W_Q4G128 = 4   /* ... per 128 elements */
+  MOE_W_Q4G128 = 4,  /* ... per 128 elements */
+  MOE_W_Q8G64 = 5    /* 8-bit affine, group 64 */
 } moe_wfmt;
 
 typedef enum { MOE_REGIME_AUTO = 0, MOE_REGIME_GEMV = 1, MOE_REGIME_TC = 2 } moe_regime;
@@ -121,6 +122,11 @@ typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GEGLU_TANH = 1 } moe_act;
  *     [E][rows][cols/32] or [E][rows][cols/128]. They run on the
  *     weight-streaming and fused-decode kernels; the tensor-core kernels take
  *     group 64, so a forward that would use them runs weight-streaming.
+ *   MOE_W_Q8G64 (8-bit affine; mlxcel PR #275, "Multi-bit handling"; DS4Server
+ *   issue #112, "Kernel contract": 4 or 8 bits):
+ *     w_gu uint32 [E][2F][d/4], w_dn uint32 [E][d][F/4], byte j of a word is
+ *     element j; s_*, b_* bf16 [E][rows][cols/64]; value = scale * q + bias.
+ *     It runs on the weight-streaming SIMT kernels only.
  *   act: moe_act, the gate activation of every expert (0, SwiGLU, when the
  *     struct is zero-initialised); other values: MOE_ERR_INVALID_ARG. */
 typedef struct {

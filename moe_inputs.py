@@ -58,7 +58,7 @@ class Workload:
     k: int
     F: int
     act: str          # "f32" | "bf16"
-    wfmt: str         # "f32" | "bf16" | "q4" (group 64) | "q4g32" | "q4g128"
+    wfmt: str         # "f32" | "bf16" | "q4" (group 64) | "q4g32" | "q4g128" | "q8"
     bias: str = "none"  # "none" | "normal0.5" | "zipf1.1"
     note: str = ""
 
@@ -127,6 +127,26 @@ def quantize_q4g64(w: torch.Tensor, group: int = GROUP):
     # reinterpret the low 32 bits as uint32 storage
     packed = torch.where(packed >= 2**31, packed - 2**32, packed).to(torch.int32)
     return packed.view(torch.uint32), scale, bias
+
+
+def quantize_q8g64(w: torch.Tensor):
+    """Encode fp32 weights [..., n, K] into the packed 8-bit affine format:
+    per group of 64 inputs scale = bf16((max - min) / 255), bias = bf16(min),
+    q = clamp(round_half_even((w - bias) / scale), 0, 255), byte j of each
+    uint32 word = element j (data generation only)."""
+    *lead, K = w.shape
+    assert K % GROUP == 0
+    wg = w.float().reshape(*lead, K // GROUP, GROUP)
+    mn = wg.amin(dim=-1)
+    mx = wg.amax(dim=-1)
+    scale = ((mx - mn) / 255.0).clamp_min(1e-8).to(torch.bfloat16)
+    bias = mn.to(torch.bfloat16)
+    q = torch.round((wg - bias.float().unsqueeze(-1)) / scale.float().unsqueeze(-1))
+    q = q.clamp_(0, 255).to(torch.int64).reshape(*lead, K // 4, 4)
+    shifts = torch.arange(4, device=w.device, dtype=torch.int64) * 8
+    words = (q << shifts).sum(dim=-1)
+    words = torch.where(words >= 2**31, words - 2**32, words).to(torch.int32)
+    return words.view(torch.uint32), scale, bias
 
 
 def pack_nibbles(q: torch.Tensor) -> torch.Tensor:
@@ -204,6 +224,11 @@ def make_experts(wl: Workload, seed: int, device="cpu") -> Experts:
         elif wl.wfmt == "bf16":
             gu.append(wgu.to(torch.bfloat16))
             dn.append(wdn.to(torch.bfloat16))
+        elif wl.wfmt == "q8":
+            p, s, b = quantize_q8g64(wgu)
+            gu.append(p); sgu.append(s); bgu.append(b)
+            p, s, b = quantize_q8g64(wdn)
+            dn.append(p); sdn.append(s); bdn.append(b)
         elif q4_group(wl.wfmt):
             p, s, b = quantize_q4g64(wgu, q4_group(wl.wfmt))
             gu.append(p); sgu.append(s); bgu.append(b)

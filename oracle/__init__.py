@@ -34,7 +34,7 @@ _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liborc_moe.so")
 
 ACT = {"f32": 0, "bf16": 1}
-WFMT = {"f32": 0, "bf16": 1, "q4": 2, "q4g32": 3, "q4g128": 4}
+WFMT = {"f32": 0, "bf16": 1, "q4": 2, "q4g32": 3, "q4g128": 4, "q8": 5}
 
 
 def build(force: bool = False) -> str:

@@ -60,7 +60,8 @@
 enum { ORC_F32 = 0, ORC_BF16 = 1 };             /* activation / dense dtypes */
 /* 4-bit affine with group 64 (ORC_W_Q4), 32 or 128 input elements per
  * scale and bias (the group sizes of DS4Server issue #112, "Kernel contract") */
-enum { ORC_W_F32 = 0, ORC_W_BF16 = 1, ORC_W_Q4 = 2, ORC_W_Q4G32 = 3, ORC_W_Q4G128 = 4 };
+enum { ORC_W_F32 = 0, ORC_W_BF16 = 1, ORC_W_Q4 = 2, ORC_W_Q4G32 = 3, ORC_W_Q4G128 = 4,
+       ORC_W_Q8 = 5 /* 8-bit affine, group 64: byte j of a word is element j */ };
 
 static int q4_group(int fmt) {
     return fmt == ORC_W_Q4 ? 64 : fmt == ORC_W_Q4G32 ? 32 : fmt == ORC_W_Q4G128 ? 128 : 0;
@@ -93,6 +94,12 @@ static double weight_value(const orc_wmat* m, int e, int r, int c) {
     size_t row = (size_t)e * m->rows + r;
     if (m->fmt == ORC_W_F32) return (double)((const float*)m->w)[row * m->cols + c];
     if (m->fmt == ORC_W_BF16) return bf16_value(((const uint16_t*)m->w)[row * m->cols + c]);
+    if (m->fmt == ORC_W_Q8) {
+        uint32_t word8 = ((const uint32_t*)m->w)[row * (m->cols / 4) + c / 4];
+        int q8 = (int)((word8 >> (8 * (c % 4))) & 0xFFu);
+        size_t g8 = row * (m->cols / 64) + c / 64;
+        return bf16_value(m->s[g8]) * (double)q8 + bf16_value(m->b[g8]);
+    }
     uint32_t word = ((const uint32_t*)m->w)[row * (m->cols / 8) + c / 8];
     int q = (int)((word >> (4 * (c % 8))) & 0xFu);
     const int gs = q4_group(m->fmt);

@@ -126,8 +126,9 @@ def _dev(*ts):
             raise ValueError("inputs must be contiguous CUDA tensors")
 
 
-W_Q4G32, W_Q4G128 = 3, 4
-_FMT = {"f32": W_F32, "bf16": W_BF16, "q4": W_Q4G64, "q4g32": W_Q4G32, "q4g128": W_Q4G128}
+W_Q4G32, W_Q4G128, W_Q8G64 = 3, 4, 5
+_FMT = {"f32": W_F32, "bf16": W_BF16, "q4": W_Q4G64, "q4g32": W_Q4G32, "q4g128": W_Q4G128,
+        "q8": W_Q8G64}
 ACT_SWIGLU, ACT_GEGLU_TANH = 0, 1
 _ACT = {"swiglu": ACT_SWIGLU, "geglu": ACT_GEGLU_TANH}
 
@@ -278,11 +279,13 @@ def pack_gate_up(fmt, w_g, w_u, s_g=None, b_g=None, s_u=None, b_u=None, stream=N
     _dev(w_g, w_u, s_g, b_g, s_u, b_u)
     E, F = w_g.shape[0], w_g.shape[1]
     fmt_c = _FMT[fmt] if isinstance(fmt, str) else int(fmt)
-    d = {W_F32: w_g.shape[2], W_BF16: w_g.shape[2], W_Q4G64: w_g.shape[2] * 8}[fmt_c]
+    per_word = {W_Q4G64: 8, W_Q4G32: 8, W_Q4G128: 8, W_Q8G64: 4}.get(fmt_c, 1)
+    d = w_g.shape[2] * per_word
+    group = {W_Q4G64: 64, W_Q4G32: 32, W_Q4G128: 128, W_Q8G64: 64}.get(fmt_c, 0)
     w_gu = torch.empty((E, 2 * F) + tuple(w_g.shape[2:]), dtype=w_g.dtype, device=w_g.device)
     s_gu = b_gu = None
-    if fmt_c == W_Q4G64:
-        s_gu = torch.empty((E, 2 * F, d // 64), dtype=s_g.dtype, device=s_g.device)
+    if group:
+        s_gu = torch.empty((E, 2 * F, d // group), dtype=s_g.dtype, device=s_g.device)
         b_gu = torch.empty_like(s_gu)
     _check(lib.moe_pack_gate_up(fmt_c, E, d, F, _ptr(w_g), _ptr(s_g), _ptr(b_g), _ptr(w_u),
                                 _ptr(s_u), _ptr(b_u), _ptr(w_gu), _ptr(s_gu), _ptr(b_gu),

@@ -62,6 +62,10 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
       if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
       if (ex->d % q4_group(ex->fmt) || ex->F % q4_group(ex->fmt)) return MOE_ERR_UNSUPPORTED;
       break;
+    case MOE_W_Q8G64:
+      if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
+      break;
     default:
       return MOE_ERR_INVALID_ARG;
   }
@@ -294,8 +298,9 @@ moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const
     case MOE_W_Q4G64:
     case MOE_W_Q4G32:
     case MOE_W_Q4G128:
-      row_bytes = (size_t)d / 2;
-      if (d % q4_group(fmt)) return MOE_ERR_UNSUPPORTED;
+    case MOE_W_Q8G64:
+      row_bytes = fmt == MOE_W_Q8G64 ? (size_t)d : (size_t)d / 2;
+      if (d % wq_group(fmt)) return MOE_ERR_UNSUPPORTED;
       if (!s_g || !b_g || !s_u || !b_u || !s_gu || !b_gu) return MOE_ERR_INVALID_ARG;
       break;
     default: return MOE_ERR_INVALID_ARG;
@@ -312,8 +317,8 @@ moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const
                              cudaMemcpyDeviceToDevice, s);
   };
   cudaError_t e = pack(w_g, w_u, w_gu, row_bytes);
-  if (e == cudaSuccess && q4_group(fmt)) {
-    const size_t srb = (size_t)(d / q4_group(fmt)) * 2;   // one row's bf16 scales (or biases)
+  if (e == cudaSuccess && wq_group(fmt)) {
+    const size_t srb = (size_t)(d / wq_group(fmt)) * 2;   // one row's bf16 scales (or biases)
     e = pack(s_g, s_u, s_gu, srb);
     if (e == cudaSuccess) e = pack(b_g, b_u, b_gu, srb);
   }

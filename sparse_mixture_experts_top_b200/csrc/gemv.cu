@@ -50,6 +50,15 @@ template <> struct WDecode<MOE_W_Q4G64> {
   }
 };
 
+template <> struct WDecode<MOE_W_Q8G64> {
+  static constexpr int EPW = 4;
+  // value = scale * q + bias, q = byte j of the word (element j)
+  __device__ __forceinline__ static void run(uint32_t w, float s, float b, float* out) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[j] = fmaf(s, (float)((w >> (8 * j)) & 0xFFu), b);
+  }
+};
+
 // The hidden rows h between the two projections: fp16 for bf16 activations
 // (the tensor-core operand format, 11-bit precision), fp32 for fp32.
 template <typename TA> struct HType { using T = float; };
@@ -63,8 +72,12 @@ __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t v) {
 template <typename TA, int N>
 __device__ __forceinline__ void load_act(const TA* p, float* out) {
   if constexpr (std::is_same<TA, __half>::value) {
-    static_assert(N == 2 || N == 8, "fp16 rows come in words of 2 or 8");
-    if constexpr (N == 8) {
+    static_assert(N == 2 || N == 4 || N == 8, "fp16 rows come in words of 2, 4 or 8");
+    if constexpr (N == 4) {
+      uint2 v = *reinterpret_cast<const uint2*>(p);
+      float2 a = f16x2_to_f32x2(v.x), b = f16x2_to_f32x2(v.y);
+      out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+    } else if constexpr (N == 8) {
       uint4 v = ldg_v4(p);
       float2 a = f16x2_to_f32x2(v.x), b = f16x2_to_f32x2(v.y);
       float2 c = f16x2_to_f32x2(v.z), d = f16x2_to_f32x2(v.w);
@@ -75,8 +88,12 @@ __device__ __forceinline__ void load_act(const TA* p, float* out) {
       out[0] = a.x; out[1] = a.y;
     }
   } else if constexpr (sizeof(TA) == 2) {
-    static_assert(N == 2 || N == 8, "bf16 activations come in words of 2 or 8");
-    if constexpr (N == 8) {
+    static_assert(N == 2 || N == 4 || N == 8, "bf16 activations come in words of 2, 4 or 8");
+    if constexpr (N == 4) {
+      uint2 v = *reinterpret_cast<const uint2*>(p);
+      float2 a = bf16x2_to_f32x2(v.x), b = bf16x2_to_f32x2(v.y);
+      out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+    } else if constexpr (N == 8) {
       uint4 v = ldg_v4(p);
       float2 a = bf16x2_to_f32x2(v.x), b = bf16x2_to_f32x2(v.y);
       float2 c = bf16x2_to_f32x2(v.z), d = bf16x2_to_f32x2(v.w);
@@ -98,7 +115,7 @@ __device__ __forceinline__ void load_act(const TA* p, float* out) {
 template <int FMT>
 __device__ __forceinline__ void scale_bias(const uint16_t* s, const uint16_t* b, size_t row,
                                            int K, int elem, int gs, float& sv, float& bv) {
-  if constexpr (FMT == MOE_W_Q4G64) {
+  if constexpr (FMT == MOE_W_Q4G64 || FMT == MOE_W_Q8G64) {
     size_t g = row * (size_t)(K / gs) + elem / gs;
     sv = bf16_bits_to_f32(__ldg(s + g));
     bv = bf16_bits_to_f32(__ldg(b + g));
@@ -277,10 +294,11 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
   launch_pdl(swiglu_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const TA*)x, row_map, row_off, tile_off, BM, \
                                                    ex.E, ex.d, ex.F, w, sc, bi,                  \
                                                    (typename HType<TA>::T*)h, ex.act,          \
-                                                   q4_group(ex.fmt), status)
+                                                   wq_group(ex.fmt), status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_SWIGLU(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_SWIGLU(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && q4_group(ex.fmt)) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q4G64);
+  else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q8G64) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q8G64);
   else return cudaErrorInvalidValue;
 #undef MOE_SWIGLU
   return cudaGetLastError();
@@ -300,10 +318,11 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
   launch_pdl(down_gemv_kernel<TA, FMT>, grid, 256, 0, s, (const typename HType<TA>::T*)h, row_off,    \
                                                  tile_off, BM, ex.E, ex.d, ex.F, w, sc, bi,     \
                                                  (typename HType<TA>::T*)ys,                \
-                                                 q4_group(ex.fmt), status)
+                                                 wq_group(ex.fmt), status)
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_DOWN(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && q4_group(ex.fmt)) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
+  else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q8G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q8G64);
   else return cudaErrorInvalidValue;
 #undef MOE_DOWN
   return cudaGetLastError();

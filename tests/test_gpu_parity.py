@@ -383,6 +383,33 @@ def test_forward_q4_group_sizes_prefill_shape(moe, orc, wfmt, T):
     assert moe.device_status() == moe.OK
 
 
+# ------------------------------------------------------------------ 8-bit affine
+
+def test_grouped_stages_q8(moe, orc):
+    """8-bit affine weights (mlxcel PR #275, "Multi-bit handling") through the
+    weight-streaming gate|up and down kernels."""
+    wl = mi.workload("decode_t32", T=32, wfmt="q8")
+    layer, idx = _stage_setup(wl, 32, 31, 0.0)
+    st = moe.sort_rows(idx.to(DEV), wl.E, 8)
+    h = moe.grouped_swiglu(layer.x, st, wl.k, layer.experts, regime=1)
+    ref_st = orc.sort_rows(idx.numpy(), wl.E, 8)
+    hx = _host(layer.experts)
+    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    # the SIMT kernel dequantises in fp32: 2^-24 per weight
+    assert_h_close(h, href, g, u, ga, ua, wl.d, 2.0 ** -24, U_F16, TOL_BF16, "h[q8]")
+    ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1)
+    yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    assert_ys_close(ys, yref, habs, 2.0 ** -24, TOL_BF16, "ys[q8]", u_ys=U_F16)
+
+
+@pytest.mark.parametrize("name,T", [("decode_t1", 1), ("prefill", 64)])
+def test_forward_q8(moe, orc, name, T):
+    layer = mi.make_layer(mi.workload(name, T=T, wfmt="q8"), seed=9, device=DEV)
+    _forward_and_compare(moe, orc, layer)
+
+
 def test_forward_deterministic(moe):
     layer = mi.make_layer("decode_t32", seed=3, device=DEV)
     a = moe.forward(layer.x, layer.w_router, None, layer.experts, layer.wl.k)
@@ -390,13 +417,14 @@ def test_forward_deterministic(moe):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["acceptance", "prefill"])
-def test_tensor_core_forward_repeats_bit_exact(moe, name):
-    """The tensor-core path gives the same bits on every repeat. A raw weight
+@pytest.mark.parametrize("name", ["acceptance", "prefill", "decode_t1", "decode_t32"])
+def test_forward_repeats_bit_exact(moe, name):
+    """Every path gives the same bits on every repeat (tensor-core kernels for
+    acceptance and prefill, the fused decode kernel for decode). A raw weight
     stage released before the dequantising warps' shared-memory loads had
     read it let the next TMA overwrite its first rows under them: a few
     features of one tile came out wrong in about one run in five (bf16
-    weights); 24 repeats catch that with near certainty."""
+    weights); 24 repeats catch a race of that rate with near certainty."""
     layer = mi.make_layer(name, seed=0, device=DEV)
     wl = layer.wl
     ws = moe.forward_workspace(layer.x, layer.experts, wl.k)

@@ -107,6 +107,29 @@ def test_q4_other_group_sizes_dequantise_to_the_encoded_weights(orc, fmt):
             assert abs(got - float(w[0, r, c])) <= 0.5 * step * (1 + 1e-2) + 1e-6, (r, c)
 
 
+def test_q8_dequantises_to_the_encoded_weights(orc):
+    """8-bit affine (mlxcel PR #275, "Multi-bit handling"): every element of
+    the oracle's dequantisation is within half a quantisation step (plus the
+    bf16 rounding of scale and bias) of the fp32 weight the generator encoded.
+    A wrong byte index or group index takes another element's code or another
+    group's scale and misses by far more."""
+    K = 256
+    torch.manual_seed(2)
+    spread = (torch.arange(K // 64, dtype=torch.float32) + 1.0).repeat_interleave(64) / 4
+    w = (torch.rand(1, 3, K) * 2 - 1) * spread
+    p, s, b = mi.quantize_q8g64(w)
+    ex = mi.Experts("q8", 1, K, 2, p, torch.zeros(1, K, 1, dtype=torch.uint32), s, b)
+    for r in range(3):
+        for c in range(K):
+            step = float(s[0, r, c // 64].float())
+            bias = float(b[0, r, c // 64].float())
+            got = orc.weight_value(ex, "gu", 0, r, c)
+            # half a step, plus what the bf16 rounding of scale (2^-9 relative,
+            # over 255 steps) and bias can leave at the clamped ends of a group
+            bound = 0.5 * step + 255 * step * 2.0 ** -9 + abs(bias) * 2.0 ** -8 + 1e-6
+            assert abs(got - float(w[0, r, c])) <= bound, (r, c)
+
+
 def test_q4_encoder_roundtrip_is_close(orc):
     """Generator sanity (not a pin of the oracle): dequantised weights stay
     within half a quantisation step of the fp32 weights they encode."""
