@@ -57,7 +57,7 @@ class Workload:
     E: int
     k: int
     F: int
-    act: str          # "f32" | "bf16"
+    act: str          # "f32" | "bf16" | "f16"
     wfmt: str         # "f32" | "bf16" | "q4" (group 64) | "q4g32" | "q4g128" | "q8"
     bias: str = "none"  # "none" | "normal0.5" | "zipf1.1"
     note: str = ""
@@ -96,7 +96,7 @@ def _gen(seed: int, tid: int, sub: int, device) -> torch.Generator:
 
 
 def _act_dtype(act: str) -> torch.dtype:
-    return {"f32": torch.float32, "bf16": torch.bfloat16}[act]
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[act]
 
 
 def q4_group(wfmt: str) -> int:

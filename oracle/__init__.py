@@ -33,7 +33,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liborc_moe.so")
 
-ACT = {"f32": 0, "bf16": 1}
+ACT = {"f32": 0, "bf16": 1, "f16": 2}
 WFMT = {"f32": 0, "bf16": 1, "q4": 2, "q4g32": 3, "q4g128": 4, "q8": 5}
 
 
@@ -113,11 +113,14 @@ def _p(a):
 
 
 def _act_code(a) -> int:
-    """0 for fp32 storage, 1 for bf16 (passed as uint16 words)."""
+    """0 for fp32 storage, 1 for bf16 (passed as uint16 words), 2 for IEEE
+    binary16 (numpy float16, passed as its own 16-bit words)."""
     if a.dtype == np.float32:
         return ACT["f32"]
     if a.dtype == np.uint16:
         return ACT["bf16"]
+    if a.dtype == np.float16:
+        return ACT["f16"]
     raise TypeError(f"activation dtype {a.dtype} not supported")
 
 

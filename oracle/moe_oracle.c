@@ -57,7 +57,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_F32 = 0, ORC_BF16 = 1 };             /* activation / dense dtypes */
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_F16 = 2 }; /* activation / dense dtypes */
 /* 4-bit affine with group 64 (ORC_W_Q4), 32 or 128 input elements per
  * scale and bias (the group sizes of DS4Server issue #112, "Kernel contract") */
 enum { ORC_W_F32 = 0, ORC_W_BF16 = 1, ORC_W_Q4 = 2, ORC_W_Q4G32 = 3, ORC_W_Q4G128 = 4,
@@ -75,8 +75,20 @@ static double bf16_value(uint16_t h) {
     return (double)f;
 }
 
+/* an IEEE 754 binary16 value: sign, 5 exponent bits (bias 15), 10 fraction
+ * bits; exponent 0 is subnormal (2^-14 * fraction / 1024), 31 is inf/NaN */
+static double f16_value(uint16_t h) {
+    const int sign = h >> 15, ex = (h >> 10) & 0x1F, fr = h & 0x3FF;
+    double v;
+    if (ex == 0) v = ldexp((double)fr, -24);
+    else if (ex == 31) v = fr ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + fr), ex - 25);
+    return sign ? -v : v;
+}
+
 static double act_value(const void* p, int dt, size_t i) {
     if (dt == ORC_F32) return (double)((const float*)p)[i];
+    if (dt == ORC_F16) return f16_value(((const uint16_t*)p)[i]);
     return bf16_value(((const uint16_t*)p)[i]);
 }
 

@@ -164,6 +164,37 @@ def test_logits_bf16_match_library_matmul(orc):
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
 
 
+def test_f16_activations_decode_every_finite_half(orc):
+    """Every finite IEEE binary16 pattern, read as an activation against a
+    unit router weight, comes back as its exact value: checked against
+    Python's own half-precision unpacking and a few closed forms (1, the
+    smallest subnormal 2^-24, the largest finite 65504, -2, a negative subnormal, the smallest normal)."""
+    import struct
+    bits = np.arange(65536, dtype=np.uint32)
+    finite = ((bits >> 10) & 0x1F) != 0x1F
+    bits = bits[finite].astype(np.uint16)
+    x = bits.view(np.float16).reshape(-1, 1)
+    got = orc.router_logits(x, np.ones((1, 1), np.float16), None)[:, 0]
+    ref = np.array([struct.unpack("<e", struct.pack("<H", int(b)))[0] for b in bits])
+    np.testing.assert_array_equal(got, ref)
+    by_bits = dict(zip(bits.tolist(), got.tolist()))
+    assert by_bits[0x3C00] == 1.0
+    assert by_bits[0x0001] == 2.0 ** -24
+    assert by_bits[0x7BFF] == 65504.0
+    assert by_bits[0xC000] == -2.0
+    assert by_bits[0x8001] == -(2.0 ** -24)
+    assert by_bits[0x0400] == 2.0 ** -14       # smallest normal
+
+
+def test_logits_f16_match_library_matmul(orc):
+    wl = mi.workload("decode_t32", d=256, E=16, act="f16")
+    L = mi.make_layer(wl, seed=2)
+    assert L.x.dtype == torch.float16
+    got = orc.router_logits(L.x, L.w_router, None)
+    ref = L.x.double().numpy() @ L.w_router.double().numpy().T
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
 # ------------------------------------------------------------ top-k
 
 def _golden_topk_cases():
