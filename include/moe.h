@@ -47,8 +47,8 @@
  *     device status word; read and clear it with moe_device_status().
  *   - T = 0 is valid: the call returns MOE_OK and launches nothing.
  *   - Preconditions: 1 <= k <= min(E, 32); E <= 1024; d and F multiples of 64;
- *     q4 and bf16 expert weights need bf16 activations, f32 weights need f32
- *     activations. Violations return MOE_ERR_INVALID_ARG or
+ *     bf16 expert weights need bf16 activations, f32 weights need f32
+ *     activations, quantised (q4 / q8) weights take bf16 or fp16 ones. Violations return MOE_ERR_INVALID_ARG or
  *     MOE_ERR_UNSUPPORTED.
  *   - All layouts are row-major with the stated shapes; buffers must be
  *     16-byte aligned.
@@ -58,11 +58,11 @@
  *   MOE_REGIME_GEMV: weight-streaming kernels, every selected expert's bytes
  *     read once per step, for few tokens per expert (decode);
  *   MOE_REGIME_TC: tensor-core grouped GEMM (tcgen05 / TMEM, TMA-staged
- *     operands) for many tokens per expert (prefill); bf16 activations,
- *     bf16 or q4 weights, d a multiple of 256, F of 128 (q4: of 256);
+ *     operands) for many tokens per expert (prefill); bf16 activations with
+ *     bf16 or q4 (group 64) weights, or fp16 activations with q4 weights, d a multiple of 256, F of 128 (q4: of 256);
  *     other shapes return MOE_ERR_UNSUPPORTED;
  *   MOE_REGIME_AUTO: GEMV when T*k <= 8*E or the shape is not one the
- *     tensor-core kernels tile, else TC (bf16) or GEMV (f32).
+ *     tensor-core kernels tile, else TC (bf16 / fp16) or GEMV (f32).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -87,7 +87,8 @@ typedef enum {
                               operands (|x| or |h| >= 65520; device status) */
 } moe_status;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype; /* activations */
+/* activations (x, the router weight, y): fp32, bf16 or IEEE binary16 */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_F16 = 2 } moe_dtype;
 
 typedef enum {
   MOE_W_F32 = 0,
@@ -212,16 +213,16 @@ moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, i
  *   x        (device) [T][d], dtype dt
  *   row_map, row_off, tile_off: as written by moe_sort_rows with the same BM
  *            (the tensor-core regime needs BM = 128)
- *   h        (device, out) [T*k][F]: fp16 for bf16 activations, fp32 for fp32:
+ *   h        (device, out) [T*k][F]: fp16 for 16-bit activations, fp32 for fp32:
  *            h[i][f] = act(g) * u (experts->act: silu or tanh-GELU),
  *            g = x[row_map[i]] . w_gu[e][f],
  *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
  *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, k, d, dt)
  *            bytes (the token rows in fp16: x converted, or, in the
  *            tensor-core regime, gathered into sorted row order); required
- *            for bf16 activations, may be NULL for fp32
+ *            for 16-bit activations, may be NULL for fp32
  * fp32 accumulation; h rounded once. The tensor-core regime multiplies fp16
- * operands (x converted exactly from bf16 when |x| < 65520, weights
+ * operands (fp16 x as is, bf16 x converted exactly when |x| < 65520, weights
  * dequantised to fp16); values outside fp16 range are reported as
  * MOE_ERR_RANGE in the device status. */
 size_t moe_grouped_swiglu_workspace(int T, int k, int d, moe_dtype dt);
@@ -232,10 +233,10 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
 
 /* Grouped down projection over rows already sorted by expert (DS4Server
  * issue #112, switch_linear with sorted indices).
- *   h        (device) [T*k][F]: fp16 for bf16 activations (dt = MOE_BF16),
+ *   h        (device) [T*k][F]: fp16 for 16-bit activations (MOE_BF16, MOE_F16),
  *            fp32 for fp32 -- as moe_grouped_swiglu writes it
  *   ys       (device, out) [T*k][d]: ys[i][o] = h[i] . w_dn[e][o], fp32
- *            accumulation, stored in fp16 for bf16 activations (its 11-bit
+ *            accumulation, stored in fp16 for 16-bit activations (its 11-bit
  *            rounding is far below the final bf16 rounding of y; values
  *            outside fp16 range are reported as MOE_ERR_RANGE in the device
  *            status) and in fp32 for fp32 activations */
@@ -248,7 +249,7 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
  * #112, _scatter_unsort; "5.5 real sparse MoE kernels (Metal)", scatter_add
  * equivalent): y[t][o] = sum_{j=0..k-1} w[t][j] * ys[inv_order[t*k+j]][o],
  * summed in fp32 in j order, rounded once to dt.
- *   ys (device) [T*k][d]: fp16 for dt = MOE_BF16, fp32 for MOE_F32 (as
+ *   ys (device) [T*k][d]: fp16 for MOE_BF16 / MOE_F16, fp32 for MOE_F32 (as
  *      moe_grouped_down writes it); inv_order (device) [T*k];
  *      topk_w (device) [T][k] fp32
  *   y  (device, out) [T][d], dtype dt */

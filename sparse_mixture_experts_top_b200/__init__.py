@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(7)
-F32, BF16 = 0, 1
+F32, BF16, F16 = 0, 1, 2
 W_F32, W_BF16, W_Q4G64 = 0, 1, 2
 REGIME_AUTO, REGIME_GEMV, REGIME_TC = 0, 1, 2
 
@@ -112,12 +112,17 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
+
+
+def _dt_of(dtype) -> int:
+    if dtype not in _DT:
+        raise TypeError(f"activations must be bfloat16, float16 or float32, got {dtype}")
+    return _DT[dtype]
+
+
 def _dt(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
-        return BF16
-    if t.dtype == torch.float32:
-        return F32
-    raise TypeError(f"activations must be bfloat16 or float32, got {t.dtype}")
+    return _dt_of(t.dtype)
 
 
 def _dev(*ts):
@@ -200,11 +205,11 @@ def sort_rows(topk_idx, E, BM, stream=None) -> SortTables:
 
 
 def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, ws=None, stream=None):
-    """-> h [T*k, F]: fp16 for bf16 x, fp32 for fp32 x"""
+    """-> h [T*k, F]: fp16 for bf16 or fp16 x, fp32 for fp32 x"""
     _dev(x)
     T = x.shape[0]
     ex = experts_struct(experts)
-    hdt = torch.float16 if x.dtype == torch.bfloat16 else torch.float32
+    hdt = torch.float32 if x.dtype == torch.float32 else torch.float16
     h = torch.empty(T * k, experts.F, dtype=hdt, device=x.device)
     nws = lib.moe_grouped_swiglu_workspace(T, k, experts.d, _dt(x))
     if ws is None:
@@ -217,10 +222,11 @@ def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, ws=Non
 
 
 def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, stream=None):
-    """-> ys [T*k, d]: fp16 for bf16 activations (fp16 h), fp32 for fp32"""
+    """-> ys [T*k, d]: fp16 for 16-bit activations (fp16 h), fp32 for fp32"""
     _dev(h)
     ex = experts_struct(experts)
-    # h is fp16 exactly when the activations are bf16; ys has h's dtype
+    # h is fp16 exactly when the activations are 16-bit; ys has h's dtype,
+    # and the step is the same for bf16 and fp16 activations
     adt = BF16 if h.dtype == torch.float16 else F32
     ys = torch.empty(T * k, experts.d, dtype=h.dtype, device=h.device)
     _check(lib.moe_grouped_down(_ptr(h), adt, _ptr(tables.row_off), _ptr(tables.tile_off),
@@ -230,15 +236,15 @@ def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, strea
 
 
 def combine(ys, inv_order, topk_w, T, k, dtype=torch.bfloat16, stream=None):
-    """-> y [T, d] in `dtype` from ys [T*k, d] (fp16 for bf16 `dtype`, fp32 for fp32)"""
+    """-> y [T, d] in `dtype` from ys [T*k, d] (fp16 for 16-bit `dtype`, fp32 for fp32)"""
     _dev(ys, inv_order, topk_w)
-    want = torch.float16 if dtype == torch.bfloat16 else torch.float32
+    want = torch.float32 if dtype == torch.float32 else torch.float16
     if ys.dtype != want:
         raise TypeError(f"ys must be {want} for {dtype} outputs")
     d = ys.shape[1]
     y = torch.empty(T, d, dtype=dtype, device=ys.device)
     _check(lib.moe_combine(_ptr(ys), _ptr(inv_order), _ptr(topk_w), T, k, d,
-                           BF16 if dtype == torch.bfloat16 else F32, _ptr(y),
+                           _dt_of(dtype), _ptr(y),
                            _stream(stream)), "moe_combine")
     return y
 
@@ -247,7 +253,7 @@ def combine(ys, inv_order, topk_w, T, k, dtype=torch.bfloat16, stream=None):
 
 def forward_layout(T, d, E, k, F, dtype, regime=REGIME_AUTO) -> WsLayout:
     L = WsLayout()
-    dt = BF16 if dtype == torch.bfloat16 else F32
+    dt = _dt_of(dtype)
     _check(lib.moe_forward_layout(T, d, E, k, F, dt, regime, ctypes.byref(L)), "moe_forward_layout")
     return L
 

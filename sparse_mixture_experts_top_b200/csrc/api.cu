@@ -26,7 +26,7 @@ static int* status_ptr() {
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static inline size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
-static inline size_t act_size(int dt) { return dt == MOE_BF16 ? 2 : 4; }
+static inline size_t act_size(int dt) { return dt == MOE_F32 ? 4 : 2; }
 
 static moe_status launched(cudaError_t e) {
   if (e == cudaSuccess) return MOE_OK;
@@ -58,12 +58,12 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
     case MOE_W_Q4G64:
     case MOE_W_Q4G32:
     case MOE_W_Q4G128:
-      if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
       if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
       if (ex->d % q4_group(ex->fmt) || ex->F % q4_group(ex->fmt)) return MOE_ERR_UNSUPPORTED;
       break;
     case MOE_W_Q8G64:
-      if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
       if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
       break;
     default:
@@ -72,17 +72,17 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
   return MOE_OK;
 }
 
-static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16; }
+static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16 || dt == MOE_F16; }
 
 // The regime a call runs: AUTO picks the weight-streaming kernels when there
 // are at most 8 routed rows per expert on average, or for fp32 activations
-// (the tensor-core kernels take bf16 operands).
+// (the tensor-core kernels take 16-bit operands).
 static int resolve_regime(int regime, long long R, int E, int dt, int d = 128, int F = 128,
                           int fmt = MOE_W_Q4G64) {
   if (regime == MOE_REGIME_GEMV || regime == MOE_REGIME_TC) return regime;
   // the tensor-core kernels tile d by 256 and F by 128 and take bf16 or q4 weights
-  if (!tc_shape_supported(d, F, fmt)) return MOE_REGIME_GEMV;
-  if (dt != MOE_BF16) return MOE_REGIME_GEMV;
+  if (!tc_shape_supported(d, F, fmt, dt)) return MOE_REGIME_GEMV;
+  if (dt == MOE_F32) return MOE_REGIME_GEMV;
   return (R <= 8LL * E) ? MOE_REGIME_GEMV : MOE_REGIME_TC;
 }
 
@@ -92,11 +92,14 @@ static int block_m_for(int regime, long long R, int E) {
 }
 
 // gate|up in the weight-streaming regime: the q4 tensor-core GEMV when it
-// applies (x converted to fp16 into x16 first), else the SIMT kernel
+// applies (bf16 x converted to fp16 into x16 first; fp16 x read in place),
+// else the SIMT kernel
 static cudaError_t swiglu_gemv(const void* x, int dt, int T, const uint32_t* rmap,
                                const int32_t* roff, const int32_t* toff, int BM, int R,
                                const moe_experts& ex, void* h, void* x16, int* stp,
                                cudaStream_t s) {
+  if (gemv_q4_mma_ok(ex, dt, BM) && dt == MOE_F16)
+    return launch_swiglu_q4_mma(x, rmap, roff, toff, BM, R, ex, h, stp, s);
   if (gemv_q4_mma_ok(ex, dt, BM) && x16) {
     cudaError_t e = launch_to_f16(x, (long long)T * ex.d, x16, stp, s);
     if (e != cudaSuccess) return e;
@@ -165,8 +168,8 @@ moe_status moe_route(const void* x, moe_dtype dt, const void* w_router, const fl
   if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaErrorNotSupported;
-  if (dt == MOE_BF16) e = launch_router_logits_tc(x, w_router, router_bias, T, d, E, logits,
-                                                  status_ptr(), s);
+  if (dt != MOE_F32) e = launch_router_logits_tc(x, dt, w_router, router_bias, T, d, E, logits,
+                                                 status_ptr(), s);
   if (e == cudaErrorNotSupported)
     e = launch_router_logits(x, dt, w_router, router_bias, T, d, E, logits, s);
   if (e != cudaSuccess) return launched(e);
@@ -199,7 +202,7 @@ size_t moe_grouped_swiglu_workspace(int T, int k, int d, moe_dtype dt) {
   if (T < 0 || k < 1 || d <= 0) return 0;
   // fp16 token rows: T rows (weight-streaming regime) or the T*k rows in
   // sorted order (tensor-core regime)
-  return dt == MOE_BF16 ? up256((size_t)T * k * d * 2) : 0;
+  return dt != MOE_F32 ? up256((size_t)T * k * d * 2) : 0;
 }
 
 moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, int BM,
@@ -233,15 +236,15 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
   const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt);
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
-    if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    if (!tc_shape_supported(experts->d, experts->F, experts->fmt)) return MOE_ERR_UNSUPPORTED;
+    if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (!tc_shape_supported(experts->d, experts->F, experts->fmt, dt)) return MOE_ERR_UNSUPPORTED;
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
     if (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, k, experts->d, dt))
       return MOE_ERR_WORKSPACE;
-    return launched(launch_swiglu_tc(x, T, row_map, row_off, tile_off, (int)R, *experts, h, ws,
+    return launched(launch_swiglu_tc(x, dt, T, row_map, row_off, tile_off, (int)R, *experts, h, ws,
                                      status_ptr(), s));
   }
-  if (dt == MOE_BF16 &&
+  if (dt != MOE_F32 &&
       (!ws || !aligned16(ws) || ws_bytes < moe_grouped_swiglu_workspace(T, k, experts->d, dt)))
     return MOE_ERR_WORKSPACE;
   return launched(swiglu_gemv(x, dt, T, row_map, row_off, tile_off, BM, (int)R, *experts, h, ws,
@@ -265,8 +268,8 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
   const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt);
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
-    if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    if (!tc_shape_supported(experts->d, experts->F, experts->fmt)) return MOE_ERR_UNSUPPORTED;
+    if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (!tc_shape_supported(experts->d, experts->F, experts->fmt, dt)) return MOE_ERR_UNSUPPORTED;
     if (BM != tc_block_m()) return MOE_ERR_INVALID_ARG;
     return launched(launch_down_tc(h, row_off, tile_off, (int)R, *experts, ys, status_ptr(), s));
   }
@@ -353,13 +356,13 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.row_off = take((size_t)(E + 1) * 4);
   L.tile_off = take((size_t)(E + 1) * 4);
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
-  L.h = take((size_t)R * F * a);      // fp16 (bf16 activations) or fp32
-  L.ys = take((size_t)R * d * a);     // fp16 (bf16 activations) or fp32
+  L.h = take((size_t)R * F * a);      // fp16 (16-bit activations) or fp32
+  L.ys = take((size_t)R * d * a);     // fp16 (16-bit activations) or fp32
   L.regime = resolve_regime(regime, R, E, dt, d, F);
   L.BM = block_m_for(L.regime, R, E);
-  // fp16 token rows: x converted (weight-streaming) or gathered in sorted
-  // row order (tensor cores)
-  L.x16 = take(dt != MOE_BF16 ? 0 : (size_t)(L.regime == MOE_REGIME_TC ? R : T) * d * 2);
+  // fp16 token rows: x converted (weight-streaming), or permuted (the
+  // one-launch path), or gathered in sorted row order (tensor cores)
+  L.x16 = take(dt == MOE_F32 ? 0 : (size_t)(L.regime == MOE_REGIME_TC ? R : T) * d * 2);
   L.total = off;
   *out = L;
   return MOE_OK;
@@ -388,11 +391,11 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
   if (st != MOE_OK) return st;
   if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  if (L.regime == MOE_REGIME_TC && dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (L.regime == MOE_REGIME_TC && dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
   // the layout assumes q4 weights; other formats the tensor-core kernels do
   // not tile take the weight-streaming kernels (which accept any BM)
   int regime_run = L.regime;
-  if (regime_run == MOE_REGIME_TC && !tc_shape_supported(d, F, experts->fmt)) {
+  if (regime_run == MOE_REGIME_TC && !tc_shape_supported(d, F, experts->fmt, dt)) {
     if (regime == MOE_REGIME_TC) return MOE_ERR_UNSUPPORTED;
     regime_run = MOE_REGIME_GEMV;
   }
@@ -419,11 +422,11 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
   // few tokens: the whole layer in one cooperative launch (its grid barrier
   // counter lives in the sort scratch, which that path does not use)
   if (regime_run == MOE_REGIME_GEMV && decode_fused_ok(T, k, E, d, F, experts->fmt, dt)) {
-    e = launch_decode_fused(x, w_router, router_bias, *experts, T, k, L.BM, logits, idx, w, order,
+    e = launch_decode_fused(x, dt, w_router, router_bias, *experts, T, k, L.BM, logits, idx, w, order,
                             inv, rmap, counts, roff, toff, x16, h, ys, y, (unsigned*)sws, stp, s);
     if (e != cudaErrorNotSupported) return launched(e);
   }
-  if (dt == MOE_BF16) e = launch_router_logits_tc(x, w_router, router_bias, T, d, E, logits, stp, s);
+  if (dt != MOE_F32) e = launch_router_logits_tc(x, dt, w_router, router_bias, T, d, E, logits, stp, s);
   if (e == cudaErrorNotSupported)
     e = launch_router_logits(x, dt, w_router, router_bias, T, d, E, logits, s);
   if (e != cudaSuccess) return launched(e);
@@ -432,14 +435,14 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
       cudaSuccess)
     return launched(e);
   if (regime_run == MOE_REGIME_TC) {
-    if ((e = launch_swiglu_tc(x, T, rmap, roff, toff, (int)R, *experts, h, x16, stp, s)) !=
+    if ((e = launch_swiglu_tc(x, dt, T, rmap, roff, toff, (int)R, *experts, h, x16, stp, s)) !=
         cudaSuccess)
       return launched(e);
     if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s)) != cudaSuccess)
       return launched(e);
   } else {
     if ((e = swiglu_gemv(x, dt, T, rmap, roff, toff, L.BM, (int)R, *experts, h,
-                         dt == MOE_BF16 ? x16 : nullptr, stp, s)) != cudaSuccess)
+                         dt == MOE_F32 ? nullptr : x16, stp, s)) != cudaSuccess)
       return launched(e);
     if ((e = down_gemv(h, dt, roff, toff, L.BM, (int)R, *experts, ys, stp, s)) != cudaSuccess)
       return launched(e);

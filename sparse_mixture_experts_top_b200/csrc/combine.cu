@@ -6,13 +6,15 @@
 // Scope -- in) adds the expert outputs with threadgroup atomics; here each
 // output element is owned by one thread, which gathers its k rows through
 // inv_order and sums them in j order -- no atomics, deterministic.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
 namespace moe {
 
 // One thread per 8 consecutive outputs of one token: k gathers of 8 ys values
-// (fp16 for bf16 activations, fp32 for fp32), fp32 fused multiply-adds in j
+// (fp16 for 16-bit activations, fp32 for fp32), fp32 fused multiply-adds in j
 // order, one rounding to TA.
 template <typename TA, typename TY>
 __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ ys,
@@ -54,11 +56,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ ys,
   }
   TA* dst = y + (size_t)t * d + o;
   if constexpr (sizeof(TA) == 2) {
+    constexpr bool kF16 = std::is_same<TA, __half>::value;
     uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
+    out.x = kF16 ? pack_f16x2(acc[0], acc[1]) : pack_bf16x2(acc[0], acc[1]);
+    out.y = kF16 ? pack_f16x2(acc[2], acc[3]) : pack_bf16x2(acc[2], acc[3]);
+    out.z = kF16 ? pack_f16x2(acc[4], acc[5]) : pack_bf16x2(acc[4], acc[5]);
+    out.w = kF16 ? pack_f16x2(acc[6], acc[7]) : pack_bf16x2(acc[6], acc[7]);
     *reinterpret_cast<uint4*>(dst) = out;
   } else {
     *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -74,6 +77,9 @@ cudaError_t launch_combine(const void* ys, const uint32_t* inv_order, const floa
   if (dt == MOE_BF16)
     launch_pdl(combine_kernel<__nv_bfloat16, __half>, blocks, 256, 0, s, (const __half*)ys,
                inv_order, w, T, k, d, (__nv_bfloat16*)y);
+  else if (dt == MOE_F16)
+    launch_pdl(combine_kernel<__half, __half>, blocks, 256, 0, s, (const __half*)ys, inv_order, w,
+               T, k, d, (__half*)y);
   else
     launch_pdl(combine_kernel<float, float>, blocks, 256, 0, s, (const float*)ys, inv_order, w, T,
                k, d, (float*)y);

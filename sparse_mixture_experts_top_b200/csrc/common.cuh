@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -43,6 +44,19 @@ template <> struct Act<__nv_bfloat16> {
     p[i] = __float2bfloat16_rn(v);
   }
 };
+template <> struct Act<__half> {
+  static __device__ __forceinline__ float load(const __half* p, size_t i) {
+    return __half2float(p[i]);
+  }
+  static __device__ __forceinline__ void store(__half* p, size_t i, float v) {
+    p[i] = __float2half_rn(v);
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 // silu(g) * u with silu(g) = g * sigmoid(g) = g / (1 + exp(-g)); the fast
 // division (2 ulp; 0 once 1 + exp(-g) passes 2^126, i.e. silu below 1e-36 in

@@ -68,8 +68,8 @@ constexpr long long kWaitCycles = 2000000000LL;
 constexpr int kRedBytes = 2 * kNg * kGw * 32 * 4 * 4;
 
 struct Params {
-  const __nv_bfloat16* x;                     // [T][d]
-  const __nv_bfloat16* wr;                    // [E][d]
+  const uint16_t* x;                          // [T][d] bf16, or fp16 when xf16
+  const uint16_t* wr;                         // [E][d] same type as x
   const float* rbias;                         // [E] or null
   const uint32_t* w_gu;                       // [E][2F][d/8] q4 words
   const uint16_t* s_gu;                       // [E][2F][d/gs] bf16
@@ -92,7 +92,8 @@ struct Params {
   __half* x16;                                // [T][d]
   __half* h;                                  // [R][F]
   __half* ys;                                 // [R][d], sorted row order
-  __nv_bfloat16* y;                           // [T][d]
+  uint16_t* y;                                // [T][d] same type as x
+  int xf16;                                   // activations are fp16 (else bf16)
   unsigned* sync;                             // grid barrier counter, zero before launch
   int* status;
 };
@@ -457,24 +458,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
       // stored as the pairs (e0,e4) (e1,e5) (e2,e6) (e3,e7), the K order of
       // the weight dequantisation
-      float e[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        e[2 * j] = __uint_as_float(w4[j] << 16);
-        e[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
-      }
       uint32_t o[4];
+      if (p.xf16) {
+        // already fp16: pair the low (even j) or high (odd j) halves of
+        // words j/2 and j/2 + 2
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (!(fabsf(e[j]) < 65520.f && fabsf(e[j + 4]) < 65520.f))
-          report_status(p.status, MOE_ERR_RANGE);
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(e[j + 4]), "f"(e[j]));
+        for (int j = 0; j < 4; ++j)
+          o[j] = __byte_perm(w4[j >> 1], w4[(j >> 1) + 2], (j & 1) ? 0x7632 : 0x5410);
+      } else {
+        float e[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          e[2 * j] = __uint_as_float(w4[j] << 16);
+          e[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (!(fabsf(e[j]) < 65520.f && fabsf(e[j + 4]) < 65520.f))
+            report_status(p.status, MOE_ERR_RANGE);
+          asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(e[j + 4]), "f"(e[j]));
+        }
       }
       xo[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     // router logits: a warp per (expert e, token t); per lane the 8-element
     // chunks lane, lane + 32, ... of the row in order, fp32 sums of exact
-    // bf16 products, then a warp sum. All of a lane's chunks are loaded
+    // bf16 (or fp16) products, then a warp sum. All of a lane's chunks are loaded
     // before the first product.
     constexpr int kMaxC = 2048 / 256;          // 16-byte chunks per lane at d = 2048
     const int nc8 = d / 8;
@@ -497,7 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const uint32_t wb[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float2 fa = bf16x2_to_f32x2(wa[q]), fb = bf16x2_to_f32x2(wb[q]);
+            const float2 fa = p.xf16 ? __half22float2(*reinterpret_cast<const __half2*>(&wa[q]))
+                                     : bf16x2_to_f32x2(wa[q]);
+            const float2 fb = p.xf16 ? __half22float2(*reinterpret_cast<const __half2*>(&wb[q]))
+                                     : bf16x2_to_f32x2(wb[q]);
             acc = fmaf(fb.x, fa.x, acc);
             acc = fmaf(fb.y, fa.y, acc);
           }
@@ -769,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!grid_barrier(p.sync, 3, &s_abort, p.status)) ok = false;
 
     // combine: y[t][o .. o+7] = sum over j of w[t][j] * ys[inv[t*k + j]][o ..
-    // o+7], fp32 fused multiply-adds in j order, one rounding to bf16
+    // o+7], fp32 fused multiply-adds in j order, one rounding to bf16 (fp16)
     if (ok) {
       const int per_row = d / 8;
       for (int i = blockIdx.x * (kCw * 32) + threadIdx.x; i < T * per_row; i += G * kCw * 32) {
@@ -790,10 +802,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           }
         }
         uint4 out;
-        out.x = pack_bf16x2(acc8[0], acc8[1]);
-        out.y = pack_bf16x2(acc8[2], acc8[3]);
-        out.z = pack_bf16x2(acc8[4], acc8[5]);
-        out.w = pack_bf16x2(acc8[6], acc8[7]);
+        if (p.xf16) {
+          uint32_t o4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __half2 hq = __floats2half2_rn(acc8[2 * q], acc8[2 * q + 1]);
+            o4[q] = *reinterpret_cast<const uint32_t*>(&hq);
+          }
+          out = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        } else {
+          out.x = pack_bf16x2(acc8[0], acc8[1]);
+          out.y = pack_bf16x2(acc8[2], acc8[3]);
+          out.z = pack_bf16x2(acc8[4], acc8[5]);
+          out.w = pack_bf16x2(acc8[6], acc8[7]);
+        }
         *reinterpret_cast<uint4*>(p.y + (size_t)t * d + o) = out;
       }
     }
@@ -845,25 +867,26 @@ static int sm_count() {
 
 bool decode_fused_ok(int T, int k, int E, int d, int F, int fmt, int dt) {
   using namespace dec;
-  return q4_group(fmt) != 0 && dt == MOE_BF16 && T >= 1 && T <= kMaxT && T * k <= kMaxR &&
+  return q4_group(fmt) != 0 && (dt == MOE_BF16 || dt == MOE_F16) && T >= 1 && T <= kMaxT && T * k <= kMaxR &&
          E <= kMaxE && k <= 32 && d % 128 == 0 && F % 128 == 0 && d <= 2048 && F <= 2048;
 }
 
 size_t decode_smem_bytes() { return dec::kSlots * dec::kSlotBytes + dec::kRedBytes + 128; }
 
-cudaError_t launch_decode_fused(const void* x, const void* w_router, const float* bias,
+cudaError_t launch_decode_fused(const void* x, int dt, const void* w_router, const float* bias,
                                 const moe_experts& ex, int T, int k, int BM, float* logits,
                                 int32_t* idx, float* w, uint32_t* order, uint32_t* inv_order,
                                 uint32_t* row_map, int32_t* counts, int32_t* row_off,
                                 int32_t* tile_off, void* x16, void* h, void* ys, void* y,
                                 unsigned* sync, int* status, cudaStream_t s) {
   using namespace dec;
-  if (!decode_fused_ok(T, k, ex.E, ex.d, ex.F, ex.fmt, MOE_BF16)) return cudaErrorNotSupported;
+  if (!decode_fused_ok(T, k, ex.E, ex.d, ex.F, ex.fmt, dt)) return cudaErrorNotSupported;
   const int G = sm_count();
   if (G <= 0) return cudaErrorNoDevice;
   Params p{};
-  p.x = (const __nv_bfloat16*)x;
-  p.wr = (const __nv_bfloat16*)w_router;
+  p.x = (const uint16_t*)x;
+  p.wr = (const uint16_t*)w_router;
+  p.xf16 = dt == MOE_F16;
   p.rbias = bias;
   p.w_gu = (const uint32_t*)ex.w_gu;
   p.s_gu = (const uint16_t*)ex.s_gu;
@@ -892,7 +915,7 @@ cudaError_t launch_decode_fused(const void* x, const void* w_router, const float
   p.x16 = (__half*)x16;
   p.h = (__half*)h;
   p.ys = (__half*)ys;
-  p.y = (__nv_bfloat16*)y;
+  p.y = (uint16_t*)y;
   p.sync = sync;
   p.status = status;
   const size_t smem = decode_smem_bytes();

@@ -59,10 +59,11 @@ template <> struct WDecode<MOE_W_Q8G64> {
   }
 };
 
-// The hidden rows h between the two projections: fp16 for bf16 activations
+// The hidden rows h between the two projections: fp16 for 16-bit activations
 // (the tensor-core operand format, 11-bit precision), fp32 for fp32.
 template <typename TA> struct HType { using T = float; };
 template <> struct HType<__nv_bfloat16> { using T = __half; };
+template <> struct HType<__half> { using T = __half; };
 
 __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t v) {
   return __half22float2(*reinterpret_cast<const __half2*>(&v));
@@ -299,6 +300,8 @@ cudaError_t launch_swiglu_gemv(const void* x, int dt, const uint32_t* row_map,
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_SWIGLU(__nv_bfloat16, MOE_W_BF16);
   else if (dt == MOE_BF16 && q4_group(ex.fmt)) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q4G64);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q8G64) MOE_SWIGLU(__nv_bfloat16, MOE_W_Q8G64);
+  else if (dt == MOE_F16 && q4_group(ex.fmt)) MOE_SWIGLU(__half, MOE_W_Q4G64);
+  else if (dt == MOE_F16 && ex.fmt == MOE_W_Q8G64) MOE_SWIGLU(__half, MOE_W_Q8G64);
   else return cudaErrorInvalidValue;
 #undef MOE_SWIGLU
   return cudaGetLastError();
@@ -319,10 +322,13 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
                                                  tile_off, BM, ex.E, ex.d, ex.F, w, sc, bi,     \
                                                  (typename HType<TA>::T*)ys,                \
                                                  wq_group(ex.fmt), status)
+  // the down projection reads and writes fp16 for both 16-bit activation
+  // types: one instantiation serves both
+  const bool a16 = dt == MOE_BF16 || dt == MOE_F16;
   if (dt == MOE_F32 && ex.fmt == MOE_W_F32) MOE_DOWN(float, MOE_W_F32);
   else if (dt == MOE_BF16 && ex.fmt == MOE_W_BF16) MOE_DOWN(__nv_bfloat16, MOE_W_BF16);
-  else if (dt == MOE_BF16 && q4_group(ex.fmt)) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
-  else if (dt == MOE_BF16 && ex.fmt == MOE_W_Q8G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q8G64);
+  else if (a16 && q4_group(ex.fmt)) MOE_DOWN(__nv_bfloat16, MOE_W_Q4G64);
+  else if (a16 && ex.fmt == MOE_W_Q8G64) MOE_DOWN(__nv_bfloat16, MOE_W_Q8G64);
   else return cudaErrorInvalidValue;
 #undef MOE_DOWN
   return cudaGetLastError();
@@ -330,7 +336,7 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
 
 
 // ===================================================================
-// q4 weights, bf16 activations: tensor-core GEMV (mma.sync m16n8k16, fp16
+// q4 weights, 16-bit activations (fp16 operands): tensor-core GEMV (mma.sync m16n8k16, fp16
 // operands, fp32 accumulate) for tiles of at most 16 token rows.
 //
 // A CTA of 4 warps owns one block of 16 weight rows of one tile -- for the
@@ -531,7 +537,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_q4_mma_kernel(
 }
 
 bool gemv_q4_mma_ok(const moe_experts& ex, int dt, int BM) {
-  return q4_group(ex.fmt) != 0 && dt == MOE_BF16 && BM <= kMmaMaxRows && ex.d % 128 == 0 &&
+  return q4_group(ex.fmt) != 0 && (dt == MOE_BF16 || dt == MOE_F16) && BM <= kMmaMaxRows && ex.d % 128 == 0 &&
          ex.F % 128 == 0;
 }
 

@@ -11,9 +11,10 @@ namespace moe {
 // Router logits L[T][E] = x[T][d] . w_router[E][d]^T + bias, fp32 out.
 cudaError_t launch_router_logits(const void* x, int dt, const void* w_router, const float* bias,
                                  int T, int d, int E, float* logits, cudaStream_t s);
-// Tensor-core router (bf16 only); returns cudaErrorNotSupported when the
-// shape is outside what the kernel tiles (caller then uses the SIMT one).
-cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const float* bias, int T,
+// Tensor-core router (bf16 or fp16 x and router weight); returns
+// cudaErrorNotSupported when the shape is outside what the kernel tiles
+// (caller then uses the SIMT one).
+cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router, const float* bias, int T,
                                     int d, int E, float* logits, int* status, cudaStream_t s);
 
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
@@ -45,8 +46,9 @@ cudaError_t launch_down_gemv(const void* h, int dt, const int32_t* row_off,
                              const int32_t* tile_off, int BM, int R, const moe_experts& ex,
                              void* ys, int* status, cudaStream_t s);
 
-// q4 weights with bf16 activations and at most 16 rows per tile: mma.sync
-// fp16 GEMV (x16: activations converted to fp16; h fp16 in, ys fp16 out).
+// q4 weights with 16-bit activations and at most 16 rows per tile: mma.sync
+// fp16 GEMV (x16: fp16 activations, converted from bf16 or the caller's own;
+// h fp16 in, ys fp16 out).
 bool gemv_q4_mma_ok(const moe_experts& ex, int dt, int BM);
 cudaError_t launch_swiglu_q4_mma(const void* x16, const uint32_t* row_map, const int32_t* row_off,
                                  const int32_t* tile_off, int BM, int R, const moe_experts& ex,
@@ -58,26 +60,26 @@ cudaError_t launch_down_q4_mma(const void* h, const int32_t* row_off, const int3
 // are reported as MOE_ERR_RANGE
 cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cudaStream_t s);
 
-// Tensor-core grouped kernels (bf16 activations; bf16 or q4 weights).
-// BM must equal tc_block_m().
+// Tensor-core grouped kernels (bf16 activations with bf16 or q4 weights,
+// fp16 activations with q4 weights). BM must equal tc_block_m().
 int tc_block_m();
-// whether the tensor-core kernels tile these expert shapes
-bool tc_shape_supported(int d, int F, int fmt);
+// whether the tensor-core kernels tile these expert shapes and types
+bool tc_shape_supported(int d, int F, int fmt, int dt);
 // xs16: R*d fp16 scratch that receives the token rows of the R sorted rows,
-// gathered through row_map and converted from bf16
-cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
+// gathered through row_map (converted when x is bf16)
+cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
                              void* xs16, int* status, cudaStream_t s);
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
                            const moe_experts& ex, void* ys, int* status, cudaStream_t s);
 
-// The decode layer fused into one cooperative launch (q4 experts, bf16
-// activations, T <= 32, T*k <= 256, E <= 256, d and F multiples of 128 and at
+// The decode layer fused into one cooperative launch (q4 experts, bf16 or
+// fp16 activations, T <= 32, T*k <= 256, E <= 256, d and F multiples of 128 and at
 // most 2048). Writes the same workspace tables as the separate stages (logits,
 // top-k, sort tables, x16, h, ys in fp16) and y; `sync` is a 4-byte scratch
 // word.
 bool decode_fused_ok(int T, int k, int E, int d, int F, int fmt, int dt);
-cudaError_t launch_decode_fused(const void* x, const void* w_router, const float* bias,
+cudaError_t launch_decode_fused(const void* x, int dt, const void* w_router, const float* bias,
                                 const moe_experts& ex, int T, int k, int BM, float* logits,
                                 int32_t* idx, float* w, uint32_t* order, uint32_t* inv_order,
                                 uint32_t* row_map, int32_t* counts, int32_t* row_off,

@@ -121,6 +121,9 @@ cudaError_t launch_router_logits(const void* x, int dt, const void* w_router, co
     if (dt == MOE_BF16)
       launch_pdl(router_gemv_kernel<__nv_bfloat16>, blocks, 256, 0, s, 
           (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, T, d, E, logits);
+    else if (dt == MOE_F16)
+      launch_pdl(router_gemv_kernel<__half>, blocks, 256, 0, s, (const __half*)x,
+                 (const __half*)w_router, bias, T, d, E, logits);
     else
       launch_pdl(router_gemv_kernel<float>, blocks, 256, 0, s, (const float*)x, (const float*)w_router,
                                                        bias, T, d, E, logits);
@@ -129,6 +132,9 @@ cudaError_t launch_router_logits(const void* x, int dt, const void* w_router, co
     if (dt == MOE_BF16)
       launch_pdl(router_tile_kernel<__nv_bfloat16>, grid, 256, 0, s, 
           (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, T, d, E, logits);
+    else if (dt == MOE_F16)
+      launch_pdl(router_tile_kernel<__half>, grid, 256, 0, s, (const __half*)x,
+                 (const __half*)w_router, bias, T, d, E, logits);
     else
       launch_pdl(router_tile_kernel<float>, grid, 256, 0, s, (const float*)x, (const float*)w_router,
                                                      bias, T, d, E, logits);

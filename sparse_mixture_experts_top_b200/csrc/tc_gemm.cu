@@ -116,6 +116,7 @@ struct Params {
   int out_ld;          // elements per output row
   int m_limit;         // valid weight rows per group (router: E)
   int act;             // gate|up: the GLU's gate activation (moe_act)
+  int router_f16;      // router: x and the router weight are fp16 (else bf16)
   const float* bias;   // router bias or null
   int* status;
 };
@@ -616,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int unit, r0, nv, e;
       decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
       const int n = mma_n(nv);
-      const uint32_t idesc = idesc_mma(n, !ROUTER);
+      const uint32_t idesc = idesc_mma(n, !ROUTER || p.router_f16);
       // tiles of <= 64 rows alternate between the two 128-column buffers
       // (matrix q at +64q); larger ones take both (matrix q at +128q)
       const bool small = n <= 64;
@@ -899,12 +900,14 @@ static int num_sms() {
 }
 
 // raw weight-tile map over a stack of `rows` weight rows of K elements
-static bool weight_map(CUtensorMap* m, int fmt, const void* w, long long rows, int K) {
+// (16-bit rows are bf16, or fp16 for an fp16 router weight)
+static bool weight_map(CUtensorMap* m, int fmt, const void* w, long long rows, int K,
+                       bool f16 = false) {
   if (fmt == MOE_W_Q4G64)
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / 8, rows, (uint64_t)K / 2, 32, BMW,
                     CU_TENSOR_MAP_SWIZZLE_128B);
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, rows, (uint64_t)K * 2, 64, BMW,
-                  CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w,
+                  K, rows, (uint64_t)K * 2, 64, BMW, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // bf16 -> fp16, 8 values per thread; values that do not round to a finite
@@ -937,8 +940,9 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ i
 // sorted rows per block (8 values per thread per load); values that do not round to a
 // finite fp16 are reported as MOE_ERR_RANGE (they become +-inf). PERM stores
 // every 8 consecutive elements in the order (0, 4, 1, 5, 2, 6, 3, 7), the K
-// order of dequant_word_perm.
-template <bool PERM>
+// order of dequant_word_perm. SRC16 takes fp16 rows, copied (and permuted)
+// as they are.
+template <bool PERM, bool SRC16 = false>
 __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict__ x,
                                                          const uint32_t* __restrict__ row_map,
                                                          long long R, int d8,
@@ -955,6 +959,22 @@ __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict
   for (int c = threadIdx.x & 63; c < d8; c += 64) {
     const uint4 v = __ldg(src + c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if constexpr (SRC16) {
+      // halves 2j (low) and 2j+1 (high) of word j; the permuted pairs are
+      // (e_j, e_{j+4}) = low or high halves of words j/2 and j/2 + 2
+      if (PERM) {
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t a = w[j >> 1], b = w[(j >> 1) + 2];
+          o[j] = (j & 1) ? __byte_perm(a, b, 0x7632) : __byte_perm(a, b, 0x5410);
+        }
+        dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+      } else {
+        dst[c] = v;
+      }
+      continue;
+    }
     float f[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -1001,22 +1021,23 @@ static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub
 // Shapes the kernels tile: gate|up units are 128 features (F % 128), down
 // units 256 output rows (d % 256); K (d or F) a multiple of 128 for the
 // k-block pairs, and of 256 for q4 raw stages.
-static bool tc_shape_ok(const moe_experts& ex) {
+static bool tc_shape_ok(const moe_experts& ex, int dt) {
   if (ex.d % 256 || ex.F % 128) return false;
+  if (dt != MOE_BF16 && dt != MOE_F16) return false;
   if (ex.fmt == MOE_W_Q4G64) return ex.F % 256 == 0;
-  return ex.fmt == MOE_W_BF16;
+  return ex.fmt == MOE_W_BF16 && dt == MOE_BF16;
 }
 
 }  // namespace tc
 
 int tc_block_m() { return tc::BN; }
 
-bool tc_shape_supported(int d, int F, int fmt) {
+bool tc_shape_supported(int d, int F, int fmt, int dt) {
   moe_experts ex{};
   ex.d = d;
   ex.F = F;
   ex.fmt = (moe_wfmt)fmt;
-  return tc::tc_shape_ok(ex);
+  return tc::tc_shape_ok(ex, dt);
 }
 
 cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cudaStream_t s) {
@@ -1027,18 +1048,22 @@ cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cu
   return cudaGetLastError();
 }
 
-cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, const int32_t* row_off,
-                             const int32_t* tile_off, int R, const moe_experts& ex, void* h,
-                             void* xs16, int* status, cudaStream_t s) {
+cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_map,
+                             const int32_t* row_off, const int32_t* tile_off, int R,
+                             const moe_experts& ex, void* h, void* xs16, int* status,
+                             cudaStream_t s) {
   using namespace tc;
-  if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
+  if (!tc_shape_ok(ex, dt)) return cudaErrorNotSupported;
   (void)T;
   if (R <= 0) return cudaSuccess;
   // the expert GEMMs take fp16 operands in row-sorted order: x gathered
-  // through row_map and converted once into xs16 [R][d]
+  // through row_map (and converted once, from bf16) into xs16 [R][d]
   // q4 weights are dequantised in a permuted K order, so are the token rows
   const unsigned gblocks = (unsigned)((R + 3) / 4);
-  if (ex.fmt == MOE_W_Q4G64)
+  if (ex.fmt == MOE_W_Q4G64 && dt == MOE_F16)
+    launch_pdl(gather_f16_kernel<true, true>, gblocks, 256, 0, s, (const uint4*)x, row_map,
+               (long long)R, ex.d / 8, (uint4*)xs16, status);
+  else if (ex.fmt == MOE_W_Q4G64)
     launch_pdl(gather_f16_kernel<true>, gblocks, 256, 0, s, (const uint4*)x, row_map, (long long)R,
                ex.d / 8, (uint4*)xs16, status);
   else
@@ -1075,7 +1100,8 @@ cudaError_t launch_swiglu_tc(const void* x, int T, const uint32_t* row_map, cons
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
                            const moe_experts& ex, void* ys, int* status, cudaStream_t s) {
   using namespace tc;
-  if (!tc_shape_ok(ex)) return cudaErrorNotSupported;
+  // h is fp16 whatever the activations' type
+  if (!tc_shape_ok(ex, ex.fmt == MOE_W_Q4G64 ? MOE_F16 : MOE_BF16)) return cudaErrorNotSupported;
   if (R <= 0) return cudaSuccess;
   CUtensorMap ta;
   if (!weight_map(&ta, ex.fmt, ex.w_dn, (long long)ex.E * ex.d, ex.F)) return cudaErrorInvalidValue;
@@ -1102,15 +1128,19 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   return run<MOE_W_BF16, EPI_STORE, false>(p, ta, ub, s);
 }
 
-cudaError_t launch_router_logits_tc(const void* x, const void* w_router, const float* bias, int T,
-                                    int d, int E, float* logits, int* status, cudaStream_t s) {
+cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router, const float* bias,
+                                    int T, int d, int E, float* logits, int* status,
+                                    cudaStream_t s) {
   using namespace tc;
   // few tokens: the weight-streaming kernel is faster than a 128-row tile
   if (T < 256 || d % 128 != 0) return cudaErrorNotSupported;
+  if (dt != MOE_BF16 && dt != MOE_F16) return cudaErrorNotSupported;
+  const bool f16 = dt == MOE_F16;
   CUtensorMap ta;
-  if (!weight_map(&ta, MOE_W_BF16, w_router, E, d)) return cudaErrorInvalidValue;
+  if (!weight_map(&ta, MOE_W_BF16, w_router, E, d, f16)) return cudaErrorInvalidValue;
   Params p{};
-  if (!token_maps(p, x, true, T, d)) return cudaErrorInvalidValue;
+  if (!token_maps(p, x, !f16, T, d)) return cudaErrorInvalidValue;
+  p.router_f16 = f16;
   p.E = 1;
   p.n_rows = T;
   // units of two 128-row blocks of experts; rows past E are zero-filled by

@@ -72,6 +72,11 @@ def test_forward_rejects_bad_arguments_without_launching(moe):
     assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(bad), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
     # q4 weights with fp32 activations
     assert L.moe_forward(fake, moe.F32, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
+    # bf16 or fp32 weights with fp16 activations
+    for fmt in (moe.W_BF16, moe.W_F32):
+        assert L.moe_forward(fake, moe.F16, fake, P, ctypes.byref(_ex(moe, fmt=fmt)), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_UNSUPPORTED
+    # unknown activation dtype
+    assert L.moe_forward(fake, 3, fake, P, ctypes.byref(ex), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
     # unknown weight format
     bad = _ex(moe, fmt=7)
     assert L.moe_forward(fake, moe.BF16, fake, P, ctypes.byref(bad), 4, 2, fake, fake, 1 << 30, 0, P) == moe.ERR_INVALID_ARG
@@ -143,3 +148,6 @@ def test_forward_layout_is_consistent(moe):
         assert L.h + T * k * F * 2 <= L.ys
         assert L.BM >= 1 and L.regime in (moe.REGIME_GEMV, moe.REGIME_TC)
         assert moe.lib.moe_forward_workspace(T, d, E, k, F, moe.BF16, 0) == L.total
+        # fp16 activations take the same layout as bf16 ones
+        L16 = moe.forward_layout(T, d, E, k, F, __import__("torch").float16)
+        assert (L16.total, L16.x16, L16.regime, L16.BM) == (L.total, L.x16, L.regime, L.BM)

@@ -67,7 +67,10 @@ def test_topk_signed_zero_and_nan(moe, orc):
                                     ("prefill", 256), ("skewed", 64), ("acceptance", 100),
                                     ("prefill", 2048), ("skewed", 520), ("acceptance", 512)])
 def test_route_logits_and_selection(moe, orc, name, T):
-    wl = mi.workload(name, T=T)
+    _check_route(moe, orc, mi.workload(name, T=T), T)
+
+
+def _check_route(moe, orc, wl, T):
     g = torch.Generator().manual_seed(11)
     x = torch.randn(T, wl.d, generator=g).to(mi._act_dtype(wl.act))
     wr = (torch.randn(wl.E, wl.d, generator=g) / wl.d ** 0.5).to(x.dtype)
@@ -144,7 +147,8 @@ STAGE_CASES = [
 
 
 def _stage_setup(wl, T, seed, skew):
-    layer = mi.make_layer(mi.workload(wl.name, T=T), seed=seed, device=DEV)
+    # the workload as given (activation type, weight format), with T tokens
+    layer = mi.make_layer(mi.Workload(**{**wl.__dict__, "T": T}), seed=seed, device=DEV)
     idx = mi.random_topk_idx(T, wl.E, wl.k, seed=seed + 1, skew=skew)
     return layer, idx
 
@@ -188,14 +192,15 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
 
 
 @pytest.mark.parametrize("T,k,d,dt", [(1, 8, 2048, torch.bfloat16), (16, 2, 128, torch.float32),
-                                      (2048, 10, 2048, torch.bfloat16), (5, 3, 64, torch.bfloat16)])
+                                      (2048, 10, 2048, torch.bfloat16), (5, 3, 64, torch.bfloat16),
+                                      (1, 8, 2048, torch.float16), (300, 10, 2048, torch.float16)])
 def test_combine_parity(moe, orc, T, k, d, dt):
     E = max(k, 16)
     idx = mi.random_topk_idx(T, E, k, seed=31)
     st = orc.sort_rows(idx.numpy(), E, 8)
-    # ys arrive in fp16 for bf16 outputs, fp32 for fp32
+    # ys arrive in fp16 for 16-bit outputs, fp32 for fp32
     ys = mi.random_ys(T * k, d, seed=32,
-                      dtype=torch.float16 if dt == torch.bfloat16 else torch.float32)
+                      dtype=torch.float32 if dt == torch.float32 else torch.float16)
     w = mi.random_weights(T, k, seed=33)
     inv = torch.from_numpy(st.inv_order.view(np.int32)).view(torch.uint32)
     y = moe.combine(ys.to(DEV), inv.to(DEV), w.to(DEV), T, k, dtype=dt)
@@ -203,7 +208,8 @@ def test_combine_parity(moe, orc, T, k, d, dt):
     g = to_np(y).astype(np.float64)
     # an fp32 sum of k products (each rounding <= 2^-24 relative of the
     # partial sum), then one rounding to the output dtype
-    u = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -24   # unit roundoff (8 / 24-bit precision)
+    # unit roundoff of the output type (8-, 11- or 24-bit precision)
+    u = {torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11, torch.float32: 2.0 ** -24}[dt]
     mag = np.abs(w.double().numpy())[:, :, None] * np.abs(ys.double().numpy()[st.inv_order.reshape(T, k)])
     bound = u * np.abs(yref) + (k + 1) * 2.0 ** -24 * mag.sum(axis=1) * (1 + u)
     assert (np.abs(g - yref) <= bound).all()
@@ -408,6 +414,64 @@ def test_grouped_stages_q8(moe, orc):
 def test_forward_q8(moe, orc, name, T):
     layer = mi.make_layer(mi.workload(name, T=T, wfmt="q8"), seed=9, device=DEV)
     _forward_and_compare(moe, orc, layer)
+
+
+# ------------------------------------------------------------------ fp16 activations
+
+@pytest.mark.parametrize("name,T", [("decode_t32", 32), ("prefill", 512), ("skewed", 300)])
+def test_route_f16(moe, orc, name, T):
+    """IEEE half activations and router weight: the weight-streaming router
+    (32 tokens) and the tensor-core one (fp16 operands, 300 and 512 tokens)."""
+    _check_route(moe, orc, mi.workload(name, T=T, act="f16"), T)
+
+
+@pytest.mark.parametrize("name,T,regime,BM,wfmt", [
+    ("decode_t32", 32, 1, 8, "q4"),          # mma.sync GEMV, x read in place
+    ("decode_t32", 32, 1, 32, "q4"),         # SIMT GEMV (tiles above 16 rows)
+    ("decode_t32", 32, 1, 8, "q8"),          # SIMT GEMV, 8-bit weights
+    ("prefill", 600, 2, 128, "q4"),          # tcgen05 kernels, fp16 gather
+])
+def test_grouped_stages_f16(moe, orc, name, T, regime, BM, wfmt):
+    wl = mi.workload(name, T=T, act="f16", wfmt=wfmt)
+    layer, idx = _stage_setup(wl, T, 41, 0.2)
+    assert layer.x.dtype == torch.float16
+    st = moe.sort_rows(idx.to(DEV), wl.E, BM)
+    h = moe.grouped_swiglu(layer.x, st, wl.k, layer.experts, regime=regime)
+    assert h.dtype == torch.float16
+    ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
+    hx = _host(layer.experts)
+    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    # the SIMT kernels dequantise in fp32, the tensor-core ones to fp16
+    simt = BM > 16 or wfmt == "q8"
+    u_w = 2.0 ** -24 if simt else U_F16
+    assert_h_close(h, href, g, u, ga, ua, wl.d, u_w, U_F16, TOL_BF16, f"h[f16 {name} {wfmt}]")
+    ys = moe.grouped_down(h, st, T, wl.k, layer.experts, regime=regime)
+    yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    assert_ys_close(ys, yref, habs, u_w, TOL_BF16, f"ys[f16 {name} {wfmt}]", u_ys=U_F16)
+    assert moe.device_status() == moe.OK
+
+
+@pytest.mark.parametrize("name,T,wfmt", [("decode_t1", 1, "q4"), ("decode_t32", 32, "q4"),
+                                         ("decode_t32", 32, "q4g128"), ("decode_t1", 1, "q8"),
+                                         ("prefill", 300, "q4")])
+def test_forward_f16(moe, orc, name, T, wfmt):
+    """The whole layer on fp16 activations: the one-launch decode kernel (q4,
+    up to 32 tokens), the separate weight-streaming stages (q8; 300 tokens)."""
+    layer = mi.make_layer(mi.workload(name, T=T, act="f16", wfmt=wfmt), seed=12, device=DEV)
+    y = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, layer.wl.k)
+    assert y.dtype == torch.float16
+    _forward_and_compare(moe, orc, layer)
+    assert moe.device_status() == moe.OK
+
+
+def test_forward_f16_prefill_tensor_cores(moe, orc):
+    layer = mi.make_layer(mi.workload("prefill", act="f16"), seed=13, device=DEV)
+    rng = np.random.default_rng(5)
+    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(2048, 64, replace=False)),
+                         regime=2)
+    assert moe.device_status() == moe.OK
 
 
 def test_forward_deterministic(moe):
