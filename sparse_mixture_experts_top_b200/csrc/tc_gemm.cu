@@ -70,9 +70,11 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kDqWarp0 = 8;
 constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at the B200's clocks
 
-// EPI_STORE: the router stores fp32 logits (+ p.bias when set), the down
-// projection fp16 ys
-enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
+// EPI_SWIGLU / EPI_GEGLU: gate|up, h = act(gate) * up in fp16, the gate
+// activation fixed at compile time (a runtime choice in the unrolled
+// epilogue cost the SwiGLU kernel a fifth of its speed); EPI_STORE: the
+// router stores fp32 logits (+ p.bias when set), the down projection fp16 ys
+enum { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_GEGLU = 2 };
 
 template <int FMT>
 struct Cfg {
@@ -115,7 +117,6 @@ struct Params {
   void* out;
   int out_ld;          // elements per output row
   int m_limit;         // valid weight rows per group (router: E)
-  int act;             // gate|up: the GLU's gate activation (moe_act)
   int router_f16;      // router: x and the router weight are fp16 (else bf16)
   const float* bias;   // router bias or null
   int* status;
@@ -678,7 +679,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
       const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
       // 16 columns of both accumulators at a time
-      if (EPI == EPI_SWIGLU) {
+      if (EPI != EPI_STORE) {
+        constexpr int kAct = EPI == EPI_GEGLU ? MOE_ACT_GEGLU_TANH : MOE_ACT_SWIGLU;
         const int orow = unit * p.unit_rows + m;          // feature of this thread
         __half* hp = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + orow;
         for (int n0 = 0; n0 < nv; n0 += 16) {
@@ -688,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const __half v =
-                __float2half_rn(glu(p.act, __uint_as_float(a0[j]), __uint_as_float(a1[j])));
+                __float2half_rn(glu(kAct, __uint_as_float(a0[j]), __uint_as_float(a1[j])));
             if (j < lim) {
               hmax = max(hmax, (uint32_t)__half_as_ushort(v) & 0x7FFFu);
               hp[(size_t)(n0 + j) * p.out_ld] = v;
@@ -818,7 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               // gate|up reads token rows the gather wrote in permuted order
-              if (EPI == EPI_SWIGLU) dequant_word_perm(ws[i], s2, b2, vals + 4 * i);
+              if (EPI != EPI_STORE) dequant_word_perm(ws[i], s2, b2, vals + 4 * i);
               else dequant_word(ws[i], s2, b2, vals + 4 * i);
             }
           } else {
@@ -1090,11 +1092,14 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.out = h;
   p.out_ld = ex.F;
   p.m_limit = ex.F;
-  p.act = ex.act;
   p.status = status;
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_SWIGLU, false>(p, ta, ub, s);
-  return run<MOE_W_BF16, EPI_SWIGLU, false>(p, ta, ub, s);
+  const bool geglu = ex.act == MOE_ACT_GEGLU_TANH;
+  if (ex.fmt == MOE_W_Q4G64)
+    return geglu ? run<MOE_W_Q4G64, EPI_GEGLU, false>(p, ta, ub, s)
+                 : run<MOE_W_Q4G64, EPI_SWIGLU, false>(p, ta, ub, s);
+  return geglu ? run<MOE_W_BF16, EPI_GEGLU, false>(p, ta, ub, s)
+               : run<MOE_W_BF16, EPI_SWIGLU, false>(p, ta, ub, s);
 }
 
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
