@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(256) down_gemv_kernel(
       const float v = warp_sum(acc[j]);
       if (lane == 0 && j < nr) {
         if (sizeof(typename HType<TA>::T) == 2) {
-          // fp16 ys (bf16 activations): out-of-range values are reported
+          // fp16 ys (16-bit activations): out-of-range values are reported
           if (!(fabsf(v) < 65520.f)) report_status(status, MOE_ERR_RANGE);
           reinterpret_cast<__half*>(ys)[(size_t)(rb + j) * d + o] = __float2half_rn(v);
         } else {
