@@ -186,6 +186,20 @@ def test_f16_activations_decode_every_finite_half(orc):
     assert by_bits[0x0400] == 2.0 ** -14       # smallest normal
 
 
+@pytest.mark.parametrize("act", ["f16", "bf16"])
+def test_16bit_forward_equals_f32_forward_on_same_values(orc, act):
+    """The whole layer on 16-bit activations equals the layer on fp32
+    activations holding the same values (both exact in fp32): the oracle reads
+    x and the router weight through the 16-bit decoding at every use."""
+    wl = mi.workload("tiny", T=7, d=128, E=4, k=2, F=64, wfmt="q4", act=act)
+    L = mi.make_layer(wl, seed=4)
+    a = orc.forward(L.x, L.w_router, L.router_bias, L.experts, wl.k)
+    b = orc.forward(L.x.float(), L.w_router.float(), L.router_bias, L.experts, wl.k)
+    np.testing.assert_array_equal(a.idx, b.idx)
+    np.testing.assert_array_equal(a.y, b.y)
+    np.testing.assert_array_equal(a.logits64, b.logits64)
+
+
 def test_logits_f16_match_library_matmul(orc):
     wl = mi.workload("decode_t32", d=256, E=16, act="f16")
     L = mi.make_layer(wl, seed=2)
