@@ -136,6 +136,22 @@ def test_pack_gate_up_rejects_bad_arguments(moe):
     assert L.moe_pack_gate_up(moe.W_Q4G64, 2, 64, 64, fake, P, fake, fake, fake, fake, fake, fake, fake, P) == moe.ERR_INVALID_ARG
 
 
+def test_regime_choice(moe):
+    """AUTO takes the tensor-core kernels for many rows per expert with 16-bit
+    activations, the weight-streaming ones for few rows or fp32."""
+    torch = __import__("torch")
+    prefill = (2048, 2048, 512, 10, 512)       # 40 rows per expert
+    decode = (32, 2048, 128, 8, 768)           # 2 rows per expert
+    for dt in (torch.bfloat16, torch.float16):
+        assert moe.forward_layout(*prefill, dt).regime == moe.REGIME_TC
+        assert moe.forward_layout(*decode, dt).regime == moe.REGIME_GEMV
+    assert moe.forward_layout(*prefill, torch.float32).regime == moe.REGIME_GEMV
+    # an explicit regime is kept
+    assert moe.forward_layout(*decode, torch.bfloat16, moe.REGIME_TC).regime == moe.REGIME_TC
+    with pytest.raises(TypeError):
+        moe.forward_layout(*decode, torch.int8)
+
+
 def test_forward_layout_is_consistent(moe):
     for (T, d, E, k, F) in [(1, 2048, 128, 8, 768), (2048, 2048, 512, 10, 512), (16, 128, 8, 2, 256)]:
         L = moe.forward_layout(T, d, E, k, F, __import__("torch").bfloat16)
