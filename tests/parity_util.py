@@ -28,28 +28,18 @@ def rms(a) -> float:
     return float(np.sqrt(np.mean(a * a))) if a.size else 0.0
 
 
-def assert_close_rms(gpu, ref, tol, what="", rounded_to=None):
-    """max |gpu - ref| <= tol * RMS(ref). With rounded_to="bf16" (an
-    intermediate the kernel stores in bf16) each element may in addition
-    differ by one bf16 rounding of its own value, 2^-8 * |ref| (twice the
-    half-ulp bound, for the fp32 error it is added to)."""
+def assert_close_rms(gpu, ref, tol, what=""):
+    """max |gpu - ref| <= tol * RMS(ref)."""
     g = to_np(gpu).astype(np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (what, g.shape, r.shape)
     assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
     if r.size == 0:
         return 0.0
-    err = np.abs(g - r)
+    e = float(np.abs(g - r).max())
     bound = tol * rms(r)
-    if rounded_to == "bf16":
-        excess = err - (bound + 2.0 ** -8 * np.abs(r))
-        i = int(np.argmax(excess))
-        assert excess.flat[i] <= 0, (f"{what}: |err| {err.flat[i]:.3e} at {i} (ref {r.flat[i]:.4e}) > "
-                                     f"{tol} * RMS {rms(r):.3e} + 2^-8 |ref|")
-    else:
-        e = float(err.max())
-        assert e <= bound, f"{what}: max|err| {e:.3e} > {tol} * RMS {rms(r):.3e} = {bound:.3e}"
-    return float(err.max()) / max(rms(r), 1e-300)
+    assert e <= bound, f"{what}: max|err| {e:.3e} > {tol} * RMS {rms(r):.3e} = {bound:.3e}"
+    return e / max(rms(r), 1e-300)
 
 
 def topk_ref(logits_np, k):
@@ -88,44 +78,59 @@ def _act_and_slope(g, act):
     return g * sig, sig * (1.0 + g * (1.0 - sig))
 
 
+def _check_stage(gpu, ref, elem_bound, tol, what):
+    """The two rules every intermediate stage (h, ys) must meet:
+    (a) the contract's rule for floating outputs, max |gpu - ref| <= tol *
+        RMS(ref), over the whole tensor; and
+    (b) per element, |gpu - ref| <= 2 * (the first-order effect of the
+        roundings the kernel documents) + 1e-3 * RMS(ref). The factor 2 and
+        the small floor cover second-order terms and fp16 subnormals; (b) is
+        far tighter than (a) for most elements, so an error confined to a few
+        small elements (a wrong token row, a swapped feature) fails it even
+        where it stays under (a)."""
+    g = to_np(gpu).astype(np.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
+    if ref.size == 0:
+        return 0.0
+    err = np.abs(g - ref)
+    r = rms(ref)
+    e = float(err.max())
+    assert e <= tol * r, f"{what}: max|err| {e:.3e} > {tol} * RMS {r:.3e} = {tol * r:.3e}"
+    bound = 2.0 * elem_bound + 1e-3 * r
+    i = int(np.argmax(err - bound))
+    assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "
+                                          f"(ref {ref.flat[i]:.4e}) > per-element bound "
+                                          f"{bound.flat[i]:.3e}")
+    return e / max(r, 1e-300)
+
+
 def assert_h_close(h_gpu, href, g, u, ga, ua, d, u_w, u_h, tol, what="", act="swiglu"):
     """h = act(g) * u as the kernels compute it: weights rounded to the
     operand format before the products (unit roundoff u_w, so |dg| <= u_w *
-    sum |x w|; 0 when the weights are exact in it), products accumulated in
-    fp32 (2 d 2^-24 * sum |x w| with margin), h rounded once to its storage
-    format (u_h |h|). The first-order bound per element is
-        tol * RMS(h) + u_h |h| + |u act'(g)| dg + |act(g)| du."""
-    gh = to_np(h_gpu).astype(np.float64)
-    assert gh.shape == href.shape, (what, gh.shape, href.shape)
-    assert np.isfinite(gh).all(), f"{what}: non-finite GPU output"
-    if href.size == 0:
-        return 0.0
-    acc = 2.0 * d * 2.0 ** -24
+    sum |x w|; 0 when the weights are exact in it), d products accumulated in
+    fp32 (at most d 2^-24 * sum |x w|), h rounded once to its storage format
+    (u_h |h|). The first-order effect per element is
+        u_h |h| + |u act'(g)| dg + |act(g)| du,
+    checked as _check_stage's rule (b), next to the contract's rule (a)."""
+    href = np.asarray(href, dtype=np.float64)
+    acc = d * 2.0 ** -24
     dg = (u_w + acc) * ga
     du = (u_w + acc) * ua
     a, da = _act_and_slope(g, act)
-    bound = tol * rms(href) + u_h * np.abs(href) + np.abs(u * da) * dg + np.abs(a) * du
-    err = np.abs(gh - href)
-    i = int(np.argmax(err - bound))
-    assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "
-                                          f"(ref {href.flat[i]:.4e}) > bound {bound.flat[i]:.3e}")
-    return float(err.max()) / max(rms(href), 1e-300)
+    elem = u_h * np.abs(href) + np.abs(u * da) * dg + np.abs(a) * du
+    return _check_stage(h_gpu, href, elem, tol, what)
 
 
-def assert_ys_close(ys_gpu, yref, habs, u_w, tol, what="", u_ys=0.0):
-    """ys = h . W_d^T accumulated in fp32: weights rounded to the operand
-    format (unit roundoff u_w) add at most u_w * sum |h w|; storing ys in a
-    format of unit roundoff u_ys adds u_ys * |ys| (+ half its smallest
-    subnormal step, 2^-25 for fp16)."""
-    g = to_np(ys_gpu).astype(np.float64)
-    assert g.shape == yref.shape and np.isfinite(g).all(), what
-    if yref.size == 0:
-        return 0.0
-    bound = tol * rms(yref) + u_w * habs
+def assert_ys_close(ys_gpu, yref, habs, u_w, tol, what="", u_ys=0.0, F=0):
+    """ys = h . W_d^T accumulated in fp32 over F products: weights rounded to
+    the operand format (unit roundoff u_w) add at most u_w * sum |h w|, the
+    fp32 sum at most F 2^-24 * sum |h w|, and storing ys in a format of unit
+    roundoff u_ys adds u_ys |ys| (+ half the smallest fp16 subnormal step,
+    2^-25). Checked as _check_stage's rules (a) and (b)."""
+    yref = np.asarray(yref, dtype=np.float64)
+    assert F > 0, "F: the length of the down projection's sums"
+    elem = (u_w + F * 2.0 ** -24) * habs
     if u_ys:
-        bound = bound + u_ys * np.abs(yref) + 2.0 ** -25
-    err = np.abs(g - yref)
-    i = int(np.argmax(err - bound))
-    assert err.flat[i] <= bound.flat[i], (f"{what}: |err| {err.flat[i]:.3e} at {i} "
-                                          f"(ref {yref.flat[i]:.4e}) > bound {bound.flat[i]:.3e}")
-    return float(err.max()) / max(rms(yref), 1e-300)
+        elem = elem + u_ys * np.abs(yref) + 2.0 ** -25
+    return _check_stage(ys_gpu, yref, elem, tol, what)

@@ -188,7 +188,7 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
     habs = orc.expert_down_abs(hin.double().numpy(), ref_st.row_off, hx)
     u_w = U_F16 if mi.q4_group(wl.wfmt) else 0.0
     u_ys = U_F16 if wl.act == "bf16" else 0.0
-    assert_ys_close(ys, yref, habs, u_w, _tol(wl.act), f"ys[{name}]", u_ys=u_ys)
+    assert_ys_close(ys, yref, habs, u_w, _tol(wl.act), f"ys[{name}]", u_ys=u_ys, F=wl.F)
 
 
 @pytest.mark.parametrize("T,k,d,dt", [(1, 8, 2048, torch.bfloat16), (16, 2, 128, torch.float32),
@@ -375,7 +375,7 @@ def test_grouped_stages_q4_group_sizes(moe, orc, wfmt):
     ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1)
     yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
     habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
-    assert_ys_close(ys, yref, habs, U_F16, TOL_BF16, f"ys[{wfmt}]", u_ys=U_F16)
+    assert_ys_close(ys, yref, habs, U_F16, TOL_BF16, f"ys[{wfmt}]", u_ys=U_F16, F=wl.F)
 
 
 @pytest.mark.parametrize("wfmt,T", [("q4g128", 300), ("q4g32", 1024)])
@@ -407,7 +407,7 @@ def test_grouped_stages_q8(moe, orc):
     ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1)
     yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
     habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
-    assert_ys_close(ys, yref, habs, 2.0 ** -24, TOL_BF16, "ys[q8]", u_ys=U_F16)
+    assert_ys_close(ys, yref, habs, 2.0 ** -24, TOL_BF16, "ys[q8]", u_ys=U_F16, F=wl.F)
 
 
 @pytest.mark.parametrize("name,T", [("decode_t1", 1), ("prefill", 64)])
@@ -449,7 +449,7 @@ def test_grouped_stages_f16(moe, orc, name, T, regime, BM, wfmt):
     ys = moe.grouped_down(h, st, T, wl.k, layer.experts, regime=regime)
     yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
     habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
-    assert_ys_close(ys, yref, habs, u_w, TOL_BF16, f"ys[f16 {name} {wfmt}]", u_ys=U_F16)
+    assert_ys_close(ys, yref, habs, u_w, TOL_BF16, f"ys[f16 {name} {wfmt}]", u_ys=U_F16, F=wl.F)
     assert moe.device_status() == moe.OK
 
 

@@ -446,3 +446,97 @@ def test_zipf_bias_gives_stated_skew(orc):
     counts = np.bincount(idx.reshape(-1), minlength=wl.E)
     assert counts.max() > 10 * counts.mean()
     assert (counts == 0).any()
+
+
+# ------------------------------------------------------------ error-bound helpers
+
+def _decode_q4_by_definition(words, scales, biases, group):
+    """A test-side decoding of 4-bit affine weights written from the format's
+    definition alone: element j of a 32-bit word is bits [4j, 4j+3], groups of
+    `group` consecutive input elements share one bf16 scale and bias, value =
+    scale * q + bias. Shares nothing with the oracle's decoder."""
+    w = words.view(torch.int32).numpy().astype(np.int64) & 0xFFFFFFFF      # [..., K/8]
+    q = np.stack([(w >> (4 * j)) & 0xF for j in range(8)], axis=-1)        # [..., K/8, 8]
+    q = q.reshape(*w.shape[:-1], w.shape[-1] * 8).astype(np.float64)       # [..., K]
+    s = np.repeat(scales.double().numpy(), group, axis=-1)
+    b = np.repeat(biases.double().numpy(), group, axis=-1)
+    return s * q + b
+
+
+def _expert_weights_fp64(ex, which):
+    """[E, rows, cols] fp64 values of an expert stack ("gu" or "dn")."""
+    w = ex.w_gu if which == "gu" else ex.w_dn
+    if mi.q4_group(ex.fmt):
+        s, b = (ex.s_gu, ex.b_gu) if which == "gu" else (ex.s_dn, ex.b_dn)
+        return _decode_q4_by_definition(w, s, b, mi.q4_group(ex.fmt))
+    return w.double().numpy()
+
+
+def _routed_tables(orc, T, E, k, seed):
+    """Sort tables of a skewed random routing with at least one empty expert,
+    so that row_map is not the identity and expert blocks differ in size."""
+    idx = mi.random_topk_idx(T, E - 1, k, seed=seed, skew=0.6).numpy()
+    idx = np.where(idx >= 2, idx + 1, idx).astype(np.int32)        # expert 2 gets no rows
+    st = orc.sort_rows(idx, E, 4)
+    assert (st.counts == 0).any() and len(set(st.counts.tolist())) > 2
+    assert (st.row_map != np.arange(T * k) // k).any()
+    return st
+
+
+@pytest.mark.parametrize("wfmt,act", [("f32", "f32"), ("bf16", "bf16"), ("q4", "bf16"),
+                                      ("q4g32", "f16")])
+def test_expert_gate_up_against_library_matmul(orc, wfmt, act):
+    """orc.expert_gate_up (the pre-activations and the absolute-product sums
+    the GPU parity tests build their per-element bounds from) against torch
+    fp64 matmuls on a test-side decoding of the weights: for every expert e
+    and its sorted rows i, with X = x[row_map[i]],
+        g = X Wg_e^T, u = X Wu_e^T, ga = |X| |Wg_e|^T, ua = |X| |Wu_e|^T,
+    Wg_e = rows 0..F-1 and Wu_e = rows F..2F-1 of expert e's fused block.
+    A swapped gate/up, a dropped fabs, a row read without row_map or another
+    expert's weights each fail it. And h from orc.expert_swiglu is silu(g) u
+    from torch's silu on the same g and u."""
+    T, E, k, d, F = 40, 6, 3, 128, 64
+    wl = mi.workload("tiny", T=T, d=d, E=E, k=k, F=F, wfmt=wfmt, act=act)
+    L = mi.make_layer(wl, seed=17)
+    st = _routed_tables(orc, T, E, k, seed=18)
+    g, u, ga, ua = orc.expert_gate_up(L.x, st.row_map, st.row_off, L.experts)
+    W = _expert_weights_fp64(L.experts, "gu")                       # [E, 2F, d]
+    x = L.x.double().numpy()
+    for e in range(E):
+        r0, r1 = int(st.row_off[e]), int(st.row_off[e + 1])
+        X = torch.from_numpy(x[st.row_map[r0:r1].astype(np.int64)])
+        Wg, Wu = torch.from_numpy(W[e, :F]), torch.from_numpy(W[e, F:])
+        for got, want in ((g, X @ Wg.T), (u, X @ Wu.T), (ga, X.abs() @ Wg.abs().T),
+                          (ua, X.abs() @ Wu.abs().T)):
+            np.testing.assert_allclose(got[r0:r1], want.numpy(), rtol=1e-12, atol=1e-13)
+    assert (ga >= np.abs(g)).all() and (ua >= np.abs(u)).all()
+    h = orc.expert_swiglu(L.x, st.row_map, st.row_off, L.experts)
+    gt, ut = torch.from_numpy(g), torch.from_numpy(u)
+    np.testing.assert_allclose(h, (torch.nn.functional.silu(gt) * ut).numpy(), rtol=1e-12,
+                               atol=1e-14)
+
+
+@pytest.mark.parametrize("wfmt", ["f32", "q4", "q4g128"])
+def test_expert_down_and_abs_against_library_matmul(orc, wfmt):
+    """orc.expert_down and orc.expert_down_abs against torch fp64 matmuls on a
+    test-side decoding of the weights: for the sorted rows i of expert e,
+    ys = h Wd_e^T and |h| |Wd_e|^T. Rows of h carry random signs, so a
+    dropped fabs changes the sums; the expert blocks differ in size, so a
+    wrong row_off or expert fails."""
+    T, E, k, d, F = 30, 5, 2, 128, 128
+    wl = mi.workload("tiny", T=T, d=d, E=E, k=k, F=F, wfmt=wfmt,
+                     act="f32" if wfmt == "f32" else "bf16")
+    L = mi.make_layer(wl, seed=19)
+    st = _routed_tables(orc, T, E, k, seed=20)
+    h = mi.random_rows(T * k, F, seed=21, dtype=torch.float32).double().numpy()
+    assert (h < 0).any() and (h > 0).any()
+    ys = orc.expert_down(h, st.row_off, L.experts)
+    habs = orc.expert_down_abs(h, st.row_off, L.experts)
+    W = _expert_weights_fp64(L.experts, "dn")                       # [E, d, F]
+    for e in range(E):
+        r0, r1 = int(st.row_off[e]), int(st.row_off[e + 1])
+        H, Wd = torch.from_numpy(h[r0:r1]), torch.from_numpy(W[e])
+        np.testing.assert_allclose(ys[r0:r1], (H @ Wd.T).numpy(), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(habs[r0:r1], (H.abs() @ Wd.abs().T).numpy(), rtol=1e-12,
+                                   atol=1e-13)
+    assert (habs >= np.abs(ys)).all()
