@@ -176,6 +176,36 @@ def time_device(fn, steps, warmup, flush):
     return [a.elapsed_time(b) for a, b in zip(starts, ends)]
 
 
+def time_layer(moe, layer, k, steps, warmup, flush, pk):
+    """One workload's whole-layer forward, graph-replayed and timed like the
+    headline step (L2 flushed before every step): ms per step, tokens/s, and
+    the layer's algorithmic bytes (the experts with at least one routed row,
+    read once, + x + y) and flops (6 R d F) as fractions of the peaks."""
+    wl = layer.wl
+    ws = moe.forward_workspace(layer.x, layer.experts, k)
+    y = torch.empty(wl.T, wl.d, dtype=layer.x.dtype, device=layer.x.device)
+    fwd = lambda: moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, k,
+                              ws=ws, out=y)
+    fwd()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    torch.cuda.synchronize()
+    ms = statistics.mean(time_device(g.replay, steps, warmup, flush))
+    L = moe.forward_layout(wl.T, wl.d, wl.E, k, wl.F, layer.x.dtype, wl.wfmt)
+    counts = ws[L.counts:L.counts + wl.E * 4].view(torch.int32).cpu().numpy()
+    active = int((counts > 0).sum())
+    nbytes = active * expert_bytes(layer.experts) + 2 * wl.T * wl.d * layer.x.element_size()
+    flops = 6.0 * wl.T * k * wl.d * wl.F
+    del g
+    return {"T": wl.T, "k": k, "ms": ms, "us_per_layer": ms * 1e3,
+            "tokens_per_s": wl.T / (ms * 1e-3), "active_experts": active,
+            "regime": {1: "gemv", 2: "tcgen05"}.get(L.regime, "?"),
+            "bytes": nbytes, "flops": flops,
+            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "tensor_frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]}
+
+
 def run_ours(args, rank, world, local_rank):
     import sparse_mixture_experts_top_b200 as moe
     dev = torch.device("cuda", local_rank)
@@ -189,7 +219,7 @@ def run_ours(args, rank, world, local_rank):
     y = torch.empty(T, wl.d, dtype=layer.x.dtype, device=dev)
     flush = (torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
              torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev))
-    L = moe.forward_layout(T, wl.d, wl.E, k, wl.F, layer.x.dtype)
+    L = moe.forward_layout(T, wl.d, wl.E, k, wl.F, layer.x.dtype, wl.wfmt)
 
     def fwd():
         moe.forward(layer.x, layer.w_router, layer.router_bias, ex, k, ws=ws, out=y)
@@ -252,57 +282,37 @@ def run_ours(args, rank, world, local_rank):
 
     ms_e2e = time_device(e2e, args.steps, args.warmup, flush)
 
-    # decode rows (T = 1 and T = 32), same procedure
-    decode = {}
-    if not args.no_decode:
-        for name in ("decode_t1", "decode_t32"):
-            dl = mi.make_layer(name, seed=args.seed + 1000 * rank, device=dev)
-            dws = moe.forward_workspace(dl.x, dl.experts, dl.wl.k)
-            dy = torch.empty(dl.wl.T, dl.wl.d, dtype=dl.x.dtype, device=dev)
-            f2 = lambda: moe.forward(dl.x, dl.w_router, dl.router_bias, dl.experts, dl.wl.k,
-                                     ws=dws, out=dy)
-            f2()
-            g2 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g2):
-                f2()
-            torch.cuda.synchronize()
-            dms = statistics.mean(time_device(g2.replay, max(args.steps, 20), args.warmup, flush))
-            dL = moe.forward_layout(dl.wl.T, dl.wl.d, dl.wl.E, dl.wl.k, dl.wl.F, dl.x.dtype)
-            dcounts = dws[dL.counts:dL.counts + dl.wl.E * 4].view(torch.int32).cpu().numpy()
-            dbytes = int((dcounts > 0).sum()) * expert_bytes(dl.experts) + 2 * dl.wl.T * dl.wl.d * 2
-            decode[name] = {"tokens_per_s": dl.wl.T / (dms * 1e-3), "us_per_layer": dms * 1e3,
-                            "selected_expert_bytes": dbytes,
-                            "hbm_frac": dbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"]}
-            del dl, dws, g2
-
-    # sparse (top-k) against dense soft routing (k = E: every expert, full
-    # softmax weights) at the PRD's acceptance shape, through the same call
-    dense = {}
+    # the other workloads, each as one graph-replayed forward timed the same
+    # way: decode at T = 1 and T = 32, the acceptance shape (sparse top-2 and
+    # dense soft routing, k = E) and the large skewed layer
+    extra = {}
+    names = [] if args.no_decode else ["decode_t1", "decode_t32"]
     if not args.no_dense:
-        al = mi.make_layer("acceptance", seed=args.seed + 1000 * rank, device=dev)
-        times = {}
-        for kk in (al.wl.k, al.wl.E):
-            aws = moe.forward_workspace(al.x, al.experts, kk)
-            ay = torch.empty(al.wl.T, al.wl.d, dtype=al.x.dtype, device=dev)
-            f3 = lambda: moe.forward(al.x, al.w_router, None, al.experts, kk, ws=aws, out=ay)
-            f3()
-            g3 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g3):
-                f3()
-            torch.cuda.synchronize()
-            times[kk] = statistics.mean(time_device(g3.replay, max(args.steps, 20), args.warmup,
-                                                    flush))
-            del g3, aws
-        wlA = al.wl
+        names.append("acceptance")
+    if not args.no_skewed:
+        names.append("skewed")
+    for name in names:
+        other = mi.make_layer(name, seed=args.seed + 1000 * rank, device=dev)
+        ks = [other.wl.k] + ([other.wl.E] if name == "acceptance" else [])
+        for kk in ks:
+            key = name if kk == other.wl.k else name + "_dense"
+            extra[key] = time_layer(moe, other, kk, max(args.steps, 20), args.warmup, flush, pk)
+        del other
+        torch.cuda.empty_cache()
+    decode = {n: extra[n] for n in ("decode_t1", "decode_t32") if n in extra}
+    dense = {}
+    if "acceptance" in extra:
+        wlA = mi.WORKLOADS["acceptance"]
+        sp, dn = extra["acceptance"]["ms"], extra["acceptance_dense"]["ms"]
         dense = {"workload": f"acceptance: T={wlA.T} d={wlA.d} E={wlA.E} F={wlA.F} bf16 experts",
-                 "sparse_k": wlA.k, "sparse_ms": times[wlA.k], "dense_ms": times[wlA.E],
-                 "speedup": times[wlA.E] / times[wlA.k], "target": 1.5}
-        del al
+                 "sparse_k": wlA.k, "sparse_ms": sp, "dense_ms": dn, "speedup": dn / sp,
+                 "target": 1.5}
 
     step_ms = statistics.mean(ms)
     res = {"ms": step_ms, "ms_eager": statistics.mean(ms_eager), "ms_e2e": statistics.mean(ms_e2e),
            "ms_swiglu": statistics.mean(ms_swiglu), "achieved_gbs": achieved_gbs,
            "tflops_swiglu": tflops, "gu_bytes": gu_bytes, "clocks": clocks, "decode": decode, "sparse_vs_dense": dense,
+           "acceptance": extra.get("acceptance"), "skewed": extra.get("skewed"),
            "active": active, "regime": regime, "BM": L.BM, "pk": pk, "pk_kind": pk_kind,
            "layer_bytes": active * expert_bytes(ex) + 2 * T * wl.d * 2,
            "layer_flops": 6.0 * T * k * wl.d * wl.F}
@@ -350,6 +360,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-skewed", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -419,6 +430,8 @@ def main():
             "gpu_launches": kernels_per_forward(wl.T, wl.k, res["regime"] == 2) * args.steps,
             "clocks": res["clocks"],
             "decode": res["decode"],
+            "acceptance": res["acceptance"],
+            "skewed": res["skewed"],
             "sparse_vs_dense": res["sparse_vs_dense"],
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -43,8 +43,11 @@
  *   - Argument errors are detected on the host before any launch and returned
  *     synchronously; nothing is launched then. MOE_ERR_CUDA reports a launch
  *     error (cudaGetLastError after the launches).
- *   - Device-side errors (a bounded wait that ran out) are recorded in a
- *     device status word; read and clear it with moe_device_status().
+ *   - Device-side errors (a bounded wait that ran out, a value outside the
+ *     fp16 range of the expert GEMMs) are recorded in one status word per
+ *     device and per process: every call on that device, on any stream or
+ *     host thread, reports into the same word, and the first error since
+ *     the last read is kept. Read and clear it with moe_device_status().
  *   - T = 0 is valid: the call returns MOE_OK and launches nothing.
  *   - Preconditions: 1 <= k <= min(E, 32); E <= 1024; d and F multiples of 64;
  *     bf16 expert weights need bf16 activations, f32 weights need f32
@@ -52,7 +55,13 @@
  *     MOE_ERR_UNSUPPORTED.
  *   - All layouts are row-major with the stated shapes; buffers must be
  *     16-byte aligned.
- *   - Calls are reentrant; the library holds no per-call state.
+ *   - Calls are reentrant and keep no state between calls, apart from the
+ *     device status word above, the no-allocation sort's scratch array
+ *     (moe_sort_rows_noalloc) and the wait bound (moe_set_wait_cycles).
+ *   - The library looks up the device addresses of its own device variables
+ *     (the status word, the no-allocation scratch) once per device and keeps
+ *     them for the life of the process; a cudaDeviceReset() followed by
+ *     further calls is not supported.
  *
  * Regimes: moe_grouped_swiglu / moe_grouped_down / moe_forward take a regime.
  *   MOE_REGIME_GEMV: weight-streaming kernels, every selected expert's bytes
@@ -196,7 +205,9 @@ moe_status moe_sort_rows(const int32_t* topk_idx, int T, int k, int E, int BM, u
  *     no cudaMalloc, cudaFree or any allocating routine.
  *   Set-up: the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture. MOE_ERR_CUDA if the lookup fails.
+ *     before any stream capture. MOE_ERR_CUDA if the lookup fails. The
+ *     address is kept for the life of the process (see the conventions:
+ *     cudaDeviceReset is not supported).
  *   Sharing: every call uses the same array. Calls that may overlap on the
  *     GPU (other streams, other host threads) race and corrupt each other's
  *     result; serialise them. The array keeps the last call's contents; the
@@ -263,25 +274,60 @@ moe_status moe_combine(const void* ys, const uint32_t* inv_order, const float* t
  *   y   (device, out) [T][d], dtype dt
  *   ws  (device) workspace of moe_forward_workspace(...) bytes; it holds the
  *       intermediates at the offsets moe_forward_layout() reports */
-size_t moe_forward_workspace(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime);
+size_t moe_forward_workspace(int T, int d, int E, int k, int F, moe_dtype dt, moe_wfmt wfmt,
+                             moe_regime regime);
 moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const float* router_bias,
                        const moe_experts* experts, int T, int k, void* y, void* ws,
                        size_t ws_bytes, moe_regime regime, moe_stream_t stream);
 
 /* Where moe_forward keeps each intermediate inside its workspace (byte
- * offsets), the regime it resolves to and the BM it sorts with. */
+ * offsets), the regime it resolves to for experts of weight format wfmt and
+ * the BM it sorts with. moe_forward_workspace(...) is its `total`; 0 when the
+ * arguments are invalid. */
 typedef struct {
   size_t logits, topk_idx, topk_w, order, inv_order, row_map, counts, row_off, tile_off;
   size_t sort_ws, h, ys, x16, total;
   int32_t regime; /* resolved: MOE_REGIME_GEMV or MOE_REGIME_TC */
   int32_t BM;
 } moe_ws_layout;
-moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime,
-                              moe_ws_layout* out /* (host, out) */);
+moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_wfmt wfmt,
+                              moe_regime regime, moe_ws_layout* out /* (host, out) */);
 
-/* Read the device status word (MOE_OK or the first device-side error since
- * the last read) and reset it. Synchronises the current device. */
+/* Token rows per tile (BM) of the tensor-core regime: moe_grouped_swiglu and
+ * moe_grouped_down in that regime need tile_off written by moe_sort_rows with
+ * this BM (DS4Server issue #112, "Kernel contract": per-expert tile prefix
+ * table). The weight-streaming regime takes any BM >= 1. */
+int moe_sort_block_m(void);
+
+/* Read the current device's status word (MOE_OK or the first device-side
+ * error since the last read, from any stream) and reset it. Synchronises the
+ * current device. */
 moe_status moe_device_status(void);
+
+/* Bound of the device-side waits, in SM cycles. Every kernel that waits
+ * (for a copy, an MMA, another warp role or another CTA) gives up after this
+ * many cycles, records MOE_ERR_TIMEOUT in the device status word, finishes
+ * the copies and MMAs it has in flight, releases its tensor memory and
+ * returns; the caller reads the status with moe_device_status(). The bound is
+ * one value for the whole process, read by every launch after the call. 0
+ * restores the default, 2e9 cycles (about one second at the B200's clocks);
+ * a short bound is for tests that make the waits of a real forward run out.
+ * The source pages have no counterpart to this call.
+ * Negative values: MOE_ERR_INVALID_ARG. */
+moe_status moe_set_wait_cycles(long long cycles);
+
+/* Test support, no counterpart on the source pages: launches a one-block
+ * kernel whose single wait can never be satisfied, with a bound of `cycles`
+ * (>= 1), using the library's own wait code, so that a test can see a
+ * bounded wait run out and the kernel return with MOE_ERR_TIMEOUT recorded
+ * in the device status word.
+ *   which 0: the mbarrier wait of the tensor-core grouped kernels;
+ *         1: the mbarrier wait of the fused decode kernel;
+ *         2: the grid barrier of the fused decode kernel; scratch (device,
+ *            16-byte aligned, >= 4 bytes) holds its counter
+ * Asynchronous on `stream`; MOE_OK when launched. */
+moe_status moe_selftest_wait_timeout(int which, long long cycles, void* scratch,
+                                     moe_stream_t stream);
 
 /* Pack separate gate and up projections into the fused [gate|up] layout the
  * kernels read (w_gu rows 0..F-1 gate, F..2F-1 up of every expert).

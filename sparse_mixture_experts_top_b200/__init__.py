@@ -25,11 +25,11 @@ W_F32, W_BF16, W_Q4G64 = 0, 1, 2
 REGIME_AUTO, REGIME_GEMV, REGIME_TC = 0, 1, 2
 
 EXPORTS = ("moe_route", "moe_topk", "moe_sort_rows_workspace", "moe_sort_rows",
-           "moe_sort_rows_noalloc",
+           "moe_sort_rows_noalloc", "moe_sort_block_m",
            "moe_grouped_swiglu_workspace", "moe_grouped_swiglu", "moe_grouped_down",
            "moe_combine", "moe_forward_workspace", "moe_pack_gate_up",
            "moe_forward", "moe_forward_layout", "moe_device_status", "moe_status_str",
-           "moe_version")
+           "moe_version", "moe_set_wait_cycles", "moe_selftest_wait_timeout")
 
 
 class MoeError(RuntimeError):
@@ -69,13 +69,20 @@ def _load():
                                      P]
     L.moe_grouped_down.argtypes = [P, I, P, P, I, I, I, ctypes.POINTER(Experts), P, I, P]
     L.moe_combine.argtypes = [P, P, P, I, I, I, I, P, P]
-    L.moe_forward_workspace.argtypes = [I, I, I, I, I, I, I]
+    L.moe_forward_workspace.argtypes = [I, I, I, I, I, I, I, I]
     L.moe_forward_workspace.restype = S
     L.moe_forward.argtypes = [P, I, P, P, ctypes.POINTER(Experts), I, I, P, P, S, I, P]
-    L.moe_forward_layout.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(WsLayout)]
+    L.moe_forward_layout.argtypes = [I, I, I, I, I, I, I, I, ctypes.POINTER(WsLayout)]
+    L.moe_sort_block_m.argtypes = []
+    L.moe_sort_block_m.restype = ctypes.c_int
+    L.moe_sort_rows_noalloc.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P]
     L.moe_pack_gate_up.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, P, P]
     L.moe_pack_gate_up.restype = ctypes.c_int
     L.moe_device_status.argtypes = []
+    L.moe_set_wait_cycles.argtypes = [ctypes.c_longlong]
+    L.moe_set_wait_cycles.restype = ctypes.c_int
+    L.moe_selftest_wait_timeout.argtypes = [I, ctypes.c_longlong, P, P]
+    L.moe_selftest_wait_timeout.restype = ctypes.c_int
     L.moe_status_str.argtypes = [I]
     L.moe_status_str.restype = ctypes.c_char_p
     L.moe_version.restype = ctypes.c_char_p
@@ -221,13 +228,23 @@ def grouped_swiglu(x, tables: SortTables, k, experts, regime=REGIME_AUTO, ws=Non
     return h
 
 
-def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, stream=None):
-    """-> ys [T*k, d]: fp16 for 16-bit activations (fp16 h), fp32 for fp32"""
+def grouped_down(h, tables: SortTables, T, k, experts, regime=REGIME_AUTO, stream=None,
+                 dtype=None):
+    """-> ys [T*k, d]: fp16 for 16-bit activations (fp16 h), fp32 for fp32.
+    `dtype` is the layer's activation type (torch.bfloat16, torch.float16 or
+    torch.float32); it may be left out for fp32 h, which only fp32
+    activations produce."""
     _dev(h)
     ex = experts_struct(experts)
-    # h is fp16 exactly when the activations are 16-bit; ys has h's dtype,
-    # and the step is the same for bf16 and fp16 activations
-    adt = BF16 if h.dtype == torch.float16 else F32
+    if dtype is None:
+        if h.dtype != torch.float32:
+            raise TypeError("grouped_down: pass dtype, the activation type (bf16 or fp16) "
+                            "the fp16 h was computed from")
+        dtype = torch.float32
+    adt = _dt_of(dtype)
+    want = torch.float32 if adt == F32 else torch.float16
+    if h.dtype != want:
+        raise TypeError(f"h must be {want} for {dtype} activations")
     ys = torch.empty(T * k, experts.d, dtype=h.dtype, device=h.device)
     _check(lib.moe_grouped_down(_ptr(h), adt, _ptr(tables.row_off), _ptr(tables.tile_off),
                                 tables.BM, T, k, ctypes.byref(ex), _ptr(ys), regime,
@@ -251,16 +268,29 @@ def combine(ys, inv_order, topk_w, T, k, dtype=torch.bfloat16, stream=None):
 
 # ------------------------------------------------------------------ forward
 
-def forward_layout(T, d, E, k, F, dtype, regime=REGIME_AUTO) -> WsLayout:
+def _fmt_code(fmt) -> int:
+    return _FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def forward_layout(T, d, E, k, F, dtype, wfmt, regime=REGIME_AUTO) -> WsLayout:
+    """moe_forward's workspace layout for experts of weight format `wfmt`
+    (a name such as "q4", or a moe_wfmt code)."""
     L = WsLayout()
     dt = _dt_of(dtype)
-    _check(lib.moe_forward_layout(T, d, E, k, F, dt, regime, ctypes.byref(L)), "moe_forward_layout")
+    _check(lib.moe_forward_layout(T, d, E, k, F, dt, _fmt_code(wfmt), regime, ctypes.byref(L)),
+           "moe_forward_layout")
     return L
+
+
+def sort_block_m() -> int:
+    """BM of the tensor-core regime (moe_sort_block_m)."""
+    return lib.moe_sort_block_m()
 
 
 def forward_workspace(x, experts, k, regime=REGIME_AUTO):
     """A workspace tensor large enough for moe_forward on these shapes."""
-    L = forward_layout(x.shape[0], experts.d, experts.E, k, experts.F, x.dtype, regime)
+    L = forward_layout(x.shape[0], experts.d, experts.E, k, experts.F, x.dtype, experts.fmt,
+                       regime)
     return torch.empty(max(L.total, 256), dtype=torch.uint8, device=x.device)
 
 
@@ -302,3 +332,8 @@ def pack_gate_up(fmt, w_g, w_u, s_g=None, b_g=None, s_u=None, b_u=None, stream=N
 def device_status() -> int:
     """Status word of device-side errors since the last read (resets it)."""
     return lib.moe_device_status()
+
+
+def set_wait_cycles(cycles: int):
+    """Bound of every device-side wait, in SM cycles (0: the default, ~1 s)."""
+    _check(lib.moe_set_wait_cycles(int(cycles)), "moe_set_wait_cycles")

@@ -1,6 +1,7 @@
 // C ABI entry points: argument checks, workspace carving, launch sequences.
 // Every check runs on the host before the first launch; nothing here reads
 // device memory or synchronises a stream (except moe_device_status).
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -22,6 +23,14 @@ static int* status_ptr() {
     ptrs[dev] = static_cast<int*>(p);
   }
   return ptrs[dev];
+}
+
+// bound of every device-side wait for work, in SM cycles; 0 = the default
+static std::atomic<long long> g_wait_cycles{0};
+
+long long wait_cycles() {
+  const long long v = g_wait_cycles.load(std::memory_order_relaxed);
+  return v > 0 ? v : kDefaultWaitCycles;
 }
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -145,6 +154,23 @@ moe_status moe_device_status(void) {
   const int zero = 0;
   if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
   return (moe_status)v;
+}
+
+moe_status moe_set_wait_cycles(long long cycles) {
+  if (cycles < 0) return MOE_ERR_INVALID_ARG;
+  g_wait_cycles.store(cycles, std::memory_order_relaxed);
+  return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(int which, long long cycles, void* scratch,
+                                     moe_stream_t stream) {
+  if (which < 0 || which > 2 || cycles < 1) return MOE_ERR_INVALID_ARG;
+  if (which == 2 && (!scratch || !aligned16(scratch))) return MOE_ERR_INVALID_ARG;
+  int* stp = status_ptr();
+  if (!stp) return MOE_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (which == 0) return launched(launch_tc_wait_selftest(cycles, stp, s));
+  return launched(launch_decode_wait_selftest(which, cycles, (unsigned*)scratch, stp, s));
 }
 
 moe_status moe_topk(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
@@ -328,10 +354,13 @@ moe_status moe_pack_gate_up(int fmt, int E, int d, int F, const void* w_g, const
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime,
-                              moe_ws_layout* out) {
+int moe_sort_block_m(void) { return tc_block_m(); }
+
+moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, moe_wfmt wfmt,
+                              moe_regime regime, moe_ws_layout* out) {
   if (!out) return MOE_ERR_INVALID_ARG;
   if (!valid_dt(dt)) return MOE_ERR_INVALID_ARG;
+  if (wfmt < MOE_W_F32 || wfmt > MOE_W_Q8G64) return MOE_ERR_INVALID_ARG;
   moe_status st = check_dims(T, d, E, k);
   if (st != MOE_OK) return st;
   if (F <= 0) return MOE_ERR_INVALID_ARG;
@@ -358,7 +387,7 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
   L.h = take((size_t)R * F * a);      // fp16 (16-bit activations) or fp32
   L.ys = take((size_t)R * d * a);     // fp16 (16-bit activations) or fp32
-  L.regime = resolve_regime(regime, R, E, dt, d, F);
+  L.regime = resolve_regime(regime, R, E, dt, d, F, wfmt);
   L.BM = block_m_for(L.regime, R, E);
   // fp16 token rows: x converted (weight-streaming), or permuted (the
   // one-launch path), or gathered in sorted row order (tensor cores)
@@ -368,9 +397,10 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   return MOE_OK;
 }
 
-size_t moe_forward_workspace(int T, int d, int E, int k, int F, moe_dtype dt, moe_regime regime) {
+size_t moe_forward_workspace(int T, int d, int E, int k, int F, moe_dtype dt, moe_wfmt wfmt,
+                             moe_regime regime) {
   moe_ws_layout L;
-  if (moe_forward_layout(T, d, E, k, F, dt, regime, &L) != MOE_OK) return 0;
+  if (moe_forward_layout(T, d, E, k, F, dt, wfmt, regime, &L) != MOE_OK) return 0;
   return L.total;
 }
 
@@ -387,18 +417,15 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
   if (!x || !w_router || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   moe_ws_layout L;
-  st = moe_forward_layout(T, d, E, k, F, dt, regime, &L);
+  st = moe_forward_layout(T, d, E, k, F, dt, (moe_wfmt)experts->fmt, regime, &L);
   if (st != MOE_OK) return st;
   if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  if (L.regime == MOE_REGIME_TC && dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
-  // the layout assumes q4 weights; other formats the tensor-core kernels do
-  // not tile take the weight-streaming kernels (which accept any BM)
-  int regime_run = L.regime;
-  if (regime_run == MOE_REGIME_TC && !tc_shape_supported(d, F, experts->fmt, dt)) {
-    if (regime == MOE_REGIME_TC) return MOE_ERR_UNSUPPORTED;
-    regime_run = MOE_REGIME_GEMV;
-  }
+  // AUTO resolves to TC only for shapes and formats the tensor-core kernels
+  // tile; an explicit TC request for others is refused
+  const int regime_run = L.regime;
+  if (regime_run == MOE_REGIME_TC && !tc_shape_supported(d, F, experts->fmt, dt))
+    return MOE_ERR_UNSUPPORTED;
 
   char* base = static_cast<char*>(ws);
   float* logits = (float*)(base + L.logits);

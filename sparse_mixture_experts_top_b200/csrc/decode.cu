@@ -96,6 +96,7 @@ struct Params {
   int xf16;                                   // activations are fp16 (else bf16)
   unsigned* sync;                             // grid barrier counter, zero before launch
   int* status;
+  long long wait_limit;                       // SM cycles a wait for work may take
 };
 
 // ------------------------------------------------------------------ PTX
@@ -124,16 +125,20 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait; false when it ran out or (honor_abort) the kernel is aborting
+// bounded wait (at most `limit` SM cycles); false when it ran out or
+// (honor_abort) the kernel is aborting. Waits for work take the launch's bound
+// (Params::wait_limit); the producer's final wait for its copies in flight
+// keeps the full bound, so no copy lands after the CTA has exited.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int* status, bool honor_abort = true) {
+                                       int* status, bool honor_abort = true,
+                                       long long limit = kWaitCycles) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 15u) == 0) {
       if (honor_abort && *abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         report_status(status, MOE_ERR_TIMEOUT);
         return false;
@@ -220,9 +225,11 @@ __device__ __forceinline__ void group_sync(int grp) {
 
 // Grid-wide barrier of the compute warps of all CTAs: a counter that only
 // grows (zeroed before the launch); barrier n waits for n * gridDim.x
-// arrivals. Bounded: on expiry the status gets MOE_ERR_TIMEOUT.
+// arrivals. Bounded (`limit` SM cycles): on expiry the status gets
+// MOE_ERR_TIMEOUT. A CTA that is aborting still arrives, so the others are
+// not kept waiting for it.
 __device__ __noinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, long long limit) {
   compute_sync();
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
@@ -235,7 +242,7 @@ __device__ __noinline__ bool grid_barrier(unsigned* ctr, unsigned n, volatile in
       unsigned v;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
       if (v >= target) break;
-      if (*abort_flag || clock64() - t0 > kWaitCycles) {
+      if (*abort_flag || clock64() - t0 > limit) {
         if (!*abort_flag) report_status(status, MOE_ERR_TIMEOUT);
         *abort_flag = 1;
         ok = 0;
@@ -520,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
   }
   bool ok = true;
-  if (warp < kCw) ok = grid_barrier(p.sync, 1, &s_abort, p.status);
+  if (warp < kCw) ok = grid_barrier(p.sync, 1, &s_abort, p.status, p.wait_limit);
   __syncthreads();
   if (s_abort) ok = false;
 
@@ -607,7 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       for (; s < nseq; ++s) {
         const int slot = s % kSlots;
         if (s >= kSlots &&
-            !mbar_wait(smem_u32(empty + slot), ((s / kSlots) - 1) & 1, &s_abort, p.status))
+            !mbar_wait(smem_u32(empty + slot), ((s / kSlots) - 1) & 1, &s_abort, p.status, true,
+                       p.wait_limit))
           break;
         const uint32_t dst = smem_u32(ring + slot * kSlotBytes);
         const uint32_t bar = smem_u32(full + slot);
@@ -686,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     for (int s = grp; s < pl.nB; s += kNg) {
       const int slot = s % kSlots;
       ok = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(full + slot), (s / kSlots) & 1,
-                                                   &s_abort, p.status));
+                                                   &s_abort, p.status, true, p.wait_limit));
       ok = group_sync_and(grp, ok);
       if (!ok) break;
       const uint8_t* sp = ring + slot * kSlotBytes;
@@ -726,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (lane == 0) mbar_arrive(smem_u32(empty + slot));
     }
     // all of h is written before any CTA reads it
-    if (!grid_barrier(p.sync, 2, &s_abort, p.status)) ok = false;
+    if (!grid_barrier(p.sync, 2, &s_abort, p.status, p.wait_limit)) ok = false;
 
     // down -> ys (fp16, sorted row order): an item is dr output rows of active
     // expert a against the expert's h rows; with 32 rows, warps 0-1 of the
@@ -738,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     for (int s = pl.nB + (((grp - pl.nB) % kNg) + kNg) % kNg; s < nseq; s += kNg) {
       const int slot = s % kSlots;
       ok = __all_sync(0xffffffffu, ok && mbar_wait(smem_u32(full + slot), (s / kSlots) & 1,
-                                                   &s_abort, p.status));
+                                                   &s_abort, p.status, true, p.wait_limit));
       ok = group_sync_and(grp, ok);
       if (!ok) break;
       const uint8_t* sp = ring + slot * kSlotBytes;
@@ -778,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (lane == 0) mbar_arrive(smem_u32(empty + slot));
     }
     // all of ys is written before any CTA reads it
-    if (!grid_barrier(p.sync, 3, &s_abort, p.status)) ok = false;
+    if (!grid_barrier(p.sync, 3, &s_abort, p.status, p.wait_limit)) ok = false;
 
     // combine: y[t][o .. o+7] = sum over j of w[t][j] * ys[inv[t*k + j]][o ..
     // o+7], fp32 fused multiply-adds in j order, one rounding to bf16 (fp16)
@@ -854,6 +862,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   }
 }
 
+// Test support: each kind of bounded wait of this file, made to run out. The
+// mbarrier expects two arrivals and gets one; the grid barrier of a one-CTA
+// grid waits for arrivals number 1 and 2 of barrier 2 after only one. Both
+// must give up after `limit` cycles, record MOE_ERR_TIMEOUT and return.
+__global__ void __launch_bounds__(kThreads, 1) wait_selftest_kernel(int which, long long limit,
+                                                                    unsigned* ctr, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int s_abort;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 2);
+    s_abort = 0;
+    *ctr = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __threadfence();
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  if (which == 1) {
+    if (threadIdx.x == 0) {
+      mbar_arrive(smem_u32(&bar));
+      mbar_wait(smem_u32(&bar), 0, &s_abort, status, true, limit);
+    }
+  } else if (warp < kCw) {
+    grid_barrier(ctr, 2, &s_abort, status, limit);
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------------ host
 
 static int sm_count() {
@@ -864,6 +900,12 @@ static int sm_count() {
 }
 
 }  // namespace dec
+
+cudaError_t launch_decode_wait_selftest(int which, long long limit, unsigned* ctr, int* status,
+                                        cudaStream_t s) {
+  dec::wait_selftest_kernel<<<1, dec::kThreads, 0, s>>>(which, limit, ctr, status);
+  return cudaGetLastError();
+}
 
 bool decode_fused_ok(int T, int k, int E, int d, int F, int fmt, int dt) {
   using namespace dec;
@@ -918,6 +960,7 @@ cudaError_t launch_decode_fused(const void* x, int dt, const void* w_router, con
   p.y = (uint16_t*)y;
   p.sync = sync;
   p.status = status;
+  p.wait_limit = wait_cycles();
   const size_t smem = decode_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

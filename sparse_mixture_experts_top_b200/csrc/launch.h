@@ -8,6 +8,16 @@
 
 namespace moe {
 
+// SM cycles a device-side wait for work may take before the kernel records
+// MOE_ERR_TIMEOUT and aborts (moe_set_wait_cycles; about one second unless set)
+constexpr long long kDefaultWaitCycles = 2000000000LL;
+long long wait_cycles();
+
+// Test support: make one kind of bounded wait run out (see moe_selftest_wait_timeout)
+cudaError_t launch_tc_wait_selftest(long long limit, int* status, cudaStream_t s);
+cudaError_t launch_decode_wait_selftest(int which, long long limit, unsigned* ctr, int* status,
+                                        cudaStream_t s);
+
 // Router logits L[T][E] = x[T][d] . w_router[E][d]^T + bias, fp32 out.
 cudaError_t launch_router_logits(const void* x, int dt, const void* w_router, const float* bias,
                                  int T, int d, int E, float* logits, cudaStream_t s);

@@ -120,6 +120,7 @@ struct Params {
   int router_f16;      // router: x and the router weight are fp16 (else bf16)
   const float* bias;   // router bias or null
   int* status;
+  long long wait_limit;  // SM cycles a wait for work may take (moe_set_wait_cycles)
 };
 
 // ------------------------------------------------------------------ PTX
@@ -164,16 +165,23 @@ __device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, ui
   return ok != 0;
 }
 
-// Bounded wait for the phase of `parity` to complete. Returns false when the
-// kernel is aborting (another role timed out) or this wait ran out.
+// Bounded wait for the phase of `parity` to complete: at most `limit` SM
+// cycles. Returns false when the kernel is aborting (another role timed out;
+// ignored when !honor_abort) or this wait ran out. Waits for work use the
+// launch's bound (Params::wait_limit); the waits for copies and MMAs still in
+// flight before the CTA exits keep the full bound, so that nothing lands in
+// shared memory or TMEM after the CTA has released it. A bound below ~50 us
+// also drops the sleep hint, so the wait notices its deadline promptly.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, bool honor_abort = true) {
+                                          int* status, bool honor_abort = true,
+                                          long long limit = kWaitCycles) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
+  const bool sleep = limit >= 100000;
   for (;;) {
-    if (mbar_try_sleep(bar, parity, 20000u)) return true;
+    if (sleep ? mbar_try_sleep(bar, parity, 20000u) : mbar_try(bar, parity)) return true;
     if (honor_abort && *abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       report_status(status, MOE_ERR_TIMEOUT);
       return false;
@@ -185,8 +193,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // converged for the .sync.aligned tcgen05 instructions that follow.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, int* status,
-                                               bool honor_abort = true) {
-  const bool r = mbar_wait(bar, parity, abort_flag, status, honor_abort);
+                                               bool honor_abort = true,
+                                               long long limit = kWaitCycles) {
+  const bool r = mbar_wait(bar, parity, abort_flag, status, honor_abort, limit);
   return __all_sync(0xffffffffu, r);
 }
 
@@ -509,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kr = 0; kr < nkr && ok; ++kr) {
         const int rs = raw_it % C::NR;
         ok = mbar_wait_warp(smem_u32(raw_empty + rs), ((raw_it / C::NR) & 1) ^ 1, abort_flag,
-                            p.status);
+                            p.status, true, p.wait_limit);
         if (!ok) break;
         if (C::Q4) {
           // the stage's scales and biases (4 groups of each weight row), 8
@@ -580,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int bs = j % NB;
           if (j >= (uint32_t)NB) {
             const uint32_t pr = (j - NB) >> 1;
-            ok = mbar_wait(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status);
+            ok = mbar_wait(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status, true, p.wait_limit);
             if (!ok) break;
           }
           const uint32_t bar = smem_u32(b_full + bs / 2);
@@ -626,9 +635,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool use0 = !small || b == 0, use1 = !small || b == 1;
       // the epilogue has drained the buffers' previous tiles
       if (use0 && uses0 > 0)
-        ok = mbar_wait_warp(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status);
+        ok = mbar_wait_warp(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
       if (ok && use1 && uses1 > 0)
-        ok = mbar_wait_warp(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status);
+        ok = mbar_wait_warp(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
       if (!ok) break;
       tc_fence_after();
       const uint32_t dcol = tm + (small ? b * 128u + q * 64u : q * 128u);
@@ -637,8 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // waits, eight MMAs and one release per pair. The pair's two A stages
       // complete one barrier; both B stages share another.
       for (int kb = 0; kb < nka && ok; kb += 2) {
-        ok = mbar_wait_warp(afull0 + (ss >> 1) * 8, sph, abort_flag, p.status) &&
-             mbar_wait_warp(smem_u32(b_full + bs / 2), bph, abort_flag, p.status);
+        ok = mbar_wait_warp(afull0 + (ss >> 1) * 8, sph, abort_flag, p.status, true, p.wait_limit) &&
+             mbar_wait_warp(smem_u32(b_full + bs / 2), bph, abort_flag, p.status, true, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t acol = a_col0 + ss * (uint32_t)C::A_COLS;
@@ -673,8 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool small = mma_n(nv) <= 64;
       const uint32_t b = small ? nb : 0u;
       const bool use0 = !small || b == 0, use1 = !small || b == 1;
-      if (use0 && !mbar_wait_warp(smem_u32(acc_full + 0), uses0 & 1, abort_flag, p.status)) break;
-      if (use1 && !mbar_wait_warp(smem_u32(acc_full + 1), uses1 & 1, abort_flag, p.status)) break;
+      if (use0 && !mbar_wait_warp(smem_u32(acc_full + 0), uses0 & 1, abort_flag, p.status, true, p.wait_limit)) break;
+      if (use1 && !mbar_wait_warp(smem_u32(acc_full + 1), uses1 & 1, abort_flag, p.status, true, p.wait_limit)) break;
       tc_fence_after();
       const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
       const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
@@ -771,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       for (int kr = 0; kr < nkr && ok; ++kr) {
         const int rs = raw_it % C::NR;
-        ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status);
+        ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status, true, p.wait_limit);
         if (!ok) break;
         // my half row: 4 chunks of 16 B in the 128-byte swizzle
         const uint32_t rowa = raw_base + rs * C::RAW_BYTES + q * C::RAW_MAT + m * 128;
@@ -837,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t as = stage % NS;
           if (stage >= (uint32_t)NS) {      // the slot's previous k-block is released
             const uint32_t pr = (stage - NS) >> 1;
-            ok = mbar_wait_warp(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status);
+            ok = mbar_wait_warp(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status, true, p.wait_limit);
             if (!ok) break;
           }
           tc_fence_after();
@@ -860,6 +869,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
   }
+}
+
+// Test support: the mbarrier wait of this file made to run out. The barrier
+// expects two arrivals and gets one, so the wait must give up after `limit`
+// cycles, record MOE_ERR_TIMEOUT and return.
+__global__ void wait_selftest_kernel(long long limit, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 2);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_arrive(smem_u32(&bar));
+  __syncwarp();
+  mbar_wait_warp(smem_u32(&bar), 0, &abort_flag, status, true, limit);
 }
 
 // ------------------------------------------------------------------ host
@@ -1034,6 +1060,11 @@ static bool tc_shape_ok(const moe_experts& ex, int dt) {
 
 int tc_block_m() { return tc::BN; }
 
+cudaError_t launch_tc_wait_selftest(long long limit, int* status, cudaStream_t s) {
+  tc::wait_selftest_kernel<<<1, 32, 0, s>>>(limit, status);
+  return cudaGetLastError();
+}
+
 bool tc_shape_supported(int d, int F, int fmt, int dt) {
   moe_experts ex{};
   ex.d = d;
@@ -1093,6 +1124,7 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.out_ld = ex.F;
   p.m_limit = ex.F;
   p.status = status;
+  p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
   const bool geglu = ex.act == MOE_ACT_GEGLU_TANH;
   if (ex.fmt == MOE_W_Q4G64)
@@ -1128,6 +1160,7 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.out_ld = ex.d;
   p.m_limit = ex.d;
   p.status = status;
+  p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
   if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE, false>(p, ta, ub, s);
   return run<MOE_W_BF16, EPI_STORE, false>(p, ta, ub, s);
@@ -1160,6 +1193,7 @@ cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router,
   p.m_limit = E;
   p.bias = bias;
   p.status = status;
+  p.wait_limit = wait_cycles();
   // token tiles small enough that at least half of the SMs get a unit: every
   // unit streams the same weight rows through one SM, so more, shorter
   // units spread the router over the GPU (down to 16 rows, the MMA's least N)

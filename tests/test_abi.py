@@ -138,23 +138,47 @@ def test_pack_gate_up_rejects_bad_arguments(moe):
 
 def test_regime_choice(moe):
     """AUTO takes the tensor-core kernels for many rows per expert with 16-bit
-    activations, the weight-streaming ones for few rows or fp32."""
+    activations and a weight format they tile, the weight-streaming ones for
+    few rows, fp32, or formats the tensor-core kernels do not take."""
     torch = __import__("torch")
     prefill = (2048, 2048, 512, 10, 512)       # 40 rows per expert
     decode = (32, 2048, 128, 8, 768)           # 2 rows per expert
     for dt in (torch.bfloat16, torch.float16):
-        assert moe.forward_layout(*prefill, dt).regime == moe.REGIME_TC
-        assert moe.forward_layout(*decode, dt).regime == moe.REGIME_GEMV
-    assert moe.forward_layout(*prefill, torch.float32).regime == moe.REGIME_GEMV
+        assert moe.forward_layout(*prefill, dt, "q4").regime == moe.REGIME_TC
+        assert moe.forward_layout(*decode, dt, "q4").regime == moe.REGIME_GEMV
+    assert moe.forward_layout(*prefill, torch.float32, "f32").regime == moe.REGIME_GEMV
+    # bf16 weights: F % 256 == 128 is a shape the tensor-core kernels tile
+    # (q4 needs F % 256 == 0)
+    acc = (512, 2048, 8, 2, 640)
+    assert moe.forward_layout(*acc, torch.bfloat16, "bf16").regime == moe.REGIME_TC
+    assert moe.forward_layout(*acc, torch.bfloat16, "q4").regime == moe.REGIME_GEMV
     # an explicit regime is kept
-    assert moe.forward_layout(*decode, torch.bfloat16, moe.REGIME_TC).regime == moe.REGIME_TC
+    assert moe.forward_layout(*decode, torch.bfloat16, "q4", moe.REGIME_TC).regime == moe.REGIME_TC
     with pytest.raises(TypeError):
-        moe.forward_layout(*decode, torch.int8)
+        moe.forward_layout(*decode, torch.int8, "q4")
+    # an unknown weight format is refused
+    L = moe.WsLayout()
+    assert moe.lib.moe_forward_layout(*decode, moe.BF16, 9, 0, ctypes.byref(L)) == moe.ERR_INVALID_ARG
+
+
+def test_sort_block_m_is_the_tensor_core_tile(moe):
+    """moe_sort_block_m is the BM the tensor-core regime needs: the layout of a
+    forward that resolves to that regime sorts with it, and a stage call in
+    that regime with another BM is refused."""
+    torch = __import__("torch")
+    bm = moe.sort_block_m()
+    assert bm == 128
+    L = moe.forward_layout(2048, 2048, 512, 10, 512, torch.bfloat16, "q4")
+    assert L.regime == moe.REGIME_TC and L.BM == bm
+    fake = ctypes.c_void_p(0x10000)
+    ex = _ex(moe, d=256)
+    assert moe.lib.moe_grouped_down(fake, moe.BF16, fake, fake, bm // 2, 4, 2, ctypes.byref(ex),
+                                    fake, 2, P) == moe.ERR_INVALID_ARG
 
 
 def test_forward_layout_is_consistent(moe):
     for (T, d, E, k, F) in [(1, 2048, 128, 8, 768), (2048, 2048, 512, 10, 512), (16, 128, 8, 2, 256)]:
-        L = moe.forward_layout(T, d, E, k, F, __import__("torch").bfloat16)
+        L = moe.forward_layout(T, d, E, k, F, __import__("torch").bfloat16, "q4")
         offs = [L.logits, L.topk_idx, L.topk_w, L.order, L.inv_order, L.row_map, L.counts,
                 L.row_off, L.tile_off, L.sort_ws, L.h, L.ys, L.x16]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
@@ -163,7 +187,7 @@ def test_forward_layout_is_consistent(moe):
         assert L.x16 + (T * k if L.regime == moe.REGIME_TC else T) * d * 2 <= L.total
         assert L.h + T * k * F * 2 <= L.ys
         assert L.BM >= 1 and L.regime in (moe.REGIME_GEMV, moe.REGIME_TC)
-        assert moe.lib.moe_forward_workspace(T, d, E, k, F, moe.BF16, 0) == L.total
+        assert moe.lib.moe_forward_workspace(T, d, E, k, F, moe.BF16, moe.W_Q4G64, 0) == L.total
         # fp16 activations take the same layout as bf16 ones
-        L16 = moe.forward_layout(T, d, E, k, F, __import__("torch").float16)
+        L16 = moe.forward_layout(T, d, E, k, F, __import__("torch").float16, "q4")
         assert (L16.total, L16.x16, L16.regime, L16.BM) == (L.total, L.x16, L.regime, L.BM)

@@ -179,7 +179,8 @@ def test_grouped_down_parity(moe, orc, name, T, regime, BM, skew):
     st = moe.sort_rows(idx.to(DEV), wl.E, BM)
     hin = mi.random_rows(T * wl.k, wl.F, seed=23,
                          dtype=torch.float16 if wl.act == "bf16" else torch.float32)
-    ys = moe.grouped_down(hin.to(DEV), st, T, wl.k, layer.experts, regime=regime)
+    ys = moe.grouped_down(hin.to(DEV), st, T, wl.k, layer.experts, regime=regime,
+                          dtype=layer.x.dtype)
     ref_st = orc.sort_rows(idx.numpy(), wl.E, BM)
     hx = _host(layer.experts)
     yref = orc.expert_down(hin.double().numpy(), ref_st.row_off, hx)
@@ -372,7 +373,7 @@ def test_grouped_stages_q4_group_sizes(moe, orc, wfmt):
     href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
     g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
     assert_h_close(h, href, g, u, ga, ua, wl.d, U_F16, U_F16, TOL_BF16, f"h[{wfmt}]")
-    ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1)
+    ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1, dtype=layer.x.dtype)
     yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
     habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
     assert_ys_close(ys, yref, habs, U_F16, TOL_BF16, f"ys[{wfmt}]", u_ys=U_F16, F=wl.F)
@@ -404,7 +405,7 @@ def test_grouped_stages_q8(moe, orc):
     g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
     # the SIMT kernel dequantises in fp32: 2^-24 per weight
     assert_h_close(h, href, g, u, ga, ua, wl.d, 2.0 ** -24, U_F16, TOL_BF16, "h[q8]")
-    ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1)
+    ys = moe.grouped_down(h, st, 32, wl.k, layer.experts, regime=1, dtype=layer.x.dtype)
     yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
     habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
     assert_ys_close(ys, yref, habs, 2.0 ** -24, TOL_BF16, "ys[q8]", u_ys=U_F16, F=wl.F)
@@ -446,7 +447,7 @@ def test_grouped_stages_f16(moe, orc, name, T, regime, BM, wfmt):
     simt = BM > 16 or wfmt == "q8"
     u_w = 2.0 ** -24 if simt else U_F16
     assert_h_close(h, href, g, u, ga, ua, wl.d, u_w, U_F16, TOL_BF16, f"h[f16 {name} {wfmt}]")
-    ys = moe.grouped_down(h, st, T, wl.k, layer.experts, regime=regime)
+    ys = moe.grouped_down(h, st, T, wl.k, layer.experts, regime=regime, dtype=layer.x.dtype)
     yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
     habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
     assert_ys_close(ys, yref, habs, u_w, TOL_BF16, f"ys[f16 {name} {wfmt}]", u_ys=U_F16, F=wl.F)
@@ -513,7 +514,7 @@ def test_forward_intermediates_match_stage_calls(moe):
     wl = layer.wl
     ws = moe.forward_workspace(layer.x, layer.experts, wl.k)
     moe.forward(layer.x, layer.w_router, None, layer.experts, wl.k, ws=ws)
-    L = moe.forward_layout(wl.T, wl.d, wl.E, wl.k, wl.F, layer.x.dtype)
+    L = moe.forward_layout(wl.T, wl.d, wl.E, wl.k, wl.F, layer.x.dtype, wl.wfmt)
     R = wl.T * wl.k
     seg = lambda off, n, dt: ws[off:off + n * 4].view(dt)
     _, idx, _ = moe.route(layer.x, layer.w_router, None, wl.k)

@@ -46,6 +46,9 @@ def test_noalloc_sort_matches_workspace_sort_on_two_calls_in_a_row(moe):
     # that uses the scratch); second call: different sizes and ids, so any
     # stale per-chunk count from the first call would change the result
     cases = [(2048, 512, 10, 128, 0.02, 1), (1500, 64, 6, 64, 0.3, 2)]
+    # then the documented limit, which fills the whole scratch: 32,768 rows
+    # (32 chunks) over 1,024 experts
+    cases.append((4096, 1024, 8, 128, 0.0, 3))
     for T, E, k, BM, skew, seed in cases:
         idx = mi.random_topk_idx(T, E, k, seed=seed, skew=skew).cuda()
         got = _noalloc(moe, idx, E, BM)
@@ -61,4 +64,7 @@ def test_noalloc_sort_rejects_sizes_beyond_its_scratch(moe):
     fake = ctypes.c_void_p(0x10000)
     # 32768 rows is the limit; 32769 is refused on the host, before any launch
     assert moe.lib.moe_sort_rows_noalloc(fake, 32769, 1, 8, 128, fake, fake, fake, fake, fake,
+                                         fake, None) == moe.ERR_UNSUPPORTED
+    # 1,024 experts is the limit; 1,025 is refused the same way
+    assert moe.lib.moe_sort_rows_noalloc(fake, 16, 2, 1025, 128, fake, fake, fake, fake, fake,
                                          fake, None) == moe.ERR_UNSUPPORTED
