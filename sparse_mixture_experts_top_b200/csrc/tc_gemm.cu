@@ -108,6 +108,8 @@ struct Params {
   int n_units;         // units (pairs of weight matrices) per token tile
   int unit_rows;       // weight rows from one unit to the next
   int mat_off;         // row offset of matrix 1 from matrix 0 inside a unit
+  int row_step;        // rows from one row of a matrix to the next: 1, or 2 when
+                       // matrix 0 takes the even and matrix 1 the odd rows
   int K;               // reduction length
   int rows_per_group;  // weight rows per expert in the stacked tensor
   int G;               // q4 groups per weight row (K / 64)
@@ -531,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < BMW / 32; ++j) {
               const int m = lane + 32 * j;
-              long long grow = (mat ? wrow1 : wrow0) + m;
+              long long grow = (mat ? wrow1 : wrow0) + (long long)m * p.row_step;
               if (grow >= p.w_rows) grow = p.w_rows - 1;
               const uint32_t o = (uint32_t)((mat * BMW + m) * 8);
               asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sdst + o),
@@ -727,22 +729,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          // the down projection's units are 256 whole rows of d (d % 256 == 0)
-          __half* op = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + orow0;
+          // the down projection's units are 256 whole rows of d (d % 256 ==
+          // 0): matrix 0 holds the even, matrix 1 the odd output features,
+          // so this thread's two features are adjacent and each token's
+          // pair goes out as one 4-byte store (a warp writes 128 contiguous
+          // bytes of a ys row)
+          const int of = unit * p.unit_rows + 2 * m;
+          uint32_t* op = reinterpret_cast<uint32_t*>(reinterpret_cast<__half*>(p.out) +
+                                                     (size_t)r0 * p.out_ld + of);
+          const size_t ld2 = (size_t)p.out_ld / 2;
           for (int n0 = 0; n0 < nv; n0 += 16) {
             uint32_t a0[16], a1[16];
             tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
             const int lim = nv - n0;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const __half v0 = __float2half_rn(__uint_as_float(a0[j]));
-              const __half v1 = __float2half_rn(__uint_as_float(a1[j]));
+              const uint32_t v = f16x2_pack(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
               if (j < lim) {
-                hmax = max(hmax, max((uint32_t)__half_as_ushort(v0) & 0x7FFFu,
-                                     (uint32_t)__half_as_ushort(v1) & 0x7FFFu));
-                __half* o = op + (size_t)(n0 + j) * p.out_ld;
-                o[0] = v0;
-                o[BMW] = v1;
+                hmax = max(hmax, max(v & 0x7FFFu, (v >> 16) & 0x7FFFu));
+                op[(size_t)(n0 + j) * ld2] = v;
               }
             }
           }
@@ -908,13 +913,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // `row_bytes`, box (box_inner, box_outer).
 static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
                      uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                     CUtensorMapSwizzle sw) {
+                     CUtensorMapSwizzle sw, uint32_t outer_step = 1) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
+  // with an outer traversal stride of s the box spans box_outer rows and
+  // loads every s-th of them (box_outer / s rows)
   cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
+  cuuint32_t estr[2] = {1, outer_step};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -929,13 +936,15 @@ static int num_sms() {
 
 // raw weight-tile map over a stack of `rows` weight rows of K elements
 // (16-bit rows are bf16, or fp16 for an fp16 router weight)
+// (row_step 2: each load takes every other row, 128 of 256)
 static bool weight_map(CUtensorMap* m, int fmt, const void* w, long long rows, int K,
-                       bool f16 = false) {
+                       bool f16 = false, uint32_t row_step = 1) {
   if (fmt == MOE_W_Q4G64)
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / 8, rows, (uint64_t)K / 2, 32, BMW,
-                    CU_TENSOR_MAP_SWIZZLE_128B);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / 8, rows, (uint64_t)K / 2, 32,
+                    BMW * row_step, CU_TENSOR_MAP_SWIZZLE_128B, row_step);
   return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w,
-                  K, rows, (uint64_t)K * 2, 64, BMW, CU_TENSOR_MAP_SWIZZLE_128B);
+                  K, rows, (uint64_t)K * 2, 64, BMW * row_step, CU_TENSOR_MAP_SWIZZLE_128B,
+                  row_step);
 }
 
 // bf16 -> fp16, 8 values per thread; values that do not round to a finite
@@ -1114,6 +1123,7 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.n_units = ex.F / BMW;
   p.unit_rows = BMW;
   p.mat_off = ex.F;
+  p.row_step = 1;
   p.K = ex.d;
   p.rows_per_group = 2 * ex.F;
   p.G = ex.d / 64;
@@ -1141,7 +1151,9 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   if (!tc_shape_ok(ex, ex.fmt == MOE_W_Q4G64 ? MOE_F16 : MOE_BF16)) return cudaErrorNotSupported;
   if (R <= 0) return cudaSuccess;
   CUtensorMap ta;
-  if (!weight_map(&ta, ex.fmt, ex.w_dn, (long long)ex.E * ex.d, ex.F)) return cudaErrorInvalidValue;
+  // matrix 0 = the unit's even output rows, matrix 1 = its odd rows
+  if (!weight_map(&ta, ex.fmt, ex.w_dn, (long long)ex.E * ex.d, ex.F, false, 2))
+    return cudaErrorInvalidValue;
   Params p{};
   if (!token_maps(p, h, false, R, ex.F)) return cudaErrorInvalidValue;
   p.row_off = row_off;
@@ -1149,7 +1161,8 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.E = ex.E;
   p.n_units = ex.d / (2 * BMW);
   p.unit_rows = 2 * BMW;
-  p.mat_off = BMW;
+  p.mat_off = 1;
+  p.row_step = 2;
   p.K = ex.F;
   p.rows_per_group = ex.d;
   p.G = ex.F / 64;
@@ -1186,6 +1199,7 @@ cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router,
   p.n_units = (E + 2 * BMW - 1) / (2 * BMW);
   p.unit_rows = 2 * BMW;
   p.mat_off = BMW;
+  p.row_step = 1;
   p.K = d;
   p.w_rows = E;
   p.out = logits;
