@@ -180,16 +180,19 @@ __device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
 // s*q + b, rounded once. Nibbles 0 and 4 (bits 0-3, 16-19) are ORed into the
 // mantissa of fp16 1024.0, whose last place is 1; nibbles 1 and 5 (bits 4-7,
 // 20-23) into that of fp16 64.0, whose last place is 1/16, so both pairs
-// read magic + q; the word shifted by 8 gives nibbles 2, 6 and 3, 7 the same
-// way. The magic is subtracted exactly and one fused multiply-add applies
-// scale and bias: 5 integer and 8 fp16 operations per 8 weights.
+// read magic + q. A byte permute puts bytes 1 and 3 (e3:e2, e7:e6) under the
+// exponent of 1024, giving 1024 + 16 e3 + e2; its bits 4-7 ORed into 64.0
+// give 64 + e3, and e2 = (1024 + 16 e3 + e2) - 16 (64 + e3) exactly. The
+// magic is subtracted exactly and one fused multiply-add applies scale and
+// bias: 4 integer and 8 fp16 operations per 8 weights.
 __device__ __forceinline__ void q4_word_perm(uint32_t w, uint32_t s2, uint32_t b2, uint32_t* o) {
-  const uint32_t c1024 = 0x64006400u, c64 = 0x54005400u;
-  const uint32_t w8 = w >> 8;
+  const uint32_t c1024 = 0x64006400u, c64 = 0x54005400u, m16 = 0xCC00CC00u;   // -16.0
+  const uint32_t hi = __byte_perm(w, 0x64646464u, 0x4341);
+  const uint32_t d = (hi & 0x00F000F0u) | c64;
   o[0] = h2_fma(h2_sub((w & 0x000F000Fu) | c1024, c1024), s2, b2);
   o[1] = h2_fma(h2_sub((w & 0x00F000F0u) | c64, c64), s2, b2);
-  o[2] = h2_fma(h2_sub((w8 & 0x000F000Fu) | c1024, c1024), s2, b2);
-  o[3] = h2_fma(h2_sub((w8 & 0x00F000F0u) | c64, c64), s2, b2);
+  o[2] = h2_fma(h2_fma(d, m16, hi), s2, b2);
+  o[3] = h2_fma(h2_sub(d, c64), s2, b2);
 }
 
 // Orderable 32-bit image of a float: larger float -> larger key; -0 -> +0;

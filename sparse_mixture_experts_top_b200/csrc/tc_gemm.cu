@@ -372,19 +372,23 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t b
 // word. A nibble at bits 0..3 of a 16-bit half becomes the mantissa of
 // fp16 1024.0 (0x6400 | q = 1024 + q); one at bits 4..7 becomes mantissa
 // bits 4..7 of fp16 64.0, whose last place is 1/16 (0x5400 | 16q = 64 + q).
-// Each pair is then one AND-OR, half of the words are shifted once, the
-// magic number is subtracted exactly and one fused multiply-add applies the
-// scale and bias: 5 integer operations per word instead of 9. The other
-// operand must use the same order: within every 8 consecutive K elements,
-// position p holds element (0, 4, 1, 5, 2, 6, 3, 7)[p].
+// Pairs (e0,e4) and (e1,e5) are one AND-OR each. For (e2,e6) and (e3,e7) a
+// byte permute puts bytes 1 and 3 of the word (e3:e2, e7:e6) under the
+// exponent of 1024, giving 1024 + 16 e3 + e2 (and e7, e6); one AND-OR of that
+// gives 64 + e3, and e2 = (1024 + 16 e3 + e2) - 16 (64 + e3) exactly. The
+// magic numbers are subtracted exactly and one fused multiply-add applies
+// the scale and bias, rounding once: 4 integer and 8 fp16 operations per
+// word. The other operand must use the same order: within every 8
+// consecutive K elements, position p holds element (0, 4, 1, 5, 2, 6, 3, 7)[p].
 __device__ __forceinline__ void dequant_word_perm(uint32_t w, uint32_t s2, uint32_t b2,
                                                   uint32_t* out) {
-  const uint32_t w8 = w >> 8;
-  const uint32_t c1024 = 0x64006400u, c64 = 0x54005400u;
+  const uint32_t c1024 = 0x64006400u, c64 = 0x54005400u, m16 = 0xCC00CC00u;   // -16.0
+  const uint32_t hi = __byte_perm(w, 0x64646464u, 0x4341);                   // 1024 + 16 e3 + e2
+  const uint32_t d = (hi & 0x00F000F0u) | c64;                               // 64 + e3
   out[0] = f16x2_fma(f16x2_sub((w & 0x000F000Fu) | c1024, c1024), s2, b2);    // e0, e4
   out[1] = f16x2_fma(f16x2_sub((w & 0x00F000F0u) | c64, c64), s2, b2);        // e1, e5
-  out[2] = f16x2_fma(f16x2_sub((w8 & 0x000F000Fu) | c1024, c1024), s2, b2);   // e2, e6
-  out[3] = f16x2_fma(f16x2_sub((w8 & 0x00F000F0u) | c64, c64), s2, b2);       // e3, e7
+  out[2] = f16x2_fma(f16x2_fma(d, m16, hi), s2, b2);                          // e2, e6
+  out[3] = f16x2_fma(f16x2_sub(d, c64), s2, b2);                              // e3, e7
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
