@@ -283,7 +283,10 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
 /* Where moe_forward keeps each intermediate inside its workspace (byte
  * offsets), the regime it resolves to for experts of weight format wfmt and
  * the BM it sorts with. moe_forward_workspace(...) is its `total`; 0 when the
- * arguments are invalid. */
+ * arguments are invalid. With q4 experts the whole-layer call may keep h and
+ * the fp16 token rows x16 with every 8 consecutive elements in the order
+ * (0, 4, 1, 5, 2, 6, 3, 7), the K order its kernels dequantise in; the
+ * routing and sort tables have the layouts moe_route and moe_sort_rows give. */
 typedef struct {
   size_t logits, topk_idx, topk_w, order, inv_order, row_map, counts, row_off, tile_off;
   size_t sort_ws, h, ys, x16, total;

@@ -462,10 +462,11 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
       cudaSuccess)
     return launched(e);
   if (regime_run == MOE_REGIME_TC) {
-    if ((e = launch_swiglu_tc(x, dt, T, rmap, roff, toff, (int)R, *experts, h, x16, stp, s)) !=
-        cudaSuccess)
+    // h stays in the q4 dequant's permuted K order between the two kernels
+    if ((e = launch_swiglu_tc(x, dt, T, rmap, roff, toff, (int)R, *experts, h, x16, stp, s,
+                              true)) != cudaSuccess)
       return launched(e);
-    if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s)) != cudaSuccess)
+    if ((e = launch_down_tc(h, roff, toff, (int)R, *experts, ys, stp, s, true)) != cudaSuccess)
       return launched(e);
   } else {
     if ((e = swiglu_gemv(x, dt, T, rmap, roff, toff, L.BM, (int)R, *experts, h,

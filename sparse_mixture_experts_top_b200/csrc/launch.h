@@ -77,11 +77,14 @@ int tc_block_m();
 bool tc_shape_supported(int d, int F, int fmt, int dt);
 // xs16: R*d fp16 scratch that receives the token rows of the R sorted rows,
 // gathered through row_map (converted when x is bf16)
+// h_perm (q4 experts): h kept in the permuted K order of the q4 dequant
+// between the two calls (the whole-layer call); otherwise feature order
 cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_map, const int32_t* row_off,
                              const int32_t* tile_off, int R, const moe_experts& ex, void* h,
-                             void* xs16, int* status, cudaStream_t s);
+                             void* xs16, int* status, cudaStream_t s, bool h_perm = false);
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
-                           const moe_experts& ex, void* ys, int* status, cudaStream_t s);
+                           const moe_experts& ex, void* ys, int* status, cudaStream_t s,
+                           bool h_perm = false);
 
 // The decode layer fused into one cooperative launch (q4 experts, bf16 or
 // fp16 activations, T <= 32, T*k <= 256, E <= 256, d and F multiples of 128 and at

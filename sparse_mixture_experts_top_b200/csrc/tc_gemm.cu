@@ -74,7 +74,22 @@ constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at the B200's clocks
 // activation fixed at compile time (a runtime choice in the unrolled
 // epilogue cost the SwiGLU kernel a fifth of its speed); EPI_STORE: the
 // router stores fp32 logits (+ p.bias when set), the down projection fp16 ys
-enum { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_GEGLU = 2 };
+// The _HP forms keep h in the permuted K order of dequant_word_perm (within
+// every 8 consecutive features, position p holds feature (0, 4, 1, 5, 2, 6,
+// 3, 7)[p]): the gate|up kernel writes it so, and the down kernel then
+// dequantises its q4 weights in that order too -- 4 integer operations per
+// word instead of 9. The whole-layer call uses them; the stage calls keep h
+// in feature order.
+enum { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_GEGLU = 2, EPI_SWIGLU_HP = 3, EPI_GEGLU_HP = 4,
+       EPI_STORE_HP = 5 };
+template <int EPI> struct Epi {
+  static constexpr bool glu = EPI != EPI_STORE && EPI != EPI_STORE_HP;
+  static constexpr bool geglu = EPI == EPI_GEGLU || EPI == EPI_GEGLU_HP;
+  static constexpr bool perm_out = EPI == EPI_SWIGLU_HP || EPI == EPI_GEGLU_HP;
+  // weights dequantised in the permuted K order (the B rows are x16, or h
+  // kept permuted)
+  static constexpr bool perm_deq = glu || EPI == EPI_STORE_HP;
+};
 
 template <int FMT>
 struct Cfg {
@@ -694,9 +709,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
       const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
       // 16 columns of both accumulators at a time
-      if (EPI != EPI_STORE) {
-        constexpr int kAct = EPI == EPI_GEGLU ? MOE_ACT_GEGLU_TANH : MOE_ACT_SWIGLU;
-        const int orow = unit * p.unit_rows + m;          // feature of this thread
+      if (Epi<EPI>::glu) {
+        constexpr int kAct = Epi<EPI>::geglu ? MOE_ACT_GEGLU_TANH : MOE_ACT_SWIGLU;
+        int orow = unit * p.unit_rows + m;                // feature of this thread
+        // feature 8g + i at position 8g + 2 (i % 4) + i / 4 (unit_rows % 8 == 0)
+        if (Epi<EPI>::perm_out) orow = (orow & ~7) | ((orow & 3) << 1) | ((orow >> 2) & 1);
         __half* hp = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + orow;
         for (int n0 = 0; n0 < nv; n0 += 16) {
           uint32_t a0[16], a1[16];
@@ -837,8 +854,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              // gate|up reads token rows the gather wrote in permuted order
-              if (EPI != EPI_STORE) dequant_word_perm(ws[i], s2, b2, vals + 4 * i);
+              // gate|up reads token rows the gather wrote in permuted order,
+              // the _HP down a permuted h
+              if (Epi<EPI>::perm_deq) dequant_word_perm(ws[i], s2, b2, vals + 4 * i);
               else dequant_word(ws[i], s2, b2, vals + 4 * i);
             }
           } else {
@@ -1097,7 +1115,7 @@ cudaError_t launch_to_f16(const void* x, long long n, void* x16, int* status, cu
 cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_map,
                              const int32_t* row_off, const int32_t* tile_off, int R,
                              const moe_experts& ex, void* h, void* xs16, int* status,
-                             cudaStream_t s) {
+                             cudaStream_t s, bool h_perm) {
   using namespace tc;
   if (!tc_shape_ok(ex, dt)) return cudaErrorNotSupported;
   (void)T;
@@ -1141,6 +1159,9 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
   const bool geglu = ex.act == MOE_ACT_GEGLU_TANH;
+  if (ex.fmt == MOE_W_Q4G64 && h_perm)
+    return geglu ? run<MOE_W_Q4G64, EPI_GEGLU_HP, false>(p, ta, ub, s)
+                 : run<MOE_W_Q4G64, EPI_SWIGLU_HP, false>(p, ta, ub, s);
   if (ex.fmt == MOE_W_Q4G64)
     return geglu ? run<MOE_W_Q4G64, EPI_GEGLU, false>(p, ta, ub, s)
                  : run<MOE_W_Q4G64, EPI_SWIGLU, false>(p, ta, ub, s);
@@ -1149,7 +1170,8 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
 }
 
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
-                           const moe_experts& ex, void* ys, int* status, cudaStream_t s) {
+                           const moe_experts& ex, void* ys, int* status, cudaStream_t s,
+                           bool h_perm) {
   using namespace tc;
   // h is fp16 whatever the activations' type
   if (!tc_shape_ok(ex, ex.fmt == MOE_W_Q4G64 ? MOE_F16 : MOE_BF16)) return cudaErrorNotSupported;
@@ -1179,6 +1201,7 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.status = status;
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
+  if (ex.fmt == MOE_W_Q4G64 && h_perm) return run<MOE_W_Q4G64, EPI_STORE_HP, false>(p, ta, ub, s);
   if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE, false>(p, ta, ub, s);
   return run<MOE_W_BF16, EPI_STORE, false>(p, ta, ub, s);
 }
