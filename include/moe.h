@@ -68,8 +68,9 @@
  *     read once per step, for few tokens per expert (decode);
  *   MOE_REGIME_TC: tensor-core grouped GEMM (tcgen05 / TMEM, TMA-staged
  *     operands) for many tokens per expert (prefill); bf16 activations with
- *     bf16 or q4 (group 64) weights, or fp16 activations with q4 weights, d a multiple of 256, F of 128 (q4: of 256);
- *     other shapes return MOE_ERR_UNSUPPORTED;
+ *     bf16 weights, or bf16 / fp16 activations with any quantised format
+ *     (q4 groups 32/64/128, q8 group 64); d a multiple of 256, F of 128 (q4:
+ *     of 256); other shapes return MOE_ERR_UNSUPPORTED;
  *   MOE_REGIME_AUTO: GEMV when T*k <= 8*E or the shape is not one the
  *     tensor-core kernels tile, else TC (bf16 / fp16) or GEMV (f32).
  */
@@ -129,14 +130,15 @@ typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GEGLU_TANH = 1 } moe_act;
  *     value = scale[group] * q + bias[group].
  *   MOE_W_Q4G32 / MOE_W_Q4G128: the same with groups of 32 or 128 (DS4Server
  *     issue #112, "Kernel contract": group 32/64/128); s_* and b_* are
- *     [E][rows][cols/32] or [E][rows][cols/128]. They run on the
- *     weight-streaming and fused-decode kernels; the tensor-core kernels take
- *     group 64, so a forward that would use them runs weight-streaming.
+ *     [E][rows][cols/32] or [E][rows][cols/128]. Every kernel family takes
+ *     them (weight-streaming, fused decode, tensor cores).
  *   MOE_W_Q8G64 (8-bit affine; mlxcel PR #275, "Multi-bit handling"; DS4Server
  *   issue #112, "Kernel contract": 4 or 8 bits):
  *     w_gu uint32 [E][2F][d/4], w_dn uint32 [E][d][F/4], byte j of a word is
  *     element j; s_*, b_* bf16 [E][rows][cols/64]; value = scale * q + bias.
- *     It runs on the weight-streaming SIMT kernels only.
+ *     It runs on the weight-streaming SIMT kernels and the tensor cores.
+ *   Quantised formats: the scale and bias arrays are 16-byte aligned, like
+ *     every other buffer.
  *   act: moe_act, the gate activation of every expert (0, SwiGLU, when the
  *     struct is zero-initialised); other values: MOE_ERR_INVALID_ARG. */
 typedef struct {

@@ -69,11 +69,17 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
     case MOE_W_Q4G128:
       if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
       if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
+      if (!aligned16(ex->s_gu) || !aligned16(ex->b_gu) || !aligned16(ex->s_dn) ||
+          !aligned16(ex->b_dn))
+        return MOE_ERR_INVALID_ARG;
       if (ex->d % q4_group(ex->fmt) || ex->F % q4_group(ex->fmt)) return MOE_ERR_UNSUPPORTED;
       break;
     case MOE_W_Q8G64:
       if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
       if (!ex->s_gu || !ex->b_gu || !ex->s_dn || !ex->b_dn) return MOE_ERR_INVALID_ARG;
+      if (!aligned16(ex->s_gu) || !aligned16(ex->b_gu) || !aligned16(ex->s_dn) ||
+          !aligned16(ex->b_dn))
+        return MOE_ERR_INVALID_ARG;
       break;
     default:
       return MOE_ERR_INVALID_ARG;

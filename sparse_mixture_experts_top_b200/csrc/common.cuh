@@ -77,12 +77,12 @@ __device__ __forceinline__ float glu(int act, float g, float u) {
 }
 
 // Elements per scale and bias of a 4-bit format (moe_wfmt), 0 for the others
-__host__ __device__ __forceinline__ int q4_group(int fmt) {
+__host__ __device__ constexpr int q4_group(int fmt) {
   return fmt == MOE_W_Q4G64 ? 64 : fmt == MOE_W_Q4G32 ? 32 : fmt == MOE_W_Q4G128 ? 128 : 0;
 }
 
 // Elements per scale and bias of any quantised format (4- or 8-bit), 0 else
-__host__ __device__ __forceinline__ int wq_group(int fmt) {
+__host__ __device__ constexpr int wq_group(int fmt) {
   return fmt == MOE_W_Q8G64 ? 64 : q4_group(fmt);
 }
 

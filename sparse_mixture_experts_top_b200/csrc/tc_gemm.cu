@@ -93,19 +93,29 @@ template <int EPI> struct Epi {
 
 template <int FMT>
 struct Cfg {
-  static constexpr bool Q4 = FMT == MOE_W_Q4G64;
-  static constexpr int KR = Q4 ? 256 : 64;                  // K elements per raw stage
+  static constexpr bool Q4 = q4_group(FMT) != 0;            // 4-bit, groups of 32, 64 or 128
+  static constexpr bool Q8 = FMT == MOE_W_Q8G64;            // 8-bit, groups of 64
+  static constexpr bool QUANT = Q4 || Q8;
+  static constexpr int GS = Q4 ? q4_group(FMT) : 64;        // K elements per scale and bias
+  // K elements per raw stage (its rows are 128 bytes)
+  static constexpr int KR = Q4 ? 256 : Q8 ? 128 : 64;
   static constexpr int RAW_MAT = BMW * 128;                 // one matrix: 128 rows x 128 bytes
   static constexpr int RAW_BYTES = 2 * RAW_MAT;
-  static constexpr int A_PER_RAW = KR / KA;                 // 4 (q4) or 1 (bf16)
+  static constexpr int A_PER_RAW = KR / KA;                 // 4 (q4), 2 (q8) or 1 (bf16)
   static constexpr int NR = 3;                              // raw stages
+  // bytes of one row's scales (or biases) in a raw stage: 16, 8 or 4 (q4 g32,
+  // g64, g128), 4 (q8)
+  static constexpr int SB = QUANT ? (KR / GS) * 2 : 0;
   static constexpr int ACC_COLS = 2 * BN;                   // two accumulators of up to 128 columns
   static constexpr int A_COLS = 2 * (KA / 2);               // TMEM columns of one A stage (2 matrices)
   static constexpr int B_BYTES = BN * 128;
-  // q4 scales then biases of a raw stage: [2 arrays][2 matrices][128 rows][4 groups] bf16
-  static constexpr int SCL_BYTES = Q4 ? 2 * 2 * BMW * 4 * 2 : 0;
+  // scales then biases of a raw stage: [2 arrays][2 matrices][128 rows][SB bytes]
+  static constexpr int SCL_BYTES = QUANT ? 2 * 2 * BMW * SB : 0;
   static constexpr int TABLES = 2 * (kMaxE + 1) * 4;
-  static constexpr int SMEM = 1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES + NR * SCL_BYTES;
+  // (the scale ring starts 128-byte aligned after the tables: its rows of up
+  // to 16 bytes are copied and read as 16-byte vectors)
+  static constexpr int SMEM =
+      1024 + NR * RAW_BYTES + NB * B_BYTES + 1024 + TABLES + 128 + NR * SCL_BYTES;
   static_assert(ACC_COLS + NS * A_COLS <= 512, "accumulators and A stages must fit TMEM");
   static_assert(NS % 2 == 0, "A stages are released in pairs");
   static_assert(NS <= 2 * NP && NB <= 2 * NP, "a ring may not outrun its release barriers");
@@ -406,6 +416,17 @@ __device__ __forceinline__ void dequant_word_perm(uint32_t w, uint32_t s2, uint3
   out[3] = f16x2_fma(f16x2_sub(d, c64), s2, b2);                              // e3, e7
 }
 
+// 4 bytes of one word (element j in byte j) -> 2 fp16 pairs of s * q + b in K
+// order: a byte permute puts each byte under the exponent of fp16 1024.0
+// (0x64qq = 1024 + q, exact for q <= 255), the magic is subtracted exactly and
+// one fused multiply-add applies scale and bias, rounding once.
+__device__ __forceinline__ void dequant_word_q8(uint32_t w, uint32_t s2, uint32_t b2,
+                                                uint32_t* out) {
+  const uint32_t c1024 = 0x64006400u;
+  out[0] = f16x2_fma(f16x2_sub(__byte_perm(w, 0x64646464u, 0x4140), c1024), s2, b2);  // q0, q1
+  out[1] = f16x2_fma(f16x2_sub(__byte_perm(w, 0x64646464u, 0x4342), c1024), s2, b2);  // q2, q3
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -474,22 +495,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sink = smem_u32(bar_area + 512);
   int* s_toff = reinterpret_cast<int*>(bar_area + 1024);
   int* s_roff = s_toff + kMaxE + 1;
-  // q4 scale ring: raw stage rs holds scales [2][128][4] then biases [2][128][4]
-  const uint32_t scl_base = smem_u32(s_roff + kMaxE + 1);
+  // scale ring: raw stage rs holds scales [2][128][SB bytes] then biases,
+  // 128-byte aligned
+  const uint32_t scl_base = (smem_u32(s_roff + kMaxE + 1) + 127u) & ~127u;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NR; ++i) {
-      // q4: the TMA arrive + the 32 lanes' cp.async arrivals for the scales
-      mbar_init(smem_u32(raw_full + i), C::Q4 ? 33 : 1);
+      // quantised: the TMA arrive + the 32 lanes' cp.async arrivals for the scales
+      mbar_init(smem_u32(raw_full + i), C::QUANT ? 33 : 1);
       mbar_init(smem_u32(raw_empty + i), 16);   // the 16 dequant warps
     }
-    // one barrier per A stage pair of a matrix: q4, each stage of the pair is
-    // written by the 4 warps of one half (8 arrivals); bf16, each stage by
-    // the 8 warps of both halves (16 arrivals)
-    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::Q4 ? 8 : 16);
+    // one barrier per A stage pair of a matrix: quantised, each stage of the
+    // pair is written by the 4 warps of one half (8 arrivals); bf16, each
+    // stage by the 8 warps of both halves (16 arrivals)
+    for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::QUANT ? 8 : 16);
     for (int i = 0; i < NB / 2; ++i) mbar_init(smem_u32(b_full + i), 1);
     for (int i = 0; i < NP; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
     for (int i = 0; i < 2; ++i) {
@@ -541,11 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait_warp(smem_u32(raw_empty + rs), ((raw_it / C::NR) & 1) ^ 1, abort_flag,
                             p.status, true, p.wait_limit);
         if (!ok) break;
-        if (C::Q4) {
-          // the stage's scales and biases (4 groups of each weight row), 8
-          // bytes per row and array, copied by the 32 lanes; each lane's
-          // arrival fires when its copies have landed. Rows past the end of
-          // the stacked tensor (never stored) read the last row instead.
+        if (C::QUANT) {
+          // the stage's scales and biases (KR / GS groups of each weight
+          // row), SB bytes per row and array, copied by the 32 lanes; each
+          // lane's arrival fires when its copies have landed. Rows past the
+          // end of the stacked tensor (never stored) read the last row instead.
           const uint32_t sdst = scl_base + rs * C::SCL_BYTES;
 #pragma unroll
           for (int mat = 0; mat < 2; ++mat)
@@ -554,13 +576,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int m = lane + 32 * j;
               long long grow = (mat ? wrow1 : wrow0) + (long long)m * p.row_step;
               if (grow >= p.w_rows) grow = p.w_rows - 1;
-              const uint32_t o = (uint32_t)((mat * BMW + m) * 8);
-              asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sdst + o),
-                           "l"(p.scales + grow * p.G + 4 * kr)
+              const uint32_t o = (uint32_t)((mat * BMW + m) * C::SB);
+              const long long g0 = grow * p.G + (long long)(C::KR / C::GS) * kr;
+              asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(sdst + o),
+                           "l"(p.scales + g0), "n"(C::SB)
                            : "memory");
-              asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+              asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(
                                sdst + C::SCL_BYTES / 2 + o),
-                           "l"(p.biases + grow * p.G + 4 * kr)
+                           "l"(p.biases + g0), "n"(C::SB)
                            : "memory");
             }
           asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
@@ -571,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rows past the end of the tensor are filled with zeros by the TMA
           const uint32_t dst = raw_base + rs * C::RAW_BYTES;
           const uint32_t bar = smem_u32(raw_full + rs);
-          const int x = kr * (C::Q4 ? C::KR / 8 : C::KR);
+          const int x = kr * (C::Q4 ? C::KR / 8 : C::Q8 ? C::KR / 4 : C::KR);
           mbar_arrive_tx(bar, C::RAW_BYTES);
           tma_load_2d(dst, &tmA, x, (int)wrow0, bar);
           tma_load_2d(dst + C::RAW_MAT, &tmA, x, (int)wrow1, bar);
@@ -791,8 +814,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // k-blocks hf and 2 + hf of every raw stage (chunks 2hf, 2hf + 1 and
     // 4 + 2hf, 5 + 2hf of the row), so both halves fill a k-block pair
     // together and the MMAs of one pair overlap the conversion of the next;
-    // bf16: half hf converts K elements 32hf .. 32hf + 31 of the raw stage's
-    // single A stage.
+    // q8: half hf converts k-block hf (chunks 4hf .. 4hf + 3); bf16: half hf
+    // converts K elements 32hf .. 32hf + 31 of the raw stage's single A stage.
     const int dw = warp - kDqWarp0;                   // 0..15
     const int q = (dw >> 2) & 1;                      // matrix
     const int hf = dw >> 3;                           // half of the raw stage
@@ -817,25 +840,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int chunk = C::Q4 ? 2 * hf + c + (c & 2) : 4 * hf + c;
           wv[c] = lds128(rowa + (((uint32_t)chunk ^ (uint32_t)sw) << 4));
         }
-        uint32_t sc = 0, bi = 0;
-        if (C::Q4) {
-          // this row's scales and biases of groups hf and 2 + hf (its two
-          // k-blocks), each a bf16 in the low half
-          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * 8);
-          uint32_t s01, s23, b01, b23;
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s01), "=r"(s23) : "r"(so));
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                       : "=r"(b01), "=r"(b23)
-                       : "r"(so + C::SCL_BYTES / 2));
-          sc = hf ? ((s01 >> 16) | (s23 & 0xFFFF0000u)) : ((s01 & 0xFFFFu) | (s23 << 16));
-          bi = hf ? ((b01 >> 16) | (b23 & 0xFFFF0000u)) : ((b01 & 0xFFFFu) | (b23 << 16));
+        // this row's scales and biases for the warp's A stage j, as bf16 in
+        // the low half (and, groups of 32, the second group of the k-block
+        // in the high half)
+        uint32_t sg[2] = {0u, 0u}, bg[2] = {0u, 0u};
+        if (C::QUANT) {
+          const uint32_t so = scl_base + rs * C::SCL_BYTES + (uint32_t)((q * BMW + m) * C::SB);
+          const uint32_t bo = so + C::SCL_BYTES / 2;
+          if (C::SB == 16) {             // q4 g32: k-block kb has groups 2kb, 2kb + 1
+            uint32_t sv[4], bv[4];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(sv[0]), "=r"(sv[1]), "=r"(sv[2]), "=r"(sv[3]) : "r"(so));
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(bv[0]), "=r"(bv[1]), "=r"(bv[2]), "=r"(bv[3]) : "r"(bo));
+            sg[0] = hf ? sv[1] : sv[0];
+            sg[1] = hf ? sv[3] : sv[2];
+            bg[0] = hf ? bv[1] : bv[0];
+            bg[1] = hf ? bv[3] : bv[2];
+          } else if (C::SB == 8) {       // q4 g64: group kb
+            uint32_t s01, s23, b01, b23;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s01), "=r"(s23) : "r"(so));
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b01), "=r"(b23) : "r"(bo));
+            sg[0] = hf ? (s01 >> 16) : (s01 & 0xFFFFu);
+            sg[1] = hf ? (s23 >> 16) : (s23 & 0xFFFFu);
+            bg[0] = hf ? (b01 >> 16) : (b01 & 0xFFFFu);
+            bg[1] = hf ? (b23 >> 16) : (b23 & 0xFFFFu);
+          } else {                       // 2 groups: q4 g128 (kb / 2), q8 (kb)
+            uint32_t s01, b01;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(s01) : "r"(so));
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b01) : "r"(bo));
+            if (C::Q4) {
+              sg[0] = s01 & 0xFFFFu, sg[1] = s01 >> 16;
+              bg[0] = b01 & 0xFFFFu, bg[1] = b01 >> 16;
+            } else {
+              sg[0] = hf ? (s01 >> 16) : (s01 & 0xFFFFu);
+              bg[0] = hf ? (b01 >> 16) : (b01 & 0xFFFFu);
+            }
+          }
         }
         // A shared-memory load has read its data only once an instruction has
         // consumed its destination registers; until then the next TMA into
         // this stage can overwrite rows the load has not read yet (seen on
         // the first rows the TMA writes). So the loaded words are folded into
         // one value stored to a scratch word before the stage is released.
-        uint32_t fold = sc ^ bi;
+        uint32_t fold = sg[0] ^ sg[1] ^ bg[0] ^ bg[1];
 #pragma unroll
         for (int c = 0; c < 4; ++c) fold ^= wv[c].x ^ wv[c].y ^ wv[c].z ^ wv[c].w;
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sink + 4u * (uint32_t)warp), "r"(fold)
@@ -847,17 +895,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t vals[32];
           if (C::Q4) {
             // my chunks 2j, 2j + 1 hold the 64 elements of k-block hf + 2j of
-            // the raw stage, group 4kr + hf + 2j
-            const uint32_t s2 = f16x2_from_bf16(j ? (sc >> 16) : (sc & 0xFFFFu));
-            const uint32_t b2 = f16x2_from_bf16(j ? (bi >> 16) : (bi & 0xFFFFu));
+            // the raw stage; groups of 32: words 0-3 and 4-7 have a group each
+            const uint32_t s2 = f16x2_from_bf16(sg[j] & 0xFFFFu);
+            const uint32_t b2 = f16x2_from_bf16(bg[j] & 0xFFFFu);
+            const uint32_t s2h = C::GS == 32 ? f16x2_from_bf16(sg[j] >> 16) : s2;
+            const uint32_t b2h = C::GS == 32 ? f16x2_from_bf16(bg[j] >> 16) : b2;
             const uint4 w0 = wv[2 * j], w1 = wv[2 * j + 1];
             const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               // gate|up reads token rows the gather wrote in permuted order,
               // the _HP down a permuted h
-              if (Epi<EPI>::perm_deq) dequant_word_perm(ws[i], s2, b2, vals + 4 * i);
-              else dequant_word(ws[i], s2, b2, vals + 4 * i);
+              const uint32_t si = i < 4 ? s2 : s2h, bi = i < 4 ? b2 : b2h;
+              if (Epi<EPI>::perm_deq) dequant_word_perm(ws[i], si, bi, vals + 4 * i);
+              else dequant_word(ws[i], si, bi, vals + 4 * i);
+            }
+          } else if (C::Q8) {
+            // the 64 bytes of k-block hf, in K order
+            const uint32_t s2 = f16x2_from_bf16(sg[0]), b2 = f16x2_from_bf16(bg[0]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t w4[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dequant_word_q8(w4[i], s2, b2, vals + 8 * c + 2 * i);
             }
           } else {
             // bf16 weights: 32 elements of the k-block; fp16 operands for
@@ -869,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 4; ++i) vals[4 * c + i] = ROUTER ? w4[i] : bf16x2_to_f16x2(w4[i]);
             }
           }
-          const uint32_t stage = a_it + (C::Q4 ? hf + 2 * j : 0);
+          const uint32_t stage = a_it + (C::Q4 ? hf + 2 * j : C::Q8 ? hf : 0);
           const uint32_t as = stage % NS;
           if (stage >= (uint32_t)NS) {      // the slot's previous k-block is released
             const uint32_t pr = (stage - NS) >> 1;
@@ -877,8 +937,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
           }
           tc_fence_after();
-          const uint32_t col = C::ACC_COLS + as * C::A_COLS + q * (KA / 2) + (C::Q4 ? 0 : hf * 16);
-          if (C::Q4) tmem_st32_sync(tl + col, vals);
+          const uint32_t col = C::ACC_COLS + as * C::A_COLS + q * (KA / 2) + (C::QUANT ? 0 : hf * 16);
+          if (C::QUANT) tmem_st32_sync(tl + col, vals);
           else tmem_st16_sync(tl + col, vals);
           tc_fence_before();
           __syncwarp();
@@ -961,9 +1021,12 @@ static int num_sms() {
 // (row_step 2: each load takes every other row, 128 of 256)
 static bool weight_map(CUtensorMap* m, int fmt, const void* w, long long rows, int K,
                        bool f16 = false, uint32_t row_step = 1) {
-  if (fmt == MOE_W_Q4G64)
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / 8, rows, (uint64_t)K / 2, 32,
-                    BMW * row_step, CU_TENSOR_MAP_SWIZZLE_128B, row_step);
+  if (q4_group(fmt) || fmt == MOE_W_Q8G64) {
+    // uint32 words: 8 (q4) or 4 (q8) elements each; rows of 128 bytes per box
+    const int per = fmt == MOE_W_Q8G64 ? 4 : 8;
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, w, K / per, rows, (uint64_t)K * 4 / per,
+                    32, BMW * row_step, CU_TENSOR_MAP_SWIZZLE_128B, row_step);
+  }
   return make_map(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w,
                   K, rows, (uint64_t)K * 2, 64, BMW * row_step, CU_TENSOR_MAP_SWIZZLE_128B,
                   row_step);
@@ -1077,13 +1140,35 @@ static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub
   return cudaGetLastError();
 }
 
+// The kernel for the experts' weight format. The _HP forms are built for
+// the q4 formats only (they permute h for the q4 dequant).
+template <int EPI, bool ROUTER>
+static cudaError_t run_fmt(int fmt, const Params& p, const CUtensorMap& a, long long ub,
+                           cudaStream_t s) {
+  constexpr bool hp = EPI == EPI_SWIGLU_HP || EPI == EPI_GEGLU_HP || EPI == EPI_STORE_HP;
+  switch (fmt) {
+    case MOE_W_Q4G64: return run<MOE_W_Q4G64, EPI, ROUTER>(p, a, ub, s);
+    case MOE_W_Q4G32: return run<MOE_W_Q4G32, EPI, ROUTER>(p, a, ub, s);
+    case MOE_W_Q4G128: return run<MOE_W_Q4G128, EPI, ROUTER>(p, a, ub, s);
+    default: break;
+  }
+  if constexpr (!hp) {
+    if (fmt == MOE_W_Q8G64) return run<MOE_W_Q8G64, EPI, ROUTER>(p, a, ub, s);
+    if (fmt == MOE_W_BF16) return run<MOE_W_BF16, EPI, ROUTER>(p, a, ub, s);
+  }
+  return cudaErrorNotSupported;
+}
+
 // Shapes the kernels tile: gate|up units are 128 features (F % 128), down
 // units 256 output rows (d % 256); K (d or F) a multiple of 128 for the
-// k-block pairs, and of 256 for q4 raw stages.
+// k-block pairs (q8 raw stages), and of 256 for q4 raw stages. Quantised
+// weights need their scale and bias arrays 16-byte aligned (the scales of a
+// raw stage are copied in pieces of up to 16 bytes).
 static bool tc_shape_ok(const moe_experts& ex, int dt) {
   if (ex.d % 256 || ex.F % 128) return false;
   if (dt != MOE_BF16 && dt != MOE_F16) return false;
-  if (ex.fmt == MOE_W_Q4G64) return ex.F % 256 == 0;
+  if (q4_group(ex.fmt)) return ex.F % 256 == 0;
+  if (ex.fmt == MOE_W_Q8G64) return true;
   return ex.fmt == MOE_W_BF16 && dt == MOE_BF16;
 }
 
@@ -1124,12 +1209,16 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   // through row_map (and converted once, from bf16) into xs16 [R][d]
   // q4 weights are dequantised in a permuted K order, so are the token rows
   const unsigned gblocks = (unsigned)((R + 3) / 4);
-  if (ex.fmt == MOE_W_Q4G64 && dt == MOE_F16)
+  const bool q4 = q4_group(ex.fmt) != 0;
+  if (q4 && dt == MOE_F16)
     launch_pdl(gather_f16_kernel<true, true>, gblocks, 256, 0, s, (const uint4*)x, row_map,
                (long long)R, ex.d / 8, (uint4*)xs16, status);
-  else if (ex.fmt == MOE_W_Q4G64)
+  else if (q4)
     launch_pdl(gather_f16_kernel<true>, gblocks, 256, 0, s, (const uint4*)x, row_map, (long long)R,
                ex.d / 8, (uint4*)xs16, status);
+  else if (dt == MOE_F16)
+    launch_pdl(gather_f16_kernel<false, true>, gblocks, 256, 0, s, (const uint4*)x, row_map,
+               (long long)R, ex.d / 8, (uint4*)xs16, status);
   else
     launch_pdl(gather_f16_kernel<false>, gblocks, 256, 0, s, (const uint4*)x, row_map, (long long)R,
                ex.d / 8, (uint4*)xs16, status);
@@ -1148,7 +1237,7 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.row_step = 1;
   p.K = ex.d;
   p.rows_per_group = 2 * ex.F;
-  p.G = ex.d / 64;
+  p.G = wq_group(ex.fmt) ? ex.d / wq_group(ex.fmt) : 0;
   p.w_rows = (long long)ex.E * 2 * ex.F;
   p.scales = (const uint16_t*)ex.s_gu;
   p.biases = (const uint16_t*)ex.b_gu;
@@ -1159,14 +1248,13 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
   const bool geglu = ex.act == MOE_ACT_GEGLU_TANH;
-  if (ex.fmt == MOE_W_Q4G64 && h_perm)
-    return geglu ? run<MOE_W_Q4G64, EPI_GEGLU_HP, false>(p, ta, ub, s)
-                 : run<MOE_W_Q4G64, EPI_SWIGLU_HP, false>(p, ta, ub, s);
-  if (ex.fmt == MOE_W_Q4G64)
-    return geglu ? run<MOE_W_Q4G64, EPI_GEGLU, false>(p, ta, ub, s)
-                 : run<MOE_W_Q4G64, EPI_SWIGLU, false>(p, ta, ub, s);
-  return geglu ? run<MOE_W_BF16, EPI_GEGLU, false>(p, ta, ub, s)
-               : run<MOE_W_BF16, EPI_SWIGLU, false>(p, ta, ub, s);
+  // h in the permuted K order only for q4 weights (the down kernel then
+  // dequantises in that order)
+  if (q4 && h_perm)
+    return geglu ? run_fmt<EPI_GEGLU_HP, false>(ex.fmt, p, ta, ub, s)
+                 : run_fmt<EPI_SWIGLU_HP, false>(ex.fmt, p, ta, ub, s);
+  return geglu ? run_fmt<EPI_GEGLU, false>(ex.fmt, p, ta, ub, s)
+               : run_fmt<EPI_SWIGLU, false>(ex.fmt, p, ta, ub, s);
 }
 
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
@@ -1191,7 +1279,7 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.row_step = 2;
   p.K = ex.F;
   p.rows_per_group = ex.d;
-  p.G = ex.F / 64;
+  p.G = wq_group(ex.fmt) ? ex.F / wq_group(ex.fmt) : 0;
   p.w_rows = (long long)ex.E * ex.d;
   p.scales = (const uint16_t*)ex.s_dn;
   p.biases = (const uint16_t*)ex.b_dn;
@@ -1201,9 +1289,8 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.status = status;
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
-  if (ex.fmt == MOE_W_Q4G64 && h_perm) return run<MOE_W_Q4G64, EPI_STORE_HP, false>(p, ta, ub, s);
-  if (ex.fmt == MOE_W_Q4G64) return run<MOE_W_Q4G64, EPI_STORE, false>(p, ta, ub, s);
-  return run<MOE_W_BF16, EPI_STORE, false>(p, ta, ub, s);
+  if (q4_group(ex.fmt) && h_perm) return run_fmt<EPI_STORE_HP, false>(ex.fmt, p, ta, ub, s);
+  return run_fmt<EPI_STORE, false>(ex.fmt, p, ta, ub, s);
 }
 
 cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router, const float* bias,

@@ -381,9 +381,10 @@ def test_grouped_stages_q4_group_sizes(moe, orc, wfmt):
 
 @pytest.mark.parametrize("wfmt,T", [("q4g128", 300), ("q4g32", 1024)])
 def test_forward_q4_group_sizes_prefill_shape(moe, orc, wfmt, T):
-    """Prefill shapes: 300 tokens run the weight-streaming tensor-core GEMV;
-    1,024 tokens would take the tcgen05 kernels, which take group 64 only,
-    so the forward runs the weight-streaming kernels with 128-row tiles."""
+    """Prefill shapes: 300 tokens (7.5 rows per expert) run the
+    weight-streaming kernels; 1,024 tokens resolve to the tcgen05 kernels."""
+    L = moe.forward_layout(T, 2048, 512, 10, 512, torch.bfloat16, wfmt)
+    assert L.regime == (moe.REGIME_TC if T == 1024 else moe.REGIME_GEMV)
     layer = mi.make_layer(mi.workload("prefill", T=T, wfmt=wfmt), seed=8, device=DEV)
     rng = np.random.default_rng(3)
     _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(T, 32, replace=False)))
@@ -522,4 +523,64 @@ def test_forward_intermediates_match_stage_calls(moe):
     st = moe.sort_rows(idx, wl.E, L.BM)
     assert torch.equal(seg(L.order, R, torch.int32), st.order.view(torch.int32))
     assert torch.equal(seg(L.tile_off, wl.E + 1, torch.int32), st.tile_off)
+    assert moe.device_status() == moe.OK
+
+
+# ------------------------------------------------------------------ other formats on the tensor cores
+
+TC_FORMAT_CASES = [
+    # workload, T, weight format, activations, skew
+    ("prefill", 600, "q4g32", "bf16", 0.3),
+    ("prefill", 600, "q4g128", "bf16", 0.0),
+    ("prefill", 600, "q8", "bf16", 0.3),
+    ("prefill", 600, "q8", "f16", 0.0),
+    ("skewed", 24, "q4g32", "bf16", 0.3),      # d = 7168: 28 raw stages per unit
+]
+
+
+@pytest.mark.parametrize("name,T,wfmt,act,skew", TC_FORMAT_CASES)
+def test_tc_stages_other_formats(moe, orc, name, T, wfmt, act, skew):
+    """q4 with groups of 32 and 128, and 8-bit affine weights, through the
+    tcgen05 gate|up and down kernels (DS4Server issue #112, "Kernel
+    contract": 4 or 8 bits, groups 32/64/128; mlxcel PR #275, "Multi-bit
+    handling"). Weights are dequantised to fp16 operands (u_w = 2^-11)."""
+    wl = mi.workload(name, T=T, wfmt=wfmt, act=act)
+    layer, idx = _stage_setup(wl, T, 51, skew)
+    st = moe.sort_rows(idx.to(DEV), wl.E, moe.sort_block_m())
+    h = moe.grouped_swiglu(layer.x, st, wl.k, layer.experts, regime=moe.REGIME_TC)
+    ref_st = orc.sort_rows(idx.numpy(), wl.E, moe.sort_block_m())
+    hx = _host(layer.experts)
+    href = orc.expert_swiglu(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    g, u, ga, ua = orc.expert_gate_up(layer.x.cpu(), ref_st.row_map, ref_st.row_off, hx)
+    assert_h_close(h, href, g, u, ga, ua, wl.d, U_F16, U_F16, TOL_BF16, f"h[{name} {wfmt} {act}]")
+    ys = moe.grouped_down(h, st, T, wl.k, layer.experts, regime=moe.REGIME_TC, dtype=layer.x.dtype)
+    yref = orc.expert_down(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    habs = orc.expert_down_abs(to_np(h).astype(np.float64), ref_st.row_off, hx)
+    assert_ys_close(ys, yref, habs, U_F16, TOL_BF16, f"ys[{name} {wfmt} {act}]", u_ys=U_F16,
+                    F=wl.F)
+    assert moe.device_status() == moe.OK
+
+
+@pytest.mark.parametrize("wfmt,act", [("q4g32", "bf16"), ("q4g128", "f16"), ("q8", "bf16")])
+def test_forward_other_formats_tensor_cores(moe, orc, wfmt, act):
+    """The whole layer at the prefill shape resolves to the tcgen05 kernels
+    for these formats and matches the oracle on sampled tokens."""
+    wl = mi.workload("prefill", wfmt=wfmt, act=act)
+    L = moe.forward_layout(wl.T, wl.d, wl.E, wl.k, wl.F, mi._act_dtype(act), wfmt)
+    assert L.regime == moe.REGIME_TC
+    layer = mi.make_layer(wl, seed=17, device=DEV)
+    rng = np.random.default_rng(7)
+    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(wl.T, 48, replace=False)))
+    assert moe.device_status() == moe.OK
+
+
+@pytest.mark.parametrize("wfmt", ["q4g32", "q8"])
+def test_forward_other_formats_repeat_bit_exact(moe, wfmt):
+    layer = mi.make_layer(mi.workload("prefill", T=1024, wfmt=wfmt), seed=3, device=DEV)
+    wl = layer.wl
+    ws = moe.forward_workspace(layer.x, layer.experts, wl.k)
+    ref = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, wl.k, ws=ws).clone()
+    for _ in range(8):
+        y = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, wl.k, ws=ws)
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
     assert moe.device_status() == moe.OK
