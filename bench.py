@@ -40,8 +40,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one gate|up launch on the prefill workload,
 # from an ncu capture of that kernel (the stage call's grouped_tc_kernel<2, 0,
 # 0> as of the commit that adds q4 g32/g128 and q8 to the tcgen05 kernels:
-# 675.21 MB read + 21.13 MB written; profiles/grouped_gate_up_q4_prefill_ncu.md);
-# to be retaken whenever that kernel changes
+# 675.21 MB read + 21.13 MB written); to be retaken whenever that kernel
+# changes
 GATE_UP_TRAFFIC = {"prefill": 696339456}
 L2_FLUSH_BYTES = 256 << 20
 
