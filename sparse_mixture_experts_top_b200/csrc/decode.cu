@@ -60,7 +60,6 @@ constexpr int kSlots = 10;                    // weight ring slots
 // gate|up item at d = 2048: 16 KB of words + up to 4 KB of scales and biases
 // (group 32)
 constexpr int kSlotBytes = 20 * 1024;
-constexpr int kTg = 8;                        // tokens per router work unit (one W_r row read)
 constexpr long long kWaitCycles = 2000000000LL;
 
 // shared memory after the ring: the groups' partial accumulators (double

@@ -26,6 +26,7 @@
 namespace moe {
 
 constexpr int kChunk = 1024;   // slots per block (32 warps x 32 lanes)
+constexpr size_t kScanSmemMax = 160 * 1024;   // dynamic shared memory of the scan block
 
 static inline int num_chunks(long long R) { return (int)((R + kChunk - 1) / kChunk); }
 
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(1024) sort_count_kernel(const int32_t* __restr
 }
 
 __global__ void __launch_bounds__(1024) sort_scan_kernel(const int32_t* __restrict__ chunk_cnt,
-                                                         int nchunks, int E, int BM,
+                                                         int nchunks, int E, int BM, bool stage_fits,
                                                          int32_t* __restrict__ chunk_base,
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ row_off,
@@ -171,11 +172,20 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(const int32_t* __restri
   extern __shared__ int sm[];
   int* cnt = sm;
   int* tiles = sm + E;
+  // the chunk counts, staged in shared memory by all threads at once when
+  // they fit (one round of independent loads instead of a chain of
+  // nchunks dependent ones per expert), else read from global memory
+  int* stage = sm + 2 * E;
+  const bool staged = stage_fits;
   __shared__ int warp_tmp[32];
   __shared__ int totals[2];
+  if (staged)
+    for (int i = threadIdx.x; i < nchunks * E; i += blockDim.x) stage[i] = chunk_cnt[i];
+  __syncthreads();
+  const int32_t* cc = staged ? stage : chunk_cnt;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
-    for (int b = 0; b < nchunks; ++b) c += chunk_cnt[(size_t)b * E + e];
+    for (int b = 0; b < nchunks; ++b) c += cc[(size_t)b * E + e];
     cnt[e] = c;
     counts[e] = c;
     tiles[e] = (c + BM - 1) / BM;
@@ -189,7 +199,7 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(const int32_t* __restri
     int base = cnt[e];
     for (int b = 0; b < nchunks; ++b) {
       chunk_base[(size_t)b * E + e] = base;
-      base += chunk_cnt[(size_t)b * E + e];
+      base += cc[(size_t)b * E + e];
     }
   }
   if (threadIdx.x == 0) {
@@ -230,8 +240,13 @@ cudaError_t launch_sort_rows(const int32_t* idx, int T, int k, int E, int BM, ui
   int32_t* chunk_cnt = reinterpret_cast<int32_t*>(ws);
   int32_t* chunk_base = chunk_cnt + (size_t)nch * E;
   launch_pdl(sort_count_kernel, nch, 1024, E * sizeof(int), s, idx, R, E, chunk_cnt);
-  launch_pdl(sort_scan_kernel, 1, 1024, smem2, s, chunk_cnt, nch, E, BM, chunk_base, counts, row_off,
-                                          tile_off);
+  // the scan stages the chunk counts in shared memory when they fit
+  const size_t stage_bytes = (size_t)nch * E * sizeof(int);
+  const bool fits = smem2 + stage_bytes <= kScanSmemMax;
+  const size_t smem_scan = smem2 + (fits ? stage_bytes : 0);
+  cudaFuncSetAttribute(sort_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_scan);
+  launch_pdl(sort_scan_kernel, 1, 1024, smem_scan, s, chunk_cnt, nch, E, BM, fits, chunk_base, counts,
+                                          row_off, tile_off);
   cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)(E * sizeof(int) + wtab));
   launch_pdl(sort_scatter_kernel, nch, 1024, E * sizeof(int) + wtab, s, idx, R, k, E, chunk_base, order,

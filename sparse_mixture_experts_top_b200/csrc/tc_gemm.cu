@@ -9,13 +9,13 @@
 //
 // B200 design (one persistent CTA per SM, 24 warps). A unit of work is one
 // token tile x two 128-row weight matrices: gate and up rows of the same
-// features (gate|up), or two adjacent 128-row blocks (down, router).
+// features (gate|up), or the even and odd rows of a 256-row block (down).
 //   * swap-AB: the MMA's M = 128 weight rows, N = the tile's token rows
 //     (<= 128, rounded up to 16 per tile), so few rows cost few tensor cycles;
 //   * warp 0: TMA of the raw weight tiles (q4 words or bf16, 128-byte rows)
 //     of both matrices, and cp.async of the q4 scales and biases;
 //   * warp 2: one TMA per k-block of the tile's token rows, from a row-sorted
-//     16-bit copy (x gathered through row_map, or h, or x for the router),
+//     fp16 copy (x gathered through row_map, or h),
 //     with one tensor map per tile height (16, 32, ..., 128 rows);
 //   * warps 8..23 (dequant, 8 per matrix): each thread owns one weight row
 //     (one TMEM lane) and half of every raw stage, dequantises w = s*q + b
@@ -28,14 +28,15 @@
 //     accumulator. Two issuers, because at small N one thread cannot issue
 //     MMAs as fast as the tensor core completes them;
 //   * warps 4..7 (epilogue): tcgen05.ld of both accumulators, SwiGLU to fp16
-//     (gate|up) or fp32 stores (down; router logits + bias). Tiles of at most
+//     (gate|up) or fp16 ys (down). Tiles of at most
 //     64 rows alternate between two accumulator buffers, so the epilogue of
 //     one overlaps the MMAs of the next.
 // The expert GEMMs multiply fp16 operands (x converted once from bf16,
 // weights dequantised to fp16, h stored in fp16): 11-bit operands keep the
 // rounding of the dequantised weights and of h 8x below bf16's; values
-// outside the fp16 range are reported as MOE_ERR_RANGE. The router keeps its
-// bf16 operands, which are exact there.
+// outside the fp16 range are reported as MOE_ERR_RANGE. The router logits
+// have their own kernel below (router_tc_kernel): no dequantisation, both
+// operands staged by TMA, kept in bf16, whose products are exact in fp32.
 // Every mbarrier wait is bounded (about a second): on expiry the kernel
 // records MOE_ERR_TIMEOUT in the status word, all roles leave their loops,
 // copies in flight are waited for (bounded), TMEM is freed, and it returns.
@@ -73,7 +74,7 @@ constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at the B200's clocks
 // EPI_SWIGLU / EPI_GEGLU: gate|up, h = act(gate) * up in fp16, the gate
 // activation fixed at compile time (a runtime choice in the unrolled
 // epilogue cost the SwiGLU kernel a fifth of its speed); EPI_STORE: the
-// router stores fp32 logits (+ p.bias when set), the down projection fp16 ys
+// down projection stores fp16 ys.
 // The _HP forms keep h in the permuted K order of dequant_word_perm (within
 // every 8 consecutive features, position p holds feature (0, 4, 1, 5, 2, 6,
 // 3, 7)[p]): the gate|up kernel writes it so, and the down kernel then
@@ -127,9 +128,7 @@ struct Params {
   CUtensorMap tmB[NBOX];     // token rows [rows][K] 16-bit; map i: box 64 x 16(i+1), 128B swizzle
   const int32_t* row_off;
   const int32_t* tile_off;
-  int E;               // groups (experts); 1 for the router
-  int n_rows;          // router: tokens T
-  int row_tile;        // router: tokens per tile (16, 32, 64 or 128)
+  int E;               // groups (experts)
   int n_units;         // units (pairs of weight matrices) per token tile
   int unit_rows;       // weight rows from one unit to the next
   int mat_off;         // row offset of matrix 1 from matrix 0 inside a unit
@@ -143,9 +142,6 @@ struct Params {
   const uint16_t* biases;
   void* out;
   int out_ld;          // elements per output row
-  int m_limit;         // valid weight rows per group (router: E)
-  int router_f16;      // router: x and the router weight are fp16 (else bf16)
-  const float* bias;   // router bias or null
   int* status;
   long long wait_limit;  // SM cycles a wait for work may take (moe_set_wait_cycles)
 };
@@ -439,30 +435,21 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 
 // Work item u -> (unit within the tile, first sorted row r0, valid rows nv,
 // expert e), with the prefix tables read from their shared-memory copies.
-template <bool ROUTER>
 __device__ __forceinline__ void decode_unit(const Params& p, const int* s_toff, const int* s_roff,
                                             int u, int& unit, int& r0, int& nv, int& e) {
   const int tau = u / p.n_units;
   unit = u - tau * p.n_units;
-  if (ROUTER) {
-    e = 0;
-    r0 = tau * p.row_tile;
-    nv = min(p.row_tile, p.n_rows - r0);
-  } else {
-    int lo = 0, hi = p.E - 1;      // largest e with tile_off[e] <= tau
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_toff[mid] <= tau) lo = mid; else hi = mid - 1;
-    }
-    e = lo;
-    r0 = s_roff[e] + (tau - s_toff[e]) * BN;
-    nv = min(BN, s_roff[e + 1] - r0);
+  int lo = 0, hi = p.E - 1;      // largest e with tile_off[e] <= tau
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_toff[mid] <= tau) lo = mid; else hi = mid - 1;
   }
+  e = lo;
+  r0 = s_roff[e] + (tau - s_toff[e]) * BN;
+  nv = min(BN, s_roff[e + 1] - r0);
 }
 
-template <bool ROUTER>
 __device__ __forceinline__ int total_units(const Params& p, const int* s_toff) {
-  if (ROUTER) return ((p.n_rows + p.row_tile - 1) / p.row_tile) * p.n_units;
   return s_toff[p.E] * p.n_units;
 }
 
@@ -471,7 +458,7 @@ __device__ __forceinline__ int mma_n(int nv) { return max(16, (nv + 15) & ~15); 
 
 // ------------------------------------------------------------------ kernel
 
-template <int FMT, int EPI, bool ROUTER>
+template <int FMT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA) {
   using C = Cfg<FMT>;
@@ -533,18 +520,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // what earlier kernels wrote
   pdl_wait();
   pdl_launch();
-  if (!ROUTER) {
-    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
-      s_toff[i] = __ldg(p.tile_off + i);
-      s_roff[i] = __ldg(p.row_off + i);
-    }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    s_toff[i] = __ldg(p.tile_off + i);
+    s_roff[i] = __ldg(p.row_off + i);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int total = total_units<ROUTER>(p, s_toff);
+  const int total = total_units(p, s_toff);
   const int nkr = p.K / C::KR;           // raw stages per unit
   const int nka = p.K / KA;              // k-blocks per unit (even: K % 128 == 0)
 
@@ -554,9 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int unit, r0, nv, e;
-      decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
-      const long long wrow0 = (ROUTER ? 0LL : (long long)e * p.rows_per_group) +
-                              (long long)unit * p.unit_rows;
+      decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
+      const long long wrow0 = (long long)e * p.rows_per_group + (long long)unit * p.unit_rows;
       const long long wrow1 = wrow0 + p.mat_off;
       for (int kr = 0; kr < nkr && ok; ++kr) {
         const int rs = raw_it % C::NR;
@@ -626,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
         int unit, r0, nv, e;
-        decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+        decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
         const int n = mma_n(nv);
         const CUtensorMap* tm = &p.tmB[n / 16 - 1];
         for (int kb = 0; kb < nka && ok; kb += 2) {
@@ -669,9 +653,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t afull0 = smem_u32(a_full + q * NS);
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int unit, r0, nv, e;
-      decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+      decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
       const int n = mma_n(nv);
-      const uint32_t idesc = idesc_mma(n, !ROUTER || p.router_f16);
+      const uint32_t idesc = idesc_mma(n, true);
       // tiles of <= 64 rows alternate between the two 128-column buffers
       // (matrix q at +64q); larger ones take both (matrix q at +128q)
       const bool small = n <= 64;
@@ -722,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t hmax = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       int unit, r0, nv, e;
-      decode_unit<ROUTER>(p, s_toff, s_roff, u, unit, r0, nv, e);
+      decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
       const bool small = mma_n(nv) <= 64;
       const uint32_t b = small ? nb : 0u;
       const bool use0 = !small || b == 0, use1 = !small || b == 1;
@@ -753,46 +737,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        const int orow0 = unit * p.unit_rows + m;
-        const int orow1 = orow0 + BMW;
-        const bool ok0 = orow0 < p.m_limit, ok1 = orow1 < p.m_limit;
-        if (ROUTER) {
-          const float bv0 = (ok0 && p.bias) ? __ldg(p.bias + orow0) : 0.f;
-          const float bv1 = (ok1 && p.bias) ? __ldg(p.bias + orow1) : 0.f;
-          float* op = reinterpret_cast<float*>(p.out) + (size_t)r0 * p.out_ld + orow0;
-          for (int n0 = 0; n0 < nv; n0 += 16) {
-            uint32_t a0[16], a1[16];
-            tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
+        // the down projection's units are 256 whole rows of d (d % 256 ==
+        // 0): matrix 0 holds the even, matrix 1 the odd output features,
+        // so this thread's two features are adjacent and each token's
+        // pair goes out as one 4-byte store (a warp writes 128 contiguous
+        // bytes of a ys row)
+        const int of = unit * p.unit_rows + 2 * m;
+        uint32_t* op = reinterpret_cast<uint32_t*>(reinterpret_cast<__half*>(p.out) +
+                                                   (size_t)r0 * p.out_ld + of);
+        const size_t ld2 = (size_t)p.out_ld / 2;
+        for (int n0 = 0; n0 < nv; n0 += 16) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
+          const int lim = nv - n0;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (n0 + j < nv) {
-                float* o = op + (size_t)(n0 + j) * p.out_ld;
-                if (ok0) o[0] = __uint_as_float(a0[j]) + bv0;
-                if (ok1) o[BMW] = __uint_as_float(a1[j]) + bv1;
-              }
-            }
-          }
-        } else {
-          // the down projection's units are 256 whole rows of d (d % 256 ==
-          // 0): matrix 0 holds the even, matrix 1 the odd output features,
-          // so this thread's two features are adjacent and each token's
-          // pair goes out as one 4-byte store (a warp writes 128 contiguous
-          // bytes of a ys row)
-          const int of = unit * p.unit_rows + 2 * m;
-          uint32_t* op = reinterpret_cast<uint32_t*>(reinterpret_cast<__half*>(p.out) +
-                                                     (size_t)r0 * p.out_ld + of);
-          const size_t ld2 = (size_t)p.out_ld / 2;
-          for (int n0 = 0; n0 < nv; n0 += 16) {
-            uint32_t a0[16], a1[16];
-            tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
-            const int lim = nv - n0;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const uint32_t v = f16x2_pack(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
-              if (j < lim) {
-                hmax = max(hmax, max(v & 0x7FFFu, (v >> 16) & 0x7FFFu));
-                op[(size_t)(n0 + j) * ld2] = v;
-              }
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t v = f16x2_pack(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
+            if (j < lim) {
+              hmax = max(hmax, max(v & 0x7FFFu, (v >> 16) & 0x7FFFu));
+              op[(size_t)(n0 + j) * ld2] = v;
             }
           }
         }
@@ -926,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) {
               const uint32_t w4[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
 #pragma unroll
-              for (int i = 0; i < 4; ++i) vals[4 * c + i] = ROUTER ? w4[i] : bf16x2_to_f16x2(w4[i]);
+              for (int i = 0; i < 4; ++i) vals[4 * c + i] = bf16x2_to_f16x2(w4[i]);
             }
           }
           const uint32_t stage = a_it + (C::Q4 ? hf + 2 * j : C::Q8 ? hf : 0);
@@ -955,6 +918,227 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ router
+
+// Router logits on the tensor cores, both operands staged in shared memory
+// by TMA: logits[t][e] = sum_k x[t][k] * W_r[e][k] (+ bias[e]), fp32
+// accumulation of exact bf16 (or fp16) products. ("5.5 real sparse MoE
+// kernels (Metal)", Scope -- in: router logits, softmax, top-k.)
+// A unit is 128 experts (the MMA's M: router weight rows) x one tile of rn
+// tokens (its N: x rows); the CTA streams both through a ring of RST stages
+// of one 64-wide k-block each. Warp 0 loads, warp 1 issues the MMAs (one
+// elected lane), warps 2..5 move the accumulator out: lane = expert, so a
+// warp's 32 lanes store 128 contiguous bytes of one token's logits. Two
+// accumulator buffers let the epilogue of one unit overlap the MMAs of the
+// next. Nothing is converted on the way: unlike the expert GEMMs, whose
+// weights must be dequantised, both operands go to the tensor core as loaded.
+constexpr int RST = 6;                         // k-block stages
+constexpr int kRThreads = 192;                 // 6 warps
+constexpr int R_A_BYTES = BMW * 128;           // 128 weight rows x 64 elements
+constexpr int R_B_BYTES = BN * 128;            // up to 128 token rows x 64 elements
+constexpr int R_STAGE = R_A_BYTES + R_B_BYTES;
+constexpr int R_SMEM = 1024 + RST * R_STAGE + 256;
+static_assert(R_SMEM <= 232448, "shared memory per CTA");
+
+struct RouterParams {
+  int T, E, K;
+  int rn;              // token rows per tile (MMA N): 16, 32, 64 or 128
+  int n_mblk;          // 128-expert blocks
+  int n_units;         // n_mblk x token tiles
+  float* logits;       // [T][E]
+  const float* bias;   // [E] or null
+  int f16;             // x and W_r are fp16 (else bf16)
+  int* status;
+  long long wait_limit;
+};
+
+// D[tmem] (+)= A[smem] * B[smem]^T for one 64-deep k-block (four K-steps of
+// 16; both descriptors advance 32 bytes inside the 128-byte swizzle atom);
+// accumulate unless `first`. Warp-uniform operands, one elected lane issues.
+__device__ __forceinline__ void mma_kblock_ss(uint32_t d, uint32_t alo, uint32_t ahi, uint32_t blo,
+                                              uint32_t bhi, uint32_t idesc, uint32_t first) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt, e;\n\t.reg .b64 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.eq.b32 pf, %6, 0;\n\t"
+      "setp.ne.b32 pt, %5, 0;\n\t"
+      "mov.b64 a0, {%1, %2};\n\tmov.b64 b0, {%3, %4};\n\t"
+      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
+      "mov.b64 a1, {%1, %2};\n\tmov.b64 b1, {%3, %4};\n\t"
+      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
+      "mov.b64 a2, {%1, %2};\n\tmov.b64 b2, {%3, %4};\n\t"
+      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
+      "mov.b64 a3, {%1, %2};\n\tmov.b64 b3, {%3, %4};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a0, b0, %5, pf;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %5, pt;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %5, pt;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %5, pt;\n\t}\n"
+      : "+r"(d), "+r"(alo), "+r"(ahi), "+r"(blo), "+r"(bhi)
+      : "r"(idesc), "r"(first)
+      : "memory");
+}
+
+// 16 columns of this warp's 32 lanes from one TMEM address, and the wait
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t (&a)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
+        "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]),
+        "=r"(a[14]), "=r"(a[15])
+      : "r"(ta)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    router_tc_kernel(const __grid_constant__ RouterParams p, const __grid_constant__ CUtensorMap tmW,
+                     const __grid_constant__ CUtensorMap tmX) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  const uint32_t st_base = smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + RST * R_STAGE);   // [RST]
+  uint64_t* empty = full + RST;                                         // [RST]
+  uint64_t* acc_full = empty + RST;                                     // [2]
+  uint64_t* acc_empty = acc_full + 2;                                   // [2]
+  uint64_t* drain = acc_empty + 2;                                      // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < RST; ++i) {
+      mbar_init(smem_u32(full + i), 1);    // the loader's arrive + the copies' bytes
+      mbar_init(smem_u32(empty + i), 1);   // the MMAs' commit
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(acc_full + i), 1);
+      mbar_init(smem_u32(acc_empty + i), 4);   // the 4 epilogue warps
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+  }
+  if (warp == 1) {
+    // two accumulator buffers of up to 128 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();
+  pdl_launch();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = p.K / KA;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads (TMA)
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const int mb = u % p.n_mblk, tt = u / p.n_mblk;
+        for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+          const uint32_t s = it % RST;
+          if (it >= (uint32_t)RST) {
+            ok = mbar_wait(smem_u32(empty + s), ((it / RST) - 1) & 1, abort_flag, p.status, true,
+                           p.wait_limit);
+            if (!ok) break;
+          }
+          const uint32_t dst = st_base + s * R_STAGE;
+          const uint32_t bar = smem_u32(full + s);
+          // rows past E or T are zero-filled and never stored
+          mbar_arrive_tx(bar, (uint32_t)(R_A_BYTES + p.rn * 128));
+          tma_load_2d(dst, &tmW, kb * KA, mb * BMW, bar);
+          tma_load_2d(dst + R_A_BYTES, &tmX, kb * KA, tt * p.rn, bar);
+        }
+      }
+      // copies in flight complete before the CTA may exit
+      for (uint32_t i = 0; i < (uint32_t)RST && i < it; ++i) {
+        const uint32_t last = it - 1 - i;
+        mbar_wait(smem_u32(full + last % RST), (last / RST) & 1, abort_flag, p.status, false);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint32_t idesc = idesc_mma(p.rn, p.f16 != 0);
+    const uint64_t da = desc_sw128(st_base), db = desc_sw128(st_base + R_A_BYTES);
+    const uint32_t alo0 = (uint32_t)da, ahi = (uint32_t)(da >> 32);
+    const uint32_t blo0 = (uint32_t)db, bhi = (uint32_t)(db >> 32);
+    uint32_t it = 0, n_acc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++n_acc) {
+      const uint32_t buf = n_acc & 1;
+      // the epilogue has drained this buffer's previous unit
+      if (n_acc >= 2) {
+        ok = mbar_wait_warp(smem_u32(acc_empty + buf), ((n_acc >> 1) - 1) & 1, abort_flag,
+                            p.status, true, p.wait_limit);
+        if (!ok) break;
+      }
+      tc_fence_after();
+      for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+        const uint32_t s = it % RST;
+        ok = mbar_wait_warp(smem_u32(full + s), (it / RST) & 1, abort_flag, p.status, true,
+                            p.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t off = s * (uint32_t)(R_STAGE >> 4);
+        mma_kblock_ss(tm + buf * 128u, alo0 + off, ahi, blo0 + off, bhi, idesc, kb == 0);
+        mma_commit_warp(smem_u32(empty + s));
+      }
+      if (!ok) break;
+      mma_commit_warp(smem_u32(acc_full + buf));
+    }
+    // all MMAs issued complete before TMEM is released
+    mma_commit_warp(smem_u32(drain));
+    mbar_wait_warp(smem_u32(drain), 0, abort_flag, p.status, false);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int qd = warp & 3;                          // TMEM lane quadrant
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    uint32_t n_acc = 0;
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++n_acc) {
+      const int mb = u % p.n_mblk, tt = u / p.n_mblk;
+      const uint32_t buf = n_acc & 1;
+      if (!mbar_wait_warp(smem_u32(acc_full + buf), (n_acc >> 1) & 1, abort_flag, p.status, true,
+                          p.wait_limit))
+        break;
+      tc_fence_after();
+      const int e = mb * BMW + qd * 32 + lane;
+      const bool ok_e = e < p.E;
+      const float bv = (ok_e && p.bias) ? __ldg(p.bias + e) : 0.f;
+      const int t0 = tt * p.rn;
+      float* op = p.logits + (size_t)t0 * p.E + e;
+      for (int n0 = 0; n0 < p.rn; n0 += 16) {
+        uint32_t a[16];
+        tmem_ld16(tl + buf * 128u + (uint32_t)n0, a);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (ok_e && t0 + n0 + j < p.T) op[(size_t)(n0 + j) * p.E] = __uint_as_float(a[j]) + bv;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(acc_empty + buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
   }
 }
 
@@ -1128,10 +1312,10 @@ static bool token_maps(Params& p, const void* src, bool bf16, long long rows, in
   return true;
 }
 
-template <int FMT, int EPI, bool ROUTER>
+template <int FMT, int EPI>
 static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub, cudaStream_t s) {
   using C = Cfg<FMT>;
-  auto kern = grouped_tc_kernel<FMT, EPI, ROUTER>;
+  auto kern = grouped_tc_kernel<FMT, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const long long grid = units_ub < num_sms() ? units_ub : num_sms();
@@ -1142,19 +1326,19 @@ static cudaError_t run(const Params& p, const CUtensorMap& a, long long units_ub
 
 // The kernel for the experts' weight format. The _HP forms are built for
 // the q4 formats only (they permute h for the q4 dequant).
-template <int EPI, bool ROUTER>
+template <int EPI>
 static cudaError_t run_fmt(int fmt, const Params& p, const CUtensorMap& a, long long ub,
                            cudaStream_t s) {
   constexpr bool hp = EPI == EPI_SWIGLU_HP || EPI == EPI_GEGLU_HP || EPI == EPI_STORE_HP;
   switch (fmt) {
-    case MOE_W_Q4G64: return run<MOE_W_Q4G64, EPI, ROUTER>(p, a, ub, s);
-    case MOE_W_Q4G32: return run<MOE_W_Q4G32, EPI, ROUTER>(p, a, ub, s);
-    case MOE_W_Q4G128: return run<MOE_W_Q4G128, EPI, ROUTER>(p, a, ub, s);
+    case MOE_W_Q4G64: return run<MOE_W_Q4G64, EPI>(p, a, ub, s);
+    case MOE_W_Q4G32: return run<MOE_W_Q4G32, EPI>(p, a, ub, s);
+    case MOE_W_Q4G128: return run<MOE_W_Q4G128, EPI>(p, a, ub, s);
     default: break;
   }
   if constexpr (!hp) {
-    if (fmt == MOE_W_Q8G64) return run<MOE_W_Q8G64, EPI, ROUTER>(p, a, ub, s);
-    if (fmt == MOE_W_BF16) return run<MOE_W_BF16, EPI, ROUTER>(p, a, ub, s);
+    if (fmt == MOE_W_Q8G64) return run<MOE_W_Q8G64, EPI>(p, a, ub, s);
+    if (fmt == MOE_W_BF16) return run<MOE_W_BF16, EPI>(p, a, ub, s);
   }
   return cudaErrorNotSupported;
 }
@@ -1243,7 +1427,6 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.biases = (const uint16_t*)ex.b_gu;
   p.out = h;
   p.out_ld = ex.F;
-  p.m_limit = ex.F;
   p.status = status;
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
@@ -1251,10 +1434,10 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   // h in the permuted K order only for q4 weights (the down kernel then
   // dequantises in that order)
   if (q4 && h_perm)
-    return geglu ? run_fmt<EPI_GEGLU_HP, false>(ex.fmt, p, ta, ub, s)
-                 : run_fmt<EPI_SWIGLU_HP, false>(ex.fmt, p, ta, ub, s);
-  return geglu ? run_fmt<EPI_GEGLU, false>(ex.fmt, p, ta, ub, s)
-               : run_fmt<EPI_SWIGLU, false>(ex.fmt, p, ta, ub, s);
+    return geglu ? run_fmt<EPI_GEGLU_HP>(ex.fmt, p, ta, ub, s)
+                 : run_fmt<EPI_SWIGLU_HP>(ex.fmt, p, ta, ub, s);
+  return geglu ? run_fmt<EPI_GEGLU>(ex.fmt, p, ta, ub, s)
+               : run_fmt<EPI_SWIGLU>(ex.fmt, p, ta, ub, s);
 }
 
 cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t* tile_off, int R,
@@ -1285,12 +1468,11 @@ cudaError_t launch_down_tc(const void* h, const int32_t* row_off, const int32_t*
   p.biases = (const uint16_t*)ex.b_dn;
   p.out = ys;
   p.out_ld = ex.d;
-  p.m_limit = ex.d;
   p.status = status;
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
-  if (q4_group(ex.fmt) && h_perm) return run_fmt<EPI_STORE_HP, false>(ex.fmt, p, ta, ub, s);
-  return run_fmt<EPI_STORE, false>(ex.fmt, p, ta, ub, s);
+  if (q4_group(ex.fmt) && h_perm) return run_fmt<EPI_STORE_HP>(ex.fmt, p, ta, ub, s);
+  return run_fmt<EPI_STORE>(ex.fmt, p, ta, ub, s);
 }
 
 cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router, const float* bias,
@@ -1301,35 +1483,37 @@ cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router,
   if (T < 256 || d % 128 != 0) return cudaErrorNotSupported;
   if (dt != MOE_BF16 && dt != MOE_F16) return cudaErrorNotSupported;
   const bool f16 = dt == MOE_F16;
-  CUtensorMap ta;
-  if (!weight_map(&ta, MOE_W_BF16, w_router, E, d, f16)) return cudaErrorInvalidValue;
-  Params p{};
-  if (!token_maps(p, x, !f16, T, d)) return cudaErrorInvalidValue;
-  p.router_f16 = f16;
-  p.E = 1;
-  p.n_rows = T;
-  // units of two 128-row blocks of experts; rows past E are zero-filled by
-  // the TMA and never stored
-  p.n_units = (E + 2 * BMW - 1) / (2 * BMW);
-  p.unit_rows = 2 * BMW;
-  p.mat_off = BMW;
-  p.row_step = 1;
+  RouterParams p{};
+  p.T = T;
+  p.E = E;
   p.K = d;
-  p.w_rows = E;
-  p.out = logits;
-  p.out_ld = E;
-  p.m_limit = E;
+  p.n_mblk = (E + BMW - 1) / BMW;
+  // the widest token tile that still gives 3/8 of the SMs a unit: every unit
+  // streams its 128 weight rows and its x rows through one SM, and each
+  // halving of the tile re-reads the router weight once more from L2 (at
+  // T = 2048, E = 512: 128 rows on 64 SMs 13.3 us, 64 rows on 128 SMs 15.4 us)
+  int rn = BN;
+  while (rn > 16 && (long long)((T + rn - 1) / rn) * p.n_mblk < (3LL * num_sms()) / 8) rn /= 2;
+  p.rn = rn;
+  p.n_units = ((T + rn - 1) / rn) * p.n_mblk;
+  p.logits = logits;
   p.bias = bias;
+  p.f16 = f16;
   p.status = status;
   p.wait_limit = wait_cycles();
-  // token tiles small enough that at least half of the SMs get a unit: every
-  // unit streams the same weight rows through one SM, so more, shorter
-  // units spread the router over the GPU (down to 16 rows, the MMA's least N)
-  int tile = BN;
-  while (tile > 16 && (long long)((T + tile - 1) / tile) * p.n_units < num_sms() / 2) tile /= 2;
-  p.row_tile = tile;
-  const long long ub = (long long)((T + tile - 1) / tile) * p.n_units;
-  return run<MOE_W_BF16, EPI_STORE, true>(p, ta, ub, s);
+  CUtensorMap tw, tx;
+  const CUtensorMapDataType ty = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&tw, ty, w_router, (uint64_t)d, (uint64_t)E, (uint64_t)d * 2, KA, BMW,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tx, ty, x, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, KA, (uint32_t)rn,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       R_SMEM);
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
+  launch_pdl(router_tc_kernel, (unsigned)grid, kRThreads, R_SMEM, s, p, tw, tx);
+  return cudaGetLastError();
 }
 
 }  // namespace moe
