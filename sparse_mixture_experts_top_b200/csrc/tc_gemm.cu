@@ -201,9 +201,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   const bool sleep = limit >= 100000;
+  const uint32_t af = smem_u32(const_cast<const int*>(abort_flag));
   for (;;) {
     if (sleep ? mbar_try_sleep(bar, parity, 20000u) : mbar_try(bar, parity)) return true;
-    if (honor_abort && *abort_flag) return false;
+    uint32_t aborting;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(aborting) : "r"(af) : "memory");
+    if (honor_abort && aborting) return false;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
       report_status(status, MOE_ERR_TIMEOUT);
@@ -269,6 +272,9 @@ __device__ __forceinline__ void mma_kblock(uint32_t d0, uint32_t a0, uint32_t bl
       : "r"(idesc), "r"(first)
       : "memory");
 }
+
+// address of barrier i of an array of 8-byte mbarriers at shared address base
+__device__ __forceinline__ uint32_t bar_at(uint32_t base, uint32_t i) { return base + 8u * i; }
 
 // tcgen05.commit from one elected lane of a converged warp
 __device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
@@ -478,6 +484,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;                               // [2] one per issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // shared-memory addresses of the barrier arrays
+  const uint32_t raw_full_s = smem_u32(raw_full);
+  const uint32_t raw_empty_s = smem_u32(raw_empty);
+  const uint32_t b_full_s = smem_u32(b_full);
+  const uint32_t s_empty_s = smem_u32(s_empty);
+  const uint32_t acc_full_s = smem_u32(acc_full);
+  const uint32_t acc_empty_s = smem_u32(acc_empty);
+  const uint32_t drain_s = smem_u32(drain);
   // one scratch word per warp (see the dequant role)
   const uint32_t sink = smem_u32(bar_area + 512);
   int* s_toff = reinterpret_cast<int*>(bar_area + 1024);
@@ -492,19 +506,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NR; ++i) {
       // quantised: the TMA arrive + the 32 lanes' cp.async arrivals for the scales
-      mbar_init(smem_u32(raw_full + i), C::QUANT ? 33 : 1);
-      mbar_init(smem_u32(raw_empty + i), 16);   // the 16 dequant warps
+      mbar_init(bar_at(raw_full_s, i), C::QUANT ? 33 : 1);
+      mbar_init(bar_at(raw_empty_s, i), 16);   // the 16 dequant warps
     }
     // one barrier per A stage pair of a matrix: quantised, each stage of the
     // pair is written by the 4 warps of one half (8 arrivals); bf16, each
     // stage by the 8 warps of both halves (16 arrivals)
     for (int i = 0; i < 2 * NS; ++i) mbar_init(smem_u32(a_full + i), C::QUANT ? 8 : 16);
-    for (int i = 0; i < NB / 2; ++i) mbar_init(smem_u32(b_full + i), 1);
-    for (int i = 0; i < NP; ++i) mbar_init(smem_u32(s_empty + i), 2);   // both issuers
+    for (int i = 0; i < NB / 2; ++i) mbar_init(bar_at(b_full_s, i), 1);
+    for (int i = 0; i < NP; ++i) mbar_init(bar_at(s_empty_s, i), 2);   // both issuers
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(acc_full + i), 2);    // both issuers
-      mbar_init(smem_u32(acc_empty + i), 4);   // the 4 epilogue warps
-      mbar_init(smem_u32(drain + i), 1);
+      mbar_init(bar_at(acc_full_s, i), 2);    // both issuers
+      mbar_init(bar_at(acc_empty_s, i), 4);   // the 4 epilogue warps
+      mbar_init(bar_at(drain_s, i), 1);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -535,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ raw weights (TMA)
-    uint32_t raw_it = 0;
+    uint32_t raw_it = 0, rs = 0, rph = 0;      // stages issued; ring slot and its phase
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int unit, r0, nv, e;
@@ -543,9 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long wrow0 = (long long)e * p.rows_per_group + (long long)unit * p.unit_rows;
       const long long wrow1 = wrow0 + p.mat_off;
       for (int kr = 0; kr < nkr && ok; ++kr) {
-        const int rs = raw_it % C::NR;
-        ok = mbar_wait_warp(smem_u32(raw_empty + rs), ((raw_it / C::NR) & 1) ^ 1, abort_flag,
-                            p.status, true, p.wait_limit);
+        ok = mbar_wait_warp(bar_at(raw_empty_s, rs), rph ^ 1, abort_flag, p.status, true,
+                            p.wait_limit);
         if (!ok) break;
         if (C::QUANT) {
           // the stage's scales and biases (KR / GS groups of each weight
@@ -571,19 +584,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                            : "memory");
             }
           asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                           smem_u32(raw_full + rs))
+                           bar_at(raw_full_s, rs))
                        : "memory");
         }
         if (lane == 0) {
           // rows past the end of the tensor are filled with zeros by the TMA
           const uint32_t dst = raw_base + rs * C::RAW_BYTES;
-          const uint32_t bar = smem_u32(raw_full + rs);
+          const uint32_t bar = bar_at(raw_full_s, rs);
           const int x = kr * (C::Q4 ? C::KR / 8 : C::Q8 ? C::KR / 4 : C::KR);
           mbar_arrive_tx(bar, C::RAW_BYTES);
           tma_load_2d(dst, &tmA, x, (int)wrow0, bar);
           tma_load_2d(dst + C::RAW_MAT, &tmA, x, (int)wrow1, bar);
         }
         ++raw_it;
+        if (++rs == (uint32_t)C::NR) { rs = 0; rph ^= 1; }
       }
     }
     // copies in flight: wait (bounded, also when aborting) for the last
@@ -592,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (uint32_t i = 0; i < (uint32_t)C::NR && i < raw_it; ++i) {
         const uint32_t last = raw_it - 1 - i;
-        mbar_wait(smem_u32(raw_full + last % C::NR), (last / C::NR) & 1, abort_flag, p.status, false);
+        mbar_wait(bar_at(raw_full_s, last % C::NR), (last / C::NR) & 1, abort_flag, p.status, false);
       }
     }
     __syncwarp();
@@ -617,10 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int bs = j % NB;
           if (j >= (uint32_t)NB) {
             const uint32_t pr = (j - NB) >> 1;
-            ok = mbar_wait(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status, true, p.wait_limit);
+            ok = mbar_wait(bar_at(s_empty_s, pr % NP), (pr / NP) & 1, abort_flag, p.status, true, p.wait_limit);
             if (!ok) break;
           }
-          const uint32_t bar = smem_u32(b_full + bs / 2);
+          const uint32_t bar = bar_at(b_full_s, bs / 2);
           mbar_arrive_tx(bar, (uint32_t)n * 256u);
           tma_load_2d(b_base + bs * C::B_BYTES, tm, kb * KA, r0, bar);
           tma_load_2d(b_base + (bs + 1) * C::B_BYTES, tm, (kb + 1) * KA, r0, bar);
@@ -629,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (uint32_t i = 0; i < (uint32_t)NB && i < j; i += 2) {
         const uint32_t last = (j - 2 - i) / 2;      // pair index
-        mbar_wait(smem_u32(b_full + last % (NB / 2)), (last / (NB / 2)) & 1, abort_flag, p.status,
+        mbar_wait(bar_at(b_full_s, last % (NB / 2)), (last / (NB / 2)) & 1, abort_flag, p.status,
                   false);
       }
     }
@@ -663,9 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool use0 = !small || b == 0, use1 = !small || b == 1;
       // the epilogue has drained the buffers' previous tiles
       if (use0 && uses0 > 0)
-        ok = mbar_wait_warp(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
+        ok = mbar_wait_warp(bar_at(acc_empty_s, 0), (uses0 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
       if (ok && use1 && uses1 > 0)
-        ok = mbar_wait_warp(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
+        ok = mbar_wait_warp(bar_at(acc_empty_s, 1), (uses1 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
       if (!ok) break;
       tc_fence_after();
       const uint32_t dcol = tm + (small ? b * 128u + q * 64u : q * 128u);
@@ -675,26 +689,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // complete one barrier; both B stages share another.
       for (int kb = 0; kb < nka && ok; kb += 2) {
         ok = mbar_wait_warp(afull0 + (ss >> 1) * 8, sph, abort_flag, p.status, true, p.wait_limit) &&
-             mbar_wait_warp(smem_u32(b_full + bs / 2), bph, abort_flag, p.status, true, p.wait_limit);
+             mbar_wait_warp(bar_at(b_full_s, bs / 2), bph, abort_flag, p.status, true, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t acol = a_col0 + ss * (uint32_t)C::A_COLS;
         const uint32_t blo = blo0 + bs * (uint32_t)(C::B_BYTES >> 4);
         mma_kblock(dcol, acol, blo, bhi, idesc, kb == 0);
         mma_kblock(dcol, acol + C::A_COLS, blo + (C::B_BYTES >> 4), bhi, idesc, 0);
-        mma_commit_warp(smem_u32(s_empty + (kg >> 1) % NP));   // release k-block pair kg / 2
+        mma_commit_warp(bar_at(s_empty_s, (kg >> 1) % NP));   // release k-block pair kg / 2
         kg += 2;
         if ((ss += 2) == (uint32_t)NS) { ss = 0; sph ^= 1; }
         if ((bs += 2) == (uint32_t)NB) { bs = 0; bph ^= 1; }
       }
       if (!ok) break;
-      if (use0) { mma_commit_warp(smem_u32(acc_full + 0)); ++uses0; }
-      if (use1) { mma_commit_warp(smem_u32(acc_full + 1)); ++uses1; }
+      if (use0) { mma_commit_warp(bar_at(acc_full_s, 0)); ++uses0; }
+      if (use1) { mma_commit_warp(bar_at(acc_full_s, 1)); ++uses1; }
       if (small) nb ^= 1u;
     }
     // all MMAs issued by this warp complete before TMEM is released
-    mma_commit_warp(smem_u32(drain + q));
-    mbar_wait_warp(smem_u32(drain + q), 0, abort_flag, p.status, false);
+    mma_commit_warp(bar_at(drain_s, q));
+    mbar_wait_warp(bar_at(drain_s, q), 0, abort_flag, p.status, false);
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;
@@ -710,8 +724,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool small = mma_n(nv) <= 64;
       const uint32_t b = small ? nb : 0u;
       const bool use0 = !small || b == 0, use1 = !small || b == 1;
-      if (use0 && !mbar_wait_warp(smem_u32(acc_full + 0), uses0 & 1, abort_flag, p.status, true, p.wait_limit)) break;
-      if (use1 && !mbar_wait_warp(smem_u32(acc_full + 1), uses1 & 1, abort_flag, p.status, true, p.wait_limit)) break;
+      if (use0 && !mbar_wait_warp(bar_at(acc_full_s, 0), uses0 & 1, abort_flag, p.status, true, p.wait_limit)) break;
+      if (use1 && !mbar_wait_warp(bar_at(acc_full_s, 1), uses1 & 1, abort_flag, p.status, true, p.wait_limit)) break;
       tc_fence_after();
       const uint32_t c0 = tl + (small ? b * 128u : 0u);         // matrix 0
       const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);  // matrix 1
@@ -763,8 +777,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (use0) mbar_arrive(smem_u32(acc_empty + 0));
-        if (use1) mbar_arrive(smem_u32(acc_empty + 1));
+        if (use0) mbar_arrive(bar_at(acc_empty_s, 0));
+        if (use1) mbar_arrive(bar_at(acc_empty_s, 1));
       }
       if (use0) ++uses0;
       if (use1) ++uses1;
@@ -787,12 +801,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
     const uint32_t afull = smem_u32(a_full + q * NS);
     constexpr int NST = C::Q4 ? 2 : 1;                // A stages per raw stage of this warp
-    uint32_t raw_it = 0, a_it = 0;
+    uint32_t rs = 0, rph = 0, a_it = 0;         // raw ring slot and its phase
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       for (int kr = 0; kr < nkr && ok; ++kr) {
-        const int rs = raw_it % C::NR;
-        ok = mbar_wait_warp(smem_u32(raw_full + rs), (raw_it / C::NR) & 1, abort_flag, p.status, true, p.wait_limit);
+        ok = mbar_wait_warp(bar_at(raw_full_s, rs), rph, abort_flag, p.status, true, p.wait_limit);
         if (!ok) break;
         // my half row: 4 chunks of 16 B in the 128-byte swizzle
         const uint32_t rowa = raw_base + rs * C::RAW_BYTES + q * C::RAW_MAT + m * 128;
@@ -846,13 +859,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this stage can overwrite rows the load has not read yet (seen on
         // the first rows the TMA writes). So the loaded words are folded into
         // one value stored to a scratch word before the stage is released.
-        uint32_t fold = sg[0] ^ sg[1] ^ bg[0] ^ bg[1];
+        // (one register of each vector load: its destination registers are
+        // written together, so consuming one waits for the whole load)
+        uint32_t fold = sg[0] ^ bg[0];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) fold ^= wv[c].x ^ wv[c].y ^ wv[c].z ^ wv[c].w;
+        for (int c = 0; c < 4; ++c) fold ^= wv[c].x;
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sink + 4u * (uint32_t)warp), "r"(fold)
                      : "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(raw_empty + rs));
+        if (lane == 0) mbar_arrive(bar_at(raw_empty_s, rs));
 #pragma unroll
         for (int j = 0; j < NST; ++j) {
           uint32_t vals[32];
@@ -896,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t as = stage % NS;
           if (stage >= (uint32_t)NS) {      // the slot's previous k-block is released
             const uint32_t pr = (stage - NS) >> 1;
-            ok = mbar_wait_warp(smem_u32(s_empty + pr % NP), (pr / NP) & 1, abort_flag, p.status, true, p.wait_limit);
+            ok = mbar_wait_warp(bar_at(s_empty_s, pr % NP), (pr / NP) & 1, abort_flag, p.status, true, p.wait_limit);
             if (!ok) break;
           }
           tc_fence_after();
@@ -907,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(afull + (as >> 1) * 8);
         }
-        ++raw_it;
+        if (++rs == (uint32_t)C::NR) { rs = 0; rph ^= 1; }
         a_it += C::A_PER_RAW;
       }
     }
