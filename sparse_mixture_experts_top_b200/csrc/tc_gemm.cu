@@ -768,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j) {
             const uint32_t v = f16x2_pack(__uint_as_float(a0[j]), __uint_as_float(a1[j]));
             if (j < lim) {
-              hmax = max(hmax, max(v & 0x7FFFu, (v >> 16) & 0x7FFFu));
+              hmax = __vmaxu2(hmax, v & 0x7FFF7FFFu);    // both halves' magnitudes
               op[(size_t)(n0 + j) * ld2] = v;
             }
           }
@@ -784,7 +784,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (use1) ++uses1;
       if (small) nb ^= 1u;
     }
-    if (!__all_sync(0xffffffffu, hmax < 0x7C00u) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
+    // (down: the two 16-bit halves hold separate maxima)
+    const uint32_t hm = max(hmax & 0xFFFFu, hmax >> 16);
+    if (!__all_sync(0xffffffffu, hm < 0x7C00u) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------------------------ dequant
     // 16 warps: (matrix q, lane quadrant qd, half hf). q4: half hf converts
