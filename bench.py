@@ -38,11 +38,10 @@ import moe_inputs as mi  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one gate|up launch on the prefill workload,
-# from an ncu capture of that kernel (the stage call's grouped_tc_kernel<2, 0,
-# 0> as of the commit that adds q4 g32/g128 and q8 to the tcgen05 kernels:
-# 675.21 MB read + 21.13 MB written); to be retaken whenever that kernel
-# changes
-GATE_UP_TRAFFIC = {"prefill": 696339456}
+# from an ncu capture of that kernel (the stage call's grouped_tc_kernel<2, 0>
+# as of the commit that trims its raw-ring bookkeeping: 675.49 MB read +
+# 20.75 MB written); to be retaken whenever that kernel changes
+GATE_UP_TRAFFIC = {"prefill": 696238336}
 L2_FLUSH_BYTES = 256 << 20
 
 
