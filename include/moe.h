@@ -65,14 +65,19 @@
  *
  * Regimes: moe_grouped_swiglu / moe_grouped_down / moe_forward take a regime.
  *   MOE_REGIME_GEMV: weight-streaming kernels, every selected expert's bytes
- *     read once per step, for few tokens per expert (decode);
+ *     read once per step; moe_forward runs the whole layer as one
+ *     cooperative launch (the fused decode kernel) where that kernel applies
+ *     (q4 experts, T <= 32, T*k <= 256, E <= 256, d and F multiples of 128
+ *     up to 2048);
  *   MOE_REGIME_TC: tensor-core grouped GEMM (tcgen05 / TMEM, TMA-staged
  *     operands) for many tokens per expert (prefill); bf16 activations with
  *     bf16 weights, or bf16 / fp16 activations with any quantised format
  *     (q4 groups 32/64/128, q8 group 64); d a multiple of 256, F of 128 (q4:
  *     of 256); other shapes return MOE_ERR_UNSUPPORTED;
- *   MOE_REGIME_AUTO: GEMV when T*k <= 8*E or the shape is not one the
- *     tensor-core kernels tile, else TC (bf16 / fp16) or GEMV (f32).
+ *   MOE_REGIME_AUTO: TC wherever the tensor-core kernels tile the shape
+ *     (16-bit activations), except that moe_forward keeps the fused decode
+ *     kernel while it applies and 2*T*k < E; GEMV for everything else
+ *     (f32 activations, other shapes).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -89,16 +89,23 @@ static moe_status check_experts(const moe_experts* ex, int dt) {
 
 static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16 || dt == MOE_F16; }
 
-// The regime a call runs: AUTO picks the weight-streaming kernels when there
-// are at most 8 routed rows per expert on average, or for fp32 activations
-// (the tensor-core kernels take 16-bit operands).
-static int resolve_regime(int regime, long long R, int E, int dt, int d = 128, int F = 128,
-                          int fmt = MOE_W_Q4G64) {
+// The regime a call runs. AUTO takes the tensor-core kernels wherever they
+// tile the shape (16-bit activations; d % 256, F % 128, or % 256 for q4;
+// q4, q8 or bf16 weights), except that the whole-layer call keeps the
+// one-launch fused decode kernel while it applies and fewer than E / 2 rows
+// are routed; the weight-streaming kernels take everything else. Measured on
+// one B200 (graph-replayed forwards, L2 flushed): at E = 256, top-8 the fused
+// kernel is faster up to 12 tokens (84 against 92 us at 8) and the tensor
+// cores from 16 (117 against 124 us; 138 against 166 at 32); at E = 512,
+// top-10, where the fused kernel does not apply, the tensor cores are faster
+// from 4 tokens (60 against 76 us); with 8 bf16 experts from 1 token (86
+// against 107 us).
+static int resolve_regime(int regime, long long R, int E, int dt, int d, int F, int fmt,
+                          bool fused_decode) {
   if (regime == MOE_REGIME_GEMV || regime == MOE_REGIME_TC) return regime;
-  // the tensor-core kernels tile d by 256 and F by 128 and take bf16 or q4 weights
-  if (!tc_shape_supported(d, F, fmt, dt)) return MOE_REGIME_GEMV;
-  if (dt == MOE_F32) return MOE_REGIME_GEMV;
-  return (R <= 8LL * E) ? MOE_REGIME_GEMV : MOE_REGIME_TC;
+  if (dt == MOE_F32 || !tc_shape_supported(d, F, fmt, dt)) return MOE_REGIME_GEMV;
+  if (fused_decode && 2 * R < E) return MOE_REGIME_GEMV;
+  return MOE_REGIME_TC;
 }
 
 static int block_m_for(int regime, long long R, int E) {
@@ -265,7 +272,8 @@ moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_m
   if (!x || !row_map || !row_off || !tile_off || !h) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
   const long long R = (long long)T * k;
-  const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt);
+  const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt,
+                                false);
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
     if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
@@ -297,7 +305,8 @@ moe_status moe_grouped_down(const void* h, moe_dtype dt, const int32_t* row_off,
   if (!h || !row_off || !tile_off || !ys) return MOE_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(ys)) return MOE_ERR_INVALID_ARG;
   const long long R = (long long)T * k;
-  const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt);
+  const int rg = resolve_regime(regime, R, experts->E, dt, experts->d, experts->F, experts->fmt,
+                                false);
   cudaStream_t s = (cudaStream_t)stream;
   if (rg == MOE_REGIME_TC) {
     if (dt == MOE_F32) return MOE_ERR_UNSUPPORTED;
@@ -393,7 +402,7 @@ moe_status moe_forward_layout(int T, int d, int E, int k, int F, moe_dtype dt, m
   L.sort_ws = take(sort_workspace_bytes((int)R, E));
   L.h = take((size_t)R * F * a);      // fp16 (16-bit activations) or fp32
   L.ys = take((size_t)R * d * a);     // fp16 (16-bit activations) or fp32
-  L.regime = resolve_regime(regime, R, E, dt, d, F, wfmt);
+  L.regime = resolve_regime(regime, R, E, dt, d, F, wfmt, decode_fused_ok(T, k, E, d, F, wfmt, dt));
   L.BM = block_m_for(L.regime, R, E);
   // fp16 token rows: x converted (weight-streaming), or permuted (the
   // one-launch path), or gathered in sorted row order (tensor cores)

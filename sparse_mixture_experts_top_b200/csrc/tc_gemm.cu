@@ -1496,8 +1496,9 @@ cudaError_t launch_router_logits_tc(const void* x, int dt, const void* w_router,
                                     int T, int d, int E, float* logits, int* status,
                                     cudaStream_t s) {
   using namespace tc;
-  // few tokens: the weight-streaming kernel is faster than a 128-row tile
-  if (T < 256 || d % 128 != 0) return cudaErrorNotSupported;
+  // any token count: 8 us on one B200 from 1 to 2048 tokens at d = 2048,
+  // E = 256-512, where the SIMT tile kernel took 170 us from 65 tokens up
+  if (T < 1 || d % 128 != 0) return cudaErrorNotSupported;
   if (dt != MOE_BF16 && dt != MOE_F16) return cudaErrorNotSupported;
   const bool f16 = dt == MOE_F16;
   RouterParams p{};

@@ -240,12 +240,13 @@ def _forward_and_compare(moe, orc, layer, sample=None, regime=0):
     return assert_close_rms(to_np(y)[rows][keep], r.y[keep], _tol(wl.act), f"y[{wl.name}]")
 
 
-@pytest.mark.parametrize("name,seed", [("tiny", 0), ("tiny", 1), ("tiny", 2),
-                                       ("decode_t1", 0), ("decode_t1", 1),
-                                       ("decode_t32", 0), ("decode_t32", 2)])
-def test_forward_parity_full(moe, orc, name, seed):
+@pytest.mark.parametrize("name,seed,regime", [("tiny", 0, 0), ("tiny", 1, 0), ("tiny", 2, 0),
+                                              ("decode_t1", 0, 0), ("decode_t1", 1, 0),
+                                              # the fused decode kernel; AUTO (tensor cores)
+                                              ("decode_t32", 0, 1), ("decode_t32", 2, 0)])
+def test_forward_parity_full(moe, orc, name, seed, regime):
     layer = mi.make_layer(name, seed=seed, device=DEV)
-    _forward_and_compare(moe, orc, layer)
+    _forward_and_compare(moe, orc, layer, regime=regime)
 
 
 def test_forward_parity_acceptance(moe, orc):
@@ -313,7 +314,7 @@ def test_grouped_geglu_parity(moe, orc, name, T, regime, BM):
 def test_forward_geglu_fused_decode(moe, orc, name):
     layer = mi.make_layer(name, seed=5, device=DEV)
     layer.experts = layer.experts.with_act("geglu")
-    _forward_and_compare(moe, orc, layer)
+    _forward_and_compare(moe, orc, layer, regime=1)
 
 
 def test_forward_geglu_prefill_sampled(moe, orc):
@@ -358,7 +359,7 @@ def test_forward_q4_group_sizes_fused_decode(moe, orc, wfmt, name, T):
     """4-bit weights with groups of 32 and 128 (DS4Server issue #112, "Kernel
     contract") through the fused decode kernel."""
     layer = mi.make_layer(mi.workload(name, T=T, wfmt=wfmt), seed=6, device=DEV)
-    _forward_and_compare(moe, orc, layer)
+    _forward_and_compare(moe, orc, layer, regime=1)
 
 
 @pytest.mark.parametrize("wfmt", ["q4g32", "q4g128"])
@@ -379,15 +380,16 @@ def test_grouped_stages_q4_group_sizes(moe, orc, wfmt):
     assert_ys_close(ys, yref, habs, U_F16, TOL_BF16, f"ys[{wfmt}]", u_ys=U_F16, F=wl.F)
 
 
-@pytest.mark.parametrize("wfmt,T", [("q4g128", 300), ("q4g32", 1024)])
-def test_forward_q4_group_sizes_prefill_shape(moe, orc, wfmt, T):
-    """Prefill shapes: 300 tokens (7.5 rows per expert) run the
-    weight-streaming kernels; 1,024 tokens resolve to the tcgen05 kernels."""
-    L = moe.forward_layout(T, 2048, 512, 10, 512, torch.bfloat16, wfmt)
-    assert L.regime == (moe.REGIME_TC if T == 1024 else moe.REGIME_GEMV)
+@pytest.mark.parametrize("wfmt,T,regime", [("q4g128", 300, 1), ("q4g32", 1024, 0)])
+def test_forward_q4_group_sizes_prefill_shape(moe, orc, wfmt, T, regime):
+    """Prefill shapes: 300 tokens on the weight-streaming kernels (asked
+    for); 1,024 tokens resolve to the tcgen05 kernels."""
+    L = moe.forward_layout(T, 2048, 512, 10, 512, torch.bfloat16, wfmt, regime)
+    assert L.regime == (moe.REGIME_TC if regime == 0 else moe.REGIME_GEMV)
     layer = mi.make_layer(mi.workload("prefill", T=T, wfmt=wfmt), seed=8, device=DEV)
     rng = np.random.default_rng(3)
-    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(T, 32, replace=False)))
+    _forward_and_compare(moe, orc, layer, sample=np.sort(rng.choice(T, 32, replace=False)),
+                         regime=regime)
     assert moe.device_status() == moe.OK
 
 
@@ -459,12 +461,14 @@ def test_grouped_stages_f16(moe, orc, name, T, regime, BM, wfmt):
                                          ("decode_t32", 32, "q4g128"), ("decode_t1", 1, "q8"),
                                          ("prefill", 300, "q4")])
 def test_forward_f16(moe, orc, name, T, wfmt):
-    """The whole layer on fp16 activations: the one-launch decode kernel (q4,
-    up to 32 tokens), the separate weight-streaming stages (q8; 300 tokens)."""
+    """The whole layer on fp16 activations in the weight-streaming regime: the
+    one-launch decode kernel (q4, up to 32 tokens), the separate
+    weight-streaming stages (q8; 300 tokens)."""
     layer = mi.make_layer(mi.workload(name, T=T, act="f16", wfmt=wfmt), seed=12, device=DEV)
-    y = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, layer.wl.k)
+    y = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, layer.wl.k,
+                    regime=1)
     assert y.dtype == torch.float16
-    _forward_and_compare(moe, orc, layer)
+    _forward_and_compare(moe, orc, layer, regime=1)
     assert moe.device_status() == moe.OK
 
 
@@ -483,21 +487,24 @@ def test_forward_deterministic(moe):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["acceptance", "prefill", "decode_t1", "decode_t32"])
-def test_forward_repeats_bit_exact(moe, name):
+@pytest.mark.parametrize("name,regime", [("acceptance", 0), ("prefill", 0), ("decode_t1", 0),
+                                         ("decode_t32", 1), ("decode_t32", 0)])
+def test_forward_repeats_bit_exact(moe, name, regime):
     """Every path gives the same bits on every repeat (tensor-core kernels for
-    acceptance and prefill, the fused decode kernel for decode). A raw weight
+    acceptance, prefill and 32-token decode, the fused decode kernel for one
+    token and for 32 when asked for). A raw weight
     stage released before the dequantising warps' shared-memory loads had
     read it let the next TMA overwrite its first rows under them: a few
     features of one tile came out wrong in about one run in five (bf16
     weights); 24 repeats catch a race of that rate with near certainty."""
     layer = mi.make_layer(name, seed=0, device=DEV)
     wl = layer.wl
-    ws = moe.forward_workspace(layer.x, layer.experts, wl.k)
+    ws = moe.forward_workspace(layer.x, layer.experts, wl.k, regime)
     ref = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, wl.k,
-                      ws=ws).clone()
+                      regime=regime, ws=ws).clone()
     for _ in range(24):
-        y = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, wl.k, ws=ws)
+        y = moe.forward(layer.x, layer.w_router, layer.router_bias, layer.experts, wl.k,
+                        regime=regime, ws=ws)
         assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
     assert moe.device_status() == moe.OK
 

@@ -56,7 +56,7 @@ def _bits(y):
 
 @pytest.mark.parametrize("name,T,regime", [
     ("prefill", 600, 2),        # router, gate|up and down on the tcgen05 kernels
-    ("decode_t32", 32, 0),      # the one-launch fused decode kernel (grid barriers)
+    ("decode_t32", 32, 1),      # the one-launch fused decode kernel (grid barriers)
 ])
 def test_forward_aborts_on_short_bound_and_recovers(moe, name, T, regime):
     layer = mi.make_layer(mi.workload(name, T=T), seed=41, device="cuda")
