@@ -76,7 +76,7 @@
  *     of 256); other shapes return MOE_ERR_UNSUPPORTED;
  *   MOE_REGIME_AUTO: TC wherever the tensor-core kernels tile the shape
  *     (16-bit activations), except that moe_forward keeps the fused decode
- *     kernel while it applies and 2*T*k < E; GEMV for everything else
+ *     kernel while it applies and T*k < E; GEMV for everything else
  *     (f32 activations, other shapes).
  */
 #ifndef MOE_B200_H

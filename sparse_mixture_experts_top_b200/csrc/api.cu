@@ -92,19 +92,19 @@ static bool valid_dt(int dt) { return dt == MOE_F32 || dt == MOE_BF16 || dt == M
 // The regime a call runs. AUTO takes the tensor-core kernels wherever they
 // tile the shape (16-bit activations; d % 256, F % 128, or % 256 for q4;
 // q4, q8 or bf16 weights), except that the whole-layer call keeps the
-// one-launch fused decode kernel while it applies and fewer than E / 2 rows
-// are routed; the weight-streaming kernels take everything else. Measured on
-// one B200 (graph-replayed forwards, L2 flushed): at E = 256, top-8 the fused
-// kernel is faster up to 12 tokens (84 against 92 us at 8) and the tensor
-// cores from 16 (117 against 124 us; 138 against 166 at 32); at E = 512,
-// top-10, where the fused kernel does not apply, the tensor cores are faster
-// from 4 tokens (60 against 76 us); with 8 bf16 experts from 1 token (86
-// against 107 us).
+// one-launch fused decode kernel while it applies and fewer than E rows are
+// routed; the weight-streaming kernels take everything else. Measured on one
+// B200 (graph-replayed forwards, L2 flushed): at E = 128, top-8, F = 768 the
+// fused kernel is faster up to 12 tokens (84 against 92 us at 8, 110 against
+// 116 at 12) and the tensor cores from 16 (117 against 124 us; 138 against
+// 166 at 32); at E = 512, top-10, where the fused kernel does not apply, the
+// tensor cores are faster from 4 tokens (60 against 76 us); with 8 bf16
+// experts from 1 token (86 against 107 us).
 static int resolve_regime(int regime, long long R, int E, int dt, int d, int F, int fmt,
                           bool fused_decode) {
   if (regime == MOE_REGIME_GEMV || regime == MOE_REGIME_TC) return regime;
   if (dt == MOE_F32 || !tc_shape_supported(d, F, fmt, dt)) return MOE_REGIME_GEMV;
-  if (fused_decode && 2 * R < E) return MOE_REGIME_GEMV;
+  if (fused_decode && R < E) return MOE_REGIME_GEMV;
   return MOE_REGIME_TC;
 }
 

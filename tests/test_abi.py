@@ -139,28 +139,29 @@ def test_pack_gate_up_rejects_bad_arguments(moe):
 def test_regime_choice(moe):
     """AUTO takes the tensor-core kernels wherever they tile the shape with
     16-bit activations, except that the whole-layer call keeps the fused
-    decode kernel while it applies and fewer than E / 2 rows are routed; the
+    decode kernel while it applies and fewer than E rows are routed; the
     weight-streaming kernels for fp32 and for shapes or formats the
     tensor-core kernels do not take."""
     torch = __import__("torch")
     prefill = (2048, 2048, 512, 10, 512)       # 40 rows per expert
-    decode32 = (32, 2048, 256, 8, 512)         # 256 rows over 256 experts
-    decode8 = (8, 2048, 256, 8, 512)           # 64 rows: the fused decode kernel
+    decode = lambda T: (T, 2048, 128, 8, 768)  # the decode layer at T tokens
     small_e512 = (4, 2048, 512, 10, 512)       # 40 rows, E > 256: no fused kernel
     for dt in (torch.bfloat16, torch.float16):
         assert moe.forward_layout(*prefill, dt, "q4").regime == moe.REGIME_TC
-        assert moe.forward_layout(*decode32, dt, "q4").regime == moe.REGIME_TC
-        assert moe.forward_layout(*decode8, dt, "q4").regime == moe.REGIME_GEMV
+        for T in (1, 8, 15):                   # T k < E: the fused decode kernel
+            assert moe.forward_layout(*decode(T), dt, "q4").regime == moe.REGIME_GEMV
+        for T in (16, 32):
+            assert moe.forward_layout(*decode(T), dt, "q4").regime == moe.REGIME_TC
         assert moe.forward_layout(*small_e512, dt, "q4").regime == moe.REGIME_TC
     # the fused decode kernel takes q4 only: q8 at the same shape goes to TC
-    assert moe.forward_layout(*decode8, torch.bfloat16, "q8").regime == moe.REGIME_TC
+    assert moe.forward_layout(*decode(8), torch.bfloat16, "q8").regime == moe.REGIME_TC
     assert moe.forward_layout(*prefill, torch.float32, "f32").regime == moe.REGIME_GEMV
     # bf16 weights: F % 256 == 128 is a shape the tensor-core kernels tile
     # (q4 needs F % 256 == 0)
     acc = (512, 2048, 8, 2, 640)
     assert moe.forward_layout(*acc, torch.bfloat16, "bf16").regime == moe.REGIME_TC
     assert moe.forward_layout(*acc, torch.bfloat16, "q4").regime == moe.REGIME_GEMV
-    decode = decode8
+    decode = decode(8)
     # an explicit regime is kept
     assert moe.forward_layout(*decode, torch.bfloat16, "q4", moe.REGIME_TC).regime == moe.REGIME_TC
     with pytest.raises(TypeError):
