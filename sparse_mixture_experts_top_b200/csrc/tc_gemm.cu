@@ -276,6 +276,45 @@ __device__ __forceinline__ void mma_kblock(uint32_t d0, uint32_t a0, uint32_t bl
 // address of barrier i of an array of 8-byte mbarriers at shared address base
 __device__ __forceinline__ uint32_t bar_at(uint32_t base, uint32_t i) { return base + 8u * i; }
 
+// D[tmem] (+)= A[smem] * B[smem]^T for one 64-deep k-block (four K-steps of
+// 16; both descriptors advance 32 bytes inside the 128-byte swizzle atom);
+// accumulate unless `first`. Warp-uniform operands, one elected lane issues.
+__device__ __forceinline__ void mma_kblock_ss(uint32_t d, uint32_t alo, uint32_t ahi, uint32_t blo,
+                                              uint32_t bhi, uint32_t idesc, uint32_t first) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt, e;\n\t.reg .b64 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.eq.b32 pf, %6, 0;\n\t"
+      "setp.ne.b32 pt, %5, 0;\n\t"
+      "mov.b64 a0, {%1, %2};\n\tmov.b64 b0, {%3, %4};\n\t"
+      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
+      "mov.b64 a1, {%1, %2};\n\tmov.b64 b1, {%3, %4};\n\t"
+      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
+      "mov.b64 a2, {%1, %2};\n\tmov.b64 b2, {%3, %4};\n\t"
+      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
+      "mov.b64 a3, {%1, %2};\n\tmov.b64 b3, {%3, %4};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a0, b0, %5, pf;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %5, pt;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %5, pt;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %5, pt;\n\t}\n"
+      : "+r"(d), "+r"(alo), "+r"(ahi), "+r"(blo), "+r"(bhi)
+      : "r"(idesc), "r"(first)
+      : "memory");
+}
+
+// 16 columns of this warp's 32 lanes from one TMEM address, and the wait
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t (&a)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
+        "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]),
+        "=r"(a[14]), "=r"(a[15])
+      : "r"(ta)
+      : "memory");
+}
+
 // tcgen05.commit from one elected lane of a converged warp
 __device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
   asm volatile(
@@ -938,6 +977,209 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ bf16 gate|up
+
+// gate|up for bf16 weights and bf16 activations: nothing to dequantise, so
+// both operands go to the tensor core as loaded (mlx-lm PR #2044, "What":
+// the expert's weight tile is read once per token tile; DS4Server issue
+// #112, "Kernel contract": h = silu(gate) * up in sorted row order). A unit
+// is one token tile x the gate and up rows of 128 features, as in
+// grouped_tc_kernel; warp 0 loads each 64-wide k-block of both weight
+// matrices and of the tile's token rows (bf16, gathered without conversion)
+// by TMA into a ring of SST stages, warp 1 issues the MMAs of both matrices
+// (A and B in shared memory) into two accumulators, warps 2..5 apply the GLU.
+// The products of bf16 values are exact in fp32, so h is what the fp16
+// operand path computes.
+constexpr int SST = 4;                          // k-block stages
+constexpr int kSThreads = 192;
+constexpr int S_A_BYTES = BMW * 128;            // 128 rows x 64 elements, one matrix
+constexpr int S_STAGE = 2 * S_A_BYTES + BN * 128;
+constexpr int S_SMEM = 1024 + SST * S_STAGE + 256 + 2 * (kMaxE + 1) * 4;
+static_assert(S_SMEM <= 232448, "shared memory per CTA");
+
+template <int EPI>
+__global__ void __launch_bounds__(kSThreads, 1)
+    ss_glu_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  const uint32_t st_base = smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SST * S_STAGE);   // [SST]
+  uint64_t* empty = full + SST;                                         // [SST]
+  uint64_t* acc_full = empty + SST;                                     // [2]
+  uint64_t* acc_empty = acc_full + 2;                                   // [2]
+  uint64_t* drain = acc_empty + 2;                                      // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_toff = reinterpret_cast<int*>(smem + SST * S_STAGE + 256);
+  int* s_roff = s_toff + kMaxE + 1;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SST; ++i) {
+      mbar_init(smem_u32(full + i), 1);    // the loader's arrive + the copies' bytes
+      mbar_init(smem_u32(empty + i), 1);   // the MMAs' commit
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(acc_full + i), 1);
+      mbar_init(smem_u32(acc_empty + i), 4);   // the 4 epilogue warps
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+  }
+  if (warp == 1) {
+    // two accumulator buffers of 128 columns (gate and up of a tile of up to
+    // 64 rows each), or both for a larger tile
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();
+  pdl_launch();
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    s_toff[i] = __ldg(p.tile_off + i);
+    s_roff[i] = __ldg(p.row_off + i);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = total_units(p, s_toff);
+  const int nk = p.K / KA;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads (TMA)
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        int unit, r0, nv, e;
+        decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
+        const int n = mma_n(nv);
+        const CUtensorMap* tb = &p.tmB[n / 16 - 1];
+        const int wrow0 = (int)((long long)e * p.rows_per_group + (long long)unit * p.unit_rows);
+        for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+          const uint32_t s = it % SST;
+          if (it >= (uint32_t)SST) {
+            ok = mbar_wait(smem_u32(empty + s), ((it / SST) - 1) & 1, abort_flag, p.status, true,
+                           p.wait_limit);
+            if (!ok) break;
+          }
+          const uint32_t dst = st_base + s * S_STAGE;
+          const uint32_t bar = smem_u32(full + s);
+          // weight rows past the stacked tensor and token rows past R are
+          // zero-filled; token rows past the tile are never stored
+          mbar_arrive_tx(bar, (uint32_t)(2 * S_A_BYTES + n * 128));
+          tma_load_2d(dst, &tmA, kb * KA, wrow0, bar);
+          tma_load_2d(dst + S_A_BYTES, &tmA, kb * KA, wrow0 + p.mat_off, bar);
+          tma_load_2d(dst + 2 * S_A_BYTES, tb, kb * KA, r0, bar);
+        }
+      }
+      for (uint32_t i = 0; i < (uint32_t)SST && i < it; ++i) {
+        const uint32_t last = it - 1 - i;
+        mbar_wait(smem_u32(full + last % SST), (last / SST) & 1, abort_flag, p.status, false);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint64_t da = desc_sw128(st_base), db = desc_sw128(st_base + 2 * S_A_BYTES);
+    const uint32_t alo0 = (uint32_t)da, ahi = (uint32_t)(da >> 32);
+    const uint32_t blo0 = (uint32_t)db, bhi = (uint32_t)(db >> 32);
+    uint32_t it = 0, nb = 0, uses0 = 0, uses1 = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int unit, r0, nv, e;
+      decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
+      const int n = mma_n(nv);
+      const uint32_t idesc = idesc_mma(n, false);      // bf16 operands
+      const bool small = n <= 64;
+      const uint32_t b = small ? nb : 0u;
+      const bool use0 = !small || b == 0, use1 = !small || b == 1;
+      if (use0 && uses0 > 0)
+        ok = mbar_wait_warp(smem_u32(acc_empty + 0), (uses0 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
+      if (ok && use1 && uses1 > 0)
+        ok = mbar_wait_warp(smem_u32(acc_empty + 1), (uses1 - 1) & 1, abort_flag, p.status, true, p.wait_limit);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d0 = tm + (small ? b * 128u : 0u);           // gate
+      const uint32_t d1 = tm + (small ? b * 128u + 64u : 128u);   // up
+      for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+        const uint32_t s = it % SST;
+        ok = mbar_wait_warp(smem_u32(full + s), (it / SST) & 1, abort_flag, p.status, true,
+                            p.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t off = s * (uint32_t)(S_STAGE >> 4);
+        mma_kblock_ss(d0, alo0 + off, ahi, blo0 + off, bhi, idesc, kb == 0);
+        mma_kblock_ss(d1, alo0 + off + (S_A_BYTES >> 4), ahi, blo0 + off, bhi, idesc, kb == 0);
+        mma_commit_warp(smem_u32(empty + s));
+      }
+      if (!ok) break;
+      if (use0) { mma_commit_warp(smem_u32(acc_full + 0)); ++uses0; }
+      if (use1) { mma_commit_warp(smem_u32(acc_full + 1)); ++uses1; }
+      if (small) nb ^= 1u;
+    }
+    mma_commit_warp(smem_u32(drain));
+    mbar_wait_warp(smem_u32(drain), 0, abort_flag, p.status, false);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    constexpr int kAct = Epi<EPI>::geglu ? MOE_ACT_GEGLU_TANH : MOE_ACT_SWIGLU;
+    const int qd = warp & 3;
+    const int m = qd * 32 + lane;                     // feature of the unit
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    uint32_t nb = 0, uses0 = 0, uses1 = 0, hmax = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      int unit, r0, nv, e;
+      decode_unit(p, s_toff, s_roff, u, unit, r0, nv, e);
+      const bool small = mma_n(nv) <= 64;
+      const uint32_t b = small ? nb : 0u;
+      const bool use0 = !small || b == 0, use1 = !small || b == 1;
+      if (use0 && !mbar_wait_warp(smem_u32(acc_full + 0), uses0 & 1, abort_flag, p.status, true, p.wait_limit)) break;
+      if (use1 && !mbar_wait_warp(smem_u32(acc_full + 1), uses1 & 1, abort_flag, p.status, true, p.wait_limit)) break;
+      tc_fence_after();
+      const uint32_t c0 = tl + (small ? b * 128u : 0u);
+      const uint32_t c1 = tl + (small ? b * 128u + 64u : 128u);
+      __half* hp = reinterpret_cast<__half*>(p.out) + (size_t)r0 * p.out_ld + unit * p.unit_rows + m;
+      for (int n0 = 0; n0 < nv; n0 += 16) {
+        uint32_t a0[16], a1[16];
+        tmem_ld16x2(c0 + n0, c1 + n0, a0, a1);
+        const int lim = nv - n0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const __half v = __float2half_rn(glu(kAct, __uint_as_float(a0[j]), __uint_as_float(a1[j])));
+          if (j < lim) {
+            hmax = max(hmax, (uint32_t)__half_as_ushort(v) & 0x7FFFu);
+            hp[(size_t)(n0 + j) * p.out_ld] = v;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (use0) mbar_arrive(smem_u32(acc_empty + 0));
+        if (use1) mbar_arrive(smem_u32(acc_empty + 1));
+      }
+      if (use0) ++uses0;
+      if (use1) ++uses1;
+      if (small) nb ^= 1u;
+    }
+    if (!__all_sync(0xffffffffu, hmax < 0x7C00u) && lane == 0) report_status(p.status, MOE_ERR_RANGE);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ router
 
 // Router logits on the tensor cores, both operands staged in shared memory
@@ -972,44 +1214,7 @@ struct RouterParams {
   long long wait_limit;
 };
 
-// D[tmem] (+)= A[smem] * B[smem]^T for one 64-deep k-block (four K-steps of
-// 16; both descriptors advance 32 bytes inside the 128-byte swizzle atom);
-// accumulate unless `first`. Warp-uniform operands, one elected lane issues.
-__device__ __forceinline__ void mma_kblock_ss(uint32_t d, uint32_t alo, uint32_t ahi, uint32_t blo,
-                                              uint32_t bhi, uint32_t idesc, uint32_t first) {
-  asm volatile(
-      "{\n\t.reg .pred pf, pt, e;\n\t.reg .b64 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.eq.b32 pf, %6, 0;\n\t"
-      "setp.ne.b32 pt, %5, 0;\n\t"
-      "mov.b64 a0, {%1, %2};\n\tmov.b64 b0, {%3, %4};\n\t"
-      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
-      "mov.b64 a1, {%1, %2};\n\tmov.b64 b1, {%3, %4};\n\t"
-      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
-      "mov.b64 a2, {%1, %2};\n\tmov.b64 b2, {%3, %4};\n\t"
-      "add.u32 %1, %1, 2;\n\tadd.u32 %3, %3, 2;\n\t"
-      "mov.b64 a3, {%1, %2};\n\tmov.b64 b3, {%3, %4};\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a0, b0, %5, pf;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %5, pt;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %5, pt;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %5, pt;\n\t}\n"
-      : "+r"(d), "+r"(alo), "+r"(ahi), "+r"(blo), "+r"(bhi)
-      : "r"(idesc), "r"(first)
-      : "memory");
-}
 
-// 16 columns of this warp's 32 lanes from one TMEM address, and the wait
-__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t (&a)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
-        "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]),
-        "=r"(a[14]), "=r"(a[15])
-      : "r"(ta)
-      : "memory");
-}
 
 __global__ void __launch_bounds__(kRThreads, 1)
     router_tc_kernel(const __grid_constant__ RouterParams p, const __grid_constant__ CUtensorMap tmW,
@@ -1411,7 +1616,13 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   // q4 weights are dequantised in a permuted K order, so are the token rows
   const unsigned gblocks = (unsigned)((R + 3) / 4);
   const bool q4 = q4_group(ex.fmt) != 0;
-  if (q4 && dt == MOE_F16)
+  // bf16 weights with bf16 activations: both operands stay bf16 (the rows are
+  // gathered as they are) and go to the tensor core without conversion
+  const bool bf16_ss = ex.fmt == MOE_W_BF16 && dt == MOE_BF16;
+  if (bf16_ss)
+    launch_pdl(gather_f16_kernel<false, true>, gblocks, 256, 0, s, (const uint4*)x, row_map,
+               (long long)R, ex.d / 8, (uint4*)xs16, status);
+  else if (q4 && dt == MOE_F16)
     launch_pdl(gather_f16_kernel<true, true>, gblocks, 256, 0, s, (const uint4*)x, row_map,
                (long long)R, ex.d / 8, (uint4*)xs16, status);
   else if (q4)
@@ -1428,7 +1639,7 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   CUtensorMap ta;
   if (!weight_map(&ta, ex.fmt, ex.w_gu, (long long)ex.E * 2 * ex.F, ex.d)) return cudaErrorInvalidValue;
   Params p{};
-  if (!token_maps(p, xs16, false, R, ex.d)) return cudaErrorInvalidValue;
+  if (!token_maps(p, xs16, bf16_ss, R, ex.d)) return cudaErrorInvalidValue;
   p.row_off = row_off;
   p.tile_off = tile_off;
   p.E = ex.E;
@@ -1448,6 +1659,14 @@ cudaError_t launch_swiglu_tc(const void* x, int dt, int T, const uint32_t* row_m
   p.wait_limit = wait_cycles();
   const long long ub = max_tiles(R, ex.E, BN) * p.n_units;
   const bool geglu = ex.act == MOE_ACT_GEGLU_TANH;
+  if (bf16_ss) {
+    auto kern = geglu ? ss_glu_kernel<EPI_GEGLU> : ss_glu_kernel<EPI_SWIGLU>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM);
+    if (e != cudaSuccess) return e;
+    const long long grid = ub < num_sms() ? ub : num_sms();
+    launch_pdl(kern, (unsigned)grid, kSThreads, S_SMEM, s, p, ta);
+    return cudaGetLastError();
+  }
   // h in the permuted K order only for q4 weights (the down kernel then
   // dequantises in that order)
   if (q4 && h_perm)
