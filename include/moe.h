@@ -236,13 +236,15 @@ moe_status moe_sort_rows_noalloc(const int32_t* topk_idx, int T, int k, int E, i
  *            g = x[row_map[i]] . w_gu[e][f],
  *            u = x[row_map[i]] . w_gu[e][F+f], e = expert of row i
  *   ws       (device) scratch of moe_grouped_swiglu_workspace(T, k, d, dt)
- *            bytes (the token rows in fp16: x converted, or, in the
- *            tensor-core regime, gathered into sorted row order); required
+ *            bytes (the token rows in 16 bits: x converted to fp16, or, in
+ *            the tensor-core regime, gathered into sorted row order); required
  *            for 16-bit activations, may be NULL for fp32
  * fp32 accumulation; h rounded once. The tensor-core regime multiplies fp16
  * operands (fp16 x as is, bf16 x converted exactly when |x| < 65520, weights
  * dequantised to fp16); values outside fp16 range are reported as
- * MOE_ERR_RANGE in the device status. */
+ * MOE_ERR_RANGE in the device status. bf16 experts with bf16 activations are
+ * multiplied as bf16 (the same products, exact in fp32; no range limit on
+ * x). */
 size_t moe_grouped_swiglu_workspace(int T, int k, int d, moe_dtype dt);
 moe_status moe_grouped_swiglu(const void* x, moe_dtype dt, const uint32_t* row_map,
                               const int32_t* row_off, const int32_t* tile_off, int BM, int T, int k,
@@ -290,10 +292,12 @@ moe_status moe_forward(const void* x, moe_dtype dt, const void* w_router, const 
 /* Where moe_forward keeps each intermediate inside its workspace (byte
  * offsets), the regime it resolves to for experts of weight format wfmt and
  * the BM it sorts with. moe_forward_workspace(...) is its `total`; 0 when the
- * arguments are invalid. With q4 experts the whole-layer call may keep h and
- * the fp16 token rows x16 with every 8 consecutive elements in the order
- * (0, 4, 1, 5, 2, 6, 3, 7), the K order its kernels dequantise in; the
- * routing and sort tables have the layouts moe_route and moe_sort_rows give. */
+ * arguments are invalid. x16 holds 16-bit token rows: fp16, or bf16 as
+ * given for bf16 experts with bf16 activations on the tensor cores. With q4
+ * experts the whole-layer call may keep h and x16 with every 8 consecutive
+ * elements in the order (0, 4, 1, 5, 2, 6, 3, 7), the K order its kernels
+ * dequantise in; the routing and sort tables have the layouts moe_route and
+ * moe_sort_rows give. */
 typedef struct {
   size_t logits, topk_idx, topk_w, order, inv_order, row_map, counts, row_off, tile_off;
   size_t sort_ws, h, ys, x16, total;
