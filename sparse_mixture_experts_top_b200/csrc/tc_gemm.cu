@@ -1468,8 +1468,9 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ i
 // sorted rows per block (8 values per thread per load); values that do not round to a
 // finite fp16 are reported as MOE_ERR_RANGE (they become +-inf). PERM stores
 // every 8 consecutive elements in the order (0, 4, 1, 5, 2, 6, 3, 7), the K
-// order of dequant_word_perm. SRC16 takes fp16 rows, copied (and permuted)
-// as they are.
+// order of dequant_word_perm. SRC16 takes 16-bit rows and copies (and
+// permutes) their bits as they are: fp16 x for the fp16 operand path, bf16 x
+// for the bf16 gate|up kernel.
 template <bool PERM, bool SRC16 = false>
 __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict__ x,
                                                          const uint32_t* __restrict__ row_map,
