@@ -445,8 +445,10 @@ def main():
             return
         layer = mi.make_layer(wl, seed=args.seed, device="cpu")
         cb = cpu_baseline(layer, budget_s=min(60.0, max(5.0, 1.0 * args.steps)))
+        # ms_per_step: one step of the whole workload at the sample's rate
         line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": wl.T / cb["value"] * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic", "config": config,
                 "cpu_baseline": cb,

@@ -44,3 +44,26 @@ def test_prefill_layer_bytes_match_reported_figure():
 ])
 def test_kernels_per_forward(T, k, tc, fused, launches):
     assert bench.kernels_per_forward(T, k, tc, fused) == launches
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` (the oracle on the host's cores) prints the
+    contract's JSON line with the reference keys, on a small workload."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert abs(line["ms_per_step"] - 16 / line["value"] * 1e3) < 1e-9 * line["ms_per_step"] + 1e-12
