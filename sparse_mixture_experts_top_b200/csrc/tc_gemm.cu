@@ -1502,24 +1502,24 @@ __global__ void __launch_bounds__(256) gather_f16_kernel(const uint4* __restrict
       } else {
         dst[c] = v;
       }
-      continue;
-    }
-    float f[8];
+    } else {
+      float f[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      f[2 * j] = __uint_as_float(w[j] << 16);
-      f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-    uint32_t o[4];
+      for (int j = 0; j < 4; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+      uint32_t o[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = PERM ? f[j] : f[2 * j], hi = PERM ? f[j + 4] : f[2 * j + 1];
-      ok &= fabsf(lo) < 65520.f && fabsf(hi) < 65520.f;
-      uint32_t dd;
-      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(dd) : "f"(hi), "f"(lo));
-      o[j] = dd;
+      for (int j = 0; j < 4; ++j) {
+        const float lo = PERM ? f[j] : f[2 * j], hi = PERM ? f[j + 4] : f[2 * j + 1];
+        ok &= fabsf(lo) < 65520.f && fabsf(hi) < 65520.f;
+        uint32_t dd;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(dd) : "f"(hi), "f"(lo));
+        o[j] = dd;
+      }
+      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   if (!ok) report_status(status, MOE_ERR_RANGE);
 }
